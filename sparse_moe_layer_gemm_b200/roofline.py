@@ -1,0 +1,25 @@
+"""Roofline accounting of the MoE FFN layer forward: the bytes it must move at
+least once and the flops it must execute, per workload and routing outcome."""
+from __future__ import annotations
+
+from .workloads import Workload
+
+
+def algorithmic_bytes(wl: Workload, touched_routed: int) -> int:
+    """Bytes the layer must move at least once: the touched routed experts plus
+    the shared expert (gate, up, down), the fp32 router weight and bias, the
+    input x and the output (same dtype as x)."""
+    el_w = 2 if wl.weight_dtype == "bf16" else 4
+    el_x = 2 if wl.act_dtype == "bf16" else 4
+    H, I, Is, E = wl.hidden, wl.intermediate, wl.shared_intermediate, wl.num_experts
+    experts = touched_routed * 3 * H * I * el_w + 3 * H * Is * el_w
+    router = H * E * 4 + E * 4
+    act = 2 * wl.T * H * el_x
+    return experts + router + act
+
+
+def algorithmic_flops(wl: Workload) -> int:
+    """Multiply-adds x2 of the router and of k routed + 1 shared SwiGLU experts."""
+    H, I, Is, E, k = wl.hidden, wl.intermediate, wl.shared_intermediate, wl.num_experts, wl.top_k
+    per_tok = 2 * H * E + k * (2 * H * 2 * I + 2 * I * H) + (2 * H * 2 * Is + 2 * Is * H)
+    return wl.T * per_tok
