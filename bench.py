@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Benchmark of the Step-3.5-Flash MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode] [--secondary prefill|none]
+
+One step = one whole layer forward (router, top-k, counting sort, gather,
+grouped gate|up GEMM + SwiGLU, grouped down GEMM, combine) over one batch of
+T synthetic tokens, inputs already resident in HBM.  Weights are streamed
+from HBM every step (touched experts: ~4 GB at T=64, ~6 GB at T=4096, far
+larger than the 126 MB L2), so no L2 flush is needed between steps.
+
+Multi-GPU (torchrun): every rank holds a replica of the layer and runs its own
+batch (weak scaling, no collective on the data path); the step time is the
+max over ranks.  Prints ONE JSON line on rank 0.
+
+``--impl reference`` times the CPU fp64 oracle (the method's plain
+definition) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at T=64 and T=4096; achieved fraction of HBM/TC roofline"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode")
+    ap.add_argument("--secondary", default="prefill")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], tc=d["bf16_tflops"], tc_sustained=d.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, source="fallback")
+
+
+def _traffic_record(kernel: str, workload: str):
+    """ncu DRAM bytes per launch of `kernel`, if the committed capture still
+    matches the kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        recs = json.load(open(p))
+        rec = recs.get(f"{kernel}:{workload}")
+        if rec is None:
+            return None
+        src = os.path.join(ROOT, rec["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        return rec["bytes_per_launch"] if h == rec["source_sha256"] else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [s for s in sm if mx is None or s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle arm
+
+def _oracle_sample(wl, x_host, rw, rb, experts, rows):
+    import oracle.moe_oracle as om
+    t0 = time.perf_counter()
+    om.moe_forward_rows(rows, x_host, rw, rb, experts["w_gate"], experts["w_up"],
+                        experts["w_down"], experts["sh_gate"], experts["sh_up"],
+                        experts["sh_down"], top_k=wl.top_k, scale=wl.scale,
+                        swiglu_limit=wl.swiglu_limit, swiglu_limit_shared=wl.swiglu_limit_shared)
+    return time.perf_counter() - t0
+
+
+class _PrefetchedExperts:
+    """Host fp32 copies of the experts a sample touches (inputs in RAM before timing)."""
+
+    def __init__(self, fetch, ids):
+        self.m = {e: fetch(e) for e in ids}
+
+    def __getitem__(self, e):
+        return self.m[e]
+
+
+def _sample_inputs_host(wl, x_host, rw, rb, rows, fetch_expert, shared):
+    import oracle.moe_oracle as om
+    r = om.moe_routing(x_host[rows], rw, rb, top_k=wl.top_k, scale=wl.scale)
+    ids = sorted(set(int(e) for e in r["topk_idx"].reshape(-1)))
+    got = {e: fetch_expert(e) for e in ids}
+    experts = dict(w_gate=_PrefetchedExperts(lambda e: got[e][0], ids),
+                   w_up=_PrefetchedExperts(lambda e: got[e][1], ids),
+                   w_down=_PrefetchedExperts(lambda e: got[e][2], ids),
+                   sh_gate=shared[0], sh_up=shared[1], sh_down=shared[2])
+    return experts, len(ids)
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    from sparse_moe_layer_gemm_b200.workloads import (WORKLOADS, draw_expert, draw_router,
+                                                      draw_shared, draw_x)
+    wl = WORKLOADS[a.workload]
+    cores = len(os.sched_getaffinity(0))
+    x = draw_x(wl, "cpu").float().numpy()
+    rw, rb = (t.float().numpy() for t in draw_router(wl, "cpu"))
+    sample = 1 if wl.hidden >= 4096 else wl.T
+    rows = np.arange(sample)
+
+    def fetch(e):
+        return tuple(t.float().numpy() for t in draw_expert(wl, e, "cpu"))
+    shared = tuple(t.float().numpy() for t in draw_shared(wl, "cpu"))
+    experts, touched = _sample_inputs_host(wl, x, rw, rb, rows, fetch, shared)
+    for _ in range(a.warmup):
+        _oracle_sample(wl, x, rw, rb, experts, rows)
+    secs = [_oracle_sample(wl, x, rw, rb, experts, rows) for _ in range(a.steps)]
+    total = sum(secs)
+    value = sample * a.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": 1e3 * total / a.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "hidden": wl.hidden,
+                   "experts": wl.num_experts, "top_k": wl.top_k,
+                   "intermediate": wl.intermediate},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{sample} of {wl.T} tokens per step ({touched} routed experts "
+                                   f"+ shared, weights drawn on the host, in RAM before timing)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def _measure(layer, x, steps, warmup, stream, record_stages=True):
+    """Times exactly `steps` forwards (after `warmup`) with CUDA events on the
+    launching stream; returns (ms per step, per-stage ms per step)."""
+    import torch
+    from sparse_moe_layer_gemm_b200 import binding as B
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            layer.forward(x)
+        torch.cuda.synchronize()
+        if record_stages:
+            B.moe_set_stage_timing(layer.handle, steps)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            layer.forward(x)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    stages = None
+    if record_stages:
+        tot, n = B.moe_get_stage_times(layer.handle)
+        stages = {k: v / max(n, 1) for k, v in tot.items()}
+        B.moe_set_stage_timing(layer.handle, 0)
+    return ms, stages
+
+
+def _routing_stats(layer, x):
+    import torch
+    out, rt = layer.forward(x, routing=True)
+    torch.cuda.synchronize()
+    counts = rt["counts"].cpu()
+    return int((counts > 0).sum()), int(counts.max())
+
+
+def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step):
+    from sparse_moe_layer_gemm_b200.roofline import (algorithmic_bytes, algorithmic_flops,
+                                                     gate_up_bytes, gate_up_flops)
+    gu_ms = stages_ms["gate_up"]
+    gu_bytes = gate_up_bytes(wl, touched)
+    gu_flops = gate_up_flops(wl)
+    t_bytes = gu_bytes / (peaks["hbm"] * 1e9)
+    t_flops = gu_flops / (peaks["tc"] * 1e12)
+    if t_bytes >= t_flops:
+        ach = gu_bytes / (gu_ms * 1e-3) / 1e9
+        rl = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+              "frac": ach / peaks["hbm"]}
+    else:
+        ach = gu_flops / (gu_ms * 1e-3) / 1e12
+        rl = {"bound": "tensor", "achieved": ach, "peak": peaks["tc"], "unit": "TFLOP/s",
+              "frac": ach / peaks["tc"]}
+    rl.update({"kernel": "grouped_gemm_kernel<gate_up>", "kernel_ms": gu_ms,
+               "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
+               "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json)"
+               if peaks["source"] == "measured" else "fallback",
+               "traffic": _traffic_record("gate_up", wl.name)})
+    lb = algorithmic_bytes(wl, touched)
+    lf = algorithmic_flops(wl)
+    t_layer = max(lb / (peaks["hbm"] * 1e9), lf / (peaks["tc"] * 1e12))
+    layer = {"bound": "hbm" if lb / peaks["hbm"] >= lf / (peaks["tc"] * 1e3) else "tensor",
+             "roofline_ms": 1e3 * t_layer, "frac": 1e3 * t_layer / ms_step,
+             "bytes": lb, "flops": lf, "touched_experts": touched}
+    return rl, layer
+
+
+def run_ours(a):
+    import torch
+    import torch.distributed as dist
+    from dataclasses import replace
+    from sparse_moe_layer_gemm_b200 import binding as B
+    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS, draw_x, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B.load_library()
+    wl = WORKLOADS[a.workload]
+    peaks = _peaks()
+
+    inp = make_inputs(wl, dev)                          # weights replicated on every rank
+    x = draw_x(replace(wl, seed=rank), dev)             # each rank its own batch
+    layer = B.MoeLayer.from_workload(wl)
+    layer.load_inputs(inp)
+    stream = torch.cuda.Stream(device=dev)
+    touched, max_rows = _routing_stats(layer, x)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        gpu_id = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+    except Exception:
+        gpu_id = str(local)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(a.warmup):
+            layer.forward(x)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms, stages = _measure(layer, x, a.steps, 0, stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    err = layer.device_error()
+    if err != 0:
+        raise RuntimeError(f"device status word {err}")
+    value = world * wl.T / (ms * 1e-3)
+    kr, lr = _kernel_roofline(wl, touched, stages, peaks, ms)
+
+    e2e = None
+    if not a.no_e2e:
+        xh = x.cpu().pin_memory()
+        oh = torch.empty_like(xh).pin_memory()
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, a.warmup)):
+                layer.forward_host(xh, oh, stream=stream)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            n = a.steps
+            e0.record(stream)
+            for _ in range(n):
+                layer.forward_host(xh, oh, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        et = torch.tensor([e0.elapsed_time(e1) / n], device=dev)
+        if world > 1:
+            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        el = 2 if wl.act_dtype == "bf16" else 4
+        e2e = {"value": world * wl.T / (float(et.item()) * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": wl.T * wl.hidden * el,
+               "d2h_bytes_per_step": wl.T * wl.hidden * el,
+               "path": "moe_forward_host (pinned host x/out, copies inside the timed region)"}
+
+    secondary = None
+    if a.secondary and a.secondary != "none" and a.secondary != a.workload:
+        wl2 = WORKLOADS[a.secondary]
+        same_weights = (wl2.expert_std == wl.expert_std and wl2.weight_dtype == wl.weight_dtype
+                        and wl2.bias == wl.bias and wl2.hidden == wl.hidden)
+        if same_weights:
+            x2 = draw_x(replace(wl2, seed=rank), dev)
+            l2 = layer
+            touched2, _ = _routing_stats(l2, x2)
+            barrier()
+            ms2, st2 = _measure(l2, x2, max(3, a.steps // 10), max(3, a.warmup), stream)
+            t2 = torch.tensor([ms2], device=dev)
+            if world > 1:
+                dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+            ms2 = float(t2.item())
+            kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2)
+            secondary = {"workload": wl2.name, "T": wl2.T, "value": world * wl2.T / (ms2 * 1e-3),
+                         "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
+                         "layer_roofline": lr2, "stage_ms": st2}
+            del x2
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = _cpu_baseline_from_device(wl, inp, x)
+
+    launches = B.moe_kernel_launches(layer.handle, wl.T) * a.steps
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "hidden": wl.hidden,
+                       "experts": wl.num_experts, "top_k": wl.top_k,
+                       "intermediate": wl.intermediate, "shared_experts": 1,
+                       "parallelism": f"replicas x{world} (weak)",
+                       "l2": "inputs larger than L2: touched expert weights streamed from HBM "
+                             "every step"},
+            "roofline": kr, "layer_roofline": lr, "stage_ms": stages,
+            "routing": {"touched_experts": touched, "max_rows_per_expert": max_rows},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def _cpu_baseline_from_device(wl, inp, x):
+    """The oracle on the host cores on a bounded sample of the same batch
+    (weights copied from the device before timing)."""
+    import numpy as np
+    from sparse_moe_layer_gemm_b200.workloads import host_f32
+    xh = host_f32(x)
+    rw = host_f32(inp["router_w"])
+    rb = host_f32(inp["router_bias"])
+    sample = min(wl.T, 8)
+    rows = np.arange(sample)
+
+    def fetch(e):
+        return (host_f32(inp["w_gate"][e]), host_f32(inp["w_up"][e]), host_f32(inp["w_down"][e]))
+    shared = (host_f32(inp["sh_gate"]), host_f32(inp["sh_up"]), host_f32(inp["sh_down"]))
+    experts, touched = _sample_inputs_host(wl, xh, rw, rb, rows, fetch, shared)
+    secs = _oracle_sample(wl, xh, rw, rb, experts, rows)
+    return {"value": sample / secs, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{sample} of {wl.T} tokens of the same batch, {touched} routed experts "
+                      f"+ shared, fp64 NumPy, weights in host RAM before timing",
+            "seconds": secs}
+
+
+def main():
+    a = _args()
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_ours(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,185 @@
+/*
+ * moe.h — C ABI of libmoe.so: the forward pass of the Step-3.5-Flash sparse
+ * MoE FFN layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (sglang-jax issue #1367 "[Feature] Support Step 3.5 Flash",
+ * section "Model configuration", MoE bullet, and section "Key difficulties",
+ * item 1; llm-atlas "Step-3.5-Flash", table "Raw config fields"):
+ *
+ *   l   = x . W_r                       router logits, fp32 (need_fp32_gate)
+ *   s   = sigmoid(l)                    fp32 scores (moe_router_activation)
+ *   S   = top-k of (s + b)              the bias selects only (use_moe_router_bias)
+ *   g_j = 3 * s_{S_j} / sum_j s_{S_j}   bias-free, renormalised (norm_expert_weight),
+ *                                       scaled (moe_router_scaling_factor 3)
+ *   out = sum_j g_j * f_{S_j}(x) + f_shared(x)
+ *   f(x) = (silu(gate) * up) . W_down,  gate = x . W_gate, up = x . W_up,
+ *          with the optional clamp gate = min(gate, L), up = clip(up, -L, L)
+ *          (swiglu_limits / swiglu_limits_shared; L = 0 means no clamp).
+ *
+ * Selection order and ties: descending s + b, equal scores to the lower
+ * expert index.  The shared expert has no gate and weight 1.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers unless the name says _host.
+ *    They are owned by the caller; the library never frees or keeps them past
+ *    the call, except that a layer handle owns its own packed weight copy.
+ *  - Layouts are row-major: x [T, H], out [T, H], router_w [H, E],
+ *    router_bias [E], w_gate / w_up [E, H, I], w_down [E, I, H],
+ *    sh_gate / sh_up [H, Is], sh_down [Is, H].
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Work is enqueued on it; no entry point synchronises the host
+ *    unless its comment says so.
+ *  - Every entry point returns a moe_status_t.  Arguments are checked on the
+ *    host first; on any error nothing is enqueued and outputs are untouched.
+ *  - T = 0 is a valid no-op.
+ */
+#ifndef SPARSE_MOE_LAYER_GEMM_B200_MOE_H
+#define SPARSE_MOE_LAYER_GEMM_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,     /* null pointer, negative size, bad enum */
+  MOE_ERR_UNSUPPORTED = 2,     /* valid but outside what the kernels handle */
+  MOE_ERR_WORKSPACE = 3,       /* workspace missing, too small or misaligned */
+  MOE_ERR_CUDA = 4,            /* a CUDA runtime call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5,  /* a kernel gave up a bounded wait (device error word) */
+  MOE_ERR_NOT_LOADED = 6       /* moe_forward before moe_load_weights */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+/* Layer configuration.  Field names follow the model's config fields
+ * (llm-atlas "Step-3.5-Flash", "Raw config fields").
+ * Supported: hidden % 128 == 0, 1 <= hidden <= 16384; 1 <= num_experts <= 1024;
+ * 1 <= top_k <= min(num_experts, 32); 1 <= intermediate <= 8192;
+ * shared_intermediate == intermediate; act_dtype, weight_dtype in {F32, BF16};
+ * routed_scaling_factor finite; swiglu limits >= 0 (0 = no clamp). */
+typedef struct {
+  int hidden;                  /* H: hidden_size, 4096 */
+  int num_experts;             /* E: moe_num_experts, 288 */
+  int top_k;                   /* k: moe_top_k, 8 */
+  int intermediate;            /* I: moe_intermediate_size, 1280 */
+  int shared_intermediate;     /* Is: share_expert_dim, 1280 */
+  int norm_expert_weight;      /* 1: renormalise the top-k scores */
+  float routed_scaling_factor; /* 3.0 */
+  int use_router_bias;         /* 1: add router_bias to the scores for selection */
+  float swiglu_limit;          /* routed experts' clamp, 0 = none */
+  float swiglu_limit_shared;   /* shared expert's clamp, 0 = none */
+  int act_dtype;               /* moe_dtype_t of x and out */
+  int weight_dtype;            /* moe_dtype_t of the expert weights passed to load */
+} moe_config_t;
+
+typedef struct moe_layer moe_layer_t;
+
+/* Optional routing outputs of moe_forward (device pointers, caller-owned;
+ * any field may be NULL).  topk_idx [T, k] int32 (descending s + b),
+ * topk_w [T, k] fp32 gate weights, counts [E] int32 pairs per expert,
+ * offsets [E + 1] int32 exclusive prefix of counts, perm [T * k] int32 pair
+ * ids t * k + j grouped by expert, ascending t within an expert. */
+typedef struct {
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+} moe_routing_t;
+
+/* Host-only check of a configuration; no CUDA call.  Returns MOE_OK,
+ * MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED. */
+int moe_config_check(const moe_config_t* cfg);
+
+/* Creates a layer on the current CUDA device.  Allocates the packed weight
+ * copy (3 * (E + 1) * H * round_up(I, 128) bf16 plus the router) and a small
+ * device status word.  *out receives the handle (NULL on error). */
+int moe_create(const moe_config_t* cfg, moe_layer_t** out);
+
+/* Copies the weights into the layer's packed bf16 layout on `stream`
+ * (K-major weight rows; gate and up interleaved in blocks of 128 rows; fp32
+ * expert weights are rounded to bf16).  router_w [H, E] and router_bias [E]
+ * are fp32 and kept fp32; router_bias may be NULL (zero bias).  The expert
+ * pointers have the config's weight_dtype.  The caller's buffers may be
+ * freed once `stream` has passed this call. */
+int moe_load_weights(moe_layer_t* layer, const float* router_w, const float* router_bias,
+                     const void* w_gate, const void* w_up, const void* w_down,
+                     const void* sh_gate, const void* sh_up, const void* sh_down,
+                     void* stream);
+
+/* Device workspace bytes moe_forward needs for T tokens (caller allocates,
+ * 256-byte aligned).  Host-only. */
+int moe_workspace_size(const moe_layer_t* layer, int T, size_t* bytes);
+
+/* The layer forward: out [T, H] (act_dtype) from x [T, H] (act_dtype).
+ * Stream-ordered, no host synchronisation, capturable in a CUDA graph once
+ * the weights are loaded.  `routing` may be NULL.  x and out must not alias. */
+int moe_forward(moe_layer_t* layer, const void* x, int T, void* out,
+                void* workspace, size_t ws_bytes, void* stream,
+                const moe_routing_t* routing);
+
+/* Workspace bytes for moe_forward_host: moe_workspace_size plus device
+ * staging for x and out. */
+int moe_workspace_size_host(const moe_layer_t* layer, int T, size_t* bytes);
+
+/* The forward from and to HOST buffers: copies x_host to the device, runs
+ * moe_forward, copies the result to out_host, all on `stream`, then
+ * synchronises `stream` before returning.  Pinned host memory makes the
+ * copies asynchronous DMA; pageable memory also works. */
+int moe_forward_host(moe_layer_t* layer, const void* x_host, int T, void* out_host,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises the device, then reads and clears the layer's device status
+ * word: *device_err = 0 when no kernel reported a problem, otherwise a bit
+ * mask (1 = a bounded wait timed out in a GEMM kernel).  Returns
+ * MOE_ERR_DEVICE_TIMEOUT when the word was non-zero. */
+int moe_get_device_error(moe_layer_t* layer, int* device_err);
+
+/* Static description of a status code. */
+const char* moe_status_string(int status);
+
+/* Frees the layer and its device memory.  NULL is ignored.  Synchronises
+ * the device first. */
+void moe_destroy(moe_layer_t* layer);
+
+/* Stages of one forward, in launch order, for the stage timers below:
+ * 0 router logits, 1 top-k and gate weights, 2 counting sort (3 kernels),
+ * 3 gather of the input rows, 4 grouped gate|up GEMM + SwiGLU,
+ * 5 grouped down GEMM x gate weight, 6 combine. */
+#define MOE_NUM_STAGES 7
+
+/* Kernel launches one moe_forward makes for T tokens (0 for T = 0). */
+int moe_kernel_launches(const moe_layer_t* layer, int T);
+
+/* Per-stage device timing.  With capacity > 0 each following moe_forward
+ * records CUDA events around its stages on its own stream, for up to
+ * `capacity` forwards (later forwards are not recorded); capacity 0 turns
+ * timing off and frees the events.  Host-side setup only. */
+int moe_set_stage_timing(moe_layer_t* layer, int capacity);
+
+/* Waits for the recorded events, writes the summed milliseconds of each stage
+ * over the recorded forwards to ms[0 .. n_stages-1] (n_stages <=
+ * MOE_NUM_STAGES) and their number to *n_forwards, then starts a new
+ * recording window of the same capacity. */
+int moe_get_stage_times(moe_layer_t* layer, float* ms, int n_stages, int* n_forwards);
+
+/* One call with the layer's argument list: creates a layer, loads the
+ * weights, allocates a workspace, runs the forward on `stream`, synchronises
+ * and frees everything.  Convenient for a single forward; for repeated calls
+ * use create / load / forward.  Allocates device memory (cudaMalloc). */
+int moe_forward_oneshot(const void* x, const float* router_w, const float* router_bias,
+                        const void* w_gate, const void* w_up, const void* w_down,
+                        const void* sh_gate, const void* sh_up, const void* sh_down,
+                        int T, int H, int E, int k, int I, float scale,
+                        float swiglu_limit, float swiglu_limit_shared,
+                        int act_dtype, int weight_dtype, void* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_MOE_LAYER_GEMM_B200_MOE_H */

@@ -62,6 +62,7 @@ __all__ = [
     "gate_weights",
     "swiglu_expert",
     "expert_permutation",
+    "moe_routing",
     "moe_forward",
     "moe_forward_rows",
     "moe_forward_dense_masked",
@@ -244,6 +245,19 @@ def _route(x, router_w, router_bias, top_k, scale, norm, use_bias, forced_idx):
     s_sel = np.take_along_axis(s32, idx.astype(np.int64), axis=1)
     w = gate_weights(s_sel, scale, norm)
     return logits, beta32, idx, w
+
+
+def moe_routing(x, router_w, router_bias, *, top_k: int, scale: float = 3.0,
+                norm: bool = True, use_bias: bool = True):
+    """Routing of every token without the expert FFNs: (topk_idx, topk_w,
+    counts, offsets, perm, pos, beta32, tie_gap).  Same steps as
+    :func:`moe_forward` (sglang-jax issue #1367, "Key difficulties" item 1)."""
+    x64 = _f64(x)
+    E = np.asarray(router_w).shape[1]
+    _, beta32, idx, w = _route(x64, router_w, router_bias, top_k, scale, norm, use_bias, None)
+    counts, offsets, perm, pos = expert_permutation(idx, E)
+    return dict(topk_idx=idx, topk_w=w, counts=counts, offsets=offsets, perm=perm, pos=pos,
+                beta32=beta32, tie_gap=near_tie_gaps(beta32, top_k))
 
 
 def moe_forward(x, router_w, router_bias, w_gate, w_up, w_down,

@@ -1,0 +1,340 @@
+"""ctypes binding of libmoe.so (include/moe.h).
+
+Argument marshalling only: torch tensors are checked for device, dtype and
+contiguity and passed as raw device pointers together with torch's current
+CUDA stream.  Every step of the layer runs in the library's kernels.  If the
+library is missing, :func:`load_library` raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE_TIMEOUT = 5
+MOE_ERR_NOT_LOADED = 6
+MOE_F32 = 0
+MOE_BF16 = 1
+
+# every symbol include/moe.h declares
+EXPORTS = (
+    "moe_config_check", "moe_create", "moe_load_weights", "moe_workspace_size",
+    "moe_forward", "moe_workspace_size_host", "moe_forward_host", "moe_get_device_error",
+    "moe_status_string", "moe_destroy", "moe_forward_oneshot", "moe_kernel_launches",
+    "moe_set_stage_timing", "moe_get_stage_times",
+)
+MOE_NUM_STAGES = 7
+STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
+
+
+class moe_config_t(ctypes.Structure):
+    _fields_ = [
+        ("hidden", ctypes.c_int),
+        ("num_experts", ctypes.c_int),
+        ("top_k", ctypes.c_int),
+        ("intermediate", ctypes.c_int),
+        ("shared_intermediate", ctypes.c_int),
+        ("norm_expert_weight", ctypes.c_int),
+        ("routed_scaling_factor", ctypes.c_float),
+        ("use_router_bias", ctypes.c_int),
+        ("swiglu_limit", ctypes.c_float),
+        ("swiglu_limit_shared", ctypes.c_float),
+        ("act_dtype", ctypes.c_int),
+        ("weight_dtype", ctypes.c_int),
+    ]
+
+
+class moe_routing_t(ctypes.Structure):
+    _fields_ = [
+        ("topk_idx", ctypes.c_void_p),
+        ("topk_w", ctypes.c_void_p),
+        ("counts", ctypes.c_void_p),
+        ("offsets", ctypes.c_void_p),
+        ("perm", ctypes.c_void_p),
+    ]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Loads libmoe.so (built in-tree by ``sparse_moe_layer_gemm_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libmoe.so not found at {p}: run `python -m sparse_moe_layer_gemm_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    lib.moe_config_check.argtypes = [ctypes.POINTER(moe_config_t)]
+    lib.moe_create.argtypes = [ctypes.POINTER(moe_config_t), ctypes.POINTER(vp)]
+    lib.moe_load_weights.argtypes = [vp] * 9 + [vp]
+    lib.moe_workspace_size.argtypes = [vp, i, ctypes.POINTER(sz)]
+    lib.moe_workspace_size_host.argtypes = [vp, i, ctypes.POINTER(sz)]
+    lib.moe_forward.argtypes = [vp, vp, i, vp, vp, sz, vp, ctypes.POINTER(moe_routing_t)]
+    lib.moe_forward_host.argtypes = [vp, vp, i, vp, vp, sz, vp]
+    lib.moe_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
+    lib.moe_status_string.argtypes = [i]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_destroy.argtypes = [vp]
+    lib.moe_destroy.restype = None
+    lib.moe_forward_oneshot.argtypes = [vp] * 9 + [i] * 5 + [f] * 3 + [i, i, vp, vp]
+    lib.moe_kernel_launches.argtypes = [vp, i]
+    lib.moe_set_stage_timing.argtypes = [vp, i]
+    lib.moe_get_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i,
+                                        ctypes.POINTER(i)]
+    for name in EXPORTS:
+        if name not in ("moe_status_string", "moe_destroy"):
+            getattr(lib, name).restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().moe_status_string(int(status)).decode()
+    except RuntimeError:
+        return "libmoe.so not loaded"
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def make_config(hidden, num_experts, top_k, intermediate, shared_intermediate=None, *,
+                norm_expert_weight=True, routed_scaling_factor=3.0, use_router_bias=True,
+                swiglu_limit=0.0, swiglu_limit_shared=0.0, act_dtype=MOE_BF16,
+                weight_dtype=MOE_BF16) -> moe_config_t:
+    return moe_config_t(hidden, num_experts, top_k, intermediate,
+                        intermediate if shared_intermediate is None else shared_intermediate,
+                        int(bool(norm_expert_weight)), float(routed_scaling_factor),
+                        int(bool(use_router_bias)), float(swiglu_limit),
+                        float(swiglu_limit_shared), int(act_dtype), int(weight_dtype))
+
+
+def config_from_workload(wl) -> moe_config_t:
+    dt = {"f32": MOE_F32, "bf16": MOE_BF16}
+    return make_config(wl.hidden, wl.num_experts, wl.top_k, wl.intermediate,
+                       wl.shared_intermediate, routed_scaling_factor=wl.scale,
+                       swiglu_limit=wl.swiglu_limit, swiglu_limit_shared=wl.swiglu_limit_shared,
+                       act_dtype=dt[wl.act_dtype], weight_dtype=dt[wl.weight_dtype])
+
+
+# ----------------------------------------------------------------- raw ABI
+def moe_config_check(cfg: moe_config_t) -> int:
+    return load_library().moe_config_check(ctypes.byref(cfg))
+
+
+def moe_create(cfg: moe_config_t) -> int:
+    h = ctypes.c_void_p()
+    _check(load_library().moe_create(ctypes.byref(cfg), ctypes.byref(h)), "moe_create")
+    return h.value
+
+
+def moe_destroy(handle: int) -> None:
+    load_library().moe_destroy(ctypes.c_void_p(handle))
+
+
+def moe_workspace_size(handle: int, T: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().moe_workspace_size(ctypes.c_void_p(handle), T, ctypes.byref(n)),
+           "moe_workspace_size")
+    return n.value
+
+
+def moe_workspace_size_host(handle: int, T: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().moe_workspace_size_host(ctypes.c_void_p(handle), T, ctypes.byref(n)),
+           "moe_workspace_size_host")
+    return n.value
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def moe_load_weights(handle, router_w, router_bias, w_gate, w_up, w_down, sh_gate, sh_up,
+                     sh_down, stream=None) -> None:
+    _check(load_library().moe_load_weights(
+        ctypes.c_void_p(handle), _ptr(router_w), _ptr(router_bias), _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), _ptr(sh_gate), _ptr(sh_up), _ptr(sh_down), _stream(stream)),
+        "moe_load_weights")
+
+
+def moe_forward(handle, x, T, out, workspace, ws_bytes, stream=None, routing=None) -> int:
+    r = None if routing is None else ctypes.byref(routing)
+    return load_library().moe_forward(ctypes.c_void_p(handle), x, T, out, workspace, ws_bytes,
+                                      _stream(stream), r)
+
+
+def moe_forward_host(handle, x_host, T, out_host, workspace, ws_bytes, stream=None) -> int:
+    return load_library().moe_forward_host(ctypes.c_void_p(handle), x_host, T, out_host,
+                                           workspace, ws_bytes, _stream(stream))
+
+
+def moe_get_device_error(handle) -> int:
+    v = ctypes.c_int()
+    load_library().moe_get_device_error(ctypes.c_void_p(handle), ctypes.byref(v))
+    return v.value
+
+
+def moe_forward_oneshot(x, router_w, router_bias, w_gate, w_up, w_down, sh_gate, sh_up, sh_down,
+                        T, H, E, k, I, scale, swiglu_limit, swiglu_limit_shared, act_dtype,
+                        weight_dtype, out, stream=None) -> int:
+    return load_library().moe_forward_oneshot(
+        _ptr(x), _ptr(router_w), _ptr(router_bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(sh_gate), _ptr(sh_up), _ptr(sh_down), T, H, E, k, I, scale, swiglu_limit,
+        swiglu_limit_shared, act_dtype, weight_dtype, _ptr(out), _stream(stream))
+
+
+def moe_kernel_launches(handle, T: int) -> int:
+    return load_library().moe_kernel_launches(ctypes.c_void_p(handle), T)
+
+
+def moe_set_stage_timing(handle, capacity: int) -> None:
+    _check(load_library().moe_set_stage_timing(ctypes.c_void_p(handle), capacity),
+           "moe_set_stage_timing")
+
+
+def moe_get_stage_times(handle):
+    """-> (dict stage name -> summed ms, number of recorded forwards)."""
+    ms = (ctypes.c_float * MOE_NUM_STAGES)()
+    n = ctypes.c_int()
+    _check(load_library().moe_get_stage_times(ctypes.c_void_p(handle), ms, MOE_NUM_STAGES,
+                                              ctypes.byref(n)), "moe_get_stage_times")
+    return dict(zip(STAGE_NAMES, list(ms))), n.value
+
+
+# ----------------------------------------------------------------- layer object
+_TORCH_DT = {MOE_F32: torch.float32, MOE_BF16: torch.bfloat16}
+
+
+class MoeLayer:
+    """One layer on the current CUDA device: owns the library handle (and its
+    packed weights) and a cached device workspace."""
+
+    def __init__(self, cfg: moe_config_t):
+        if not torch.cuda.is_available():
+            raise RuntimeError("MoeLayer needs a CUDA device")
+        self.cfg = cfg
+        self.device = torch.device("cuda", torch.cuda.current_device())
+        self.handle = moe_create(cfg)
+        self._ws: Optional[torch.Tensor] = None
+
+    @classmethod
+    def from_workload(cls, wl) -> "MoeLayer":
+        return cls(config_from_workload(wl))
+
+    @property
+    def act_dtype(self) -> torch.dtype:
+        return _TORCH_DT[self.cfg.act_dtype]
+
+    def _need(self, t: torch.Tensor, name: str, dtype: torch.dtype, shape):
+        if t.device != self.device or t.dtype != dtype or not t.is_contiguous() \
+                or tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: want contiguous {dtype} {tuple(shape)} on {self.device}, "
+                             f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+    def load_weights(self, router_w, router_bias, w_gate, w_up, w_down, sh_gate, sh_up, sh_down):
+        c = self.cfg
+        H, E, I, Is = c.hidden, c.num_experts, c.intermediate, c.shared_intermediate
+        wdt = _TORCH_DT[c.weight_dtype]
+        self._need(router_w, "router_w", torch.float32, (H, E))
+        if router_bias is not None:
+            self._need(router_bias, "router_bias", torch.float32, (E,))
+        self._need(w_gate, "w_gate", wdt, (E, H, I))
+        self._need(w_up, "w_up", wdt, (E, H, I))
+        self._need(w_down, "w_down", wdt, (E, I, H))
+        self._need(sh_gate, "sh_gate", wdt, (H, Is))
+        self._need(sh_up, "sh_up", wdt, (H, Is))
+        self._need(sh_down, "sh_down", wdt, (Is, H))
+        moe_load_weights(self.handle, router_w, router_bias, w_gate, w_up, w_down, sh_gate,
+                         sh_up, sh_down)
+
+    def load_inputs(self, inp: Dict[str, torch.Tensor]):
+        self.load_weights(inp["router_w"], inp["router_bias"], inp["w_gate"], inp["w_up"],
+                          inp["w_down"], inp["sh_gate"], inp["sh_up"], inp["sh_down"])
+
+    def workspace(self, T: int, host_io: bool = False) -> torch.Tensor:
+        n = (moe_workspace_size_host if host_io else moe_workspace_size)(self.handle, T)
+        if self._ws is None or self._ws.numel() < n:
+            self._ws = torch.empty(max(n, 256), dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                routing: bool = False, stream=None):
+        T = x.shape[0]
+        self._need(x, "x", self.act_dtype, (T, self.cfg.hidden))
+        if out is None:
+            out = torch.empty_like(x)
+        else:
+            self._need(out, "out", self.act_dtype, (T, self.cfg.hidden))
+        ws = self.workspace(T)
+        r = None
+        rt = None
+        if routing:
+            k, E = self.cfg.top_k, self.cfg.num_experts
+            dev = self.device
+            rt = dict(topk_idx=torch.empty(T, k, dtype=torch.int32, device=dev),
+                      topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
+                      counts=torch.empty(E, dtype=torch.int32, device=dev),
+                      offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                      perm=torch.empty(T * k, dtype=torch.int32, device=dev))
+            r = moe_routing_t(*(rt[n].data_ptr() for n in
+                                ("topk_idx", "topk_w", "counts", "offsets", "perm")))
+        _check(moe_forward(self.handle, x.data_ptr(), T, out.data_ptr(), ws.data_ptr(),
+                           ws.numel(), stream, r), "moe_forward")
+        return (out, rt) if routing else out
+
+    def forward_host(self, x_host: torch.Tensor, out_host: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+        """Host tensors in and out (pinned for asynchronous copies); returns
+        after the result is on the host."""
+        T = x_host.shape[0]
+        if x_host.device.type != "cpu" or not x_host.is_contiguous() or x_host.dtype != self.act_dtype:
+            raise ValueError("x_host must be a contiguous host tensor of the layer's dtype")
+        if out_host is None:
+            out_host = torch.empty_like(x_host, pin_memory=x_host.is_pinned())
+        ws = self.workspace(T, host_io=True)
+        _check(moe_forward_host(self.handle, x_host.data_ptr(), T, out_host.data_ptr(),
+                                ws.data_ptr(), ws.numel(), stream), "moe_forward_host")
+        return out_host
+
+    def device_error(self) -> int:
+        return moe_get_device_error(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,535 @@
+// C ABI of libmoe.so (declared in include/moe.h): argument checks, weight
+// packing, workspace layout, tensor-map encoding and the stream-ordered
+// launch sequence of the MoE FFN layer forward:
+//   K1 router logits -> K2 top-k + weights -> K3 counting sort -> K4 gather
+//   -> K5 grouped gate|up + SwiGLU -> K6 grouped down x gate weight -> K7 combine.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+using moe::GemmParams;
+
+struct moe_layer {
+  moe_config_t cfg;
+  int device;
+  int num_sms;
+  int I_pad;
+  __nv_bfloat16* w_gu;  // [(E+1) * 2 * I_pad, H]
+  __nv_bfloat16* w_dn;  // [(E+1) * H, I_pad]
+  float* router_w;      // [H, E]
+  float* router_b;      // [E]
+  int has_bias;
+  int* status;          // device status word
+  int loaded;
+  CUtensorMap tm_gu;    // A operand of K5 (box 64 x 256)
+  CUtensorMap tm_dn;    // A operand of K6 (box 64 x 128)
+  // stage timers: capacity x (MOE_NUM_STAGES + 1) events, filled in order
+  std::vector<cudaEvent_t> events;
+  int timing_capacity;
+  int timing_recorded;
+};
+
+namespace {
+
+constexpr int kMaxTokens = 1 << 20;
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t partial, topk_idx, topk_w, masks, chunk_cnt, chunk_base, counts, row_start, tiles_gu,
+      tiles_dn, perm, pos, w_perm, x_perm, h, y, total;
+  int ksplit, nch, rows_routed, rows_xperm, rows_all;
+};
+
+int router_ksplit(int T, int H, int E, int num_sms) {
+  const int tiles = ((E + moe::kRouterExp - 1) / moe::kRouterExp) *
+                    ((T + moe::kRouterTok - 1) / moe::kRouterTok);
+  int s = 1;
+  while (tiles * s < 2 * num_sms && H / (2 * s) >= 128 && H % (2 * s * moe::kRouterKStep) == 0)
+    s *= 2;
+  return s;
+}
+
+WsLayout ws_layout(const moe_layer* L, int T) {
+  const moe_config_t& c = L->cfg;
+  const int H = c.hidden, E = c.num_experts, k = c.top_k, G = E + 1;
+  WsLayout w{};
+  w.ksplit = router_ksplit(T, H, E, L->num_sms);
+  w.nch = (T + moe::kSortChunk - 1) / moe::kSortChunk;
+  w.rows_routed = T * k;
+  w.rows_xperm = T * k + (c.act_dtype == MOE_F32 ? T : 0);
+  w.rows_all = T * k + T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  w.partial = take(static_cast<size_t>(w.ksplit) * T * E * sizeof(float));
+  w.topk_idx = take(static_cast<size_t>(T) * k * sizeof(int));
+  w.topk_w = take(static_cast<size_t>(T) * k * sizeof(float));
+  w.masks = take(static_cast<size_t>(w.nch) * E * 4 * sizeof(uint32_t));
+  w.chunk_cnt = take(static_cast<size_t>(w.nch) * E * sizeof(int));
+  w.chunk_base = take(static_cast<size_t>(w.nch) * E * sizeof(int));
+  w.counts = take(static_cast<size_t>(G) * sizeof(int));
+  w.row_start = take(static_cast<size_t>(G + 1) * sizeof(int));
+  w.tiles_gu = take(static_cast<size_t>(G + 1) * sizeof(int));
+  w.tiles_dn = take(static_cast<size_t>(G + 1) * sizeof(int));
+  w.perm = take(static_cast<size_t>(T) * k * sizeof(int));
+  w.pos = take(static_cast<size_t>(T) * k * sizeof(int));
+  w.w_perm = take(static_cast<size_t>(w.rows_all) * sizeof(float));
+  w.x_perm = take(static_cast<size_t>(w.rows_xperm) * H * 2);
+  w.h = take(static_cast<size_t>(w.rows_all) * L->I_pad * 2);
+  w.y = take(static_cast<size_t>(w.rows_all) * H * 2);
+  w.total = off;
+  return w;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows, cols] row-major, box = 64 columns (128 bytes) x box_rows, 128B swizzle,
+// out-of-range elements read as zero.
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(moe::kBK), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Makes the layer's device current for the lifetime of the guard.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = true;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      ok = false;
+      return;
+    }
+    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+#define MOE_CUDA(call)                          \
+  do {                                          \
+    if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration or size";
+    case MOE_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    case MOE_ERR_NOT_LOADED: return "weights not loaded";
+    default: return "unknown status";
+  }
+}
+
+int moe_config_check(const moe_config_t* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->num_experts <= 0 || c->top_k <= 0 || c->intermediate <= 0 ||
+      c->shared_intermediate <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if ((c->act_dtype != MOE_F32 && c->act_dtype != MOE_BF16) ||
+      (c->weight_dtype != MOE_F32 && c->weight_dtype != MOE_BF16))
+    return MOE_ERR_INVALID_ARG;
+  if (!isfinite(c->routed_scaling_factor) || !isfinite(c->swiglu_limit) ||
+      !isfinite(c->swiglu_limit_shared) || c->swiglu_limit < 0.f || c->swiglu_limit_shared < 0.f)
+    return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->num_experts) return MOE_ERR_INVALID_ARG;
+  if (c->hidden % 128 != 0 || c->hidden > 16384) return MOE_ERR_UNSUPPORTED;
+  if (c->num_experts > 1024 || c->top_k > 32 || c->intermediate > 8192) return MOE_ERR_UNSUPPORTED;
+  if (c->shared_intermediate != c->intermediate) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const int chk = moe_config_check(cfg);
+  if (chk != MOE_OK) return chk;
+  moe_layer* L = new (std::nothrow) moe_layer();
+  if (L == nullptr) return MOE_ERR_CUDA;
+  L->cfg = *cfg;
+  L->I_pad = (cfg->intermediate + 127) / 128 * 128;
+  if (cudaGetDevice(&L->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) !=
+          cudaSuccess) {
+    delete L;
+    return MOE_ERR_CUDA;
+  }
+  const size_t H = cfg->hidden, E = cfg->num_experts, Ip = L->I_pad;
+  const size_t gu_bytes = (E + 1) * 2 * Ip * H * 2, dn_bytes = (E + 1) * H * Ip * 2;
+  if (moe::gemm_configure_device() != cudaSuccess ||
+      cudaMalloc(&L->w_gu, gu_bytes) != cudaSuccess ||
+      cudaMalloc(&L->w_dn, dn_bytes) != cudaSuccess ||
+      cudaMalloc(&L->router_w, H * E * sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&L->router_b, E * sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
+      cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess) {
+    moe_destroy(L);
+    return MOE_ERR_CUDA;
+  }
+  if (!encode_bf16_2d(&L->tm_gu, L->w_gu, (E + 1) * 2 * Ip, H, 2 * moe::kBM) ||
+      !encode_bf16_2d(&L->tm_dn, L->w_dn, (E + 1) * H, Ip, moe::kBM)) {
+    moe_destroy(L);
+    return MOE_ERR_CUDA;
+  }
+  *out = L;
+  return MOE_OK;
+}
+
+int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_bias,
+                     const void* w_gate, const void* w_up, const void* w_down, const void* sh_gate,
+                     const void* sh_up, const void* sh_down, void* stream) {
+  if (L == nullptr || router_w == nullptr || w_gate == nullptr || w_up == nullptr ||
+      w_down == nullptr || sh_gate == nullptr || sh_up == nullptr || sh_down == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const moe_config_t& c = L->cfg;
+  const int H = c.hidden, E = c.num_experts, I = c.intermediate, Ip = L->I_pad;
+  const bool wb = c.weight_dtype == MOE_BF16;
+  const size_t gu_group = static_cast<size_t>(2) * Ip * H, dn_group = static_cast<size_t>(H) * Ip;
+  MOE_CUDA(cudaMemsetAsync(L->w_gu, 0, (E + 1) * gu_group * 2, st));
+  MOE_CUDA(cudaMemsetAsync(L->w_dn, 0, (E + 1) * dn_group * 2, st));
+  MOE_CUDA(moe::launch_pack_gate_up(w_gate, wb, E, H, I, Ip, 0, L->w_gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up(w_up, wb, E, H, I, Ip, 1, L->w_gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up(sh_gate, wb, 1, H, I, Ip, 0, L->w_gu + E * gu_group, st));
+  MOE_CUDA(moe::launch_pack_gate_up(sh_up, wb, 1, H, I, Ip, 1, L->w_gu + E * gu_group, st));
+  MOE_CUDA(moe::launch_pack_down(w_down, wb, E, H, I, Ip, L->w_dn, st));
+  MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, L->w_dn + E * dn_group, st));
+  MOE_CUDA(cudaMemcpyAsync(L->router_w, router_w, static_cast<size_t>(H) * E * sizeof(float),
+                           cudaMemcpyDeviceToDevice, st));
+  L->has_bias = (c.use_router_bias && router_bias != nullptr) ? 1 : 0;
+  if (L->has_bias)
+    MOE_CUDA(cudaMemcpyAsync(L->router_b, router_bias, E * sizeof(float),
+                             cudaMemcpyDeviceToDevice, st));
+  L->loaded = 1;
+  return MOE_OK;
+}
+
+int moe_workspace_size(const moe_layer_t* L, int T, size_t* bytes) {
+  if (L == nullptr || bytes == nullptr || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > kMaxTokens) return MOE_ERR_UNSUPPORTED;
+  *bytes = (T == 0) ? 0 : ws_layout(L, T).total;
+  return MOE_OK;
+}
+
+int moe_workspace_size_host(const moe_layer_t* L, int T, size_t* bytes) {
+  size_t b = 0;
+  const int r = moe_workspace_size(L, T, &b);
+  if (r != MOE_OK) return r;
+  const size_t el = (L->cfg.act_dtype == MOE_BF16) ? 2 : 4;
+  const size_t io = align_up(static_cast<size_t>(T) * L->cfg.hidden * el, kAlign);
+  *bytes = b + 2 * io;
+  return MOE_OK;
+}
+
+int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace, size_t ws_bytes,
+                void* stream, const moe_routing_t* routing) {
+  if (L == nullptr || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > kMaxTokens) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || out == nullptr || x == out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  const WsLayout w = ws_layout(L, T);
+  if (workspace == nullptr || ws_bytes < w.total || !aligned(workspace, 256))
+    return MOE_ERR_WORKSPACE;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+
+  const moe_config_t& c = L->cfg;
+  const int H = c.hidden, E = c.num_experts, k = c.top_k, G = E + 1, Ip = L->I_pad;
+  const bool xb = c.act_dtype == MOE_BF16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* partial = reinterpret_cast<float*>(ws + w.partial);
+  int* topk_idx = reinterpret_cast<int*>(ws + w.topk_idx);
+  float* topk_w = reinterpret_cast<float*>(ws + w.topk_w);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(ws + w.masks);
+  int* chunk_cnt = reinterpret_cast<int*>(ws + w.chunk_cnt);
+  int* chunk_base = reinterpret_cast<int*>(ws + w.chunk_base);
+  int* counts = reinterpret_cast<int*>(ws + w.counts);
+  int* row_start = reinterpret_cast<int*>(ws + w.row_start);
+  int* tiles_gu = reinterpret_cast<int*>(ws + w.tiles_gu);
+  int* tiles_dn = reinterpret_cast<int*>(ws + w.tiles_dn);
+  int* perm = reinterpret_cast<int*>(ws + w.perm);
+  int* pos = reinterpret_cast<int*>(ws + w.pos);
+  float* w_perm = reinterpret_cast<float*>(ws + w.w_perm);
+  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + w.x_perm);
+  __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + w.h);
+  __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(ws + w.y);
+
+  CUtensorMap tm_b, tm_bsh, tm_h;
+  if (!encode_bf16_2d(&tm_b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
+      !encode_bf16_2d(&tm_h, hbuf, w.rows_all, Ip, moe::kBBoxRows))
+    return MOE_ERR_CUDA;
+  if (xb) {
+    if (!encode_bf16_2d(&tm_bsh, x, T, H, moe::kBBoxRows)) return MOE_ERR_CUDA;
+  } else {
+    tm_bsh = tm_b;
+  }
+
+  cudaEvent_t* ev = nullptr;
+  if (L->timing_capacity > 0 && L->timing_recorded < L->timing_capacity)
+    ev = &L->events[static_cast<size_t>(L->timing_recorded++) * (MOE_NUM_STAGES + 1)];
+  auto mark = [&](int i) { return ev == nullptr ? cudaSuccess : cudaEventRecord(ev[i], st); };
+
+  MOE_CUDA(mark(0));
+  MOE_CUDA(moe::launch_router_logits(x, xb, L->router_w, partial, T, H, E, w.ksplit, st));
+  MOE_CUDA(mark(1));
+  MOE_CUDA(moe::launch_topk(partial, w.ksplit, T, E, k, L->has_bias ? L->router_b : nullptr,
+                            c.norm_expert_weight != 0, c.routed_scaling_factor, topk_idx, topk_w,
+                            st));
+  MOE_CUDA(mark(2));
+  MOE_CUDA(moe::launch_sort(topk_idx, topk_w, T, k, E, Ip / moe::kBM, H / moe::kBM, masks,
+                            chunk_cnt, chunk_base, counts, row_start, tiles_gu, tiles_dn, perm, pos,
+                            w_perm, st));
+  MOE_CUDA(mark(3));
+  MOE_CUDA(moe::launch_gather(x, xb, perm, w.rows_routed, k, T, H, !xb, x_perm, L->num_sms, st));
+  MOE_CUDA(mark(4));
+
+  GemmParams p{};
+  p.counts = counts;
+  p.row_start = row_start;
+  p.G = G;
+  p.E = E;
+  p.status = L->status;
+  p.limit = c.swiglu_limit;
+  p.limit_shared = c.swiglu_limit_shared;
+
+  p.tile_start = tiles_gu;
+  p.num_kb = H / moe::kBK;
+  p.m_tiles = Ip / moe::kBM;
+  p.a_rows_per_group = 2 * Ip;
+  p.shared_b_row0 = xb ? 0 : T * k;
+  p.out = hbuf;
+  p.out_ld = Ip;
+  p.w_perm = nullptr;
+  MOE_CUDA(moe::launch_gemm_gate_up(L->tm_gu, tm_b, tm_bsh, p, L->num_sms, st));
+  MOE_CUDA(mark(5));
+
+  p.tile_start = tiles_dn;
+  p.num_kb = Ip / moe::kBK;
+  p.m_tiles = H / moe::kBM;
+  p.a_rows_per_group = H;
+  p.shared_b_row0 = T * k;
+  p.out = ybuf;
+  p.out_ld = H;
+  p.w_perm = w_perm;
+  MOE_CUDA(moe::launch_gemm_down(L->tm_dn, tm_h, p, L->num_sms, st));
+  MOE_CUDA(mark(6));
+  MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, out, st));
+  MOE_CUDA(mark(7));
+
+  if (routing != nullptr) {
+    const size_t tk = static_cast<size_t>(T) * k;
+    if (routing->topk_idx)
+      MOE_CUDA(cudaMemcpyAsync(routing->topk_idx, topk_idx, tk * 4, cudaMemcpyDeviceToDevice, st));
+    if (routing->topk_w)
+      MOE_CUDA(cudaMemcpyAsync(routing->topk_w, topk_w, tk * 4, cudaMemcpyDeviceToDevice, st));
+    if (routing->counts)
+      MOE_CUDA(cudaMemcpyAsync(routing->counts, counts, E * 4, cudaMemcpyDeviceToDevice, st));
+    if (routing->offsets)
+      MOE_CUDA(
+          cudaMemcpyAsync(routing->offsets, row_start, (E + 1) * 4, cudaMemcpyDeviceToDevice, st));
+    if (routing->perm)
+      MOE_CUDA(cudaMemcpyAsync(routing->perm, perm, tk * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  return MOE_OK;
+}
+
+int moe_forward_host(moe_layer_t* L, const void* x_host, int T, void* out_host, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  if (L == nullptr || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (x_host == nullptr || out_host == nullptr) return MOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  int r = moe_workspace_size_host(L, T, &need);
+  if (r != MOE_OK) return r;
+  if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  const size_t el = (L->cfg.act_dtype == MOE_BF16) ? 2 : 4;
+  const size_t io_bytes = static_cast<size_t>(T) * L->cfg.hidden * el;
+  const size_t base = ws_layout(L, T).total;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* x_dev = ws + base;
+  void* out_dev = ws + base + align_up(io_bytes, kAlign);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, st));
+  r = moe_forward(L, x_dev, T, out_dev, workspace, base, stream, nullptr);
+  if (r != MOE_OK) return r;
+  MOE_CUDA(cudaMemcpyAsync(out_host, out_dev, io_bytes, cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  return MOE_OK;
+}
+
+int moe_get_device_error(moe_layer_t* L, int* device_err) {
+  if (L == nullptr || device_err == nullptr) return MOE_ERR_INVALID_ARG;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  int v = 0;
+  MOE_CUDA(cudaDeviceSynchronize());
+  MOE_CUDA(cudaMemcpy(&v, L->status, sizeof(int), cudaMemcpyDeviceToHost));
+  MOE_CUDA(cudaMemset(L->status, 0, sizeof(int)));
+  *device_err = v;
+  return v == 0 ? MOE_OK : MOE_ERR_DEVICE_TIMEOUT;
+}
+
+int moe_kernel_launches(const moe_layer_t* L, int T) {
+  if (L == nullptr || T <= 0) return 0;
+  // router, top-k, 3 sort kernels, gather, gate|up GEMM, down GEMM, combine
+  return 9;
+}
+
+namespace {
+void free_events(moe_layer* L) {
+  for (cudaEvent_t e : L->events) cudaEventDestroy(e);
+  L->events.clear();
+  L->timing_capacity = 0;
+  L->timing_recorded = 0;
+}
+}  // namespace
+
+int moe_set_stage_timing(moe_layer_t* L, int capacity) {
+  if (L == nullptr || capacity < 0) return MOE_ERR_INVALID_ARG;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  free_events(L);
+  if (capacity == 0) return MOE_OK;
+  const size_t n = static_cast<size_t>(capacity) * (MOE_NUM_STAGES + 1);
+  L->events.resize(n, nullptr);
+  for (size_t i = 0; i < n; ++i) {
+    if (cudaEventCreate(&L->events[i]) != cudaSuccess) {
+      L->events.resize(i);
+      free_events(L);
+      return MOE_ERR_CUDA;
+    }
+  }
+  L->timing_capacity = capacity;
+  L->timing_recorded = 0;
+  return MOE_OK;
+}
+
+int moe_get_stage_times(moe_layer_t* L, float* ms, int n_stages, int* n_forwards) {
+  if (L == nullptr || ms == nullptr || n_forwards == nullptr || n_stages < 0 ||
+      n_stages > MOE_NUM_STAGES)
+    return MOE_ERR_INVALID_ARG;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  for (int i = 0; i < n_stages; ++i) ms[i] = 0.f;
+  const int n = L->timing_recorded;
+  for (int f = 0; f < n; ++f) {
+    cudaEvent_t* ev = &L->events[static_cast<size_t>(f) * (MOE_NUM_STAGES + 1)];
+    MOE_CUDA(cudaEventSynchronize(ev[MOE_NUM_STAGES]));
+    for (int i = 0; i < n_stages; ++i) {
+      float t = 0.f;
+      MOE_CUDA(cudaEventElapsedTime(&t, ev[i], ev[i + 1]));
+      ms[i] += t;
+    }
+  }
+  *n_forwards = n;
+  L->timing_recorded = 0;
+  return MOE_OK;
+}
+
+void moe_destroy(moe_layer_t* L) {
+  if (L == nullptr) return;
+  {
+    DeviceGuard dg(L->device);
+    cudaDeviceSynchronize();
+    free_events(L);
+    cudaFree(L->w_gu);
+    cudaFree(L->w_dn);
+    cudaFree(L->router_w);
+    cudaFree(L->router_b);
+    cudaFree(L->status);
+  }
+  delete L;
+}
+
+int moe_forward_oneshot(const void* x, const float* router_w, const float* router_bias,
+                        const void* w_gate, const void* w_up, const void* w_down,
+                        const void* sh_gate, const void* sh_up, const void* sh_down, int T, int H,
+                        int E, int k, int I, float scale, float swiglu_limit,
+                        float swiglu_limit_shared, int act_dtype, int weight_dtype, void* out,
+                        void* stream) {
+  moe_config_t c{};
+  c.hidden = H;
+  c.num_experts = E;
+  c.top_k = k;
+  c.intermediate = I;
+  c.shared_intermediate = I;
+  c.norm_expert_weight = 1;
+  c.routed_scaling_factor = scale;
+  c.use_router_bias = router_bias != nullptr ? 1 : 0;
+  c.swiglu_limit = swiglu_limit;
+  c.swiglu_limit_shared = swiglu_limit_shared;
+  c.act_dtype = act_dtype;
+  c.weight_dtype = weight_dtype;
+  int r = moe_config_check(&c);
+  if (r != MOE_OK) return r;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_layer_t* L = nullptr;
+  r = moe_create(&c, &L);
+  if (r != MOE_OK) return r;
+  r = moe_load_weights(L, router_w, router_bias, w_gate, w_up, w_down, sh_gate, sh_up, sh_down,
+                       stream);
+  void* ws = nullptr;
+  size_t bytes = 0;
+  if (r == MOE_OK) r = moe_workspace_size(L, T, &bytes);
+  if (r == MOE_OK && cudaMalloc(&ws, bytes) != cudaSuccess) r = MOE_ERR_CUDA;
+  if (r == MOE_OK) r = moe_forward(L, x, T, out, ws, bytes, stream, nullptr);
+  if (r == MOE_OK && cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    r = MOE_ERR_CUDA;
+  if (ws != nullptr) cudaFree(ws);
+  moe_destroy(L);
+  return r;
+}
+
+}  // extern "C"

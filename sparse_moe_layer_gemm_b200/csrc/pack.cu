@@ -1,0 +1,71 @@
+// Weight packing at load time: the caller's x . W layouts become the K-major
+// bf16 operands of the grouped GEMMs.
+//   gate / up  [G][H][I]  ->  rows g * 2*I_pad + (f / 128) * 256 + half * 128 + f % 128,
+//                             columns h (ld H): each 256-row block holds 128 gate
+//                             rows then the 128 matching up rows.
+//   down       [G][I][H]  ->  rows g * H + n, columns i (ld I_pad).
+// Rows and columns past I (up to I_pad, a multiple of 128) stay zero, so the
+// padded features compute silu(0) * 0 = 0 and add nothing in the down GEMM.
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Transposes the [R][C] matrix of group blockIdx.z through a 32 x 32 tile.
+template <typename TS, bool GU>
+__global__ void __launch_bounds__(256) pack_kernel(const TS* __restrict__ src, int R, int C,
+                                                   __nv_bfloat16* __restrict__ dst, int dst_ld,
+                                                   int I_pad, int H, int half) {
+  __shared__ float tile[32][33];
+  const int g = blockIdx.z;
+  const TS* s = src + static_cast<size_t>(g) * R * C;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < R && c < C) ? to_f32(s[static_cast<size_t>(r) * C + c]) : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < C && r < R) {
+      size_t drow;
+      if (GU)
+        drow = static_cast<size_t>(g) * 2 * I_pad + (c / 128) * 256 + half * 128 + (c % 128);
+      else
+        drow = static_cast<size_t>(g) * H + c;
+      dst[drow * dst_ld + r] = __float2bfloat16_rn(tile[threadIdx.x][i]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
+                                int half, __nv_bfloat16* dst, cudaStream_t st) {
+  dim3 grid((I + 31) / 32, (H + 31) / 32, groups), block(32, 8);
+  if (w_bf16)
+    pack_kernel<__nv_bfloat16, true><<<grid, block, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), H, I, dst, H, I_pad, H, half);
+  else
+    pack_kernel<float, true><<<grid, block, 0, st>>>(static_cast<const float*>(w), H, I, dst, H,
+                                                     I_pad, H, half);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
+                             __nv_bfloat16* dst, cudaStream_t st) {
+  dim3 grid((H + 31) / 32, (I + 31) / 32, groups), block(32, 8);
+  if (w_bf16)
+    pack_kernel<__nv_bfloat16, false><<<grid, block, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), I, H, dst, I_pad, I_pad, H, 0);
+  else
+    pack_kernel<float, false><<<grid, block, 0, st>>>(static_cast<const float*>(w), I, H, dst,
+                                                      I_pad, I_pad, H, 0);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

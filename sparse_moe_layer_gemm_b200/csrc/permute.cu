@@ -1,0 +1,220 @@
+// K3: deterministic token-to-expert grouping (histogram, scan, stable scatter)
+// and K4: gather of the input rows into expert-contiguous order.
+//
+// The grouped matmul of an expert-parallel MoE ("EPMoE", sglang-jax issue
+// #1367 "Support Step 3.5 Flash", sections "Reuse map" and "Implementation
+// strategy") needs each expert's rows contiguous.  Definition kept here:
+// perm lists the pair ids t * k + j of expert 0, then expert 1, ..., each in
+// ascending t; pos[t * k + j] is the pair's slot in perm.  The shared expert
+// is group E with the T identity rows [T*k, T*k + T).
+//
+// No order-dependent atomics: each block owns kSortChunk tokens and records,
+// per expert, a 128-bit mask of its tokens that chose that expert (atomicOr
+// gives the same mask in any order).  A pair's rank inside its block is the
+// popcount of the mask bits below its token, so the scatter is stable and
+// bit-reproducible.
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kMaskWords = kSortChunk / 32;  // 4
+
+__global__ void __launch_bounds__(256) sort_hist_kernel(const int* __restrict__ topk_idx, int T,
+                                                        int k, int E, uint32_t* __restrict__ masks,
+                                                        int* __restrict__ chunk_cnt) {
+  extern __shared__ uint32_t sm[];
+  const int c = blockIdx.x;
+  const int t0 = c * kSortChunk;
+  const int nt = min(kSortChunk, T - t0);
+  for (int i = threadIdx.x; i < E * kMaskWords; i += blockDim.x) sm[i] = 0u;
+  __syncthreads();
+  for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
+    const int tl = p / k;
+    const int e = topk_idx[static_cast<size_t>(t0) * k + p];
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+      atomicOr(&sm[e * kMaskWords + (tl >> 5)], 1u << (tl & 31));
+  }
+  __syncthreads();
+  uint32_t* mo = masks + static_cast<size_t>(c) * E * kMaskWords;
+  for (int i = threadIdx.x; i < E * kMaskWords; i += blockDim.x) mo[i] = sm[i];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int n = 0;
+#pragma unroll
+    for (int q = 0; q < kMaskWords; ++q) n += __popc(sm[e * kMaskWords + q]);
+    chunk_cnt[static_cast<size_t>(c) * E + e] = n;
+  }
+}
+
+// One block.  Per expert: running offsets of the chunks; then warp 0 forms
+// the exclusive prefix over the G = E + 1 groups of the row counts and of the
+// GEMM tile counts (ceil(rows / kBN) token tiles x m_tiles weight tiles).
+__global__ void __launch_bounds__(1024) sort_scan_kernel(
+    const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int mt_gu, int mt_dn,
+    int* __restrict__ chunk_base, int* __restrict__ counts, int* __restrict__ row_start,
+    int* __restrict__ tiles_gu, int* __restrict__ tiles_dn) {
+  __shared__ int cnt_s[1025];
+  const int G = E + 1;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < nch; ++c) {
+      chunk_base[static_cast<size_t>(c) * E + e] = run;
+      run += chunk_cnt[static_cast<size_t>(c) * E + e];
+    }
+    cnt_s[e] = run;
+  }
+  if (threadIdx.x == 0) cnt_s[E] = T;
+  __syncthreads();
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  const int per = (G + 31) / 32;
+  const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+  int s_rows = 0, s_gu = 0, s_dn = 0;
+  for (int g = g0; g < g1; ++g) {
+    const int n = cnt_s[g];
+    const int nt = (n + kBN - 1) / kBN;
+    s_rows += n;
+    s_gu += nt * mt_gu;
+    s_dn += nt * mt_dn;
+  }
+  int i_rows = s_rows, i_gu = s_gu, i_dn = s_dn;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, i_rows, off);
+    const int b = __shfl_up_sync(0xffffffffu, i_gu, off);
+    const int d = __shfl_up_sync(0xffffffffu, i_dn, off);
+    if (lane >= off) {
+      i_rows += a;
+      i_gu += b;
+      i_dn += d;
+    }
+  }
+  int b_rows = i_rows - s_rows, b_gu = i_gu - s_gu, b_dn = i_dn - s_dn;
+  for (int g = g0; g < g1; ++g) {
+    const int n = cnt_s[g];
+    const int nt = (n + kBN - 1) / kBN;
+    counts[g] = n;
+    row_start[g] = b_rows;
+    tiles_gu[g] = b_gu;
+    tiles_dn[g] = b_dn;
+    b_rows += n;
+    b_gu += nt * mt_gu;
+    b_dn += nt * mt_dn;
+  }
+  if (lane == 31) {
+    row_start[G] = i_rows;
+    tiles_gu[G] = i_gu;
+    tiles_dn[G] = i_dn;
+  }
+}
+
+__global__ void __launch_bounds__(256) sort_scatter_kernel(
+    const int* __restrict__ topk_idx, const float* __restrict__ topk_w, int T, int k, int E,
+    const uint32_t* __restrict__ masks, const int* __restrict__ chunk_base,
+    const int* __restrict__ row_start, int* __restrict__ perm, int* __restrict__ pos,
+    float* __restrict__ w_perm) {
+  extern __shared__ uint32_t sm[];
+  const int c = blockIdx.x;
+  const int t0 = c * kSortChunk;
+  const int nt = min(kSortChunk, T - t0);
+  const uint32_t* mi = masks + static_cast<size_t>(c) * E * kMaskWords;
+  for (int i = threadIdx.x; i < E * kMaskWords; i += blockDim.x) sm[i] = mi[i];
+  __syncthreads();
+  for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
+    const int tl = p / k;
+    const size_t pair = static_cast<size_t>(t0) * k + p;
+    const int e = topk_idx[pair];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) continue;
+    const uint32_t* m = sm + e * kMaskWords;
+    const int wd = tl >> 5;
+    int rank = __popc(m[wd] & ((1u << (tl & 31)) - 1u));
+    for (int q = 0; q < wd; ++q) rank += __popc(m[q]);
+    const int slot = row_start[e] + chunk_base[static_cast<size_t>(c) * E + e] + rank;
+    perm[slot] = static_cast<int>(pair);
+    pos[pair] = slot;
+    w_perm[slot] = topk_w[pair];
+  }
+  const int shared0 = T * k;
+  for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) w_perm[shared0 + t0 + tl] = 1.0f;
+}
+
+__device__ __forceinline__ uint4 load8_bf16(const __nv_bfloat16* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+
+__device__ __forceinline__ uint4 load8_bf16(const float* p) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  uint4 q;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q);
+  h[0] = __floats2bfloat162_rn(a.x, a.y);
+  h[1] = __floats2bfloat162_rn(a.z, a.w);
+  h[2] = __floats2bfloat162_rn(b.x, b.y);
+  h[3] = __floats2bfloat162_rn(b.z, b.w);
+  return q;
+}
+
+// One warp per destination row, 16-byte vectors.  Rows [0, rows_routed) take
+// x[perm[r] / k]; with write_shared, rows [rows_routed, rows_routed + T) take
+// x[r - rows_routed] (the shared expert's rows, needed when x is fp32).
+template <typename TX>
+__global__ void __launch_bounds__(256) gather_kernel(const TX* __restrict__ x,
+                                                     const int* __restrict__ perm,
+                                                     int rows_routed, int k, int T, int H,
+                                                     int write_shared,
+                                                     __nv_bfloat16* __restrict__ xp) {
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int nrows = rows_routed + (write_shared ? T : 0);
+  const int nvec = H / 8;
+  for (int r = warp; r < nrows; r += nwarps) {
+    const int t = (r < rows_routed) ? perm[r] / k : r - rows_routed;
+    uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(r) * H);
+    if (static_cast<unsigned>(t) >= static_cast<unsigned>(T)) {
+      for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const TX* src = x + static_cast<size_t>(t) * H;
+    for (int v = lane; v < nvec; v += 32) dst[v] = load8_bf16(src + v * 8);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int m_tiles_gu,
+                        int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
+                        int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
+                        int* pos, float* w_perm, cudaStream_t st) {
+  const int nch = (T + kSortChunk - 1) / kSortChunk;
+  const size_t smem = static_cast<size_t>(E) * kMaskWords * sizeof(uint32_t);
+  sort_hist_kernel<<<nch, 256, smem, st>>>(topk_idx, T, k, E, masks, chunk_cnt);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  sort_scan_kernel<<<1, 1024, 0, st>>>(chunk_cnt, nch, T, k, E, m_tiles_gu, m_tiles_dn, chunk_base,
+                                       counts, row_start, tiles_gu, tiles_dn);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  sort_scatter_kernel<<<nch, 256, smem, st>>>(topk_idx, topk_w, T, k, E, masks, chunk_base,
+                                              row_start, perm, pos, w_perm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_routed, int k, int T,
+                          int H, bool write_shared, __nv_bfloat16* x_perm, int num_sms,
+                          cudaStream_t st) {
+  const int nrows = rows_routed + (write_shared ? T : 0);
+  const int want = (nrows + 7) / 8;
+  const int blocks = max(1, min(want, num_sms * 8));
+  if (x_bf16)
+    gather_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), perm,
+                                                         rows_routed, k, T, H, write_shared ? 1 : 0,
+                                                         x_perm);
+  else
+    gather_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), perm, rows_routed, k,
+                                                 T, H, write_shared ? 1 : 0, x_perm);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

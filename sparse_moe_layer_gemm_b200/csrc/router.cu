@@ -1,0 +1,220 @@
+// K1: router logits l = x . W_r in fp32, and K2: sigmoid scores, top-k on the
+// biased scores, bias-free renormalised and scaled gate weights.
+//
+// The routing order follows sglang-jax issue #1367 "Support Step 3.5 Flash",
+// section "Key difficulties", item 1: sigmoid scores in fp32; the router bias
+// only selects the top-k; the gating weights are the bias-free scores of the
+// selected experts, normalised over the top-k and multiplied by the routed
+// scaling factor (llm-atlas "Step-3.5-Flash", "Raw config fields":
+// moe_router_activation sigmoid, moe_router_scaling_factor 3,
+// norm_expert_weight true, use_moe_router_bias true, need_fp32_gate true).
+#include <float.h>
+#include <math.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ void load8_as_f32(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+
+__device__ __forceinline__ void load8_as_f32(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// One block: kRouterTok tokens x kRouterExp experts over one K slice
+// [z * kchunk, (z+1) * kchunk).  256 threads, each 4 tokens x 6 experts
+// (experts strided by 16 so a warp reads 16 consecutive weights).  x is
+// widened to fp32 exactly; products accumulate in fp32 FMAs.
+template <typename TX>
+__global__ void __launch_bounds__(256) router_logits_kernel(const TX* __restrict__ x,
+                                                            const float* __restrict__ wr,
+                                                            float* __restrict__ partial, int T,
+                                                            int H, int E, int kchunk) {
+  __shared__ __align__(16) float xs[kRouterKStep][kRouterTok + 4];
+  __shared__ __align__(16) float ws[kRouterKStep][kRouterExp];
+  const int e0 = blockIdx.x * kRouterExp;
+  const int t0 = blockIdx.y * kRouterTok;
+  const int z = blockIdx.z;
+  const int kbeg = z * kchunk;
+  const int kend = min(H, kbeg + kchunk);
+  const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
+
+  float acc[4][6];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 6; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = kbeg; k0 < kend; k0 += kRouterKStep) {
+    {  // x tile: 64 tokens x 32 k, 8 consecutive k per thread, stored k-major
+      const int tl = tid >> 2, kq = (tid & 3) * 8;
+      const int t = t0 + tl;
+      float v[8];
+      if (t < T) {
+        load8_as_f32(x + static_cast<size_t>(t) * H + k0 + kq, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) xs[kq + i][tl] = v[i];
+    }
+    for (int i = tid; i < kRouterKStep * kRouterExp; i += 256) {  // W tile: 32 k x 96 experts
+      const int kk = i / kRouterExp, ee = i % kRouterExp;
+      const int e = e0 + ee;
+      ws[kk][ee] = (e < E) ? wr[static_cast<size_t>(k0 + kk) * E + e] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kRouterKStep; ++kk) {
+      const float4 xv = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      float wv[6];
+#pragma unroll
+      for (int j = 0; j < 6; ++j) wv[j] = ws[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 6; ++j) acc[i][j] = fmaf(xa[i], wv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 6; ++j) {
+      const int e = e0 + tx + 16 * j;
+      if (e < E) partial[(static_cast<size_t>(z) * T + t) * E + e] = acc[i][j];
+    }
+  }
+}
+
+// One warp per token.  Lane l holds experts l, l + 32, ...  (MPL per lane).
+// k rounds of a warp arg-max on (selection score, lower index first) pick the
+// experts in descending order; the owner lane hands over the bias-free score.
+template <int MPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ partial, int ksplit,
+                                                   int T, int E, int k,
+                                                   const float* __restrict__ bias, int norm,
+                                                   float scale, int* __restrict__ topk_idx,
+                                                   float* __restrict__ topk_w) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+
+  float sc[MPL], be[MPL];
+#pragma unroll
+  for (int i = 0; i < MPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      float l = 0.f;
+      for (int z = 0; z < ksplit; ++z) l += partial[(static_cast<size_t>(z) * T + t) * E + e];
+      const float s = 1.0f / (1.0f + expf(-l));
+      sc[i] = s;
+      be[i] = (bias != nullptr) ? s + bias[e] : s;
+    } else {
+      sc[i] = 0.f;
+      be[i] = -INFINITY;
+    }
+  }
+
+  uint32_t taken = 0;
+  int my_idx = 0;
+  float my_s = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < MPL; ++i) {
+      const int e = lane + 32 * i;
+      const bool free_ = !((taken >> i) & 1u) && e < E;
+      if (free_ && (be[i] > bv || (be[i] == bv && e < bi))) {
+        bv = be[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if (bi >= E) bi = 0;  // only reachable with non-finite scores (unsupported input)
+    float s_sel = 0.f;
+    if ((bi & 31) == lane) {
+      const int ii = bi >> 5;
+#pragma unroll
+      for (int i = 0; i < MPL; ++i)
+        if (i == ii) {
+          taken |= 1u << i;
+          s_sel = sc[i];
+        }
+    }
+    s_sel = __shfl_sync(0xffffffffu, s_sel, bi & 31);
+    if (lane == j) {
+      my_idx = bi;
+      my_s = s_sel;
+    }
+  }
+  float sum = 0.f;
+  for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, my_s, j);
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(t) * k + lane] = my_idx;
+    topk_w[static_cast<size_t>(t) * k + lane] = norm ? (my_s / sum) * scale : my_s * scale;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router_w, float* partial,
+                                 int T, int H, int E, int ksplit, cudaStream_t st) {
+  const int kchunk = H / ksplit;
+  dim3 grid((E + kRouterExp - 1) / kRouterExp, (T + kRouterTok - 1) / kRouterTok, ksplit);
+  if (x_bf16)
+    router_logits_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), router_w, partial, T, H, E, kchunk);
+  else
+    router_logits_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), router_w,
+                                                       partial, T, H, E, kchunk);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, const float* bias,
+                        bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st) {
+  const int blocks = (T + 7) / 8;
+  const int mpl = (E + 31) / 32;
+#define MOE_TOPK(N)                                                                          \
+  topk_kernel<N><<<blocks, 256, 0, st>>>(partial, ksplit, T, E, k, bias, norm ? 1 : 0, scale, \
+                                         topk_idx, topk_w)
+  if (mpl <= 1) MOE_TOPK(1);
+  else if (mpl <= 2) MOE_TOPK(2);
+  else if (mpl <= 4) MOE_TOPK(4);
+  else if (mpl <= 8) MOE_TOPK(8);
+  else if (mpl <= 9) MOE_TOPK(9);
+  else if (mpl <= 16) MOE_TOPK(16);
+  else MOE_TOPK(32);
+#undef MOE_TOPK
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -23,3 +23,31 @@ def algorithmic_flops(wl: Workload) -> int:
     H, I, Is, E, k = wl.hidden, wl.intermediate, wl.shared_intermediate, wl.num_experts, wl.top_k
     per_tok = 2 * H * E + k * (2 * H * 2 * I + 2 * I * H) + (2 * H * 2 * Is + 2 * Is * H)
     return wl.T * per_tok
+
+
+def gate_up_bytes(wl: Workload, touched_routed: int) -> int:
+    """Bytes the grouped gate|up GEMM must move at least once: the gate and up
+    weights of the touched routed experts and of the shared expert, the input
+    rows (T x H) and the SwiGLU output h ((k + 1) rows per token x I, bf16)."""
+    el_w = 2 if wl.weight_dtype == "bf16" else 4
+    el_x = 2 if wl.act_dtype == "bf16" else 4
+    H, I = wl.hidden, wl.intermediate
+    weights = (touched_routed + 1) * 2 * H * I * el_w
+    return weights + wl.T * H * el_x + wl.T * (wl.top_k + 1) * I * 2
+
+
+def gate_up_flops(wl: Workload) -> int:
+    """2 x multiply-adds of the gate and up projections of k routed + 1 shared experts."""
+    return wl.T * (wl.top_k + 1) * 2 * wl.hidden * 2 * wl.intermediate
+
+
+def down_bytes(wl: Workload, touched_routed: int) -> int:
+    """Down weights of the touched experts + shared, h in, y out (bf16)."""
+    el_w = 2 if wl.weight_dtype == "bf16" else 4
+    H, I = wl.hidden, wl.intermediate
+    rows = wl.T * (wl.top_k + 1)
+    return (touched_routed + 1) * H * I * el_w + rows * I * 2 + rows * H * 2
+
+
+def down_flops(wl: Workload) -> int:
+    return wl.T * (wl.top_k + 1) * 2 * wl.intermediate * wl.hidden

@@ -1,0 +1,93 @@
+"""Comparison of the CUDA path with the CPU oracle (used by the GPU tests and
+by the smoke check).
+
+Bar (element by element):
+* top-k indices bit-exact, except tokens whose oracle k-th and (k+1)-th fp32
+  selection scores differ by less than TIE_BAND (several selections are then
+  correct); those are counted, and their outputs are re-checked against the
+  oracle evaluated on the GPU's selection;
+* counts, offsets and the permutation bit-exact given the selection;
+* gate weights within fp32 rounding (rtol 1e-5);
+* outputs: relative Frobenius error <= 1e-2 and max |error| <= 5e-2 * RMS(out).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+import oracle.moe_oracle as om
+
+TIE_BAND = 1e-6
+REL_FRO = 1e-2
+MAX_ABS_OVER_RMS = 5e-2
+W_RTOL = 1e-5
+
+
+@dataclass
+class ParityReport:
+    tokens: int
+    near_ties: int
+    idx_mismatch_rows: int
+    rel_fro: float
+    max_abs_over_rms: float
+    rows_checked: int
+
+    def ok(self) -> bool:
+        return self.rel_fro <= REL_FRO and self.max_abs_over_rms <= MAX_ABS_OVER_RMS
+
+
+def check_routing(gpu_rt: dict, ref: dict, top_k: int, E: int):
+    """Selection, weights and grouping.  Returns (mismatched-row mask, near-tie mask)."""
+    gidx = gpu_rt["topk_idx"]
+    tie = ref["tie_gap"] < TIE_BAND
+    mism = (gidx != ref["topk_idx"]).any(axis=1)
+    bad = np.nonzero(mism & ~tie)[0]
+    assert bad.size == 0, f"top-k differs on {bad.size} non-tied tokens, first {bad[:8]}"
+    # weights: the bias-free scores of the (same) selection, renormalised, scaled
+    ok = ~mism
+    np.testing.assert_allclose(gpu_rt["topk_w"][ok], ref["topk_w"][ok], rtol=W_RTOL, atol=1e-7)
+    # grouping: the permutation of the GPU's own selection is unique
+    counts, offsets, perm, _ = om.expert_permutation(gidx, E)
+    assert np.array_equal(gpu_rt["counts"], counts)
+    assert np.array_equal(gpu_rt["offsets"], offsets)
+    assert np.array_equal(gpu_rt["perm"], perm)
+    if not mism.any():
+        assert np.array_equal(gpu_rt["perm"], ref["perm"])
+        assert np.array_equal(gpu_rt["counts"], ref["counts"])
+    return mism, tie
+
+
+def output_errors(gpu_out: np.ndarray, ref_out: np.ndarray):
+    d = gpu_out.astype(np.float64) - ref_out
+    rel = float(np.linalg.norm(d) / max(np.linalg.norm(ref_out), 1e-300))
+    rms = float(np.sqrt(np.mean(ref_out ** 2)))
+    mx = float(np.max(np.abs(d)) / max(rms, 1e-300))
+    return rel, mx
+
+
+def compare(inp_host: dict, wl, gpu_out: np.ndarray, gpu_rt: dict,
+            rows: Optional[np.ndarray] = None, experts=None) -> ParityReport:
+    """inp_host: exact fp32 host copies of x, router_w, router_bias (and, when
+    ``experts`` is None, of all weights); ``experts`` may supply lazy
+    per-expert views (w_gate, w_up, w_down, sh_gate, sh_up, sh_down)."""
+    k, E = wl.top_k, wl.num_experts
+    x = inp_host["x"]
+    ref = om.moe_routing(x, inp_host["router_w"], inp_host["router_bias"], top_k=k,
+                         scale=wl.scale)
+    mism, tie = check_routing(gpu_rt, ref, k, E)
+    T = x.shape[0]
+    if rows is None:
+        rows = np.arange(T)
+    rows = np.unique(np.concatenate([np.asarray(rows, np.int64), np.nonzero(mism)[0]]))
+    w = experts if experts is not None else inp_host
+    res = om.moe_forward_rows(rows, x, inp_host["router_w"], inp_host["router_bias"],
+                              w["w_gate"], w["w_up"], w["w_down"], w["sh_gate"], w["sh_up"],
+                              w["sh_down"], top_k=k, scale=wl.scale,
+                              swiglu_limit=wl.swiglu_limit,
+                              swiglu_limit_shared=wl.swiglu_limit_shared,
+                              forced_idx=gpu_rt["topk_idx"][rows])
+    rel, mx = output_errors(gpu_out[rows], res.out)
+    return ParityReport(tokens=T, near_ties=int(tie.sum()), idx_mismatch_rows=int(mism.sum()),
+                        rel_fro=rel, max_abs_over_rms=mx, rows_checked=int(rows.size))
