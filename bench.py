@@ -44,6 +44,9 @@ def _args():
     ap.add_argument("--secondary", default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling case: override the number of routed experts "
+                         "(smaller device footprint for ncu captures)")
     return ap.parse_args()
 
 
@@ -270,8 +273,9 @@ def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step):
 def run_ours(a):
     import torch
     import torch.distributed as dist
-    from dataclasses import replace
     from sparse_moe_layer_gemm_b200 import binding as B
+    from sparse_moe_layer_gemm_b200.replicas import (job_throughput, max_over_ranks,
+                                                     rank_batch_workload)
     from sparse_moe_layer_gemm_b200.workloads import WORKLOADS, draw_x, make_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -284,10 +288,13 @@ def run_ours(a):
     torch.cuda.set_device(dev)
     B.load_library()
     wl = WORKLOADS[a.workload]
+    if a.experts:
+        from dataclasses import replace as _replace
+        wl = _replace(wl, num_experts=a.experts, name=f"{wl.name}_e{a.experts}")
     peaks = _peaks()
 
     inp = make_inputs(wl, dev)                          # weights replicated on every rank
-    x = draw_x(replace(wl, seed=rank), dev)             # each rank its own batch
+    x = draw_x(rank_batch_workload(wl, rank), dev)      # each rank its own batch
     layer = B.MoeLayer.from_workload(wl)
     layer.load_inputs(inp)
     stream = torch.cuda.Stream(device=dev)
@@ -314,14 +321,11 @@ def run_ours(a):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     err = layer.device_error()
     if err != 0:
         raise RuntimeError(f"device status word {err}")
-    value = world * wl.T / (ms * 1e-3)
+    value = job_throughput(wl.T, world, ms)
     kr, lr = _kernel_roofline(wl, touched, stages, peaks, ms)
 
     e2e = None
@@ -339,11 +343,9 @@ def run_ours(a):
                 layer.forward_host(xh, oh, stream=stream)
             e1.record(stream)
             torch.cuda.synchronize()
-        et = torch.tensor([e0.elapsed_time(e1) / n], device=dev)
-        if world > 1:
-            dist.all_reduce(et, op=dist.ReduceOp.MAX)
+        et = max_over_ranks(e0.elapsed_time(e1) / n, dev)
         el = 2 if wl.act_dtype == "bf16" else 4
-        e2e = {"value": world * wl.T / (float(et.item()) * 1e-3), "unit": "tokens/s",
+        e2e = {"value": job_throughput(wl.T, world, et), "unit": "tokens/s",
                "h2d_bytes_per_step": wl.T * wl.hidden * el,
                "d2h_bytes_per_step": wl.T * wl.hidden * el,
                "path": "moe_forward_host (pinned host x/out, copies inside the timed region)"}
@@ -354,17 +356,15 @@ def run_ours(a):
         same_weights = (wl2.expert_std == wl.expert_std and wl2.weight_dtype == wl.weight_dtype
                         and wl2.bias == wl.bias and wl2.hidden == wl.hidden)
         if same_weights:
-            x2 = draw_x(replace(wl2, seed=rank), dev)
+            x2 = draw_x(rank_batch_workload(wl2, rank), dev)
             l2 = layer
             touched2, _ = _routing_stats(l2, x2)
             barrier()
             ms2, st2 = _measure(l2, x2, max(3, a.steps // 10), max(3, a.warmup), stream)
-            t2 = torch.tensor([ms2], device=dev)
-            if world > 1:
-                dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-            ms2 = float(t2.item())
+            ms2 = max_over_ranks(ms2, dev)
             kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2)
-            secondary = {"workload": wl2.name, "T": wl2.T, "value": world * wl2.T / (ms2 * 1e-3),
+            secondary = {"workload": wl2.name, "T": wl2.T,
+                         "value": job_throughput(wl2.T, world, ms2),
                          "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
                          "layer_roofline": lr2, "stage_ms": st2}
             del x2
