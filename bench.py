@@ -59,22 +59,24 @@ def _peaks():
     return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, source="fallback")
 
 
-def _traffic_record(kernel: str, workload: str):
-    """ncu DRAM bytes per launch of `kernel`, if the committed capture still
-    matches the kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+def _traffic_record(kernel: str, workload: str, groups: int):
+    """ncu DRAM bytes per launch of `kernel`: the committed per-group figure
+    times the launch's groups, or None once the kernel source has changed
+    since the capture."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
     try:
-        recs = json.load(open(p))
-        rec = recs.get(f"{kernel}:{workload}")
-        if rec is None:
-            return None
-        src = os.path.join(ROOT, rec["source"])
-        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        return rec["bytes_per_launch"] if h == rec["source_sha256"] else None
+        for line in open(p):
+            f = line.split()
+            if not f or f[0].startswith("#") or f[0] != f"{kernel}:{workload}":
+                continue
+            src = os.path.join(ROOT, f[1])
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+            return int(f[3]) * groups if h == f[2] else None
     except Exception:
         return None
+    return None
 
 
 class ClockSampler:
@@ -260,7 +262,7 @@ def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step):
                "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json)"
                if peaks["source"] == "measured" else "fallback",
-               "traffic": _traffic_record("gate_up", wl.name)})
+               "traffic": _traffic_record("gate_up", wl.name, touched + 1)})
     lb = algorithmic_bytes(wl, touched)
     lf = algorithmic_flops(wl)
     t_layer = max(lb / (peaks["hbm"] * 1e9), lf / (peaks["tc"] * 1e12))
