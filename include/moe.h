@@ -178,6 +178,35 @@ int moe_forward_oneshot(const void* x, const float* router_w, const float* route
                         float swiglu_limit, float swiglu_limit_shared,
                         int act_dtype, int weight_dtype, void* out, void* stream);
 
+/* Routing without any device allocation: router logits x . W_r (fp32),
+ * sigmoid scores, top-k of score + router_bias (descending, ties to the lower
+ * index), and the gate weights scale * s / sum(s) of the selected bias-free
+ * scores (plain scale * s when norm_expert_weight is 0).  The source pages
+ * have no counterpart of this entry point: it exists for callers that cannot
+ * call cudaMalloc, such as code running under CUDA-graph capture, runtimes
+ * that own all of HBM through their own pool, or latency-critical loops where
+ * an allocation could synchronise the device.  It needs no layer handle and
+ * no workspace.
+ *
+ * x [T, H] (act_dtype, 16-byte aligned), router_w [H, E] fp32, router_bias
+ * [E] fp32 or NULL; outputs topk_idx [T, k] int32 and topk_w [T, k] fp32, all
+ * device pointers owned by the caller.  Same results as the routing outputs
+ * of moe_forward for the same configuration.
+ *
+ * Scratch: a 4 MiB static device array inside the library (1,048,576 fp32
+ * partial logits), held on every GPU that loads the library until the
+ * process exits.  T * E must not exceed 1,048,576 (MOE_ERR_UNSUPPORTED
+ * otherwise).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call uses the same array, so calls that
+ * may overlap on the GPU (different streams, or different host threads) race
+ * and must be serialised by the caller.  No cudaMalloc, cudaFree or other
+ * allocating routine is called. */
+int moe_route_static(const void* x, int act_dtype, const float* router_w,
+                     const float* router_bias, int T, int H, int E, int k,
+                     int norm_expert_weight, float routed_scaling_factor,
+                     int32_t* topk_idx, float* topk_w, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,7 @@ EXPORTS = (
     "moe_config_check", "moe_create", "moe_load_weights", "moe_workspace_size",
     "moe_forward", "moe_workspace_size_host", "moe_forward_host", "moe_get_device_error",
     "moe_status_string", "moe_destroy", "moe_forward_oneshot", "moe_kernel_launches",
-    "moe_set_stage_timing", "moe_get_stage_times",
+    "moe_set_stage_timing", "moe_get_stage_times", "moe_route_static",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -98,6 +98,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward_oneshot.argtypes = [vp] * 9 + [i] * 5 + [f] * 3 + [i, i, vp, vp]
     lib.moe_kernel_launches.argtypes = [vp, i]
     lib.moe_set_stage_timing.argtypes = [vp, i]
+    lib.moe_route_static.argtypes = [vp, i, vp, vp, i, i, i, i, i, f, vp, vp, vp]
     lib.moe_get_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i,
                                         ctypes.POINTER(i)]
     for name in EXPORTS:
@@ -228,6 +229,16 @@ def moe_get_stage_times(handle):
     _check(load_library().moe_get_stage_times(ctypes.c_void_p(handle), ms, MOE_NUM_STAGES,
                                               ctypes.byref(n)), "moe_get_stage_times")
     return dict(zip(STAGE_NAMES, list(ms))), n.value
+
+
+def moe_route_static(x, act_dtype, router_w, router_bias, T, H, E, k, norm_expert_weight,
+                     routed_scaling_factor, topk_idx, topk_w, stream=None) -> int:
+    """Routing with no device allocation (see include/moe.h): for callers
+    that cannot call cudaMalloc, e.g. under CUDA-graph capture."""
+    return load_library().moe_route_static(
+        _ptr(x), act_dtype, _ptr(router_w), _ptr(router_bias), T, H, E, k,
+        int(bool(norm_expert_weight)), float(routed_scaling_factor), _ptr(topk_idx),
+        _ptr(topk_w), _stream(stream))
 
 
 # ----------------------------------------------------------------- layer object

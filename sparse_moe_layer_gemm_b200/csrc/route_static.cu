@@ -1,0 +1,94 @@
+// moe_route_static: the routing stage (router logits, sigmoid scores, top-k on
+// the biased scores, renormalised and scaled gate weights) for callers that
+// must not allocate device memory.
+//
+// Who needs it: code that runs while a CUDA graph is being captured (a
+// cudaMalloc there invalidates the capture), runtimes that own every byte of
+// HBM through their own pool and forbid allocations behind their back, and
+// latency-critical loops where a cudaMalloc / cudaFree may synchronise the
+// whole device.  moe_forward needs a caller-provided workspace and a layer
+// handle whose creation allocates; this entry point needs neither.
+//
+// Its only scratch, the split-K partial logits, lives in the file-scope array
+// below.  Every GPU that loads the library holds it until the process exits.
+// In host code `g_route_scratch` is a host-side stand-in, not a device
+// address, so its device address is looked up once per device with
+// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+#include <math.h>
+
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+namespace {
+
+// 4 MiB: partial logits [splits][T][E] fp32.
+constexpr size_t kRouteScratchFloats = static_cast<size_t>(1) << 20;
+__device__ __align__(256) float g_route_scratch[kRouteScratchFloats];
+
+constexpr int kMaxDevices = 64;
+float* g_scratch_dev[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device (looked up the
+// first time this device is seen).
+int scratch_for_current_device(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_dev[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
+      return MOE_ERR_CUDA;
+    g_scratch_dev[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_dev[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" int moe_route_static(const void* x, int act_dtype, const float* router_w,
+                                const float* router_bias, int T, int H, int E, int k,
+                                int norm_expert_weight, float routed_scaling_factor,
+                                int32_t* topk_idx, float* topk_w, void* stream) {
+  if (T < 0 || H <= 0 || E <= 0 || k <= 0 || k > E) return MOE_ERR_INVALID_ARG;
+  if (act_dtype != MOE_F32 && act_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (!isfinite(routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0 || H > 16384 || E > 1024 || k > 32) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || router_w == nullptr || topk_idx == nullptr || topk_w == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(x) % 16 != 0) return MOE_ERR_INVALID_ARG;
+  // one split must fit: T * E fp32 partial logits
+  if (static_cast<size_t>(T) * E > kRouteScratchFloats) return MOE_ERR_UNSUPPORTED;
+
+  float* scratch = nullptr;
+  int r = scratch_for_current_device(&scratch);
+  if (r != MOE_OK) return r;
+  int dev = 0, num_sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+
+  // K splits: the rule moe_forward uses, reduced until the partials fit.
+  const int tiles = ((E + moe::kRouterExp - 1) / moe::kRouterExp) *
+                    ((T + moe::kRouterTok - 1) / moe::kRouterTok);
+  int splits = 1;
+  while (tiles * splits < 2 * num_sms && H / (2 * splits) >= 128 &&
+         H % (2 * splits * moe::kRouterKStep) == 0)
+    splits *= 2;
+  while (splits > 1 && static_cast<size_t>(splits) * T * E > kRouteScratchFloats) splits /= 2;
+
+  // Every partial the top-k reads is written first, so nothing needs clearing.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (moe::launch_router_logits(x, act_dtype == MOE_BF16, router_w, scratch, T, H, E, splits,
+                                st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe::launch_topk(scratch, splits, T, E, k, router_bias, norm_expert_weight != 0,
+                       routed_scaling_factor, topk_idx, topk_w, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
