@@ -82,13 +82,15 @@ typedef struct moe_layer moe_layer_t;
  * any field may be NULL).  topk_idx [T, k] int32 (descending s + b),
  * topk_w [T, k] fp32 gate weights, counts [E] int32 pairs per expert,
  * offsets [E + 1] int32 exclusive prefix of counts, perm [T * k] int32 pair
- * ids t * k + j grouped by expert, ascending t within an expert. */
+ * ids t * k + j grouped by expert, ascending t within an expert, logits
+ * [T, E] fp32 router logits x . W_r as used for the selection. */
 typedef struct {
   int32_t* topk_idx;
   float* topk_w;
   int32_t* counts;
   int32_t* offsets;
   int32_t* perm;
+  float* logits;
 } moe_routing_t;
 
 /* Host-only check of a configuration; no CUDA call.  Returns MOE_OK,
@@ -190,8 +192,12 @@ int moe_forward_oneshot(const void* x, const float* router_w, const float* route
  *
  * x [T, H] (act_dtype, 16-byte aligned), router_w [H, E] fp32, router_bias
  * [E] fp32 or NULL; outputs topk_idx [T, k] int32 and topk_w [T, k] fp32, all
- * device pointers owned by the caller.  Same results as the routing outputs
- * of moe_forward for the same configuration.
+ * device pointers owned by the caller.  It runs the router on the CUDA cores
+ * with the K split moe_forward uses there (below 512 tokens, or fp32 x), and
+ * gives identical results whenever T * E * H / 128 <= 1,048,576 (else it
+ * uses fewer splits).  From 512 bf16 tokens moe_forward runs the router on
+ * the tensor cores; the two then agree to fp32 rounding (the selection can
+ * differ only on tokens whose k-th and (k+1)-th scores are within ~1e-6).
  *
  * Scratch: a 4 MiB static device array inside the library (1,048,576 fp32
  * partial logits), held on every GPU that loads the library until the

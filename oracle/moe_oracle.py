@@ -254,10 +254,11 @@ def moe_routing(x, router_w, router_bias, *, top_k: int, scale: float = 3.0,
     :func:`moe_forward` (sglang-jax issue #1367, "Key difficulties" item 1)."""
     x64 = _f64(x)
     E = np.asarray(router_w).shape[1]
-    _, beta32, idx, w = _route(x64, router_w, router_bias, top_k, scale, norm, use_bias, None)
+    logits, beta32, idx, w = _route(x64, router_w, router_bias, top_k, scale, norm, use_bias,
+                                    None)
     counts, offsets, perm, pos = expert_permutation(idx, E)
     return dict(topk_idx=idx, topk_w=w, counts=counts, offsets=offsets, perm=perm, pos=pos,
-                beta32=beta32, tie_gap=near_tie_gaps(beta32, top_k))
+                beta32=beta32, tie_gap=near_tie_gaps(beta32, top_k), logits=logits)
 
 
 def moe_forward(x, router_w, router_bias, w_gate, w_up, w_down,

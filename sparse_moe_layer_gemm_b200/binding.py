@@ -61,6 +61,7 @@ class moe_routing_t(ctypes.Structure):
         ("counts", ctypes.c_void_p),
         ("offsets", ctypes.c_void_p),
         ("perm", ctypes.c_void_p),
+        ("logits", ctypes.c_void_p),
     ]
 
 
@@ -315,9 +316,10 @@ class MoeLayer:
                       topk_w=torch.empty(T, k, dtype=torch.float32, device=dev),
                       counts=torch.empty(E, dtype=torch.int32, device=dev),
                       offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
-                      perm=torch.empty(T * k, dtype=torch.int32, device=dev))
+                      perm=torch.empty(T * k, dtype=torch.int32, device=dev),
+                      logits=torch.empty(T, E, dtype=torch.float32, device=dev))
             r = moe_routing_t(*(rt[n].data_ptr() for n in
-                                ("topk_idx", "topk_w", "counts", "offsets", "perm")))
+                                ("topk_idx", "topk_w", "counts", "offsets", "perm", "logits")))
         _check(moe_forward(self.handle, x.data_ptr(), T, out.data_ptr(), ws.data_ptr(),
                            ws.numel(), stream, r), "moe_forward")
         return (out, rt) if routing else out

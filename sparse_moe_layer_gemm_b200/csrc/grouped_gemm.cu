@@ -6,6 +6,11 @@
 //                  h = silu(gate) * up, stored bf16.
 //   K6 (down):     y = (h_g . Wd_g) * w_row, the row's gate weight (1 for the
 //                  shared rows), stored bf16.
+//   K1 (router, large T):  logits = x . W_r in fp32 accuracy on the bf16 tensor
+//                  cores: W_r = W1 + W2 + W3 split into three bf16 terms that
+//                  are concatenated along K, so one accumulation over 3H gives
+//                  x.W1 + x.W2 + x.W3 (each bf16 x bf16 product is exact in
+//                  fp32; x is bf16 and needs no split); stored fp32.
 //
 // The expert FFN is the SwiGLU of sglang-jax issue #1367 "Support Step 3.5
 // Flash", section "Model configuration" (MoE bullet; clamped SwiGLU via
@@ -37,8 +42,9 @@ namespace moe {
 
 namespace {
 
-template <bool GU>
+template <int MODE>
 struct Shape {
+  static constexpr bool GU = MODE == kModeGateUp;
   static constexpr int A_ROWS = GU ? 2 * kBM : kBM;
   static constexpr int A_BYTES = A_ROWS * kBK * 2;
   static constexpr int B_BYTES = kBN * kBK * 2;
@@ -62,6 +68,14 @@ struct Tile {
 // prefix of per-group tile counts, so the group is the last g with
 // tile_start[g] <= w (empty groups are skipped naturally).
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
+  if (p.single_rows > 0) {
+    Tile t;
+    t.g = 0;
+    t.nc = w / p.m_tiles;
+    t.mt = w - t.nc * p.m_tiles;
+    t.n_valid = min(kBN, p.single_rows - t.nc * kBN);
+    return t;
+  }
   int lo = 0, hi = p.G;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -79,12 +93,22 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
   return t;
 }
 
-template <bool GU>
+__device__ __forceinline__ int total_tiles(const GemmParams& p) {
+  if (p.single_rows > 0) return p.m_tiles * ((p.single_rows + kBN - 1) / kBN);
+  return p.tile_start[p.G];
+}
+
+__device__ __forceinline__ int group_row0(const GemmParams& p, int g) {
+  return p.single_rows > 0 ? 0 : p.row_start[g];
+}
+
+template <int MODE>
 __global__ void __launch_bounds__(192, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBsh, const GemmParams p) {
-  using S = Shape<GU>;
+  using S = Shape<MODE>;
+  constexpr bool GU = S::GU;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -126,7 +150,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = p.tile_start[p.G];
+  const int total = total_tiles(p);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -141,7 +165,7 @@ __global__ void __launch_bounds__(192, 1)
         const int nbox = (n_mma + kBBoxRows - 1) / kBBoxRows;
         const bool sh = GU && t.g == p.E;
         const CUtensorMap* mb = sh ? &tmBsh : &tmB;
-        const int b_row = (sh ? p.shared_b_row0 : p.row_start[t.g]) + t.nc * kBN;
+        const int b_row = (sh ? p.shared_b_row0 : group_row0(p, t.g)) + t.nc * kBN;
         const int a_row = t.g * p.a_rows_per_group + t.mt * S::A_ROWS;
         const uint32_t bytes = S::A_BYTES + nbox * S::B_BOX_BYTES;
         bool ok = true;
@@ -157,8 +181,9 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
           const uint32_t sb = sa + S::A_BYTES;
           tma_load_2d(sa, &tmA, fb, kb * kBK, a_row, pol_a);
+          const int bk = p.b_k_wrap > 0 ? (kb * kBK) % p.b_k_wrap : kb * kBK;
           for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sb + i * S::B_BOX_BYTES, mb, fb, kb * kBK, b_row + i * kBBoxRows, pol_b);
+            tma_load_2d(sb + i * S::B_BOX_BYTES, mb, fb, bk, b_row + i * kBBoxRows, pol_b);
           ++it;
         }
         if (!ok) break;
@@ -230,9 +255,21 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * S::ACC_COLS;
       const int feat = t.mt * kBM + q * 32 + lane;
-      const size_t row0 = static_cast<size_t>(p.row_start[t.g]) + static_cast<size_t>(t.nc) * kBN;
-      __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
-      if (GU) {
+      const size_t row0 = static_cast<size_t>(group_row0(p, t.g)) + static_cast<size_t>(t.nc) * kBN;
+      if (MODE == kModeRouter) {
+        float* lp = p.out_f32 + row0 * p.out_ld + feat;
+        const bool keep = feat < p.valid_feats;
+        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+          uint32_t ra[16];
+          tmem_ld_x16(taddr + c0, ra);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (keep && c0 + i < t.n_valid)
+              lp[static_cast<size_t>(c0 + i) * p.out_ld] = __uint_as_float(ra[i]);
+        }
+      } else if (GU) {
+        __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
         const float L = (t.g == p.E) ? p.limit_shared : p.limit;
         for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
           uint32_t ra[16], rb[16];
@@ -254,6 +291,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       } else {
+        __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
         const float* wrow = p.w_perm + row0;
         for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
           uint32_t ra[16];
@@ -286,28 +324,41 @@ __global__ void __launch_bounds__(192, 1)
 
 }  // namespace
 
-size_t gemm_smem_bytes(bool gate_up) { return gate_up ? Shape<true>::SMEM : Shape<false>::SMEM; }
+size_t gemm_smem_bytes(int mode) {
+  return mode == kModeGateUp ? Shape<kModeGateUp>::SMEM
+                             : (mode == kModeDown ? Shape<kModeDown>::SMEM : Shape<kModeRouter>::SMEM);
+}
 
 cudaError_t gemm_configure_device() {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<true>,
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGateUp>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Shape<true>::SMEM));
+                                       static_cast<int>(Shape<kModeGateUp>::SMEM));
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(grouped_gemm_kernel<false>,
+  e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeDown>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(Shape<kModeDown>::SMEM));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kModeRouter>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(Shape<false>::SMEM));
+                              static_cast<int>(Shape<kModeRouter>::SMEM));
 }
 
 cudaError_t launch_gemm_gate_up(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 const CUtensorMap& tmBsh, const GemmParams& p, int grid,
                                 cudaStream_t st) {
-  grouped_gemm_kernel<true><<<grid, 192, Shape<true>::SMEM, st>>>(tmA, tmB, tmBsh, p);
+  grouped_gemm_kernel<kModeGateUp><<<grid, 192, Shape<kModeGateUp>::SMEM, st>>>(tmA, tmB, tmBsh, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                              int grid, cudaStream_t st) {
-  grouped_gemm_kernel<false><<<grid, 192, Shape<false>::SMEM, st>>>(tmA, tmB, tmB, p);
+  grouped_gemm_kernel<kModeDown><<<grid, 192, Shape<kModeDown>::SMEM, st>>>(tmA, tmB, tmB, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_router(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
+                               int grid, cudaStream_t st) {
+  grouped_gemm_kernel<kModeRouter><<<grid, 192, Shape<kModeRouter>::SMEM, st>>>(tmA, tmB, tmB, p);
   return cudaGetLastError();
 }
 

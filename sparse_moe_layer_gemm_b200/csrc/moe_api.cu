@@ -25,11 +25,14 @@ struct moe_layer {
   __nv_bfloat16* w_dn;  // [(E+1) * H, I_pad]
   float* router_w;      // [H, E]
   float* router_b;      // [E]
+  __nv_bfloat16* router_tc;  // [E_pad, 3H]: bf16 three-term split of router_w^T
+  int E_pad;
   int has_bias;
   int* status;          // device status word
   int loaded;
   CUtensorMap tm_gu;    // A operand of K5 (box 64 x 256)
   CUtensorMap tm_dn;    // A operand of K6 (box 64 x 128)
+  CUtensorMap tm_router;  // A operand of the tensor-core router (box 64 x 128)
   // stage timers: capacity x (MOE_NUM_STAGES + 1) events, filled in order
   std::vector<cudaEvent_t> events;
   int timing_capacity;
@@ -49,12 +52,13 @@ struct WsLayout {
   int ksplit, nch, rows_routed, rows_xperm, rows_all;
 };
 
-int router_ksplit(int T, int H, int E, int num_sms) {
-  const int tiles = ((E + moe::kRouterExp - 1) / moe::kRouterExp) *
-                    ((T + moe::kRouterTok - 1) / moe::kRouterTok);
-  int s = 1;
-  while (tiles * s < 2 * num_sms && H / (2 * s) >= 128 && H % (2 * s * moe::kRouterKStep) == 0)
-    s *= 2;
+// K splits of the CUDA-core router: fixed 128-wide K chunks, so a token's
+// logits do not depend on the batch it arrives in; halved (or dropped to one)
+// only if the partial logits would exceed 64 MB.
+int router_ksplit(int T, int H, int E) {
+  constexpr size_t kMaxPartialFloats = static_cast<size_t>(16) << 20;
+  int s = H / 128;
+  while (s > 1 && static_cast<size_t>(T) * E * s > kMaxPartialFloats) s = (s % 2 == 0) ? s / 2 : 1;
   return s;
 }
 
@@ -62,7 +66,7 @@ WsLayout ws_layout(const moe_layer* L, int T) {
   const moe_config_t& c = L->cfg;
   const int H = c.hidden, E = c.num_experts, k = c.top_k, G = E + 1;
   WsLayout w{};
-  w.ksplit = router_ksplit(T, H, E, L->num_sms);
+  w.ksplit = router_ksplit(T, H, E);
   w.nch = (T + moe::kSortChunk - 1) / moe::kSortChunk;
   w.rows_routed = T * k;
   w.rows_xperm = T * k + (c.act_dtype == MOE_F32 ? T : 0);
@@ -191,6 +195,7 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
   if (L == nullptr) return MOE_ERR_CUDA;
   L->cfg = *cfg;
   L->I_pad = (cfg->intermediate + 127) / 128 * 128;
+  L->E_pad = (cfg->num_experts + 127) / 128 * 128;
   if (cudaGetDevice(&L->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) !=
           cudaSuccess) {
@@ -204,13 +209,15 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
       cudaMalloc(&L->w_dn, dn_bytes) != cudaSuccess ||
       cudaMalloc(&L->router_w, H * E * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&L->router_b, E * sizeof(float)) != cudaSuccess ||
+      cudaMalloc(&L->router_tc, static_cast<size_t>(L->E_pad) * 3 * H * 2) != cudaSuccess ||
       cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
       cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
   }
   if (!encode_bf16_2d(&L->tm_gu, L->w_gu, (E + 1) * 2 * Ip, H, 2 * moe::kBM) ||
-      !encode_bf16_2d(&L->tm_dn, L->w_dn, (E + 1) * H, Ip, moe::kBM)) {
+      !encode_bf16_2d(&L->tm_dn, L->w_dn, (E + 1) * H, Ip, moe::kBM) ||
+      !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM)) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
   }
@@ -241,6 +248,7 @@ int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_
   MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, L->w_dn + E * dn_group, st));
   MOE_CUDA(cudaMemcpyAsync(L->router_w, router_w, static_cast<size_t>(H) * E * sizeof(float),
                            cudaMemcpyDeviceToDevice, st));
+  MOE_CUDA(moe::launch_pack_router(router_w, H, E, L->E_pad, L->router_tc, st));
   L->has_bias = (c.use_router_bias && router_bias != nullptr) ? 1 : 0;
   if (L->has_bias)
     MOE_CUDA(cudaMemcpyAsync(L->router_b, router_bias, E * sizeof(float),
@@ -318,11 +326,37 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   auto mark = [&](int i) { return ev == nullptr ? cudaSuccess : cudaEventRecord(ev[i], st); };
 
   MOE_CUDA(mark(0));
-  MOE_CUDA(moe::launch_router_logits(x, xb, L->router_w, partial, T, H, E, w.ksplit, st));
+  int ksplit = w.ksplit;
+  moe::TopkRefine refine{};
+  const bool tc_router = xb && T >= moe::kTcRouterMinTokens;
+  if (tc_router) {
+    // tensor-core router: one group of T rows, 3H reduction over W1 | W2 | W3
+    GemmParams r{};
+    r.single_rows = T;
+    r.E = E;
+    r.num_kb = 3 * H / moe::kBK;
+    r.m_tiles = L->E_pad / moe::kBM;
+    r.b_k_wrap = H;
+    r.out_f32 = partial;
+    r.out_ld = E;
+    r.valid_feats = E;
+    r.status = L->status;
+    const int tiles = r.m_tiles * ((T + moe::kBN - 1) / moe::kBN);
+    MOE_CUDA(moe::launch_gemm_router(L->tm_router, tm_bsh, r, tiles < L->num_sms ? tiles : L->num_sms,
+                                     st));
+    ksplit = 1;
+    refine.x = static_cast<const __nv_bfloat16*>(x);
+    refine.w_tc = L->router_tc;
+    refine.H = H;
+    refine.band = moe::router_refine_band(H);
+  } else {
+    MOE_CUDA(moe::launch_router_logits(x, xb, L->router_w, partial, T, H, E, w.ksplit, st));
+  }
   MOE_CUDA(mark(1));
-  MOE_CUDA(moe::launch_topk(partial, w.ksplit, T, E, k, L->has_bias ? L->router_b : nullptr,
+  MOE_CUDA(moe::launch_topk(partial, ksplit, T, E, k, L->has_bias ? L->router_b : nullptr,
                             c.norm_expert_weight != 0, c.routed_scaling_factor, topk_idx, topk_w,
-                            st));
+                            st, routing != nullptr ? routing->logits : nullptr,
+                            tc_router ? &refine : nullptr));
   MOE_CUDA(mark(2));
   MOE_CUDA(moe::launch_sort(topk_idx, topk_w, T, k, E, Ip / moe::kBM, H / moe::kBM, masks,
                             chunk_cnt, chunk_base, counts, row_start, tiles_gu, tiles_dn, perm, pos,
@@ -422,8 +456,9 @@ int moe_get_device_error(moe_layer_t* L, int* device_err) {
 
 int moe_kernel_launches(const moe_layer_t* L, int T) {
   if (L == nullptr || T <= 0) return 0;
-  // router, top-k, 3 sort kernels, gather, gate|up GEMM, down GEMM, combine
-  return 9;
+  // router, top-k, counting sort (one kernel up to kSortChunk tokens, else
+  // three), gather, gate|up GEMM, down GEMM, combine
+  return T <= moe::kSortChunk ? 7 : 9;
 }
 
 namespace {
@@ -487,6 +522,7 @@ void moe_destroy(moe_layer_t* L) {
     cudaFree(L->w_dn);
     cudaFree(L->router_w);
     cudaFree(L->router_b);
+    cudaFree(L->router_tc);
     cudaFree(L->status);
   }
   delete L;

@@ -25,7 +25,17 @@ constexpr int kRouterKStep = 32;
 // Chunk of tokens owned by one block of the counting sort (4 x 32-bit masks).
 constexpr int kSortChunk = 128;
 
+// Epilogue modes of the grouped GEMM kernel.
+constexpr int kModeGateUp = 0;  // h = silu(clamp(gate)) * clamp(up), bf16
+constexpr int kModeDown = 1;    // y = acc * w_perm[row], bf16
+constexpr int kModeRouter = 2;  // logits = acc, fp32, features < valid_feats
+
+// Token count from which the router runs on the tensor cores (bf16 x only).
+constexpr int kTcRouterMinTokens = 512;
+
 struct GemmParams {
+  int single_rows;        // > 0: one group of this many rows starting at row 0
+                          // (counts / row_start / tile_start unused)
   const int* counts;      // [G] rows per group (group E = the shared expert, T rows)
   const int* row_start;   // [G + 1] first row of each group in x_perm / h / y
   const int* tile_start;  // [G + 1] exclusive prefix of the group's tile counts
@@ -41,13 +51,35 @@ struct GemmParams {
   float limit;            // gate/up clamp of routed experts (<= 0: none)
   float limit_shared;     // gate/up clamp of the shared expert
   int* status;            // device status word
+  int b_k_wrap;           // > 0: B's K coordinate wraps at this value (router)
+  float* out_f32;         // router: logits [rows, out_ld]
+  int valid_feats;        // router: features (experts) actually stored
+};
+
+// Guard band (selection-score units) of the top-k after the tensor-core
+// router: experts whose approximate score is within it of the approximate
+// k-th are recomputed in fp32 on the CUDA cores.  Sized from a worst-case
+// accumulation error: 3H/16 MMA steps, each truncating at most one fp32 ulp
+// of partial sums up to magnitude 8 (2^-20), times the sigmoid's maximum
+// slope 0.25, times 2 for the two sides of the boundary -- ~3.7e-4 at
+// H = 4096, against ~2.8e-5 observed.
+__host__ __device__ constexpr float router_refine_band(int H) {
+  return 2.0f * 0.25f * (3.0f * H / 16.0f) * 9.5367431640625e-07f;
+}
+
+struct TopkRefine {
+  const __nv_bfloat16* x;     // [T, H] bf16 input rows
+  const __nv_bfloat16* w_tc;  // [E_pad, 3H] three-term split router rows
+  int H;
+  float band;                 // 0: no refinement
 };
 
 // ---- launchers (each returns the cudaGetLastError of its launch) ----
 cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router_w, float* partial,
                                  int T, int H, int E, int ksplit, cudaStream_t st);
 cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, const float* bias,
-                        bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st);
+                        bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st,
+                        float* logits_out = nullptr, const TopkRefine* refine = nullptr);
 cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int m_tiles_gu,
                         int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
                         int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
@@ -60,6 +92,10 @@ cudaError_t launch_gemm_gate_up(const CUtensorMap& tmA, const CUtensorMap& tmB,
                                 cudaStream_t st);
 cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
                              int grid, cudaStream_t st);
+cudaError_t launch_gemm_router(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
+                               int grid, cudaStream_t st);
+cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
+                               cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k, int H, bool out_bf16,
                            void* out, cudaStream_t st);
 cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
@@ -69,6 +105,6 @@ cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int 
 
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t gemm_configure_device();
-size_t gemm_smem_bytes(bool gate_up);
+size_t gemm_smem_bytes(int mode);
 
 }  // namespace moe

@@ -42,7 +42,47 @@ __global__ void __launch_bounds__(256) pack_kernel(const TS* __restrict__ src, i
   }
 }
 
+// Router weight [H][E] fp32 -> [E_pad][3H] bf16: row e holds W1 | W2 | W3
+// along K, with W1 = bf16(w), W2 = bf16(w - W1), W3 = bf16(w - W1 - W2).
+// Each residual is exact in fp32 (it keeps at most 16, then 8, significant
+// bits), and W3 holds the last 8, so W1 + W2 + W3 == w for normal w.  Rows
+// e >= E are zero.
+__global__ void __launch_bounds__(256) pack_router_kernel(const float* __restrict__ w, int H, int E,
+                                                          int E_pad,
+                                                          __nv_bfloat16* __restrict__ dst) {
+  __shared__ float tile[32][33];
+  const int e0 = blockIdx.x * 32, h0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int h = h0 + i, e = e0 + threadIdx.x;
+    tile[i][threadIdx.x] = (h < H && e < E) ? w[static_cast<size_t>(h) * E + e] : 0.f;
+  }
+  __syncthreads();
+  const size_t ld = static_cast<size_t>(3) * H;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int e = e0 + i, h = h0 + threadIdx.x;
+    if (e < E_pad && h < H) {
+      const float v = tile[threadIdx.x][i];
+      const __nv_bfloat16 b1 = __float2bfloat16_rn(v);
+      const float r1 = v - __bfloat162float(b1);
+      const __nv_bfloat16 b2 = __float2bfloat16_rn(r1);
+      const float r2 = r1 - __bfloat162float(b2);
+      const __nv_bfloat16 b3 = __float2bfloat16_rn(r2);
+      __nv_bfloat16* row = dst + static_cast<size_t>(e) * ld;
+      row[h] = b1;
+      row[H + h] = b2;
+      row[2 * H + h] = b3;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
+                               cudaStream_t st) {
+  dim3 grid((E_pad + 31) / 32, (H + 31) / 32), block(32, 8);
+  pack_router_kernel<<<grid, block, 0, st>>>(w, H, E, E_pad, dst);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
                                 int half, __nv_bfloat16* dst, cudaStream_t st) {

@@ -47,27 +47,14 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int* __restrict__ 
   }
 }
 
-// One block.  Per expert: running offsets of the chunks; then warp 0 forms
-// the exclusive prefix over the G = E + 1 groups of the row counts and of the
-// GEMM tile counts (ceil(rows / kBN) token tiles x m_tiles weight tiles).
-__global__ void __launch_bounds__(1024) sort_scan_kernel(
-    const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int mt_gu, int mt_dn,
-    int* __restrict__ chunk_base, int* __restrict__ counts, int* __restrict__ row_start,
-    int* __restrict__ tiles_gu, int* __restrict__ tiles_dn) {
-  __shared__ int cnt_s[1025];
-  const int G = E + 1;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int c = 0; c < nch; ++c) {
-      chunk_base[static_cast<size_t>(c) * E + e] = run;
-      run += chunk_cnt[static_cast<size_t>(c) * E + e];
-    }
-    cnt_s[e] = run;
-  }
-  if (threadIdx.x == 0) cnt_s[E] = T;
-  __syncthreads();
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
+// Warp-wide exclusive prefix over the G = E + 1 groups of the row counts and
+// of the GEMM tile counts (ceil(rows / kBN) token tiles x m_tiles weight
+// tiles).  Called by one full warp; cnt_s holds the G row counts.  When
+// start_s is given, the row starts are also left there for the caller.
+__device__ void scan_groups(const int* cnt_s, int G, int mt_gu, int mt_dn, int* __restrict__ counts,
+                            int* __restrict__ row_start, int* __restrict__ tiles_gu,
+                            int* __restrict__ tiles_dn, int* start_s) {
+  const int lane = threadIdx.x & 31;
   const int per = (G + 31) / 32;
   const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
   int s_rows = 0, s_gu = 0, s_dn = 0;
@@ -96,6 +83,7 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(
     const int nt = (n + kBN - 1) / kBN;
     counts[g] = n;
     row_start[g] = b_rows;
+    if (start_s != nullptr) start_s[g] = b_rows;
     tiles_gu[g] = b_gu;
     tiles_dn[g] = b_dn;
     b_rows += n;
@@ -107,6 +95,78 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(
     tiles_gu[G] = i_gu;
     tiles_dn[G] = i_dn;
   }
+}
+
+// One block.  Per expert: running offsets of the chunks; then warp 0 forms
+// the prefixes over the groups.
+__global__ void __launch_bounds__(1024) sort_scan_kernel(
+    const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int mt_gu, int mt_dn,
+    int* __restrict__ chunk_base, int* __restrict__ counts, int* __restrict__ row_start,
+    int* __restrict__ tiles_gu, int* __restrict__ tiles_dn) {
+  __shared__ int cnt_s[1025];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < nch; ++c) {
+      chunk_base[static_cast<size_t>(c) * E + e] = run;
+      run += chunk_cnt[static_cast<size_t>(c) * E + e];
+    }
+    cnt_s[e] = run;
+  }
+  if (threadIdx.x == 0) cnt_s[E] = T;
+  __syncthreads();
+  if (threadIdx.x < 32)
+    scan_groups(cnt_s, E + 1, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, nullptr);
+}
+
+// Rank of token tl among the tokens of this chunk that chose the expert whose
+// 128-bit mask is m: the number of mask bits below tl.
+__device__ __forceinline__ int chunk_rank(const uint32_t* m, int tl) {
+  const int wd = tl >> 5;
+  int rank = __popc(m[wd] & ((1u << (tl & 31)) - 1u));
+  for (int q = 0; q < wd; ++q) rank += __popc(m[q]);
+  return rank;
+}
+
+// T <= kSortChunk (decode): histogram, prefixes and stable scatter in one block.
+__global__ void __launch_bounds__(1024) sort_small_kernel(
+    const int* __restrict__ topk_idx, const float* __restrict__ topk_w, int T, int k, int E,
+    int mt_gu, int mt_dn, int* __restrict__ counts, int* __restrict__ row_start,
+    int* __restrict__ tiles_gu, int* __restrict__ tiles_dn, int* __restrict__ perm,
+    int* __restrict__ pos, float* __restrict__ w_perm) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* masks = sm;                                   // [E][4]
+  int* cnt_s = reinterpret_cast<int*>(sm + E * kMaskWords);  // [E + 1]
+  int* start_s = cnt_s + (E + 1);                         // [E + 1]
+  for (int i = threadIdx.x; i < E * kMaskWords; i += blockDim.x) masks[i] = 0u;
+  __syncthreads();
+  for (int p = threadIdx.x; p < T * k; p += blockDim.x) {
+    const int tl = p / k;
+    const int e = topk_idx[p];
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+      atomicOr(&masks[e * kMaskWords + (tl >> 5)], 1u << (tl & 31));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int n = 0;
+#pragma unroll
+    for (int q = 0; q < kMaskWords; ++q) n += __popc(masks[e * kMaskWords + q]);
+    cnt_s[e] = n;
+  }
+  if (threadIdx.x == 0) cnt_s[E] = T;
+  __syncthreads();
+  if (threadIdx.x < 32)
+    scan_groups(cnt_s, E + 1, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, start_s);
+  __syncthreads();
+  for (int p = threadIdx.x; p < T * k; p += blockDim.x) {
+    const int tl = p / k;
+    const int e = topk_idx[p];
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) continue;
+    const int slot = start_s[e] + chunk_rank(masks + e * kMaskWords, tl);
+    perm[slot] = p;
+    pos[p] = slot;
+    w_perm[slot] = topk_w[p];
+  }
+  for (int t = threadIdx.x; t < T; t += blockDim.x) w_perm[T * k + t] = 1.0f;
 }
 
 __global__ void __launch_bounds__(256) sort_scatter_kernel(
@@ -126,11 +186,8 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(
     const size_t pair = static_cast<size_t>(t0) * k + p;
     const int e = topk_idx[pair];
     if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) continue;
-    const uint32_t* m = sm + e * kMaskWords;
-    const int wd = tl >> 5;
-    int rank = __popc(m[wd] & ((1u << (tl & 31)) - 1u));
-    for (int q = 0; q < wd; ++q) rank += __popc(m[q]);
-    const int slot = row_start[e] + chunk_base[static_cast<size_t>(c) * E + e] + rank;
+    const int slot = row_start[e] + chunk_base[static_cast<size_t>(c) * E + e] +
+                     chunk_rank(sm + e * kMaskWords, tl);
     perm[slot] = static_cast<int>(pair);
     pos[pair] = slot;
     w_perm[slot] = topk_w[pair];
@@ -189,6 +246,13 @@ cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, 
                         int* pos, float* w_perm, cudaStream_t st) {
   const int nch = (T + kSortChunk - 1) / kSortChunk;
   const size_t smem = static_cast<size_t>(E) * kMaskWords * sizeof(uint32_t);
+  if (nch == 1) {
+    const size_t smem1 = smem + 2 * static_cast<size_t>(E + 1) * sizeof(int);
+    sort_small_kernel<<<1, 1024, smem1, st>>>(topk_idx, topk_w, T, k, E, m_tiles_gu, m_tiles_dn,
+                                              counts, row_start, tiles_gu, tiles_dn, perm, pos,
+                                              w_perm);
+    return cudaGetLastError();
+  }
   sort_hist_kernel<<<nch, 256, smem, st>>>(topk_idx, T, k, E, masks, chunk_cnt);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;

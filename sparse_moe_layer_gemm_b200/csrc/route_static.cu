@@ -68,19 +68,12 @@ extern "C" int moe_route_static(const void* x, int act_dtype, const float* route
   float* scratch = nullptr;
   int r = scratch_for_current_device(&scratch);
   if (r != MOE_OK) return r;
-  int dev = 0, num_sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
-
-  // K splits: the rule moe_forward uses, reduced until the partials fit.
-  const int tiles = ((E + moe::kRouterExp - 1) / moe::kRouterExp) *
-                    ((T + moe::kRouterTok - 1) / moe::kRouterTok);
-  int splits = 1;
-  while (tiles * splits < 2 * num_sms && H / (2 * splits) >= 128 &&
-         H % (2 * splits * moe::kRouterKStep) == 0)
-    splits *= 2;
-  while (splits > 1 && static_cast<size_t>(splits) * T * E > kRouteScratchFloats) splits /= 2;
+  // K splits: the rule moe_forward uses (fixed 128-wide K chunks), halved
+  // until the partials fit the array; results equal moe_forward's whenever
+  // no halving was needed (T * E * H / 128 <= 1,048,576).
+  int splits = H / 128;
+  while (splits > 1 && static_cast<size_t>(splits) * T * E > kRouteScratchFloats)
+    splits = (splits % 2 == 0) ? splits / 2 : 1;
 
   // Every partial the top-k reads is written first, so nothing needs clearing.
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -106,39 +106,28 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const TX* __restrict
   }
 }
 
-// One warp per token.  Lane l holds experts l, l + 32, ...  (MPL per lane).
-// k rounds of a warp arg-max on (selection score, lower index first) pick the
-// experts in descending order; the owner lane hands over the bias-free score.
+// k rounds of a warp arg-max on (selection score, lower index first) over the
+// scores in shared memory: lane l holds experts l, l + 32, ... (MPL per lane);
+// the owner lane hands over the bias-free score of the winner.  Lane j < k
+// ends with the j-th pick; every lane gets the k-th selection score (kth) and
+// the best remaining one after k picks (next, -inf when k == E).
 template <int MPL>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ partial, int ksplit,
-                                                   int T, int E, int k,
-                                                   const float* __restrict__ bias, int norm,
-                                                   float scale, int* __restrict__ topk_idx,
-                                                   float* __restrict__ topk_w) {
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+__device__ __forceinline__ void warp_select(const float* s_sc, const float* s_be, int E, int k,
+                                            int& my_idx, float& my_s, float& kth, float& next) {
   const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-
   float sc[MPL], be[MPL];
 #pragma unroll
   for (int i = 0; i < MPL; ++i) {
     const int e = lane + 32 * i;
-    if (e < E) {
-      float l = 0.f;
-      for (int z = 0; z < ksplit; ++z) l += partial[(static_cast<size_t>(z) * T + t) * E + e];
-      const float s = 1.0f / (1.0f + expf(-l));
-      sc[i] = s;
-      be[i] = (bias != nullptr) ? s + bias[e] : s;
-    } else {
-      sc[i] = 0.f;
-      be[i] = -INFINITY;
-    }
+    sc[i] = (e < E) ? s_sc[e] : 0.f;
+    be[i] = (e < E) ? s_be[e] : -INFINITY;
   }
-
   uint32_t taken = 0;
-  int my_idx = 0;
-  float my_s = 0.f;
-  for (int j = 0; j < k; ++j) {
+  my_idx = 0;
+  my_s = 0.f;
+  kth = -INFINITY;
+  next = -INFINITY;
+  for (int j = 0; j <= k; ++j) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
 #pragma unroll
@@ -159,6 +148,11 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
         bi = oi;
       }
     }
+    if (j == k) {  // the best score left after the k picks
+      next = bv;
+      break;
+    }
+    kth = bv;
     if (bi >= E) bi = 0;  // only reachable with non-finite scores (unsupported input)
     float s_sel = 0.f;
     if ((bi & 31) == lane) {
@@ -176,6 +170,118 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ par
       my_s = s_sel;
     }
   }
+}
+
+// One block per token.  Thread e sums the ksplit partial logits of expert e
+// (independent loads, fixed order), forms the fp32 sigmoid score s and the
+// selection score s + b in shared memory; warp 0 selects.
+//
+// After the tensor-core router (band > 0) the logits are approximations: the
+// tensor cores' fp32 accumulation over the 3H products truncates at every
+// step (errors up to ~1e-4 at H = 4096).  They are used only to rule experts
+// out.  Every expert whose approximate selection score is within `band` of
+// the approximate k-th one -- the approximate top-k included -- is a
+// candidate; one warp per candidate recomputes its logit as an fp32 dot
+// product on the CUDA cores (its router row rebuilt exactly as W1 + W2 + W3
+// from the packed three-term split; lane-strided FMA chains, fixed shuffle
+// tree).  The selection, its order and the gate weights then come from these
+// fp32 logits; non-candidates are excluded, which is exact as long as the
+// tensor-core error in the selection score stays below band / 2.
+template <int MPL>
+__global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ partial, int ksplit,
+                                                    int T, int E, int k,
+                                                    const float* __restrict__ bias, int norm,
+                                                    float scale, int* __restrict__ topk_idx,
+                                                    float* __restrict__ topk_w,
+                                                    float* __restrict__ logits_out,
+                                                    TopkRefine rf) {
+  __shared__ float s_l[32 * MPL];
+  __shared__ float s_sc[32 * MPL];
+  __shared__ float s_be[32 * MPL];
+  __shared__ int s_cand[32 * MPL];
+  __shared__ int s_ncand;
+  __shared__ float s_kth;
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const float* src = partial + static_cast<size_t>(t) * E + e;
+    const size_t zstride = static_cast<size_t>(T) * E;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int z = 0;
+    for (; z + 4 <= ksplit; z += 4) {
+      a0 += src[(z + 0) * zstride];
+      a1 += src[(z + 1) * zstride];
+      a2 += src[(z + 2) * zstride];
+      a3 += src[(z + 3) * zstride];
+    }
+    for (; z < ksplit; ++z) a0 += src[z * zstride];
+    const float l = (a0 + a1) + (a2 + a3);
+    const float s = 1.0f / (1.0f + expf(-l));
+    s_l[e] = l;
+    s_sc[e] = s;
+    s_be[e] = (bias != nullptr) ? s + bias[e] : s;
+  }
+  __syncthreads();
+  int my_idx = 0;
+  float my_s = 0.f, kth, next;
+  if (rf.band > 0.f) {
+    if (warp == 0) {
+      warp_select<MPL>(s_sc, s_be, E, k, my_idx, my_s, kth, next);
+      if (lane == 0) {
+        s_kth = kth;
+        s_ncand = 0;
+      }
+    }
+    __syncthreads();
+    const float floor_ = s_kth - rf.band;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      if (s_be[e] >= floor_)
+        s_cand[atomicAdd(&s_ncand, 1)] = e;
+      else
+        s_be[e] = -INFINITY;  // ruled out
+    }
+    __syncthreads();
+    const int n = s_ncand;
+    const int H = rf.H;
+    const __nv_bfloat16* xt = rf.x + static_cast<size_t>(t) * H;
+    for (int c = warp; c < n; c += nwarps) {
+      const int e = s_cand[c];
+      const __nv_bfloat16* w = rf.w_tc + static_cast<size_t>(e) * 3 * H;
+      float acc = 0.f;
+      for (int h0 = lane * 8; h0 < H; h0 += 256) {
+        const uint4 xq = *reinterpret_cast<const uint4*>(xt + h0);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(w + h0);
+        const uint4 q2 = *reinterpret_cast<const uint4*>(w + H + h0);
+        const uint4 q3 = *reinterpret_cast<const uint4*>(w + 2 * H + h0);
+        const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&xq);
+        const __nv_bfloat16* w1 = reinterpret_cast<const __nv_bfloat16*>(&q1);
+        const __nv_bfloat16* w2 = reinterpret_cast<const __nv_bfloat16*>(&q2);
+        const __nv_bfloat16* w3 = reinterpret_cast<const __nv_bfloat16*>(&q3);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float wv =
+              (__bfloat162float(w1[i]) + __bfloat162float(w2[i])) + __bfloat162float(w3[i]);
+          acc = fmaf(__bfloat162float(xv[i]), wv, acc);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (lane == 0) {
+        const float s = 1.0f / (1.0f + expf(-acc));
+        s_l[e] = acc;
+        s_sc[e] = s;
+        s_be[e] = (bias != nullptr) ? s + bias[e] : s;
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 0) warp_select<MPL>(s_sc, s_be, E, k, my_idx, my_s, kth, next);
+  if (logits_out != nullptr) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      logits_out[static_cast<size_t>(t) * E + e] = s_l[e];
+  }
+  if (warp != 0) return;
   float sum = 0.f;
   for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, my_s, j);
   if (lane < k) {
@@ -200,12 +306,15 @@ cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router
 }
 
 cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, const float* bias,
-                        bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st) {
-  const int blocks = (T + 7) / 8;
+                        bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st,
+                        float* logits_out, const TopkRefine* refine) {
   const int mpl = (E + 31) / 32;
-#define MOE_TOPK(N)                                                                          \
-  topk_kernel<N><<<blocks, 256, 0, st>>>(partial, ksplit, T, E, k, bias, norm ? 1 : 0, scale, \
-                                         topk_idx, topk_w)
+  const int threads = min(1024, max(32, (E + 31) / 32 * 32));
+  TopkRefine rf{};
+  if (refine != nullptr) rf = *refine;
+#define MOE_TOPK(N)                                                                       \
+  topk_kernel<N><<<T, threads, 0, st>>>(partial, ksplit, T, E, k, bias, norm ? 1 : 0, scale, \
+                                        topk_idx, topk_w, logits_out, rf)
   if (mpl <= 1) MOE_TOPK(1);
   else if (mpl <= 2) MOE_TOPK(2);
   else if (mpl <= 4) MOE_TOPK(4);

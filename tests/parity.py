@@ -8,6 +8,10 @@ Bar (element by element):
   oracle evaluated on the GPU's selection;
 * counts, offsets and the permutation bit-exact given the selection;
 * gate weights within fp32 rounding (rtol 1e-5);
+* router logits of the selected experts within LOGIT_TOL of the fp64 logits
+  (fp32 accuracy); every logit within LOGIT_TOL_APPROX (after the tensor-core
+  router, experts that cannot be selected keep its approximate logit, whose
+  error must stay well inside the top-k guard band);
 * outputs: relative Frobenius error <= 1e-2 and max |error| <= 5e-2 * RMS(out).
 """
 from __future__ import annotations
@@ -23,6 +27,8 @@ TIE_BAND = 1e-6
 REL_FRO = 1e-2
 MAX_ABS_OVER_RMS = 5e-2
 W_RTOL = 1e-5
+LOGIT_TOL = 1e-5
+LOGIT_TOL_APPROX = 4e-4
 
 
 @dataclass
@@ -33,6 +39,7 @@ class ParityReport:
     rel_fro: float
     max_abs_over_rms: float
     rows_checked: int
+    logit_max_err: float = 0.0
 
     def ok(self) -> bool:
         return self.rel_fro <= REL_FRO and self.max_abs_over_rms <= MAX_ABS_OVER_RMS
@@ -77,6 +84,13 @@ def compare(inp_host: dict, wl, gpu_out: np.ndarray, gpu_rt: dict,
     ref = om.moe_routing(x, inp_host["router_w"], inp_host["router_bias"], top_k=k,
                          scale=wl.scale)
     mism, tie = check_routing(gpu_rt, ref, k, E)
+    logit_err = 0.0
+    if "logits" in gpu_rt:
+        d = np.abs(gpu_rt["logits"].astype(np.float64) - ref["logits"])
+        sel = np.take_along_axis(d, gpu_rt["topk_idx"].astype(np.int64), axis=1)
+        logit_err = float(sel.max())
+        assert logit_err <= LOGIT_TOL, f"selected router logits off by {logit_err}"
+        assert float(d.max()) <= LOGIT_TOL_APPROX, f"router logits off by {float(d.max())}"
     T = x.shape[0]
     if rows is None:
         rows = np.arange(T)
@@ -90,4 +104,5 @@ def compare(inp_host: dict, wl, gpu_out: np.ndarray, gpu_rt: dict,
                               forced_idx=gpu_rt["topk_idx"][rows])
     rel, mx = output_errors(gpu_out[rows], res.out)
     return ParityReport(tokens=T, near_ties=int(tie.sum()), idx_mismatch_rows=int(mism.sum()),
-                        rel_fro=rel, max_abs_over_rms=mx, rows_checked=int(rows.size))
+                        rel_fro=rel, max_abs_over_rms=mx, rows_checked=int(rows.size),
+                        logit_max_err=logit_err)
