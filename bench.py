@@ -44,6 +44,8 @@ def _args():
     ap.add_argument("--secondary", default="prefill")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling case: override the token count T")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling case: override the number of routed experts "
                          "(smaller device footprint for ncu captures)")
@@ -290,9 +292,10 @@ def run_ours(a):
     torch.cuda.set_device(dev)
     B.load_library()
     wl = WORKLOADS[a.workload]
-    if a.experts:
+    if a.experts or a.tokens:
         from dataclasses import replace as _replace
-        wl = _replace(wl, num_experts=a.experts, name=f"{wl.name}_e{a.experts}")
+        wl = _replace(wl, num_experts=a.experts or wl.num_experts, T=a.tokens or wl.T,
+                      name=f"{wl.name}_e{a.experts or wl.num_experts}_t{a.tokens or wl.T}")
     peaks = _peaks()
 
     inp = make_inputs(wl, dev)                          # weights replicated on every rank

@@ -75,11 +75,13 @@ _lib: Optional[ctypes.CDLL] = None
 
 
 def load_library(path: Optional[str] = None) -> ctypes.CDLL:
-    """Loads libmoe.so (built in-tree by ``sparse_moe_layer_gemm_b200.build``)."""
+    """Loads libmoe.so: `path`, else $SPARSE_MOE_LIBRARY, else the in-tree
+    build of ``sparse_moe_layer_gemm_b200.build``."""
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = path or LIB_PATH
+    env = os.environ.get("SPARSE_MOE_LIBRARY")
+    p = path or env or LIB_PATH
     if not os.path.exists(p):
         raise RuntimeError(f"libmoe.so not found at {p}: run `python -m sparse_moe_layer_gemm_b200.build`")
     lib = ctypes.CDLL(p)

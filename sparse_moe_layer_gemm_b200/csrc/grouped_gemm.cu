@@ -6,11 +6,11 @@
 //                  h = silu(gate) * up, stored bf16.
 //   K6 (down):     y = (h_g . Wd_g) * w_row, the row's gate weight (1 for the
 //                  shared rows), stored bf16.
-//   K1 (router, large T):  logits = x . W_r in fp32 accuracy on the bf16 tensor
-//                  cores: W_r = W1 + W2 + W3 split into three bf16 terms that
-//                  are concatenated along K, so one accumulation over 3H gives
-//                  x.W1 + x.W2 + x.W3 (each bf16 x bf16 product is exact in
-//                  fp32; x is bf16 and needs no split); stored fp32.
+//   K1 (router, large T):  logits = x . W_r on the bf16 tensor cores: W_r =
+//                  W1 + W2 + W3 split into three bf16 terms concatenated along
+//                  K, so one accumulation over 3H gives x.W1 + x.W2 + x.W3
+//                  (each bf16 x bf16 product is exact in fp32; x is bf16);
+//                  stored fp32.
 //
 // The expert FFN is the SwiGLU of sglang-jax issue #1367 "Support Step 3.5
 // Flash", section "Model configuration" (MoE bullet; clamped SwiGLU via
@@ -21,19 +21,24 @@
 // Design (swap-AB): the MMA's M side (128) is always a block of weight rows,
 // the N side the group's tokens (rounded up to 16, at most 128 per tile), so
 // ragged groups of 1..21 tokens (decode) waste no more than 15 columns.
-// A tile is (group, weight block mt, token block nc); tiles of one group are
-// ordered token-block-major so all weight blocks of the same token block run
+// A tile is (group, weight tile mt, token block nc); tiles of one group are
+// ordered token-block-major so all weight tiles of the same token block run
 // together and an expert's weights stay in L2 across its token blocks.
 //
-// One persistent CTA per SM, 6 warps:
-//   warp 0     TMA producer: A = 128 (down) or 2x128 (gate, up) weight rows
-//              x 64 K, B = token rows in 32-row boxes, 128-byte swizzle,
-//              multi-stage mbarrier ring.
-//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
-//              (kind::f16, bf16 x bf16 -> fp32 in TMEM), two accumulator
-//              buffers so the epilogue of tile i overlaps the mainloop of i+1.
-//   warps 2-5  epilogue: tcgen05.ld (32 lanes x 16 columns), SwiGLU / gate
-//              weight in registers, bf16 stores.
+// One persistent CTA per SM, 4 + NI warps:
+//   warp 0        TMA producer: per stage one box of the tile's weight rows
+//                 (BLOCKS 128-feature blocks; gate|up blocks are 128 gate rows
+//                 then 128 up rows) x 64 K and one box of token rows (32 rows
+//                 for tiles of <= 32 tokens, else 128), 128-byte swizzle.
+//   warps 1..NI   tcgen05.mma issuers (kind::f16, bf16 x bf16 -> fp32 TMEM):
+//                 each owns every NI-th 128-row accumulator of the tile (gate
+//                 and up, or two weight blocks) and keeps its own stage waits
+//                 and commits, so the issue latencies of the accumulator
+//                 chains overlap; warp 1 also allocates TMEM.  Two
+//                 accumulator buffers let the epilogue of tile i overlap the
+//                 mainloop of tile i+1.
+//   last 4 warps  epilogue: tcgen05.ld (32 lanes x 16 columns), SwiGLU or
+//                 gate weight in registers, bf16 (router: fp32) stores.
 // No TMA multicast anywhere.
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
@@ -42,38 +47,56 @@ namespace moe {
 
 namespace {
 
-template <int MODE>
+// Tile shape: BLOCKS weight blocks of 128 features per tile (gate|up: each
+// block is 128 gate rows + 128 up rows), BN tokens per tile, BK = 64 reduction
+// elements (one 128-byte swizzled row) per pipeline stage.
+template <int MODE, int BLOCKS, int BN_>
 struct Shape {
   static constexpr bool GU = MODE == kModeGateUp;
-  static constexpr int A_ROWS = GU ? 2 * kBM : kBM;
-  static constexpr int A_BYTES = A_ROWS * kBK * 2;
-  static constexpr int B_BYTES = kBN * kBK * 2;
-  static constexpr int B_BOX_BYTES = kBBoxRows * kBK * 2;
+  static constexpr int BN = BN_;
+  static constexpr int BK = kBK;
+  static constexpr int ROW = BK * 2;                        // bytes per operand row in SMEM
+  static constexpr int ACCS = BLOCKS * (GU ? 2 : 1);       // 128-row accumulators per tile
+  static constexpr int NI = ACCS >= 2 ? 2 : 1;             // MMA-issuing warps
+  static constexpr int THREADS = 32 * (1 + NI + 4);
+  static constexpr int A_ROWS = kBM * ACCS;
+  static constexpr int A_BOX = GU ? 2 * kBM : kBM;         // rows per A box (the tensor maps')
+  static constexpr int A_LOADS = A_ROWS / A_BOX;
+  static constexpr int A_BYTES = A_ROWS * ROW;
+  static constexpr int B_BYTES = BN * ROW;
+  static constexpr int B_BOX_BYTES = kBBoxRows * ROW;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = GU ? 4 : 6;
-  static constexpr int ACC_COLS = GU ? 2 * kBN : kBN;  // TMEM columns per accumulator buffer
-  static constexpr int TMEM_COLS = 2 * ACC_COLS;       // two buffers
+  static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < 6 ? (200 * 1024 / STAGE_BYTES) : 6;
+  static constexpr int ACC_COLS = ACCS * BN;                // TMEM columns per accumulator buffer
+  static constexpr int NBUF = ACC_COLS <= 256 ? 2 : 1;     // double-buffered when it fits
+  static constexpr int TMEM_COLS = NBUF * ACC_COLS > 256 ? 512 : 256;
   static constexpr int BAR_BYTES = 256;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + BAR_BYTES;
   static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
-  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation");
+  static_assert(NBUF * ACC_COLS <= 512, "TMEM capacity");
+  static_assert(BN == 128, "token tile (the wide token-row box is BN rows)");
+  static_assert(A_ROWS % A_BOX == 0 && ACCS % NI == 0, "A boxes, issuer split");
+  static_assert(STAGES >= 2, "pipeline depth");
   static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay aligned");
+  // descriptor start-address field: 14 bits of (address >> 4), no carries
+  static_assert(1024 + STAGES * STAGE_BYTES + BAR_BYTES <= 256 * 1024, "descriptor range");
 };
 
 struct Tile {
   int g, mt, nc, n_valid;
 };
 
-// Tile w -> (group, weight block, token block); tile_start is the exclusive
+// Tile w -> (group, weight tile, token block); tile_start is the exclusive
 // prefix of per-group tile counts, so the group is the last g with
 // tile_start[g] <= w (empty groups are skipped naturally).
+template <int BN>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
   if (p.single_rows > 0) {
     Tile t;
     t.g = 0;
     t.nc = w / p.m_tiles;
     t.mt = w - t.nc * p.m_tiles;
-    t.n_valid = min(kBN, p.single_rows - t.nc * kBN);
+    t.n_valid = min(BN, p.single_rows - t.nc * BN);
     return t;
   }
   int lo = 0, hi = p.G;
@@ -89,12 +112,13 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
   const int local = w - p.tile_start[lo];
   t.nc = local / p.m_tiles;
   t.mt = local - t.nc * p.m_tiles;
-  t.n_valid = min(kBN, p.counts[lo] - t.nc * kBN);
+  t.n_valid = min(BN, p.counts[lo] - t.nc * BN);
   return t;
 }
 
+template <int BN>
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
-  if (p.single_rows > 0) return p.m_tiles * ((p.single_rows + kBN - 1) / kBN);
+  if (p.single_rows > 0) return p.m_tiles * ((p.single_rows + BN - 1) / BN);
   return p.tile_start[p.G];
 }
 
@@ -102,13 +126,32 @@ __device__ __forceinline__ int group_row0(const GemmParams& p, int g) {
   return p.single_rows > 0 ? 0 : p.row_start[g];
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(192, 1)
+// tcgen05.mma issue without a memory clobber: the MMA reads shared memory
+// the TMA wrote (ordered by the full-barrier wait and the tcgen05 fence) and
+// writes TMEM; its completion is ordered by the (volatile, clobbering)
+// commit that follows it.
+__device__ __forceinline__ void mma_issue(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+// tmB / tmBsh: token-row operands with kBBoxRows-row boxes; tmBw / tmBshw
+// the same tensors with BN-row boxes, used when a tile has more than
+// kBBoxRows tokens (one TMA instruction per stage instead of several).
+template <int MODE, int BLOCKS, int BN>
+__global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmBsh, const GemmParams p) {
-  using S = Shape<MODE>;
+                        const __grid_constant__ CUtensorMap tmBsh,
+                        const __grid_constant__ CUtensorMap tmBw,
+                        const __grid_constant__ CUtensorMap tmBshw, const GemmParams p) {
+  using S = Shape<MODE, BLOCKS, BN>;
   constexpr bool GU = S::GU;
+  constexpr int BK = S::BK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -127,20 +170,24 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, S::NI);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tfull0 + 8 * b, S::NI);
       mbar_init(tempty0 + 8 * b, 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, S::NI);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (GU) prefetch_tmap(&tmBsh);
+    prefetch_tmap(&tmBw);
+    if (GU) {
+      prefetch_tmap(&tmBsh);
+      prefetch_tmap(&tmBshw);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), S::TMEM_COLS);
@@ -150,24 +197,24 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = total_tiles(p);
+  const int total = total_tiles<BN>(p);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_a = l2_policy_evict_first();  // weights: streamed once
-      const uint64_t pol_b = l2_policy_evict_last();   // token rows: reused by every weight block
+      const uint64_t pol_b = l2_policy_evict_last();   // token rows: reused by every weight tile
       uint32_t it = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
         if (*abort_flag) break;
-        const Tile t = decode_tile(p, w);
+        const Tile t = decode_tile<BN>(p, w);
         const int n_mma = (t.n_valid + 15) & ~15;
-        const int nbox = (n_mma + kBBoxRows - 1) / kBBoxRows;
+        const bool wide = n_mma > kBBoxRows;  // one BN-row box, else one kBBoxRows-row box
         const bool sh = GU && t.g == p.E;
-        const CUtensorMap* mb = sh ? &tmBsh : &tmB;
-        const int b_row = (sh ? p.shared_b_row0 : group_row0(p, t.g)) + t.nc * kBN;
+        const CUtensorMap* mb = wide ? (sh ? &tmBshw : &tmBw) : (sh ? &tmBsh : &tmB);
+        const int b_row = (sh ? p.shared_b_row0 : group_row0(p, t.g)) + t.nc * BN;
         const int a_row = t.g * p.a_rows_per_group + t.mt * S::A_ROWS;
-        const uint32_t bytes = S::A_BYTES + nbox * S::B_BOX_BYTES;
+        const uint32_t bytes = S::A_BYTES + (wide ? S::B_BYTES : S::B_BOX_BYTES);
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           const uint32_t s = it % S::STAGES;
@@ -179,11 +226,11 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t fb = full0 + 8 * s;
           mbar_arrive_expect_tx(fb, bytes);
           const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
-          const uint32_t sb = sa + S::A_BYTES;
-          tma_load_2d(sa, &tmA, fb, kb * kBK, a_row, pol_a);
-          const int bk = p.b_k_wrap > 0 ? (kb * kBK) % p.b_k_wrap : kb * kBK;
-          for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sb + i * S::B_BOX_BYTES, mb, fb, bk, b_row + i * kBBoxRows, pol_b);
+#pragma unroll
+          for (int i = 0; i < S::A_LOADS; ++i)
+            tma_load_2d(sa + i * S::A_BOX * S::ROW, &tmA, fb, kb * BK, a_row + i * S::A_BOX, pol_a);
+          const int bk = p.b_k_wrap > 0 ? (kb * BK) % p.b_k_wrap : kb * BK;
+          tma_load_2d(sa + S::A_BYTES, mb, fb, bk, b_row, pol_b);
           ++it;
         }
         if (!ok) break;
@@ -195,17 +242,19 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait(full0 + 8 * s, (last / S::STAGES) & 1u, nullptr, p.status);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp <= S::NI) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
+      const int me = warp - 1;  // this warp issues accumulators me, me + NI, ...
+      const uint64_t desc0 = sdesc_k_sw<S::ROW>(smem_u32(smem));
       uint32_t it = 0, tc = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
         if (*abort_flag) break;
-        const Tile t = decode_tile(p, w);
+        const Tile t = decode_tile<BN>(p, w);
         const int n_mma = (t.n_valid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
-        const uint32_t buf = tc & 1u;
-        const uint32_t tph = (tc >> 1) & 1u;
+        const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
+        const uint32_t tph = (S::NBUF == 2 ? (tc >> 1) : tc) & 1u;
         if (!mbar_wait(tempty0 + 8 * buf, tph ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + buf * S::ACC_COLS;
@@ -218,20 +267,23 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
-          const uint32_t sb = sa + S::A_BYTES;
+          // stage descriptors: the start field advances by (byte offset >> 4)
+          const uint64_t ad = desc0 + static_cast<uint64_t>((s * S::STAGE_BYTES) >> 4);
+          const uint64_t bd = ad + static_cast<uint64_t>(S::A_BYTES >> 4);
+          const uint32_t acc0 = kb != 0 ? 1u : 0u;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t bdesc = sdesc_k_sw128(sb + kk * 32);
-            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            tc_mma_bf16(d, sdesc_k_sw128(sa + kk * 32), bdesc, idesc, acc);
-            if (GU) tc_mma_bf16(d + kBN, sdesc_k_sw128(sa + kBM * 128 + kk * 32), bdesc, idesc, acc);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+#pragma unroll
+            for (int j = 0; j < S::ACCS / S::NI; ++j) {
+              const int a = j * S::NI + me;
+              mma_issue(d + a * BN, ad + static_cast<uint64_t>((a * kBM * S::ROW + kk * 32) >> 4),
+                        bd + static_cast<uint64_t>((kk * 32) >> 4), idesc, kk == 0 ? acc0 : 1u);
+            }
           tc_commit(empty0 + 8 * s);  // frees the stage once these MMAs have read it
           ++it;
         }
         if (!ok) break;
-        tc_commit(tfull0 + 8 * buf);  // accumulator ready for the epilogue
+        tc_commit(tfull0 + 8 * buf);  // this warp's accumulators are ready
         ++tc;
       }
       if (it > 0) {  // no MMA may still be writing TMEM at deallocation
@@ -244,9 +296,9 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;  // the TMEM lane quadrant this warp may read
     uint32_t tc = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      const Tile t = decode_tile(p, w);
-      const uint32_t buf = tc & 1u;
-      const uint32_t tph = (tc >> 1) & 1u;
+      const Tile t = decode_tile<BN>(p, w);
+      const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
+      const uint32_t tph = (S::NBUF == 2 ? (tc >> 1) : tc) & 1u;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(tfull0 + 8 * buf, tph, abort_flag, p.status) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -254,54 +306,59 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * S::ACC_COLS;
-      const int feat = t.mt * kBM + q * 32 + lane;
-      const size_t row0 = static_cast<size_t>(group_row0(p, t.g)) + static_cast<size_t>(t.nc) * kBN;
-      if (MODE == kModeRouter) {
-        float* lp = p.out_f32 + row0 * p.out_ld + feat;
-        const bool keep = feat < p.valid_feats;
-        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
-          uint32_t ra[16];
-          tmem_ld_x16(taddr + c0, ra);
-          tmem_ld_wait();
+      const size_t row0 = static_cast<size_t>(group_row0(p, t.g)) + static_cast<size_t>(t.nc) * BN;
+#pragma unroll 1
+      for (int b = 0; b < BLOCKS; ++b) {
+        const int feat = (t.mt * BLOCKS + b) * kBM + q * 32 + lane;
+        if ((t.mt * BLOCKS + b) * kBM >= p.out_feats) break;  // never past the output
+        if (MODE == kModeRouter) {
+          float* lp = p.out_f32 + row0 * p.out_ld + feat;
+          const bool keep = feat < p.valid_feats;
+          for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t ra[16];
+            tmem_ld_x16(taddr + b * BN + c0, ra);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (keep && c0 + i < t.n_valid)
-              lp[static_cast<size_t>(c0 + i) * p.out_ld] = __uint_as_float(ra[i]);
-        }
-      } else if (GU) {
-        __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
-        const float L = (t.g == p.E) ? p.limit_shared : p.limit;
-        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
-          uint32_t ra[16], rb[16];
-          tmem_ld_x16(taddr + c0, ra);
-          tmem_ld_x16(taddr + kBN + c0, rb);
-          tmem_ld_wait();
+            for (int i = 0; i < 16; ++i)
+              if (keep && c0 + i < t.n_valid)
+                lp[static_cast<size_t>(c0 + i) * p.out_ld] = __uint_as_float(ra[i]);
+          }
+        } else if (GU) {
+          __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
+          const float L = (t.g == p.E) ? p.limit_shared : p.limit;
+          const uint32_t tg = taddr + (2 * b) * BN, tu = taddr + (2 * b + 1) * BN;
+          for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t ra[16], rb[16];
+            tmem_ld_x16(tg + c0, ra);
+            tmem_ld_x16(tu + c0, rb);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (c0 + i < t.n_valid) {
-              float a = __uint_as_float(ra[i]);
-              float u = __uint_as_float(rb[i]);
-              if (L > 0.f) {
-                a = fminf(a, L);
-                u = fminf(fmaxf(u, -L), L);
+            for (int i = 0; i < 16; ++i) {
+              if (c0 + i < t.n_valid) {
+                float a = __uint_as_float(ra[i]);
+                float u = __uint_as_float(rb[i]);
+                if (L > 0.f) {
+                  a = fminf(a, L);
+                  u = fminf(fmaxf(u, -L), L);
+                }
+                const float hv = a / (1.0f + __expf(-a)) * u;
+                outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(hv);
               }
-              const float hv = a / (1.0f + __expf(-a)) * u;
-              outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(hv);
             }
           }
-        }
-      } else {
-        __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
-        const float* wrow = p.w_perm + row0;
-        for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
-          uint32_t ra[16];
-          tmem_ld_x16(taddr + c0, ra);
-          tmem_ld_wait();
+        } else {
+          __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
+          const float* wrow = p.w_perm + row0;
+          for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t ra[16];
+            tmem_ld_x16(taddr + b * BN + c0, ra);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (c0 + i < t.n_valid) {
-              const float yv = __uint_as_float(ra[i]) * wrow[c0 + i];
-              outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(yv);
+            for (int i = 0; i < 16; ++i) {
+              if (c0 + i < t.n_valid) {
+                const float yv = __uint_as_float(ra[i]) * wrow[c0 + i];
+                outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(yv);
+              }
             }
           }
         }
@@ -322,43 +379,54 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// The launch configurations.  gate|up: one 128-feature block per tile (the
+// gate and up accumulators, one issuer warp each).  down: two 128-feature
+// blocks per tile when H allows (one issuer warp each; double-buffered
+// TMEM), else one.  router: one block.
+using GuCfg = Shape<kModeGateUp, 1, 128>;
+using DnCfg2 = Shape<kModeDown, 2, 128>;
+using DnCfg1 = Shape<kModeDown, 1, 128>;
+using RtCfg = Shape<kModeRouter, 1, 128>;
+
+template <typename S, int MODE, int BLOCKS>
+cudaError_t set_smem() {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BLOCKS, S::BN>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(S::SMEM));
+}
+
 }  // namespace
 
-size_t gemm_smem_bytes(int mode) {
-  return mode == kModeGateUp ? Shape<kModeGateUp>::SMEM
-                             : (mode == kModeDown ? Shape<kModeDown>::SMEM : Shape<kModeRouter>::SMEM);
-}
-
 cudaError_t gemm_configure_device() {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeGateUp>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Shape<kModeGateUp>::SMEM));
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(grouped_gemm_kernel<kModeDown>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(Shape<kModeDown>::SMEM));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kModeRouter>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(Shape<kModeRouter>::SMEM));
+  cudaError_t e;
+  if ((e = set_smem<GuCfg, kModeGateUp, 1>()) != cudaSuccess) return e;
+  if ((e = set_smem<DnCfg2, kModeDown, 2>()) != cudaSuccess) return e;
+  if ((e = set_smem<DnCfg1, kModeDown, 1>()) != cudaSuccess) return e;
+  return set_smem<RtCfg, kModeRouter, 1>();
 }
 
-cudaError_t launch_gemm_gate_up(const CUtensorMap& tmA, const CUtensorMap& tmB,
-                                const CUtensorMap& tmBsh, const GemmParams& p, int grid,
-                                cudaStream_t st) {
-  grouped_gemm_kernel<kModeGateUp><<<grid, 192, Shape<kModeGateUp>::SMEM, st>>>(tmA, tmB, tmBsh, p);
+int gemm_down_blocks(int H) { return (H / kBM) % 2 == 0 ? 2 : 1; }
+
+cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
+  grouped_gemm_kernel<kModeGateUp, 1, 128>
+      <<<grid, GuCfg::THREADS, GuCfg::SMEM, st>>>(m.a, m.b, m.bsh, m.bw, m.bshw, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
-                             int grid, cudaStream_t st) {
-  grouped_gemm_kernel<kModeDown><<<grid, 192, Shape<kModeDown>::SMEM, st>>>(tmA, tmB, tmB, p);
+cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
+                             cudaStream_t st) {
+  if (blocks == 2)
+    grouped_gemm_kernel<kModeDown, 2, 128>
+        <<<grid, DnCfg2::THREADS, DnCfg2::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, p);
+  else
+    grouped_gemm_kernel<kModeDown, 1, 128>
+        <<<grid, DnCfg1::THREADS, DnCfg1::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_router(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
-                               int grid, cudaStream_t st) {
-  grouped_gemm_kernel<kModeRouter><<<grid, 192, Shape<kModeRouter>::SMEM, st>>>(tmA, tmB, tmB, p);
+cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
+  grouped_gemm_kernel<kModeRouter, 1, 128>
+      <<<grid, RtCfg::THREADS, RtCfg::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, p);
   return cudaGetLastError();
 }
 

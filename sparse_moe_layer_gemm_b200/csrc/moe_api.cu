@@ -110,8 +110,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// bf16 [rows, cols] row-major, box = 64 columns (128 bytes) x box_rows, 128B swizzle,
-// out-of-range elements read as zero.
+// bf16 [rows, cols] row-major, box = 64 columns (128 bytes) x box_rows, 128B
+// swizzle; out-of-range elements read as zero.
 bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
@@ -310,15 +310,33 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + w.h);
   __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(ws + w.y);
 
-  CUtensorMap tm_b, tm_bsh, tm_h;
-  if (!encode_bf16_2d(&tm_b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
-      !encode_bf16_2d(&tm_h, hbuf, w.rows_all, Ip, moe::kBBoxRows))
+  // expert-GEMM weight tiles: gate|up one 128-feature block, down one or two
+  const int dn_blocks = moe::gemm_down_blocks(H);
+  const int mt_gu = Ip / moe::kBM, mt_dn = H / moe::kBM / dn_blocks;
+
+  // Token-row operands, each with kBBoxRows- and kBN-row boxes: x_perm (or x
+  // for the shared expert) for K5 and the router, h for K6.
+  moe::GemmMaps gu{}, dn{}, rt{};
+  gu.a = L->tm_gu;
+  dn.a = L->tm_dn;
+  rt.a = L->tm_router;
+  if (!encode_bf16_2d(&gu.b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
+      !encode_bf16_2d(&gu.bw, x_perm, w.rows_xperm, H, moe::kBN) ||
+      !encode_bf16_2d(&dn.b, hbuf, w.rows_all, Ip, moe::kBBoxRows) ||
+      !encode_bf16_2d(&dn.bw, hbuf, w.rows_all, Ip, moe::kBN))
     return MOE_ERR_CUDA;
   if (xb) {
-    if (!encode_bf16_2d(&tm_bsh, x, T, H, moe::kBBoxRows)) return MOE_ERR_CUDA;
+    if (!encode_bf16_2d(&gu.bsh, x, T, H, moe::kBBoxRows) ||
+        !encode_bf16_2d(&gu.bshw, x, T, H, moe::kBN))
+      return MOE_ERR_CUDA;
+    rt.b = gu.bsh;
+    rt.bw = gu.bshw;
   } else {
-    tm_bsh = tm_b;
+    gu.bsh = gu.b;
+    gu.bshw = gu.bw;
   }
+  dn.bsh = dn.b;
+  dn.bshw = dn.bw;
 
   cudaEvent_t* ev = nullptr;
   if (L->timing_capacity > 0 && L->timing_recorded < L->timing_capacity)
@@ -340,10 +358,10 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
     r.out_f32 = partial;
     r.out_ld = E;
     r.valid_feats = E;
+    r.out_feats = E;
     r.status = L->status;
     const int tiles = r.m_tiles * ((T + moe::kBN - 1) / moe::kBN);
-    MOE_CUDA(moe::launch_gemm_router(L->tm_router, tm_bsh, r, tiles < L->num_sms ? tiles : L->num_sms,
-                                     st));
+    MOE_CUDA(moe::launch_gemm_router(rt, r, tiles < L->num_sms ? tiles : L->num_sms, st));
     ksplit = 1;
     refine.x = static_cast<const __nv_bfloat16*>(x);
     refine.w_tc = L->router_tc;
@@ -358,7 +376,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
                             st, routing != nullptr ? routing->logits : nullptr,
                             tc_router ? &refine : nullptr));
   MOE_CUDA(mark(2));
-  MOE_CUDA(moe::launch_sort(topk_idx, topk_w, T, k, E, Ip / moe::kBM, H / moe::kBM, masks,
+  MOE_CUDA(moe::launch_sort(topk_idx, topk_w, T, k, E, moe::kBN, mt_gu, mt_dn, masks,
                             chunk_cnt, chunk_base, counts, row_start, tiles_gu, tiles_dn, perm, pos,
                             w_perm, st));
   MOE_CUDA(mark(3));
@@ -376,24 +394,26 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
 
   p.tile_start = tiles_gu;
   p.num_kb = H / moe::kBK;
-  p.m_tiles = Ip / moe::kBM;
+  p.m_tiles = mt_gu;
   p.a_rows_per_group = 2 * Ip;
   p.shared_b_row0 = xb ? 0 : T * k;
   p.out = hbuf;
   p.out_ld = Ip;
+  p.out_feats = Ip;
   p.w_perm = nullptr;
-  MOE_CUDA(moe::launch_gemm_gate_up(L->tm_gu, tm_b, tm_bsh, p, L->num_sms, st));
+  MOE_CUDA(moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
   MOE_CUDA(mark(5));
 
   p.tile_start = tiles_dn;
   p.num_kb = Ip / moe::kBK;
-  p.m_tiles = H / moe::kBM;
+  p.m_tiles = mt_dn;
   p.a_rows_per_group = H;
   p.shared_b_row0 = T * k;
   p.out = ybuf;
   p.out_ld = H;
+  p.out_feats = H;
   p.w_perm = w_perm;
-  MOE_CUDA(moe::launch_gemm_down(L->tm_dn, tm_h, p, L->num_sms, st));
+  MOE_CUDA(moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
   MOE_CUDA(mark(6));
   MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, out, st));
   MOE_CUDA(mark(7));

@@ -47,6 +47,7 @@ struct GemmParams {
   int shared_b_row0;      // gate/up: first row of the shared group's B operand
   __nv_bfloat16* out;     // h [rows, out_ld] or y [rows, out_ld]
   int out_ld;
+  int out_feats;          // output features (columns) that exist; larger ones are not stored
   const float* w_perm;    // down: gate weight of each row (1 for shared rows)
   float limit;            // gate/up clamp of routed experts (<= 0: none)
   float limit_shared;     // gate/up clamp of the shared expert
@@ -80,20 +81,27 @@ cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router
 cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, const float* bias,
                         bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st,
                         float* logits_out = nullptr, const TopkRefine* refine = nullptr);
-cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int m_tiles_gu,
-                        int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
+cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn,
+                        int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
                         int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
                         int* pos, float* w_perm, cudaStream_t st);
 cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_routed, int k, int T,
                           int H, bool write_shared, __nv_bfloat16* x_perm, int num_sms,
                           cudaStream_t st);
-cudaError_t launch_gemm_gate_up(const CUtensorMap& tmA, const CUtensorMap& tmB,
-                                const CUtensorMap& tmBsh, const GemmParams& p, int grid,
-                                cudaStream_t st);
-cudaError_t launch_gemm_down(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
-                             int grid, cudaStream_t st);
-cudaError_t launch_gemm_router(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmParams& p,
-                               int grid, cudaStream_t st);
+// 128-feature weight blocks per down-projection tile for hidden size H.
+int gemm_down_blocks(int H);
+
+// Tensor maps of one grouped-GEMM launch: the weight operand, the token-row
+// operand with kBBoxRows- and BN-row boxes, and the shared expert's token
+// rows (gate|up only) with both box heights.
+struct GemmMaps {
+  CUtensorMap a, b, bsh, bw, bshw;
+};
+
+cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
+cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
+                             cudaStream_t st);
+cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
 cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
                                cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k, int H, bool out_bf16,
@@ -105,6 +113,6 @@ cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int 
 
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t gemm_configure_device();
-size_t gemm_smem_bytes(int mode);
+
 
 }  // namespace moe

@@ -165,17 +165,21 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // Shared-memory matrix descriptor of a K-major operand tile stored with the
-// 128-byte swizzle: rows of 128 bytes, 8-row atoms of 1024 bytes (stride
-// byte offset 1024), leading byte offset unused (1), descriptor version 1,
-// layout type 2 (SWIZZLE_128B).  The tile base must be 1024-byte aligned;
-// advancing along K inside the atom adds the byte offset to the start field.
-__device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
+// 128-byte (ROW_BYTES = 128) or 64-byte (ROW_BYTES = 64) swizzle: one row of
+// ROW_BYTES per M/N index, 8-row atoms (stride byte offset 8 * ROW_BYTES),
+// leading byte offset unused (1), descriptor version 1, layout type 2
+// (SWIZZLE_128B) or 4 (SWIZZLE_64B).  The tile base must be aligned to its
+// atom; advancing along K inside a row adds the byte offset to the start
+// field.
+template <int ROW_BYTES>
+__device__ __forceinline__ uint64_t sdesc_k_sw(uint32_t saddr) {
+  static_assert(ROW_BYTES == 128 || ROW_BYTES == 64, "swizzle width");
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
   d |= static_cast<uint64_t>(1) << 16;
-  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>((8 * ROW_BYTES) >> 4) << 32;
   d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(2) << 61;
+  d |= static_cast<uint64_t>(ROW_BYTES == 128 ? 2 : 4) << 61;
   return d;
 }
 

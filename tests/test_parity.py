@@ -58,6 +58,16 @@ SMALL = {
     "five_tokens": replace(WORKLOADS["tiny"], name="t5", T=5, act_dtype="bf16",
                            weight_dtype="bf16"),
     "top1_of_1": replace(WORKLOADS["tiny"], name="e1", T=64, num_experts=1, top_k=1),
+    # many token tiles per group: ~525 rows per expert = four full token tiles
+    # and a ragged one; down tiles of two weight blocks
+    "large_tiles": replace(WORKLOADS["tiny"], name="lt", T=2100, hidden=512, num_experts=16,
+                           top_k=4, intermediate=256, shared_intermediate=256,
+                           act_dtype="bf16", weight_dtype="bf16", x_dist="rmsnorm_normal",
+                           swiglu_limit=0.9, swiglu_limit_shared=1.3, expert_std=0.08),
+    # H with an odd number of 128-feature blocks: down tiles of one block
+    "large_odd_hidden": replace(WORKLOADS["tiny"], name="lo", T=2048, hidden=384,
+                                num_experts=12, top_k=3, intermediate=128,
+                                shared_intermediate=128, act_dtype="bf16", weight_dtype="bf16"),
 }
 
 
