@@ -26,6 +26,7 @@ struct moe_layer {
   float* router_w;      // [H, E]
   float* router_b;      // [E]
   __nv_bfloat16* router_tc;  // [E_pad, 3H]: bf16 three-term split of router_w^T
+  float* router_t;           // [E, H]: router_w^T, fp32 (top-k candidate recomputation)
   int E_pad;
   int has_bias;
   int* status;          // device status word
@@ -204,12 +205,13 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
   }
   const size_t H = cfg->hidden, E = cfg->num_experts, Ip = L->I_pad;
   const size_t gu_bytes = (E + 1) * 2 * Ip * H * 2, dn_bytes = (E + 1) * H * Ip * 2;
-  if (moe::gemm_configure_device() != cudaSuccess ||
+  if (moe::gemm_configure_device() != cudaSuccess || moe::topk_configure_device() != cudaSuccess ||
       cudaMalloc(&L->w_gu, gu_bytes) != cudaSuccess ||
       cudaMalloc(&L->w_dn, dn_bytes) != cudaSuccess ||
       cudaMalloc(&L->router_w, H * E * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&L->router_b, E * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&L->router_tc, static_cast<size_t>(L->E_pad) * 3 * H * 2) != cudaSuccess ||
+      cudaMalloc(&L->router_t, E * H * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
       cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess) {
     moe_destroy(L);
@@ -248,7 +250,7 @@ int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_
   MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, L->w_dn + E * dn_group, st));
   MOE_CUDA(cudaMemcpyAsync(L->router_w, router_w, static_cast<size_t>(H) * E * sizeof(float),
                            cudaMemcpyDeviceToDevice, st));
-  MOE_CUDA(moe::launch_pack_router(router_w, H, E, L->E_pad, L->router_tc, st));
+  MOE_CUDA(moe::launch_pack_router(router_w, H, E, L->E_pad, L->router_tc, L->router_t, st));
   L->has_bias = (c.use_router_bias && router_bias != nullptr) ? 1 : 0;
   if (L->has_bias)
     MOE_CUDA(cudaMemcpyAsync(L->router_b, router_bias, E * sizeof(float),
@@ -364,7 +366,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
     MOE_CUDA(moe::launch_gemm_router(rt, r, tiles < L->num_sms ? tiles : L->num_sms, st));
     ksplit = 1;
     refine.x = static_cast<const __nv_bfloat16*>(x);
-    refine.w_tc = L->router_tc;
+    refine.w_t = L->router_t;
     refine.H = H;
     refine.band = moe::router_refine_band(H);
   } else {
@@ -543,6 +545,7 @@ void moe_destroy(moe_layer_t* L) {
     cudaFree(L->router_w);
     cudaFree(L->router_b);
     cudaFree(L->router_tc);
+    cudaFree(L->router_t);
     cudaFree(L->status);
   }
   delete L;

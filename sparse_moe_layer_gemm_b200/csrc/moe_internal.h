@@ -69,10 +69,10 @@ __host__ __device__ constexpr float router_refine_band(int H) {
 }
 
 struct TopkRefine {
-  const __nv_bfloat16* x;     // [T, H] bf16 input rows
-  const __nv_bfloat16* w_tc;  // [E_pad, 3H] three-term split router rows
+  const __nv_bfloat16* x;  // [T, H] bf16 input rows
+  const float* w_t;        // [E, H] fp32 router weight, transposed
   int H;
-  float band;                 // 0: no refinement
+  float band;              // 0: no refinement
 };
 
 // ---- launchers (each returns the cudaGetLastError of its launch) ----
@@ -103,7 +103,7 @@ cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, i
                              cudaStream_t st);
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
 cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
-                               cudaStream_t st);
+                               float* dst_t, cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k, int H, bool out_bf16,
                            void* out, cudaStream_t st);
 cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
@@ -113,6 +113,7 @@ cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int 
 
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t gemm_configure_device();
+cudaError_t topk_configure_device();
 
 
 }  // namespace moe

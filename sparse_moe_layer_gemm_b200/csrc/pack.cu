@@ -46,10 +46,11 @@ __global__ void __launch_bounds__(256) pack_kernel(const TS* __restrict__ src, i
 // along K, with W1 = bf16(w), W2 = bf16(w - W1), W3 = bf16(w - W1 - W2).
 // Each residual is exact in fp32 (it keeps at most 16, then 8, significant
 // bits), and W3 holds the last 8, so W1 + W2 + W3 == w for normal w.  Rows
-// e >= E are zero.
+// e >= E are zero.  Also writes the fp32 transpose [E][H] (dst_t).
 __global__ void __launch_bounds__(256) pack_router_kernel(const float* __restrict__ w, int H, int E,
                                                           int E_pad,
-                                                          __nv_bfloat16* __restrict__ dst) {
+                                                          __nv_bfloat16* __restrict__ dst,
+                                                          float* __restrict__ dst_t) {
   __shared__ float tile[32][33];
   const int e0 = blockIdx.x * 32, h0 = blockIdx.y * 32;
   for (int i = threadIdx.y; i < 32; i += 8) {
@@ -71,6 +72,7 @@ __global__ void __launch_bounds__(256) pack_router_kernel(const float* __restric
       row[h] = b1;
       row[H + h] = b2;
       row[2 * H + h] = b3;
+      if (e < E) dst_t[static_cast<size_t>(e) * H + h] = v;
     }
   }
 }
@@ -78,9 +80,9 @@ __global__ void __launch_bounds__(256) pack_router_kernel(const float* __restric
 }  // namespace
 
 cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
-                               cudaStream_t st) {
+                               float* dst_t, cudaStream_t st) {
   dim3 grid((E_pad + 31) / 32, (H + 31) / 32), block(32, 8);
-  pack_router_kernel<<<grid, block, 0, st>>>(w, H, E, E_pad, dst);
+  pack_router_kernel<<<grid, block, 0, st>>>(w, H, E, E_pad, dst, dst_t);
   return cudaGetLastError();
 }
 

@@ -182,9 +182,8 @@ __device__ __forceinline__ void warp_select(const float* s_sc, const float* s_be
 // out.  Every expert whose approximate selection score is within `band` of
 // the approximate k-th one -- the approximate top-k included -- is a
 // candidate; one warp per candidate recomputes its logit as an fp32 dot
-// product on the CUDA cores (its router row rebuilt exactly as W1 + W2 + W3
-// from the packed three-term split; lane-strided FMA chains, fixed shuffle
-// tree).  The selection, its order and the gate weights then come from these
+// product on the CUDA cores (the token's row staged in shared memory, the
+// expert's fp32 router column read as a contiguous row of W_r^T).  The selection, its order and the gate weights then come from these
 // fp32 logits; non-candidates are excluded, which is exact as long as the
 // tensor-core error in the selection score stays below band / 2.
 template <int MPL>
@@ -233,6 +232,20 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ pa
         s_ncand = 0;
       }
     }
+    // the token's input row, widened to fp32 once for all candidate warps
+    extern __shared__ float s_x[];
+    const int H = rf.H;
+    const __nv_bfloat16* xt = rf.x + static_cast<size_t>(t) * H;
+    for (int h = threadIdx.x * 8; h < H; h += blockDim.x * 8) {
+      const uint4 q = *reinterpret_cast<const uint4*>(xt + h);
+      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(hv[i]);
+        s_x[h + 2 * i] = f.x;
+        s_x[h + 2 * i + 1] = f.y;
+      }
+    }
     __syncthreads();
     const float floor_ = s_kth - rf.band;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -243,40 +256,66 @@ __global__ void __launch_bounds__(1024) topk_kernel(const float* __restrict__ pa
     }
     __syncthreads();
     const int n = s_ncand;
-    const int H = rf.H;
-    const __nv_bfloat16* xt = rf.x + static_cast<size_t>(t) * H;
     for (int c = warp; c < n; c += nwarps) {
+      // fp32 dot product with the expert's router column (a row of W_r^T):
+      // lane-strided float4 chunks, four partial sums, fixed shuffle tree
       const int e = s_cand[c];
-      const __nv_bfloat16* w = rf.w_tc + static_cast<size_t>(e) * 3 * H;
-      float acc = 0.f;
-      for (int h0 = lane * 8; h0 < H; h0 += 256) {
-        const uint4 xq = *reinterpret_cast<const uint4*>(xt + h0);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(w + h0);
-        const uint4 q2 = *reinterpret_cast<const uint4*>(w + H + h0);
-        const uint4 q3 = *reinterpret_cast<const uint4*>(w + 2 * H + h0);
-        const __nv_bfloat16* xv = reinterpret_cast<const __nv_bfloat16*>(&xq);
-        const __nv_bfloat16* w1 = reinterpret_cast<const __nv_bfloat16*>(&q1);
-        const __nv_bfloat16* w2 = reinterpret_cast<const __nv_bfloat16*>(&q2);
-        const __nv_bfloat16* w3 = reinterpret_cast<const __nv_bfloat16*>(&q3);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float wv =
-              (__bfloat162float(w1[i]) + __bfloat162float(w2[i])) + __bfloat162float(w3[i]);
-          acc = fmaf(__bfloat162float(xv[i]), wv, acc);
-        }
+      const float4* w4 = reinterpret_cast<const float4*>(rf.w_t + static_cast<size_t>(e) * H);
+      const float4* x4 = reinterpret_cast<const float4*>(s_x);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+      for (int i = lane; i < H / 4; i += 32) {
+        const float4 wv = __ldg(w4 + i);
+        const float4 xv = x4[i];
+        a0 = fmaf(xv.x, wv.x, a0);
+        a1 = fmaf(xv.y, wv.y, a1);
+        a2 = fmaf(xv.z, wv.z, a2);
+        a3 = fmaf(xv.w, wv.w, a3);
       }
+      float acc = (a0 + a1) + (a2 + a3);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
       if (lane == 0) {
-        const float s = 1.0f / (1.0f + expf(-acc));
+        const float sv = 1.0f / (1.0f + expf(-acc));
         s_l[e] = acc;
-        s_sc[e] = s;
-        s_be[e] = (bias != nullptr) ? s + bias[e] : s;
+        s_sc[e] = sv;
+        s_be[e] = (bias != nullptr) ? sv + bias[e] : sv;
       }
     }
     __syncthreads();
+    if (n <= 32) {
+      // order the candidates by rank: lane c holds candidate c; its rank is
+      // the number of candidates ahead of it (higher score, or equal score
+      // and lower index); lane with rank j supplies the j-th pick
+      if (warp == 0) {
+        const int e = lane < n ? s_cand[lane] : 0x7fffffff;
+        const float b = lane < n ? s_be[e] : -INFINITY;
+        int rank = 0;
+        for (int c = 0; c < n; ++c) {
+          const float bc = __shfl_sync(0xffffffffu, b, c);
+          const int ec = __shfl_sync(0xffffffffu, e, c);
+          rank += (bc > b || (bc == b && ec < e)) ? 1 : 0;
+        }
+        // lane j gathers the candidate of rank j
+        int pick_e = 0;
+        float pick_s = 0.f;
+        for (int c = 0; c < n; ++c) {
+          const int rc = __shfl_sync(0xffffffffu, rank, c);
+          const int ec = __shfl_sync(0xffffffffu, e, c);
+          if (rc == lane) {
+            pick_e = ec;
+            pick_s = s_sc[ec];
+          }
+        }
+        my_idx = pick_e;
+        my_s = pick_s;
+      }
+    } else if (warp == 0) {
+      warp_select<MPL>(s_sc, s_be, E, k, my_idx, my_s, kth, next);
+    }
+  } else if (warp == 0) {
+    warp_select<MPL>(s_sc, s_be, E, k, my_idx, my_s, kth, next);
   }
-  if (warp == 0) warp_select<MPL>(s_sc, s_be, E, k, my_idx, my_s, kth, next);
   if (logits_out != nullptr) {
     for (int e = threadIdx.x; e < E; e += blockDim.x)
       logits_out[static_cast<size_t>(t) * E + e] = s_l[e];
@@ -305,6 +344,19 @@ cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router
   return cudaGetLastError();
 }
 
+cudaError_t topk_configure_device() {
+  // dynamic shared memory of the candidate recomputation: one fp32 input row
+  const int bytes = 16384 * static_cast<int>(sizeof(float));
+  cudaError_t e = cudaSuccess;
+#define MOE_TOPK_ATTR(N)                                                                       \
+  if (e == cudaSuccess)                                                                        \
+    e = cudaFuncSetAttribute(topk_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  MOE_TOPK_ATTR(1) MOE_TOPK_ATTR(2) MOE_TOPK_ATTR(4) MOE_TOPK_ATTR(8) MOE_TOPK_ATTR(9)
+  MOE_TOPK_ATTR(16) MOE_TOPK_ATTR(32)
+#undef MOE_TOPK_ATTR
+  return e;
+}
+
 cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, const float* bias,
                         bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st,
                         float* logits_out, const TopkRefine* refine) {
@@ -312,9 +364,10 @@ cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, c
   const int threads = min(1024, max(32, (E + 31) / 32 * 32));
   TopkRefine rf{};
   if (refine != nullptr) rf = *refine;
-#define MOE_TOPK(N)                                                                       \
-  topk_kernel<N><<<T, threads, 0, st>>>(partial, ksplit, T, E, k, bias, norm ? 1 : 0, scale, \
-                                        topk_idx, topk_w, logits_out, rf)
+  const size_t smem = rf.band > 0.f ? static_cast<size_t>(rf.H) * sizeof(float) : 0;
+#define MOE_TOPK(N)                                                                          \
+  topk_kernel<N><<<T, threads, smem, st>>>(partial, ksplit, T, E, k, bias, norm ? 1 : 0, scale, \
+                                           topk_idx, topk_w, logits_out, rf)
   if (mpl <= 1) MOE_TOPK(1);
   else if (mpl <= 2) MOE_TOPK(2);
   else if (mpl <= 4) MOE_TOPK(4);
