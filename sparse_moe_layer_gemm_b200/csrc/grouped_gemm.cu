@@ -21,9 +21,9 @@
 // Design (swap-AB): the MMA's M side (128) is always a block of weight rows,
 // the N side the group's tokens (rounded up to 16, at most 128 per tile), so
 // ragged groups of 1..21 tokens (decode) waste no more than 15 columns.
-// A tile is (group, weight tile mt, token block nc); tiles of one group are
-// ordered token-block-major so all weight tiles of the same token block run
-// together and an expert's weights stay in L2 across its token blocks.
+// A tile is (group, weight tile mt, token block nc); the order of a group's
+// tiles (chunks of token blocks, weight-tile major inside a chunk) is
+// described at decode_tile.
 //
 // One persistent CTA per SM, 4 + NI warps:
 //   warp 0        TMA producer: per stage one box of the tile's weight rows
@@ -83,36 +83,51 @@ struct Shape {
 };
 
 struct Tile {
-  int g, mt, nc, n_valid;
+  int g, mt, nc, n_valid, nch;  // nch: token blocks of the group
 };
 
-// Tile w -> (group, weight tile, token block); tile_start is the exclusive
+// Token blocks per ordering chunk (see decode_tile).
+constexpr int kChunk = 4;
+
+// Tile w -> (group, weight tile, token block).  tile_start is the exclusive
 // prefix of per-group tile counts, so the group is the last g with
-// tile_start[g] <= w (empty groups are skipped naturally).
+// tile_start[g] <= w (empty groups are skipped naturally).  Within a group
+// the tiles run in chunks of kChunk token blocks; inside a chunk weight-tile
+// major, token-block minor.  Consecutive tiles go to different CTAs at about
+// the same time, so the (up to kChunk) readers of a weight tile share one
+// pass through L2, while a chunk's token rows (kChunk x 128 rows) stay in L2
+// across its weight tiles; an expert's weights (21 MB gate|up, 10.5 MB down)
+// stay in L2 from one chunk to the next.
 template <int BN>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
+  int g, local, rows;
   if (p.single_rows > 0) {
-    Tile t;
-    t.g = 0;
-    t.nc = w / p.m_tiles;
-    t.mt = w - t.nc * p.m_tiles;
-    t.n_valid = min(BN, p.single_rows - t.nc * BN);
-    return t;
-  }
-  int lo = 0, hi = p.G;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (p.tile_start[mid] <= w)
-      lo = mid;
-    else
-      hi = mid;
+    g = 0;
+    local = w;
+    rows = p.single_rows;
+  } else {
+    int lo = 0, hi = p.G;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.tile_start[mid] <= w)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    g = lo;
+    local = w - p.tile_start[lo];
+    rows = p.counts[lo];
   }
   Tile t;
-  t.g = lo;
-  const int local = w - p.tile_start[lo];
-  t.nc = local / p.m_tiles;
-  t.mt = local - t.nc * p.m_tiles;
-  t.n_valid = min(BN, p.counts[lo] - t.nc * BN);
+  t.g = g;
+  t.nch = (rows + BN - 1) / BN;
+  const int per_chunk = p.m_tiles * kChunk;
+  const int cc = local / per_chunk;
+  const int rem = local - cc * per_chunk;
+  const int in_chunk = min(kChunk, t.nch - cc * kChunk);  // token blocks in this chunk
+  t.mt = rem / in_chunk;
+  t.nc = cc * kChunk + (rem - t.mt * in_chunk);
+  t.n_valid = min(BN, rows - t.nc * BN);
   return t;
 }
 
@@ -202,8 +217,12 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_a = l2_policy_evict_first();  // weights: streamed once
-      const uint64_t pol_b = l2_policy_evict_last();   // token rows: reused by every weight tile
+      // weights: evict-first when only one token block reads them, else
+      // normal so the other token blocks of the group find them in L2;
+      // token rows: evict-last, every weight tile of the chunk reads them
+      const uint64_t pol_first = l2_policy_evict_first();
+      const uint64_t pol_normal = l2_policy_evict_normal();
+      const uint64_t pol_b = l2_policy_evict_last();
       uint32_t it = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
         if (*abort_flag) break;
@@ -215,6 +234,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
         const int b_row = (sh ? p.shared_b_row0 : group_row0(p, t.g)) + t.nc * BN;
         const int a_row = t.g * p.a_rows_per_group + t.mt * S::A_ROWS;
         const uint32_t bytes = S::A_BYTES + (wide ? S::B_BYTES : S::B_BOX_BYTES);
+        const uint64_t pol_a = t.nch > 1 ? pol_normal : pol_first;
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           const uint32_t s = it % S::STAGES;
@@ -349,14 +369,30 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
         } else {
           __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
           const float* wrow = p.w_perm + row0;
+          // group row offsets are arbitrary: vector loads only when aligned
+          const bool vec = (reinterpret_cast<uintptr_t>(wrow) & 15u) == 0;
           for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
             uint32_t ra[16];
             tmem_ld_x16(taddr + b * BN + c0, ra);
+            float wv[16];
+            if (vec && c0 + 16 <= t.n_valid) {  // the 16 rows' gate weights in four vector loads
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const float4 q4 = __ldg(reinterpret_cast<const float4*>(wrow + c0) + v);
+                wv[4 * v] = q4.x;
+                wv[4 * v + 1] = q4.y;
+                wv[4 * v + 2] = q4.z;
+                wv[4 * v + 3] = q4.w;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) wv[i] = c0 + i < t.n_valid ? wrow[c0 + i] : 0.f;
+            }
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               if (c0 + i < t.n_valid) {
-                const float yv = __uint_as_float(ra[i]) * wrow[c0 + i];
+                const float yv = __uint_as_float(ra[i]) * wv[i];
                 outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(yv);
               }
             }
