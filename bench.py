@@ -41,7 +41,8 @@ def _args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode")
-    ap.add_argument("--secondary", default="prefill")
+    ap.add_argument("--secondary", default="prefill,zipf_prefill",
+                    help="comma-separated further workloads measured in the same run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
@@ -355,24 +356,29 @@ def run_ours(a):
                "d2h_bytes_per_step": wl.T * wl.hidden * el,
                "path": "moe_forward_host (pinned host x/out, copies inside the timed region)"}
 
-    secondary = None
-    if a.secondary and a.secondary != "none" and a.secondary != a.workload:
-        wl2 = WORKLOADS[a.secondary]
-        same_weights = (wl2.expert_std == wl.expert_std and wl2.weight_dtype == wl.weight_dtype
-                        and wl2.bias == wl.bias and wl2.hidden == wl.hidden)
-        if same_weights:
-            x2 = draw_x(rank_batch_workload(wl2, rank), dev)
-            l2 = layer
-            touched2, _ = _routing_stats(l2, x2)
-            barrier()
-            ms2, st2 = _measure(l2, x2, max(3, a.steps // 10), max(3, a.warmup), stream)
-            ms2 = max_over_ranks(ms2, dev)
-            kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2)
-            secondary = {"workload": wl2.name, "T": wl2.T,
-                         "value": job_throughput(wl2.T, world, ms2),
-                         "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
-                         "layer_roofline": lr2, "stage_ms": st2}
-            del x2
+    secondary = []
+    for name2 in [n for n in (a.secondary or "").split(",") if n and n != "none" and n != a.workload]:
+        wl2 = WORKLOADS[name2]
+        same_experts = (wl2.expert_std == wl.expert_std and wl2.weight_dtype == wl.weight_dtype
+                        and wl2.hidden == wl.hidden and wl2.num_experts == wl.num_experts
+                        and wl2.swiglu_limit == wl.swiglu_limit)
+        if not same_experts:
+            continue
+        if wl2.bias != wl.bias:  # same experts, another router bias
+            from sparse_moe_layer_gemm_b200.workloads import draw_router
+            _, rb2 = draw_router(wl2, dev)
+            layer.load_weights(inp["router_w"], rb2, inp["w_gate"], inp["w_up"], inp["w_down"],
+                               inp["sh_gate"], inp["sh_up"], inp["sh_down"])
+        x2 = draw_x(rank_batch_workload(wl2, rank), dev)
+        touched2, _ = _routing_stats(layer, x2)
+        barrier()
+        ms2, st2 = _measure(layer, x2, max(3, a.steps // 10), max(3, a.warmup), stream)
+        ms2 = max_over_ranks(ms2, dev)
+        kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2)
+        secondary.append({"workload": wl2.name, "T": wl2.T, "value": job_throughput(wl2.T, world, ms2),
+                          "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
+                          "layer_roofline": lr2, "stage_ms": st2})
+        del x2
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
