@@ -47,6 +47,9 @@ namespace moe {
 
 namespace {
 
+// Rows per TMA-store chunk of the down epilogue (one tcgen05.ld x16).
+constexpr int kEpiRows = 16;
+
 // Tile shape: BLOCKS weight blocks of 128 features per tile (gate|up: each
 // block is 128 gate rows + 128 up rows), BN tokens per tile, BK = 64 reduction
 // elements (one 128-byte swizzled row) per pipeline stage.
@@ -71,7 +74,11 @@ struct Shape {
   static constexpr int NBUF = ACC_COLS <= 256 ? 2 : 1;     // double-buffered when it fits
   static constexpr int TMEM_COLS = NBUF * ACC_COLS > 256 ? 512 : 256;
   static constexpr int BAR_BYTES = 256;
-  static constexpr size_t SMEM = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + BAR_BYTES;
+  // down epilogue: per epilogue warp two 16-row x 32-feature bf16 staging
+  // buffers for TMA stores of y
+  static constexpr int EPI_STAGE_BYTES = MODE == kModeDown ? 4 * 2 * kEpiRows * 32 * 2 : 0;
+  static constexpr size_t SMEM =
+      1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES;
   static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
   static_assert(NBUF * ACC_COLS <= 512, "TMEM capacity");
   static_assert(BN == 128, "token tile (the wide token-row box is BN rows)");
@@ -80,6 +87,7 @@ struct Shape {
   static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay aligned");
   // descriptor start-address field: 14 bits of (address >> 4), no carries
   static_assert(1024 + STAGES * STAGE_BYTES + BAR_BYTES <= 256 * 1024, "descriptor range");
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 struct Tile {
@@ -163,7 +171,8 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBsh,
                         const __grid_constant__ CUtensorMap tmBw,
-                        const __grid_constant__ CUtensorMap tmBshw, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmBshw,
+                        const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   using S = Shape<MODE, BLOCKS, BN>;
   constexpr bool GU = S::GU;
   constexpr int BK = S::BK;
@@ -314,6 +323,11 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quadrant this warp may read
+    // down: this warp's two y staging buffers (16 rows x 32 features bf16)
+    uint8_t* epi_stage = smem + S::STAGES * S::STAGE_BYTES + S::BAR_BYTES +
+                         (warp - (1 + S::NI)) * 2 * kEpiRows * 32 * 2;
+    uint32_t chunks = 0;  // TMA-store chunks this warp has issued
+    if (MODE == kModeDown && lane == 0) prefetch_tmap(&tmOut);
     uint32_t tc = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       const Tile t = decode_tile<BN>(p, w);
@@ -389,11 +403,30 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
               for (int i = 0; i < 16; ++i) wv[i] = c0 + i < t.n_valid ? wrow[c0 + i] : 0.f;
             }
             tmem_ld_wait();
+            if (c0 + kEpiRows <= t.n_valid) {
+              // full chunk: stage [16 rows][32 features] and write it with one
+              // TMA store (the chunk's rows all belong to this group)
+              const uint32_t buf_off = (chunks & 1u) * (kEpiRows * 32 * 2);
+              if (chunks >= 2 && lane == 0) bulk_wait_group_read<1>();  // buffer free again
+              __syncwarp();
+              __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(epi_stage + buf_off);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              if (c0 + i < t.n_valid) {
-                const float yv = __uint_as_float(ra[i]) * wv[i];
-                outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(yv);
+              for (int i = 0; i < kEpiRows; ++i)
+                stg[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(ra[i]) * wv[i]);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmOut, smem_u32(stg), feat - lane, static_cast<int>(row0) + c0);
+                bulk_commit_group();
+              }
+              ++chunks;
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                if (c0 + i < t.n_valid) {
+                  const float yv = __uint_as_float(ra[i]) * wv[i];
+                  outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(yv);
+                }
               }
             }
           }
@@ -404,6 +437,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
       if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
       ++tc;
     }
+    if (MODE == kModeDown && lane == 0) bulk_wait_group_all();  // y fully written
   }
 
   tc_fence_before();
@@ -445,7 +479,7 @@ int gemm_down_blocks(int H) { return (H / kBM) % 2 == 0 ? 2 : 1; }
 
 cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
   grouped_gemm_kernel<kModeGateUp, 1, 128>
-      <<<grid, GuCfg::THREADS, GuCfg::SMEM, st>>>(m.a, m.b, m.bsh, m.bw, m.bshw, p);
+      <<<grid, GuCfg::THREADS, GuCfg::SMEM, st>>>(m.a, m.b, m.bsh, m.bw, m.bshw, m.out, p);
   return cudaGetLastError();
 }
 
@@ -453,16 +487,16 @@ cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, i
                              cudaStream_t st) {
   if (blocks == 2)
     grouped_gemm_kernel<kModeDown, 2, 128>
-        <<<grid, DnCfg2::THREADS, DnCfg2::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, p);
+        <<<grid, DnCfg2::THREADS, DnCfg2::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, m.out, p);
   else
     grouped_gemm_kernel<kModeDown, 1, 128>
-        <<<grid, DnCfg1::THREADS, DnCfg1::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, p);
+        <<<grid, DnCfg1::THREADS, DnCfg1::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, m.out, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
   grouped_gemm_kernel<kModeRouter, 1, 128>
-      <<<grid, RtCfg::THREADS, RtCfg::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, p);
+      <<<grid, RtCfg::THREADS, RtCfg::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, m.out, p);
   return cudaGetLastError();
 }
 

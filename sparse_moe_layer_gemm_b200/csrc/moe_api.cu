@@ -128,6 +128,21 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   return r == CUDA_SUCCESS;
 }
 
+// bf16 [rows, cols] row-major, box 32 columns x 16 rows, no swizzle: the
+// down epilogue's TMA stores of y.
+bool encode_bf16_store(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {32, 16};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Makes the layer's device current for the lifetime of the guard.
@@ -325,8 +340,11 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   if (!encode_bf16_2d(&gu.b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
       !encode_bf16_2d(&gu.bw, x_perm, w.rows_xperm, H, moe::kBN) ||
       !encode_bf16_2d(&dn.b, hbuf, w.rows_all, Ip, moe::kBBoxRows) ||
-      !encode_bf16_2d(&dn.bw, hbuf, w.rows_all, Ip, moe::kBN))
+      !encode_bf16_2d(&dn.bw, hbuf, w.rows_all, Ip, moe::kBN) ||
+      !encode_bf16_store(&dn.out, ybuf, w.rows_all, H))
     return MOE_ERR_CUDA;
+  gu.out = dn.out;  // unused by gate|up and the router
+  rt.out = dn.out;
   if (xb) {
     if (!encode_bf16_2d(&gu.bsh, x, T, H, moe::kBBoxRows) ||
         !encode_bf16_2d(&gu.bshw, x, T, H, moe::kBN))

@@ -92,10 +92,11 @@ cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_
 int gemm_down_blocks(int H);
 
 // Tensor maps of one grouped-GEMM launch: the weight operand, the token-row
-// operand with kBBoxRows- and BN-row boxes, and the shared expert's token
-// rows (gate|up only) with both box heights.
+// operand with kBBoxRows- and BN-row boxes, the shared expert's token rows
+// (gate|up only) with both box heights, and the output for TMA stores (down:
+// y with 32-feature x 16-row boxes, no swizzle).
 struct GemmMaps {
-  CUtensorMap a, b, bsh, bw, bshw;
+  CUtensorMap a, b, bsh, bw, bshw, out;
 };
 
 cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
