@@ -74,9 +74,9 @@ struct Shape {
   static constexpr int NBUF = ACC_COLS <= 256 ? 2 : 1;     // double-buffered when it fits
   static constexpr int TMEM_COLS = NBUF * ACC_COLS > 256 ? 512 : 256;
   static constexpr int BAR_BYTES = 256;
-  // down epilogue: per epilogue warp two 16-row x 32-feature bf16 staging
-  // buffers for TMA stores of y
-  static constexpr int EPI_STAGE_BYTES = MODE == kModeDown ? 4 * 2 * kEpiRows * 32 * 2 : 0;
+  // gate|up and down epilogues: per epilogue warp two 16-row x 32-feature
+  // bf16 staging buffers for TMA stores of h or y
+  static constexpr int EPI_STAGE_BYTES = MODE != kModeRouter ? 4 * 2 * kEpiRows * 32 * 2 : 0;
   static constexpr size_t SMEM =
       1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES;
   static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
@@ -323,11 +323,38 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // the TMEM lane quadrant this warp may read
-    // down: this warp's two y staging buffers (16 rows x 32 features bf16)
+    // this warp's two output staging buffers (16 rows x 32 features bf16)
     uint8_t* epi_stage = smem + S::STAGES * S::STAGE_BYTES + S::BAR_BYTES +
                          (warp - (1 + S::NI)) * 2 * kEpiRows * 32 * 2;
     uint32_t chunks = 0;  // TMA-store chunks this warp has issued
-    if (MODE == kModeDown && lane == 0) prefetch_tmap(&tmOut);
+    if (MODE != kModeRouter && lane == 0) prefetch_tmap(&tmOut);
+    // Writes rows [c0, c0 + 16) of this lane's output feature.  A chunk whose
+    // 16 rows all belong to the tile goes through a staging buffer and one
+    // TMA store of 16 x 32 values; a ragged one is stored directly, so no row
+    // of another group is ever written.
+    auto store_chunk = [&](const float (&v)[16], int c0, int n_valid, size_t row0, int feat,
+                           __nv_bfloat16* outp) {
+      if (c0 + kEpiRows <= n_valid) {
+        const uint32_t buf_off = (chunks & 1u) * (kEpiRows * 32 * 2);
+        if (chunks >= 2 && lane == 0) bulk_wait_group_read<1>();  // buffer free again
+        __syncwarp();
+        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(epi_stage + buf_off);
+#pragma unroll
+        for (int i = 0; i < kEpiRows; ++i) stg[i * 32 + lane] = __float2bfloat16_rn(v[i]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmOut, smem_u32(stg), feat - lane, static_cast<int>(row0) + c0);
+          bulk_commit_group();
+        }
+        ++chunks;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (c0 + i < n_valid)
+            outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(v[i]);
+      }
+    };
     uint32_t tc = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       const Tile t = decode_tile<BN>(p, w);
@@ -366,19 +393,18 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
             tmem_ld_x16(tg + c0, ra);
             tmem_ld_x16(tu + c0, rb);
             tmem_ld_wait();
+            float hv[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              if (c0 + i < t.n_valid) {
-                float a = __uint_as_float(ra[i]);
-                float u = __uint_as_float(rb[i]);
-                if (L > 0.f) {
-                  a = fminf(a, L);
-                  u = fminf(fmaxf(u, -L), L);
-                }
-                const float hv = a / (1.0f + __expf(-a)) * u;
-                outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(hv);
+              float a = __uint_as_float(ra[i]);
+              float u = __uint_as_float(rb[i]);
+              if (L > 0.f) {
+                a = fminf(a, L);
+                u = fminf(fmaxf(u, -L), L);
               }
+              hv[i] = a / (1.0f + __expf(-a)) * u;
             }
+            store_chunk(hv, c0, t.n_valid, row0, feat, outp);
           }
         } else {
           __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
@@ -403,32 +429,10 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
               for (int i = 0; i < 16; ++i) wv[i] = c0 + i < t.n_valid ? wrow[c0 + i] : 0.f;
             }
             tmem_ld_wait();
-            if (c0 + kEpiRows <= t.n_valid) {
-              // full chunk: stage [16 rows][32 features] and write it with one
-              // TMA store (the chunk's rows all belong to this group)
-              const uint32_t buf_off = (chunks & 1u) * (kEpiRows * 32 * 2);
-              if (chunks >= 2 && lane == 0) bulk_wait_group_read<1>();  // buffer free again
-              __syncwarp();
-              __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(epi_stage + buf_off);
+            float yv[16];
 #pragma unroll
-              for (int i = 0; i < kEpiRows; ++i)
-                stg[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(ra[i]) * wv[i]);
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&tmOut, smem_u32(stg), feat - lane, static_cast<int>(row0) + c0);
-                bulk_commit_group();
-              }
-              ++chunks;
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                if (c0 + i < t.n_valid) {
-                  const float yv = __uint_as_float(ra[i]) * wv[i];
-                  outp[static_cast<size_t>(c0 + i) * p.out_ld] = __float2bfloat16_rn(yv);
-                }
-              }
-            }
+            for (int i = 0; i < 16; ++i) yv[i] = __uint_as_float(ra[i]) * wv[i];
+            store_chunk(yv, c0, t.n_valid, row0, feat, outp);
           }
         }
       }
@@ -437,7 +441,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
       if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
       ++tc;
     }
-    if (MODE == kModeDown && lane == 0) bulk_wait_group_all();  // y fully written
+    if (MODE != kModeRouter && lane == 0) bulk_wait_group_all();  // h / y fully written
   }
 
   tc_fence_before();

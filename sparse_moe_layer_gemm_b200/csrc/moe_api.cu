@@ -129,7 +129,7 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 }
 
 // bf16 [rows, cols] row-major, box 32 columns x 16 rows, no swizzle: the
-// down epilogue's TMA stores of y.
+// expert GEMM epilogues' TMA stores of h and y.
 bool encode_bf16_store(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
@@ -341,10 +341,10 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
       !encode_bf16_2d(&gu.bw, x_perm, w.rows_xperm, H, moe::kBN) ||
       !encode_bf16_2d(&dn.b, hbuf, w.rows_all, Ip, moe::kBBoxRows) ||
       !encode_bf16_2d(&dn.bw, hbuf, w.rows_all, Ip, moe::kBN) ||
+      !encode_bf16_store(&gu.out, hbuf, w.rows_all, Ip) ||
       !encode_bf16_store(&dn.out, ybuf, w.rows_all, H))
     return MOE_ERR_CUDA;
-  gu.out = dn.out;  // unused by gate|up and the router
-  rt.out = dn.out;
+  rt.out = dn.out;  // unused by the router
   if (xb) {
     if (!encode_bf16_2d(&gu.bsh, x, T, H, moe::kBBoxRows) ||
         !encode_bf16_2d(&gu.bshw, x, T, H, moe::kBN))

@@ -93,7 +93,7 @@ int gemm_down_blocks(int H);
 
 // Tensor maps of one grouped-GEMM launch: the weight operand, the token-row
 // operand with kBBoxRows- and BN-row boxes, the shared expert's token rows
-// (gate|up only) with both box heights, and the output for TMA stores (down:
+// (gate|up only) with both box heights, and the output for TMA stores (h or
 // y with 32-feature x 16-row boxes, no swizzle).
 struct GemmMaps {
   CUtensorMap a, b, bsh, bw, bshw, out;
