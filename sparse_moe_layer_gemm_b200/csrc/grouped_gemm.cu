@@ -40,6 +40,7 @@
 //   last 4 warps  epilogue: tcgen05.ld (32 lanes x 16 columns), SwiGLU or
 //                 gate weight in registers, bf16 (router: fp32) stores.
 // No TMA multicast anywhere.
+#include "gemm_common.cuh"
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
 
@@ -47,8 +48,7 @@ namespace moe {
 
 namespace {
 
-// Rows per TMA-store chunk of the down epilogue (one tcgen05.ld x16).
-constexpr int kEpiRows = 16;
+using namespace gemm;
 
 // Tile shape: BLOCKS weight blocks of 128 features per tile (gate|up: each
 // block is 128 gate rows + 128 up rows), BN tokens per tile, BK = 64 reduction
@@ -76,9 +76,13 @@ struct Shape {
   static constexpr int BAR_BYTES = 256;
   // gate|up and down epilogues: per epilogue warp two 16-row x 32-feature
   // bf16 staging buffers for TMA stores of h or y
-  static constexpr int EPI_STAGE_BYTES = MODE != kModeRouter ? 4 * 2 * kEpiRows * 32 * 2 : 0;
-  static constexpr size_t SMEM =
-      1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES;
+  // (down: plus per warp the tile's BN gate weights, fp32)
+  static constexpr int EPI_STAGE_BYTES =
+      MODE != kModeRouter ? 4 * 2 * kEpiRows * 32 * 2 + (MODE == kModeDown ? 4 * BN * 4 : 0) : 0;
+  // group tables (tile_start, counts, row_start) copied to shared memory
+  static constexpr int TAB_OFFSET = STAGES * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES;
+  static constexpr int TAB_BYTES = MODE != kModeRouter ? kTabBytes : 0;
+  static constexpr size_t SMEM = 1024 + static_cast<size_t>(TAB_OFFSET) + TAB_BYTES;
   static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
   static_assert(NBUF * ACC_COLS <= 512, "TMEM capacity");
   static_assert(BN == 128, "token tile (the wide token-row box is BN rows)");
@@ -89,65 +93,6 @@ struct Shape {
   static_assert(1024 + STAGES * STAGE_BYTES + BAR_BYTES <= 256 * 1024, "descriptor range");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
-
-struct Tile {
-  int g, mt, nc, n_valid, nch;  // nch: token blocks of the group
-};
-
-// Token blocks per ordering chunk (see decode_tile).
-constexpr int kChunk = 4;
-
-// Tile w -> (group, weight tile, token block).  tile_start is the exclusive
-// prefix of per-group tile counts, so the group is the last g with
-// tile_start[g] <= w (empty groups are skipped naturally).  Within a group
-// the tiles run in chunks of kChunk token blocks; inside a chunk weight-tile
-// major, token-block minor.  Consecutive tiles go to different CTAs at about
-// the same time, so the (up to kChunk) readers of a weight tile share one
-// pass through L2, while a chunk's token rows (kChunk x 128 rows) stay in L2
-// across its weight tiles; an expert's weights (21 MB gate|up, 10.5 MB down)
-// stay in L2 from one chunk to the next.
-template <int BN>
-__device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
-  int g, local, rows;
-  if (p.single_rows > 0) {
-    g = 0;
-    local = w;
-    rows = p.single_rows;
-  } else {
-    int lo = 0, hi = p.G;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (p.tile_start[mid] <= w)
-        lo = mid;
-      else
-        hi = mid;
-    }
-    g = lo;
-    local = w - p.tile_start[lo];
-    rows = p.counts[lo];
-  }
-  Tile t;
-  t.g = g;
-  t.nch = (rows + BN - 1) / BN;
-  const int per_chunk = p.m_tiles * kChunk;
-  const int cc = local / per_chunk;
-  const int rem = local - cc * per_chunk;
-  const int in_chunk = min(kChunk, t.nch - cc * kChunk);  // token blocks in this chunk
-  t.mt = rem / in_chunk;
-  t.nc = cc * kChunk + (rem - t.mt * in_chunk);
-  t.n_valid = min(BN, rows - t.nc * BN);
-  return t;
-}
-
-template <int BN>
-__device__ __forceinline__ int total_tiles(const GemmParams& p) {
-  if (p.single_rows > 0) return p.m_tiles * ((p.single_rows + BN - 1) / BN);
-  return p.tile_start[p.G];
-}
-
-__device__ __forceinline__ int group_row0(const GemmParams& p, int g) {
-  return p.single_rows > 0 ? 0 : p.row_start[g];
-}
 
 // tcgen05.mma issue without a memory clobber: the MMA reads shared memory
 // the TMA wrote (ordered by the full-barrier wait and the tcgen05 fence) and
@@ -190,6 +135,9 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // group tables in shared memory (visible after the __syncthreads below)
+  const GemmParams gp =
+      MODE != kModeRouter ? stage_group_tables(p, reinterpret_cast<int*>(smem + S::TAB_OFFSET)) : p;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
@@ -221,7 +169,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = total_tiles<BN>(p);
+  const int total = total_tiles<BN>(gp);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -235,12 +183,12 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
       uint32_t it = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
         if (*abort_flag) break;
-        const Tile t = decode_tile<BN>(p, w);
+        const Tile t = decode_tile<BN>(gp, w);
         const int n_mma = (t.n_valid + 15) & ~15;
         const bool wide = n_mma > kBBoxRows;  // one BN-row box, else one kBBoxRows-row box
         const bool sh = GU && t.g == p.E;
         const CUtensorMap* mb = wide ? (sh ? &tmBshw : &tmBw) : (sh ? &tmBsh : &tmB);
-        const int b_row = (sh ? p.shared_b_row0 : group_row0(p, t.g)) + t.nc * BN;
+        const int b_row = (sh ? p.shared_b_row0 : group_row0(gp, t.g)) + t.nc * BN;
         const int a_row = t.g * p.a_rows_per_group + t.mt * S::A_ROWS;
         const uint32_t bytes = S::A_BYTES + (wide ? S::B_BYTES : S::B_BOX_BYTES);
         const uint64_t pol_a = t.nch > 1 ? pol_normal : pol_first;
@@ -279,7 +227,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
       uint32_t it = 0, tc = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
         if (*abort_flag) break;
-        const Tile t = decode_tile<BN>(p, w);
+        const Tile t = decode_tile<BN>(gp, w);
         const int n_mma = (t.n_valid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
         const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
@@ -326,6 +274,11 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
     // this warp's two output staging buffers (16 rows x 32 features bf16)
     uint8_t* epi_stage = smem + S::STAGES * S::STAGE_BYTES + S::BAR_BYTES +
                          (warp - (1 + S::NI)) * 2 * kEpiRows * 32 * 2;
+    // down: the tile's gate weights, loaded once per tile while the
+    // accumulators are still being computed
+    float* wbuf = reinterpret_cast<float*>(smem + S::STAGES * S::STAGE_BYTES + S::BAR_BYTES +
+                                           4 * 2 * kEpiRows * 32 * 2) +
+                  (warp - (1 + S::NI)) * BN;
     uint32_t chunks = 0;  // TMA-store chunks this warp has issued
     if (MODE != kModeRouter && lane == 0) prefetch_tmap(&tmOut);
     // Writes rows [c0, c0 + 16) of this lane's output feature.  A chunk whose
@@ -357,17 +310,28 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
     };
     uint32_t tc = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      const Tile t = decode_tile<BN>(p, w);
+      const Tile t = decode_tile<BN>(gp, w);
       const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
       const uint32_t tph = (S::NBUF == 2 ? (tc >> 1) : tc) & 1u;
+      const size_t row0 = static_cast<size_t>(group_row0(gp, t.g)) + static_cast<size_t>(t.nc) * BN;
+      float wl[BN / 32];
+      if (MODE == kModeDown) {
+#pragma unroll
+        for (int m = 0; m < BN / 32; ++m)
+          wl[m] = lane + 32 * m < t.n_valid ? __ldg(p.w_perm + row0 + lane + 32 * m) : 0.f;
+      }
       int ok = 1;
       if (lane == 0) ok = mbar_wait(tfull0 + 8 * buf, tph, abort_flag, p.status) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
+      if (MODE == kModeDown) {
+#pragma unroll
+        for (int m = 0; m < BN / 32; ++m) wbuf[lane + 32 * m] = wl[m];
+        __syncwarp();
+      }
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * S::ACC_COLS;
-      const size_t row0 = static_cast<size_t>(group_row0(p, t.g)) + static_cast<size_t>(t.nc) * BN;
 #pragma unroll 1
       for (int b = 0; b < BLOCKS; ++b) {
         const int feat = (t.mt * BLOCKS + b) * kBM + q * 32 + lane;
@@ -408,30 +372,13 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
           }
         } else {
           __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
-          const float* wrow = p.w_perm + row0;
-          // group row offsets are arbitrary: vector loads only when aligned
-          const bool vec = (reinterpret_cast<uintptr_t>(wrow) & 15u) == 0;
           for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
             uint32_t ra[16];
             tmem_ld_x16(taddr + b * BN + c0, ra);
-            float wv[16];
-            if (vec && c0 + 16 <= t.n_valid) {  // the 16 rows' gate weights in four vector loads
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const float4 q4 = __ldg(reinterpret_cast<const float4*>(wrow + c0) + v);
-                wv[4 * v] = q4.x;
-                wv[4 * v + 1] = q4.y;
-                wv[4 * v + 2] = q4.z;
-                wv[4 * v + 3] = q4.w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) wv[i] = c0 + i < t.n_valid ? wrow[c0 + i] : 0.f;
-            }
             tmem_ld_wait();
             float yv[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) yv[i] = __uint_as_float(ra[i]) * wv[i];
+            for (int i = 0; i < 16; ++i) yv[i] = __uint_as_float(ra[i]) * wbuf[c0 + i];
             store_chunk(yv, c0, t.n_valid, row0, feat, outp);
           }
         }

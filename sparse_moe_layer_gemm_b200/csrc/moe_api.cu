@@ -32,6 +32,7 @@ struct moe_layer {
   int* status;          // device status word
   int loaded;
   CUtensorMap tm_gu;    // A operand of K5 (box 64 x 256)
+  CUtensorMap tm_gu64;  // A operand of K5 on CTA pairs (box 64 x 64)
   CUtensorMap tm_dn;    // A operand of K6 (box 64 x 128)
   CUtensorMap tm_router;  // A operand of the tensor-core router (box 64 x 128)
   // stage timers: capacity x (MOE_NUM_STAGES + 1) events, filled in order
@@ -197,7 +198,7 @@ int moe_config_check(const moe_config_t* c) {
     return MOE_ERR_INVALID_ARG;
   if (c->top_k > c->num_experts) return MOE_ERR_INVALID_ARG;
   if (c->hidden % 128 != 0 || c->hidden > 16384) return MOE_ERR_UNSUPPORTED;
-  if (c->num_experts > 1024 || c->top_k > 32 || c->intermediate > 8192) return MOE_ERR_UNSUPPORTED;
+  if (c->num_experts > moe::kMaxGroups - 1 || c->top_k > 32 || c->intermediate > 8192) return MOE_ERR_UNSUPPORTED;
   if (c->shared_intermediate != c->intermediate) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -220,7 +221,9 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
   }
   const size_t H = cfg->hidden, E = cfg->num_experts, Ip = L->I_pad;
   const size_t gu_bytes = (E + 1) * 2 * Ip * H * 2, dn_bytes = (E + 1) * H * Ip * 2;
-  if (moe::gemm_configure_device() != cudaSuccess || moe::topk_configure_device() != cudaSuccess ||
+  if (moe::gemm_configure_device() != cudaSuccess ||
+      moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
+      moe::topk_configure_device() != cudaSuccess ||
       cudaMalloc(&L->w_gu, gu_bytes) != cudaSuccess ||
       cudaMalloc(&L->w_dn, dn_bytes) != cudaSuccess ||
       cudaMalloc(&L->router_w, H * E * sizeof(float)) != cudaSuccess ||
@@ -233,6 +236,7 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
     return MOE_ERR_CUDA;
   }
   if (!encode_bf16_2d(&L->tm_gu, L->w_gu, (E + 1) * 2 * Ip, H, 2 * moe::kBM) ||
+      !encode_bf16_2d(&L->tm_gu64, L->w_gu, (E + 1) * 2 * Ip, H, 64) ||
       !encode_bf16_2d(&L->tm_dn, L->w_dn, (E + 1) * H, Ip, moe::kBM) ||
       !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM)) {
     moe_destroy(L);
@@ -327,14 +331,21 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + w.h);
   __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(ws + w.y);
 
-  // expert-GEMM weight tiles: gate|up one 128-feature block, down one or two
+  // expert-GEMM tiles: on one SM, 128 tokens x gate|up one 128-feature block
+  // (down one or two); on CTA pairs (large T), 256 tokens x gate|up 128
+  // features (down 256)
+  const bool pair_gu = T >= moe::kPairMinTokens;
+  const bool pair_dn = T >= moe::kPairMinTokens && (H / moe::kBM) % 2 == 0;
   const int dn_blocks = moe::gemm_down_blocks(H);
-  const int mt_gu = Ip / moe::kBM, mt_dn = H / moe::kBM / dn_blocks;
+  const int bn_gu = pair_gu ? 2 * moe::kBN : moe::kBN;
+  const int bn_dn = pair_dn ? 2 * moe::kBN : moe::kBN;
+  const int mt_gu = Ip / moe::kBM;
+  const int mt_dn = pair_dn ? H / (2 * moe::kBM) : H / moe::kBM / dn_blocks;
 
   // Token-row operands, each with kBBoxRows- and kBN-row boxes: x_perm (or x
   // for the shared expert) for K5 and the router, h for K6.
   moe::GemmMaps gu{}, dn{}, rt{};
-  gu.a = L->tm_gu;
+  gu.a = pair_gu ? L->tm_gu64 : L->tm_gu;
   dn.a = L->tm_dn;
   rt.a = L->tm_router;
   if (!encode_bf16_2d(&gu.b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
@@ -396,7 +407,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
                             st, routing != nullptr ? routing->logits : nullptr,
                             tc_router ? &refine : nullptr));
   MOE_CUDA(mark(2));
-  MOE_CUDA(moe::launch_sort(topk_idx, topk_w, T, k, E, moe::kBN, mt_gu, mt_dn, masks,
+  MOE_CUDA(moe::launch_sort(topk_idx, topk_w, T, k, E, bn_gu, bn_dn, mt_gu, mt_dn, masks,
                             chunk_cnt, chunk_base, counts, row_start, tiles_gu, tiles_dn, perm, pos,
                             w_perm, st));
   MOE_CUDA(mark(3));
@@ -413,7 +424,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.limit_shared = c.swiglu_limit_shared;
 
   p.tile_start = tiles_gu;
-  p.num_kb = H / moe::kBK;
+  p.num_kb = H / (pair_gu ? 2 * moe::kBK : moe::kBK);
   p.m_tiles = mt_gu;
   p.a_rows_per_group = 2 * Ip;
   p.shared_b_row0 = xb ? 0 : T * k;
@@ -421,11 +432,12 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.out_ld = Ip;
   p.out_feats = Ip;
   p.w_perm = nullptr;
-  MOE_CUDA(moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
+  MOE_CUDA(pair_gu ? moe::launch_gemm_gate_up_pair(gu, p, st)
+                : moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
   MOE_CUDA(mark(5));
 
   p.tile_start = tiles_dn;
-  p.num_kb = Ip / moe::kBK;
+  p.num_kb = Ip / (pair_dn ? 2 * moe::kBK : moe::kBK);
   p.m_tiles = mt_dn;
   p.a_rows_per_group = H;
   p.shared_b_row0 = T * k;
@@ -433,7 +445,8 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.out_ld = H;
   p.out_feats = H;
   p.w_perm = w_perm;
-  MOE_CUDA(moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
+  MOE_CUDA(pair_dn ? moe::launch_gemm_down_pair(dn, p, st)
+                : moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
   MOE_CUDA(mark(6));
   MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, out, st));
   MOE_CUDA(mark(7));

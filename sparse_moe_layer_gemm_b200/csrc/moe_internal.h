@@ -22,6 +22,9 @@ constexpr int kRouterTok = 64;
 constexpr int kRouterExp = 96;
 constexpr int kRouterKStep = 32;
 
+// Groups (routed experts + the shared one) the grouped GEMM supports.
+constexpr int kMaxGroups = 1025;
+
 // Chunk of tokens owned by one block of the counting sort (4 x 32-bit masks).
 constexpr int kSortChunk = 128;
 
@@ -29,6 +32,10 @@ constexpr int kSortChunk = 128;
 constexpr int kModeGateUp = 0;  // h = silu(clamp(gate)) * clamp(up), bf16
 constexpr int kModeDown = 1;    // y = acc * w_perm[row], bf16
 constexpr int kModeRouter = 2;  // logits = acc, fp32, features < valid_feats
+
+// Token count from which the expert GEMMs run on CTA pairs (2-SM UMMA,
+// 256-token tiles; needs an even number of 128-feature blocks in H).
+constexpr int kPairMinTokens = 2048;
 
 // Token count from which the router runs on the tensor cores (bf16 x only).
 constexpr int kTcRouterMinTokens = 512;
@@ -81,8 +88,8 @@ cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router
 cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, const float* bias,
                         bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st,
                         float* logits_out = nullptr, const TopkRefine* refine = nullptr);
-cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn,
-                        int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
+cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn_gu,
+                        int bn_dn, int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
                         int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
                         int* pos, float* w_perm, cudaStream_t st);
 cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_routed, int k, int T,
@@ -103,6 +110,11 @@ cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid
 cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
                              cudaStream_t st);
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
+// CTA-pair versions (grouped_gemm_pair.cu): m.a has 64-row boxes for gate|up
+// and 128-row boxes for down; tiles of 256 tokens; num_kb = K / 128; m_tiles
+// = I_pad / 128 (gate|up) or H / 256 (down).
+cudaError_t launch_gemm_gate_up_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st);
+cudaError_t launch_gemm_down_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st);
 cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
                                float* dst_t, cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k, int H, bool out_bf16,
@@ -114,6 +126,8 @@ cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int 
 
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t gemm_configure_device();
+// also sizes the pair kernels' grid to the co-resident 2-CTA clusters
+cudaError_t gemm_pair_configure_device(int num_sms);
 cudaError_t topk_configure_device();
 
 

@@ -49,9 +49,10 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int* __restrict__ 
 
 // Warp-wide exclusive prefix over the G = E + 1 groups of the row counts and
 // of the GEMM tile counts (ceil(rows / bn) token tiles x m_tiles weight
-// tiles).  Called by one full warp; cnt_s holds the G row counts.  When
+// tiles, with each GEMM's own bn).  Called by one full warp; cnt_s holds
+// the G row counts.  When
 // start_s is given, the row starts are also left there for the caller.
-__device__ void scan_groups(const int* cnt_s, int G, int bn, int mt_gu, int mt_dn,
+__device__ void scan_groups(const int* cnt_s, int G, int bn_gu, int bn_dn, int mt_gu, int mt_dn,
                             int* __restrict__ counts,
                             int* __restrict__ row_start, int* __restrict__ tiles_gu,
                             int* __restrict__ tiles_dn, int* start_s) {
@@ -61,10 +62,9 @@ __device__ void scan_groups(const int* cnt_s, int G, int bn, int mt_gu, int mt_d
   int s_rows = 0, s_gu = 0, s_dn = 0;
   for (int g = g0; g < g1; ++g) {
     const int n = cnt_s[g];
-    const int nt = (n + bn - 1) / bn;
     s_rows += n;
-    s_gu += nt * mt_gu;
-    s_dn += nt * mt_dn;
+    s_gu += (n + bn_gu - 1) / bn_gu * mt_gu;
+    s_dn += (n + bn_dn - 1) / bn_dn * mt_dn;
   }
   int i_rows = s_rows, i_gu = s_gu, i_dn = s_dn;
 #pragma unroll
@@ -81,15 +81,14 @@ __device__ void scan_groups(const int* cnt_s, int G, int bn, int mt_gu, int mt_d
   int b_rows = i_rows - s_rows, b_gu = i_gu - s_gu, b_dn = i_dn - s_dn;
   for (int g = g0; g < g1; ++g) {
     const int n = cnt_s[g];
-    const int nt = (n + bn - 1) / bn;
     counts[g] = n;
     row_start[g] = b_rows;
     if (start_s != nullptr) start_s[g] = b_rows;
     tiles_gu[g] = b_gu;
     tiles_dn[g] = b_dn;
     b_rows += n;
-    b_gu += nt * mt_gu;
-    b_dn += nt * mt_dn;
+    b_gu += (n + bn_gu - 1) / bn_gu * mt_gu;
+    b_dn += (n + bn_dn - 1) / bn_dn * mt_dn;
   }
   if (lane == 31) {
     row_start[G] = i_rows;
@@ -101,7 +100,7 @@ __device__ void scan_groups(const int* cnt_s, int G, int bn, int mt_gu, int mt_d
 // One block.  Per expert: running offsets of the chunks; then warp 0 forms
 // the prefixes over the groups.
 __global__ void __launch_bounds__(1024) sort_scan_kernel(
-    const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int bn, int mt_gu, int mt_dn,
+    const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int bn_gu, int bn_dn, int mt_gu, int mt_dn,
     int* __restrict__ chunk_base, int* __restrict__ counts, int* __restrict__ row_start,
     int* __restrict__ tiles_gu, int* __restrict__ tiles_dn) {
   __shared__ int cnt_s[1025];
@@ -116,7 +115,7 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(
   if (threadIdx.x == 0) cnt_s[E] = T;
   __syncthreads();
   if (threadIdx.x < 32)
-    scan_groups(cnt_s, E + 1, bn, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, nullptr);
+    scan_groups(cnt_s, E + 1, bn_gu, bn_dn, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, nullptr);
 }
 
 // Rank of token tl among the tokens of this chunk that chose the expert whose
@@ -131,7 +130,7 @@ __device__ __forceinline__ int chunk_rank(const uint32_t* m, int tl) {
 // T <= kSortChunk (decode): histogram, prefixes and stable scatter in one block.
 __global__ void __launch_bounds__(1024) sort_small_kernel(
     const int* __restrict__ topk_idx, const float* __restrict__ topk_w, int T, int k, int E,
-    int bn, int mt_gu, int mt_dn, int* __restrict__ counts, int* __restrict__ row_start,
+    int bn_gu, int bn_dn, int mt_gu, int mt_dn, int* __restrict__ counts, int* __restrict__ row_start,
     int* __restrict__ tiles_gu, int* __restrict__ tiles_dn, int* __restrict__ perm,
     int* __restrict__ pos, float* __restrict__ w_perm) {
   extern __shared__ uint32_t sm[];
@@ -156,7 +155,7 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(
   if (threadIdx.x == 0) cnt_s[E] = T;
   __syncthreads();
   if (threadIdx.x < 32)
-    scan_groups(cnt_s, E + 1, bn, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, start_s);
+    scan_groups(cnt_s, E + 1, bn_gu, bn_dn, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, start_s);
   __syncthreads();
   for (int p = threadIdx.x; p < T * k; p += blockDim.x) {
     const int tl = p / k;
@@ -241,15 +240,15 @@ __global__ void __launch_bounds__(256) gather_kernel(const TX* __restrict__ x,
 
 }  // namespace
 
-cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn,
-                        int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
+cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn_gu,
+                        int bn_dn, int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
                         int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
                         int* pos, float* w_perm, cudaStream_t st) {
   const int nch = (T + kSortChunk - 1) / kSortChunk;
   const size_t smem = static_cast<size_t>(E) * kMaskWords * sizeof(uint32_t);
   if (nch == 1) {
     const size_t smem1 = smem + 2 * static_cast<size_t>(E + 1) * sizeof(int);
-    sort_small_kernel<<<1, 1024, smem1, st>>>(topk_idx, topk_w, T, k, E, bn, m_tiles_gu, m_tiles_dn,
+    sort_small_kernel<<<1, 1024, smem1, st>>>(topk_idx, topk_w, T, k, E, bn_gu, bn_dn, m_tiles_gu, m_tiles_dn,
                                               counts, row_start, tiles_gu, tiles_dn, perm, pos,
                                               w_perm);
     return cudaGetLastError();
@@ -257,7 +256,7 @@ cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, 
   sort_hist_kernel<<<nch, 256, smem, st>>>(topk_idx, T, k, E, masks, chunk_cnt);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  sort_scan_kernel<<<1, 1024, 0, st>>>(chunk_cnt, nch, T, k, E, bn, m_tiles_gu, m_tiles_dn,
+  sort_scan_kernel<<<1, 1024, 0, st>>>(chunk_cnt, nch, T, k, E, bn_gu, bn_dn, m_tiles_gu, m_tiles_dn,
                                        chunk_base,
                                        counts, row_start, tiles_gu, tiles_dn);
   err = cudaGetLastError();
