@@ -17,6 +17,7 @@ constexpr int kTabBytes = (3 * kMaxGroups + 1) * 4;
 
 struct Tile {
   int g, mt, nc, n_valid, nch;  // nch: token blocks of the group
+  int kz;                       // K part (single_rows with k_parts > 1), else 0
 };
 
 // Token blocks per ordering chunk (see decode_tile).
@@ -33,11 +34,13 @@ constexpr int kChunk = 4;
 // stay in L2 from one chunk to the next.
 template <int BN>
 __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
-  int g, local, rows;
+  int g, local, rows, kz = 0;
   if (p.single_rows > 0) {
     g = 0;
-    local = w;
     rows = p.single_rows;
+    const int per_part = p.m_tiles * ((rows + BN - 1) / BN);
+    kz = w / per_part;
+    local = w - kz * per_part;
   } else {
     int lo = 0, hi = p.G;
     while (hi - lo > 1) {
@@ -53,6 +56,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
   }
   Tile t;
   t.g = g;
+  t.kz = kz;
   t.nch = (rows + BN - 1) / BN;
   const int per_chunk = p.m_tiles * kChunk;
   const int cc = local / per_chunk;
@@ -66,7 +70,8 @@ __device__ __forceinline__ Tile decode_tile(const GemmParams& p, int w) {
 
 template <int BN>
 __device__ __forceinline__ int total_tiles(const GemmParams& p) {
-  if (p.single_rows > 0) return p.m_tiles * ((p.single_rows + BN - 1) / BN);
+  if (p.single_rows > 0)
+    return (p.k_parts > 1 ? p.k_parts : 1) * p.m_tiles * ((p.single_rows + BN - 1) / BN);
   return p.tile_start[p.G];
 }
 

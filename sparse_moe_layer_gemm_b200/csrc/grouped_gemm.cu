@@ -8,9 +8,9 @@
 //                  shared rows), stored bf16.
 //   K1 (router, large T):  logits = x . W_r on the bf16 tensor cores: W_r =
 //                  W1 + W2 + W3 split into three bf16 terms concatenated along
-//                  K, so one accumulation over 3H gives x.W1 + x.W2 + x.W3
-//                  (each bf16 x bf16 product is exact in fp32; x is bf16);
-//                  stored fp32.
+//                  K; the tiles of part z accumulate x . Wz (each bf16 x bf16
+//                  product is exact in fp32; x is bf16) and store it, fp32,
+//                  as partial z; the top-k adds the three parts.
 //
 // The expert FFN is the SwiGLU of sglang-jax issue #1367 "Support Step 3.5
 // Flash", section "Model configuration" (MoE bullet; clamped SwiGLU via
@@ -85,7 +85,7 @@ struct Shape {
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(TAB_OFFSET) + TAB_BYTES;
   static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
   static_assert(NBUF * ACC_COLS <= 512, "TMEM capacity");
-  static_assert(BN == 128, "token tile (the wide token-row box is BN rows)");
+  static_assert(BN % kBN == 0, "token tile: whole wide (kBN-row) token-row boxes");
   static_assert(A_ROWS % A_BOX == 0 && ACCS % NI == 0, "A boxes, issuer split");
   static_assert(STAGES >= 2, "pipeline depth");
   static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay aligned");
@@ -185,13 +185,17 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
         if (*abort_flag) break;
         const Tile t = decode_tile<BN>(gp, w);
         const int n_mma = (t.n_valid + 15) & ~15;
-        const bool wide = n_mma > kBBoxRows;  // one BN-row box, else one kBBoxRows-row box
+        // token rows: kBN-row boxes (as many as the MMA's N needs), else one
+        // kBBoxRows-row box
+        const bool wide = n_mma > kBBoxRows;
+        const int nbox = wide ? (n_mma + kBN - 1) / kBN : 1;
         const bool sh = GU && t.g == p.E;
         const CUtensorMap* mb = wide ? (sh ? &tmBshw : &tmBw) : (sh ? &tmBsh : &tmB);
         const int b_row = (sh ? p.shared_b_row0 : group_row0(gp, t.g)) + t.nc * BN;
         const int a_row = t.g * p.a_rows_per_group + t.mt * S::A_ROWS;
-        const uint32_t bytes = S::A_BYTES + (wide ? S::B_BYTES : S::B_BOX_BYTES);
+        const uint32_t bytes = S::A_BYTES + (wide ? nbox * kBN * S::ROW : S::B_BOX_BYTES);
         const uint64_t pol_a = t.nch > 1 ? pol_normal : pol_first;
+        const int a_k0 = t.kz * p.num_kb * BK;  // K part of a split-K tile
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           const uint32_t s = it % S::STAGES;
@@ -205,9 +209,10 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
           const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
 #pragma unroll
           for (int i = 0; i < S::A_LOADS; ++i)
-            tma_load_2d(sa + i * S::A_BOX * S::ROW, &tmA, fb, kb * BK, a_row + i * S::A_BOX, pol_a);
-          const int bk = p.b_k_wrap > 0 ? (kb * BK) % p.b_k_wrap : kb * BK;
-          tma_load_2d(sa + S::A_BYTES, mb, fb, bk, b_row, pol_b);
+            tma_load_2d(sa + i * S::A_BOX * S::ROW, &tmA, fb, a_k0 + kb * BK, a_row + i * S::A_BOX,
+                        pol_a);
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d(sa + S::A_BYTES + i * kBN * S::ROW, mb, fb, kb * BK, b_row + i * kBN, pol_b);
           ++it;
         }
         if (!ok) break;
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
         const int feat = (t.mt * BLOCKS + b) * kBM + q * 32 + lane;
         if ((t.mt * BLOCKS + b) * kBM >= p.out_feats) break;  // never past the output
         if (MODE == kModeRouter) {
-          float* lp = p.out_f32 + row0 * p.out_ld + feat;
+          float* lp = p.out_f32 + t.kz * p.part_stride + row0 * p.out_ld + feat;
           const bool keep = feat < p.valid_feats;
           for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
             uint32_t ra[16];

@@ -79,7 +79,11 @@ WsLayout ws_layout(const moe_layer* L, int T) {
     off = align_up(off + bytes, kAlign);
     return at;
   };
-  w.partial = take(static_cast<size_t>(w.ksplit) * T * E * sizeof(float));
+  // partial logits: the CUDA-core router's K splits, or the tensor-core
+  // router's three parts
+  const bool tc_router = c.act_dtype == MOE_BF16 && T >= moe::kTcRouterMinTokens;
+  const int parts = tc_router ? moe::kRouterTcParts : w.ksplit;
+  w.partial = take(static_cast<size_t>(parts) * T * E * sizeof(float));
   w.topk_idx = take(static_cast<size_t>(T) * k * sizeof(int));
   w.topk_w = take(static_cast<size_t>(T) * k * sizeof(float));
   w.masks = take(static_cast<size_t>(w.nch) * E * 4 * sizeof(uint32_t));
@@ -379,21 +383,24 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   moe::TopkRefine refine{};
   const bool tc_router = xb && T >= moe::kTcRouterMinTokens;
   if (tc_router) {
-    // tensor-core router: one group of T rows, 3H reduction over W1 | W2 | W3
+    // tensor-core router: one group of T rows; the K = 3H reduction over
+    // W1 | W2 | W3 runs as three parts (three times the tiles, a third of the
+    // k-blocks each), summed in fixed order by the top-k
     GemmParams r{};
     r.single_rows = T;
     r.E = E;
-    r.num_kb = 3 * H / moe::kBK;
+    r.num_kb = H / moe::kBK;
     r.m_tiles = L->E_pad / moe::kBM;
-    r.b_k_wrap = H;
+    r.k_parts = moe::kRouterTcParts;
+    r.part_stride = static_cast<size_t>(T) * E;
     r.out_f32 = partial;
     r.out_ld = E;
     r.valid_feats = E;
     r.out_feats = E;
     r.status = L->status;
-    const int tiles = r.m_tiles * ((T + moe::kBN - 1) / moe::kBN);
+    const int tiles = r.k_parts * r.m_tiles * ((T + moe::kBN - 1) / moe::kBN);
     MOE_CUDA(moe::launch_gemm_router(rt, r, tiles < L->num_sms ? tiles : L->num_sms, st));
-    ksplit = 1;
+    ksplit = moe::kRouterTcParts;
     refine.x = static_cast<const __nv_bfloat16*>(x);
     refine.w_t = L->router_t;
     refine.H = H;

@@ -37,8 +37,10 @@ constexpr int kModeRouter = 2;  // logits = acc, fp32, features < valid_feats
 // 256-token tiles; needs an even number of 128-feature blocks in H).
 constexpr int kPairMinTokens = 2048;
 
-// Token count from which the router runs on the tensor cores (bf16 x only).
+// Token count from which the router runs on the tensor cores (bf16 x only),
+// and the K parts of its reduction (the three bf16 terms of W_r).
 constexpr int kTcRouterMinTokens = 512;
+constexpr int kRouterTcParts = 3;
 
 struct GemmParams {
   int single_rows;        // > 0: one group of this many rows starting at row 0
@@ -59,7 +61,10 @@ struct GemmParams {
   float limit;            // gate/up clamp of routed experts (<= 0: none)
   float limit_shared;     // gate/up clamp of the shared expert
   int* status;            // device status word
-  int b_k_wrap;           // > 0: B's K coordinate wraps at this value (router)
+  int k_parts;            // single_rows: > 1 splits K into this many parts of num_kb
+                          // k-blocks (A's K offset z * num_kb * kBK, B's 0), each part
+                          // stored at out_f32 + z * part_stride (router: W1 | W2 | W3)
+  size_t part_stride;
   float* out_f32;         // router: logits [rows, out_ld]
   int valid_feats;        // router: features (experts) actually stored
 };
