@@ -74,9 +74,11 @@ def _traffic_record(kernel: str, workload: str, groups: int):
             f = line.split()
             if not f or f[0].startswith("#") or f[0] != f"{kernel}:{workload}":
                 continue
-            src = os.path.join(ROOT, f[1])
-            h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-            return int(f[3]) * groups if h == f[2] else None
+            # the kernel's sources, comma-separated: their bytes hashed in order
+            h = hashlib.sha256()
+            for src in f[1].split(","):
+                h.update(open(os.path.join(ROOT, src), "rb").read())
+            return int(f[3]) * groups if h.hexdigest() == f[2] else None
     except Exception:
         return None
     return None
@@ -261,7 +263,9 @@ def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step):
         ach = gu_flops / (gu_ms * 1e-3) / 1e12
         rl = {"bound": "tensor", "achieved": ach, "peak": peaks["tc"], "unit": "TFLOP/s",
               "frac": ach / peaks["tc"]}
-    rl.update({"kernel": "grouped_gemm_kernel<gate_up>", "kernel_ms": gu_ms,
+    # from 2048 tokens the library runs the expert GEMMs on CTA pairs
+    kname = "grouped_gemm_pair_kernel<gate_up>" if wl.T >= 2048 else "grouped_gemm_kernel<gate_up>"
+    rl.update({"kernel": kname, "kernel_ms": gu_ms,
                "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json)"
                if peaks["source"] == "measured" else "fallback",
