@@ -327,11 +327,15 @@ def run_ours(a):
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms, stages = _measure(layer, x, a.steps, 0, stream)
+    ms, _ = _measure(layer, x, a.steps, 0, stream, record_stages=False)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     ms = max_over_ranks(ms, dev)
+    # per-stage durations (and the dominant kernel's) from a second pass of
+    # the same K steps with CUDA events between the kernels; kept out of the
+    # timed region above because the events themselves cost ~4 % at T=64
+    _, stages = _measure(layer, x, a.steps, 0, stream, record_stages=True)
     err = layer.device_error()
     if err != 0:
         raise RuntimeError(f"device status word {err}")
@@ -376,8 +380,10 @@ def run_ours(a):
         x2 = draw_x(rank_batch_workload(wl2, rank), dev)
         touched2, _ = _routing_stats(layer, x2)
         barrier()
-        ms2, st2 = _measure(layer, x2, max(3, a.steps // 10), max(3, a.warmup), stream)
+        ms2, _ = _measure(layer, x2, max(3, a.steps // 10), max(3, a.warmup), stream,
+                          record_stages=False)
         ms2 = max_over_ranks(ms2, dev)
+        _, st2 = _measure(layer, x2, max(3, a.steps // 10), 0, stream)
         kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2)
         secondary.append({"workload": wl2.name, "T": wl2.T, "value": job_throughput(wl2.T, world, ms2),
                           "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,

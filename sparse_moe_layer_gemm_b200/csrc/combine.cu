@@ -5,6 +5,7 @@
 // expert).  Summed in fp32 in the fixed order j = 0..k-1 then the shared
 // row, rounded once to the output dtype: deterministic.
 #include "moe_internal.h"
+#include "moe_ptx.cuh"
 
 namespace moe {
 
@@ -38,6 +39,7 @@ template <typename TO>
 __global__ void __launch_bounds__(512) combine_kernel(const __nv_bfloat16* __restrict__ y,
                                                       const int* __restrict__ pos, int T, int k,
                                                       int H, TO* __restrict__ out) {
+  pdl_wait();  // the previous kernel's results are visible
   __shared__ int rows[33];
   const int t = blockIdx.x;
   if (threadIdx.x < k) rows[threadIdx.x] = pos[static_cast<size_t>(t) * k + threadIdx.x];
@@ -57,11 +59,10 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k,
                            void* out, cudaStream_t st) {
   const int threads = min(512, max(32, H / 8));
   if (out_bf16)
-    combine_kernel<__nv_bfloat16><<<T, threads, 0, st>>>(y, pos, T, k, H,
-                                                          static_cast<__nv_bfloat16*>(out));
-  else
-    combine_kernel<float><<<T, threads, 0, st>>>(y, pos, T, k, H, static_cast<float*>(out));
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(T), dim3(threads), 0, st, y, pos, T, k, H,
+                      static_cast<__nv_bfloat16*>(out));
+  return launch_pdl(combine_kernel<float>, dim3(T), dim3(threads), 0, st, y, pos, T, k, H,
+                    static_cast<float*>(out));
 }
 
 }  // namespace moe

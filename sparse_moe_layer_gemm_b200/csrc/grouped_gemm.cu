@@ -135,9 +135,6 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // group tables in shared memory (visible after the __syncthreads below)
-  const GemmParams gp =
-      MODE != kModeRouter ? stage_group_tables(p, reinterpret_cast<int*>(smem + S::TAB_OFFSET)) : p;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
@@ -165,6 +162,12 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), S::TMEM_COLS);
     tmem_relinquish();
   }
+  // everything above touched only this CTA's resources; from here on the
+  // previous kernel's outputs are read
+  pdl_wait();
+  // group tables in shared memory (visible after the __syncthreads below)
+  const GemmParams gp =
+      MODE != kModeRouter ? stage_group_tables(p, reinterpret_cast<int*>(smem + S::TAB_OFFSET)) : p;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -434,26 +437,22 @@ cudaError_t gemm_configure_device() {
 int gemm_down_blocks(int H) { return (H / kBM) % 2 == 0 ? 2 : 1; }
 
 cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
-  grouped_gemm_kernel<kModeGateUp, 1, 128>
-      <<<grid, GuCfg::THREADS, GuCfg::SMEM, st>>>(m.a, m.b, m.bsh, m.bw, m.bshw, m.out, p);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<kModeGateUp, 1, 128>, dim3(grid), dim3(GuCfg::THREADS),
+                    GuCfg::SMEM, st, m.a, m.b, m.bsh, m.bw, m.bshw, m.out, p);
 }
 
 cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
                              cudaStream_t st) {
   if (blocks == 2)
-    grouped_gemm_kernel<kModeDown, 2, 128>
-        <<<grid, DnCfg2::THREADS, DnCfg2::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, m.out, p);
-  else
-    grouped_gemm_kernel<kModeDown, 1, 128>
-        <<<grid, DnCfg1::THREADS, DnCfg1::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, m.out, p);
-  return cudaGetLastError();
+    return launch_pdl(grouped_gemm_kernel<kModeDown, 2, 128>, dim3(grid), dim3(DnCfg2::THREADS),
+                      DnCfg2::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
+  return launch_pdl(grouped_gemm_kernel<kModeDown, 1, 128>, dim3(grid), dim3(DnCfg1::THREADS),
+                    DnCfg1::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
-  grouped_gemm_kernel<kModeRouter, 1, 128>
-      <<<grid, RtCfg::THREADS, RtCfg::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, m.out, p);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<kModeRouter, 1, 128>, dim3(grid), dim3(RtCfg::THREADS),
+                    RtCfg::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 
 }  // namespace moe

@@ -117,7 +117,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
-  const GemmParams gp = stage_group_tables(p, reinterpret_cast<int*>(smem + S::TAB_OFFSET));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
@@ -145,6 +144,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
     tmem_alloc_pair(smem_u32(tmem_slot), S::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  // everything above touched only this pair's resources; from here on the
+  // previous kernel's outputs are read
+  pdl_wait();
+  const GemmParams gp = stage_group_tables(p, reinterpret_cast<int*>(smem + S::TAB_OFFSET));
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers initialised before any remote use
@@ -455,16 +458,15 @@ int gemm_pair_grid() { return g_pair_grid; }
 
 cudaError_t launch_gemm_gate_up_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   if (g_pair_grid <= 0) return cudaErrorInvalidConfiguration;
-  grouped_gemm_pair_kernel<kModeGateUp, 2>
-      <<<g_pair_grid, GuPair::THREADS, GuPair::SMEM, st>>>(m.a, m.b, m.bsh, m.bw, m.bshw, m.out, p);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_pair_kernel<kModeGateUp, 2>, dim3(g_pair_grid),
+                    dim3(GuPair::THREADS), GuPair::SMEM, st, m.a, m.b, m.bsh, m.bw, m.bshw, m.out,
+                    p);
 }
 
 cudaError_t launch_gemm_down_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   if (g_pair_grid <= 0) return cudaErrorInvalidConfiguration;
-  grouped_gemm_pair_kernel<kModeDown, 2>
-      <<<g_pair_grid, DnPair::THREADS, DnPair::SMEM, st>>>(m.a, m.b, m.b, m.bw, m.bw, m.out, p);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_pair_kernel<kModeDown, 2>, dim3(g_pair_grid),
+                    dim3(DnPair::THREADS), DnPair::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 
 }  // namespace moe

@@ -129,6 +129,24 @@ cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, i
 cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
                              __nv_bfloat16* dst, cudaStream_t st);
 
+// Launches `kernel` on `st` with programmatic stream serialization, so it may
+// start (up to its pdl_wait) while the previous kernel of the stream ends.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t gemm_configure_device();
 // also sizes the pair kernels' grid to the co-resident 2-CTA clusters

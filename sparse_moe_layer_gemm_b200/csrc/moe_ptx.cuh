@@ -27,6 +27,17 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- launch order
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization is launched as the previous kernel of the stream retires its
+// CTAs, and runs its prologue (barriers, TMEM, tensor-map prefetch) while that
+// kernel's tail finishes; pdl_wait blocks until the previous kernel has
+// completed and its memory operations are visible.  (No kernel triggers its
+// dependents early: measured, an early trigger made the small kernels'
+// successors occupy SMs while they still ran.)  A no-op for a kernel launched
+// without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -14,6 +14,7 @@
 // popcount of the mask bits below its token, so the scatter is stable and
 // bit-reproducible.
 #include "moe_internal.h"
+#include "moe_ptx.cuh"
 
 namespace moe {
 
@@ -24,6 +25,7 @@ constexpr int kMaskWords = kSortChunk / 32;  // 4
 __global__ void __launch_bounds__(256) sort_hist_kernel(const int* __restrict__ topk_idx, int T,
                                                         int k, int E, uint32_t* __restrict__ masks,
                                                         int* __restrict__ chunk_cnt) {
+  pdl_wait();  // the previous kernel's results are visible
   extern __shared__ uint32_t sm[];
   const int c = blockIdx.x;
   const int t0 = c * kSortChunk;
@@ -103,6 +105,7 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(
     const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int bn_gu, int bn_dn, int mt_gu, int mt_dn,
     int* __restrict__ chunk_base, int* __restrict__ counts, int* __restrict__ row_start,
     int* __restrict__ tiles_gu, int* __restrict__ tiles_dn) {
+  pdl_wait();  // the previous kernel's results are visible
   __shared__ int cnt_s[1025];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
@@ -133,6 +136,7 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(
     int bn_gu, int bn_dn, int mt_gu, int mt_dn, int* __restrict__ counts, int* __restrict__ row_start,
     int* __restrict__ tiles_gu, int* __restrict__ tiles_dn, int* __restrict__ perm,
     int* __restrict__ pos, float* __restrict__ w_perm) {
+  pdl_wait();  // the previous kernel's results are visible
   extern __shared__ uint32_t sm[];
   uint32_t* masks = sm;                                   // [E][4]
   int* cnt_s = reinterpret_cast<int*>(sm + E * kMaskWords);  // [E + 1]
@@ -174,6 +178,7 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(
     const uint32_t* __restrict__ masks, const int* __restrict__ chunk_base,
     const int* __restrict__ row_start, int* __restrict__ perm, int* __restrict__ pos,
     float* __restrict__ w_perm) {
+  pdl_wait();  // the previous kernel's results are visible
   extern __shared__ uint32_t sm[];
   const int c = blockIdx.x;
   const int t0 = c * kSortChunk;
@@ -221,6 +226,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const TX* __restrict__ x,
                                                      int rows_routed, int k, int T, int H,
                                                      int write_shared,
                                                      __nv_bfloat16* __restrict__ xp) {
+  pdl_wait();  // the previous kernel's results are visible
   const int lane = threadIdx.x & 31;
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -248,22 +254,18 @@ cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, 
   const size_t smem = static_cast<size_t>(E) * kMaskWords * sizeof(uint32_t);
   if (nch == 1) {
     const size_t smem1 = smem + 2 * static_cast<size_t>(E + 1) * sizeof(int);
-    sort_small_kernel<<<1, 1024, smem1, st>>>(topk_idx, topk_w, T, k, E, bn_gu, bn_dn, m_tiles_gu, m_tiles_dn,
-                                              counts, row_start, tiles_gu, tiles_dn, perm, pos,
-                                              w_perm);
-    return cudaGetLastError();
+    return launch_pdl(sort_small_kernel, dim3(1), dim3(1024), smem1, st, topk_idx, topk_w, T, k, E,
+                      bn_gu, bn_dn, m_tiles_gu, m_tiles_dn, counts, row_start, tiles_gu, tiles_dn,
+                      perm, pos, w_perm);
   }
-  sort_hist_kernel<<<nch, 256, smem, st>>>(topk_idx, T, k, E, masks, chunk_cnt);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(sort_hist_kernel, dim3(nch), dim3(256), smem, st, topk_idx, T, k, E,
+                               masks, chunk_cnt);
   if (err != cudaSuccess) return err;
-  sort_scan_kernel<<<1, 1024, 0, st>>>(chunk_cnt, nch, T, k, E, bn_gu, bn_dn, m_tiles_gu, m_tiles_dn,
-                                       chunk_base,
-                                       counts, row_start, tiles_gu, tiles_dn);
-  err = cudaGetLastError();
+  err = launch_pdl(sort_scan_kernel, dim3(1), dim3(1024), 0, st, chunk_cnt, nch, T, k, E, bn_gu,
+                   bn_dn, m_tiles_gu, m_tiles_dn, chunk_base, counts, row_start, tiles_gu, tiles_dn);
   if (err != cudaSuccess) return err;
-  sort_scatter_kernel<<<nch, 256, smem, st>>>(topk_idx, topk_w, T, k, E, masks, chunk_base,
-                                              row_start, perm, pos, w_perm);
-  return cudaGetLastError();
+  return launch_pdl(sort_scatter_kernel, dim3(nch), dim3(256), smem, st, topk_idx, topk_w, T, k, E,
+                    masks, chunk_base, row_start, perm, pos, w_perm);
 }
 
 cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_routed, int k, int T,
@@ -273,13 +275,12 @@ cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_
   const int want = (nrows + 7) / 8;
   const int blocks = max(1, min(want, num_sms * 8));
   if (x_bf16)
-    gather_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), perm,
-                                                         rows_routed, k, T, H, write_shared ? 1 : 0,
-                                                         x_perm);
-  else
-    gather_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), perm, rows_routed, k,
-                                                 T, H, write_shared ? 1 : 0, x_perm);
-  return cudaGetLastError();
+    return launch_pdl(gather_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(x), perm, rows_routed, k, T, H,
+                      write_shared ? 1 : 0, x_perm);
+  return launch_pdl(gather_kernel<float>, dim3(blocks), dim3(256), 0, st,
+                    static_cast<const float*>(x), perm, rows_routed, k, T, H, write_shared ? 1 : 0,
+                    x_perm);
 }
 
 }  // namespace moe

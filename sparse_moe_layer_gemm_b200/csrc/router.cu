@@ -12,6 +12,7 @@
 #include <math.h>
 
 #include "moe_internal.h"
+#include "moe_ptx.cuh"
 
 namespace moe {
 
@@ -44,6 +45,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const TX* __restrict
                                                             const float* __restrict__ wr,
                                                             float* __restrict__ partial, int T,
                                                             int H, int E, int kchunk) {
+  pdl_wait();  // the previous kernel's results are visible
   __shared__ __align__(16) float xs[kRouterKStep][kRouterTok + 4];
   __shared__ __align__(16) float ws[kRouterKStep][kRouterExp];
   const int e0 = blockIdx.x * kRouterExp;
@@ -195,6 +197,7 @@ __global__ void __launch_bounds__(1024) topk_block_kernel(const float* __restric
                                                     float* __restrict__ topk_w,
                                                     float* __restrict__ logits_out,
                                                     TopkRefine rf) {
+  pdl_wait();  // the previous kernel's results are visible
   __shared__ float s_l[32 * MPL];
   __shared__ float s_sc[32 * MPL];
   __shared__ float s_be[32 * MPL];
@@ -474,6 +477,7 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(
     const float* __restrict__ partial, int ksplit, int T, int E, int k,
     const float* __restrict__ bias, int norm, float scale, int* __restrict__ topk_idx,
     float* __restrict__ topk_w, float* __restrict__ logits_out, TopkRefine rf) {
+  pdl_wait();  // the previous kernel's results are visible
   extern __shared__ float s_bias[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_bias[e] = bias != nullptr ? bias[e] : 0.f;
   __syncthreads();
@@ -654,12 +658,10 @@ cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router
   const int kchunk = H / ksplit;
   dim3 grid((E + kRouterExp - 1) / kRouterExp, (T + kRouterTok - 1) / kRouterTok, ksplit);
   if (x_bf16)
-    router_logits_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), router_w, partial, T, H, E, kchunk);
-  else
-    router_logits_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), router_w,
-                                                       partial, T, H, E, kchunk);
-  return cudaGetLastError();
+    return launch_pdl(router_logits_kernel<__nv_bfloat16>, grid, dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(x), router_w, partial, T, H, E, kchunk);
+  return launch_pdl(router_logits_kernel<float>, grid, dim3(256), 0, st,
+                    static_cast<const float*>(x), router_w, partial, T, H, E, kchunk);
 }
 
 cudaError_t topk_configure_device() {
@@ -686,10 +688,9 @@ cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, c
   if (T < kTopkWarpMinTokens) {
     const int threads = min(1024, max(32, (E + 31) / 32 * 32));
     const size_t smem = rf.band > 0.f ? static_cast<size_t>(rf.H) * sizeof(float) : 0;
-#define MOE_TOPK(N)                                                                     \
-  topk_block_kernel<N><<<T, threads, smem, st>>>(partial, ksplit, T, E, k, bias,        \
-                                                 norm ? 1 : 0, scale, topk_idx, topk_w, \
-                                                 logits_out, rf)
+#define MOE_TOPK(N)                                                                        \
+  return launch_pdl(topk_block_kernel<N>, dim3(T), dim3(threads), smem, st, partial, ksplit, T, E, \
+                    k, bias, norm ? 1 : 0, scale, topk_idx, topk_w, logits_out, rf)
     if (mpl <= 1) MOE_TOPK(1);
     else if (mpl <= 2) MOE_TOPK(2);
     else if (mpl <= 4) MOE_TOPK(4);
@@ -703,10 +704,9 @@ cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, c
   const int blocks = (T + kTopkWarps - 1) / kTopkWarps;
   // router bias, then per warp a list of up to 32 candidates
   const size_t smem = static_cast<size_t>(E) * sizeof(float) + kTopkWarps * 32 * sizeof(int);
-#define MOE_TOPK(N)                                                                          \
-  topk_warp_kernel<N><<<blocks, 32 * kTopkWarps, smem, st>>>(partial, ksplit, T, E, k, bias, \
-                                                             norm ? 1 : 0, scale, topk_idx,  \
-                                                             topk_w, logits_out, rf)
+#define MOE_TOPK(N)                                                                            \
+  return launch_pdl(topk_warp_kernel<N>, dim3(blocks), dim3(32 * kTopkWarps), smem, st, partial,   \
+                    ksplit, T, E, k, bias, norm ? 1 : 0, scale, topk_idx, topk_w, logits_out, rf)
   if (mpl <= 1) MOE_TOPK(1);
   else if (mpl <= 2) MOE_TOPK(2);
   else if (mpl <= 4) MOE_TOPK(4);
