@@ -56,13 +56,17 @@ using namespace gemm;
 template <int MODE, int BLOCKS, int BN_>
 struct Shape {
   static constexpr bool GU = MODE == kModeGateUp;
+  // router with BLOCKS = 2: one weight block, the tile's tokens split into two
+  // halves, one accumulator (and issuer) each
+  static constexpr bool TOKSPLIT = MODE == kModeRouter && BLOCKS == 2;
   static constexpr int BN = BN_;
   static constexpr int BK = kBK;
   static constexpr int ROW = BK * 2;                        // bytes per operand row in SMEM
   static constexpr int ACCS = BLOCKS * (GU ? 2 : 1);       // 128-row accumulators per tile
   static constexpr int NI = ACCS >= 2 ? 2 : 1;             // MMA-issuing warps
   static constexpr int THREADS = 32 * (1 + NI + 4);
-  static constexpr int A_ROWS = kBM * ACCS;
+  static constexpr int A_ROWS = TOKSPLIT ? kBM : kBM * ACCS;
+  static constexpr int ACC_N = TOKSPLIT ? BN / 2 : BN;      // tokens (columns) per accumulator
   static constexpr int A_BOX = GU ? 2 * kBM : kBM;         // rows per A box (the tensor maps')
   static constexpr int A_LOADS = A_ROWS / A_BOX;
   static constexpr int A_BYTES = A_ROWS * ROW;
@@ -70,7 +74,7 @@ struct Shape {
   static constexpr int B_BOX_BYTES = kBBoxRows * ROW;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (200 * 1024 / STAGE_BYTES) < 6 ? (200 * 1024 / STAGE_BYTES) : 6;
-  static constexpr int ACC_COLS = ACCS * BN;                // TMEM columns per accumulator buffer
+  static constexpr int ACC_COLS = ACCS * ACC_N;             // TMEM columns per accumulator buffer
   static constexpr int NBUF = ACC_COLS <= 256 ? 2 : 1;     // double-buffered when it fits
   static constexpr int TMEM_COLS = NBUF * ACC_COLS > 256 ? 512 : 256;
   static constexpr int BAR_BYTES = 256;
@@ -236,8 +240,11 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
         if (*abort_flag) break;
         const Tile t = decode_tile<BN>(gp, w);
-        const int n_mma = (t.n_valid + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
+        // token-split router tiles: this issuer's half of the tokens (none
+        // for a ragged tile's empty second half: it only commits)
+        const int n_me = S::TOKSPLIT ? min(S::ACC_N, max(0, t.n_valid - me * S::ACC_N)) : t.n_valid;
+        const int n_mma = (n_me + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma > 0 ? n_mma : 16);
         const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
         const uint32_t tph = (S::NBUF == 2 ? (tc >> 1) : tc) & 1u;
         if (!mbar_wait(tempty0 + 8 * buf, tph ^ 1u, abort_flag, p.status)) break;
@@ -256,14 +263,21 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
           const uint64_t ad = desc0 + static_cast<uint64_t>((s * S::STAGE_BYTES) >> 4);
           const uint64_t bd = ad + static_cast<uint64_t>(S::A_BYTES >> 4);
           const uint32_t acc0 = kb != 0 ? 1u : 0u;
+          if (n_mma > 0) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
+            for (int kk = 0; kk < BK / 16; ++kk)
 #pragma unroll
-            for (int j = 0; j < S::ACCS / S::NI; ++j) {
-              const int a = j * S::NI + me;
-              mma_issue(d + a * BN, ad + static_cast<uint64_t>((a * kBM * S::ROW + kk * 32) >> 4),
-                        bd + static_cast<uint64_t>((kk * 32) >> 4), idesc, kk == 0 ? acc0 : 1u);
-            }
+              for (int j = 0; j < S::ACCS / S::NI; ++j) {
+                const int a = j * S::NI + me;
+                // accumulator a: its own weight rows, or (token split) its
+                // own half of the token rows
+                const int a_off = S::TOKSPLIT ? 0 : a * kBM * S::ROW;
+                const int b_off = S::TOKSPLIT ? a * S::ACC_N * S::ROW : 0;
+                mma_issue(d + a * S::ACC_N, ad + static_cast<uint64_t>((a_off + kk * 32) >> 4),
+                          bd + static_cast<uint64_t>((b_off + kk * 32) >> 4), idesc,
+                          kk == 0 ? acc0 : 1u);
+              }
+          }
           tc_commit(empty0 + 8 * s);  // frees the stage once these MMAs have read it
           ++it;
         }
@@ -342,18 +356,22 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * S::ACC_COLS;
 #pragma unroll 1
       for (int b = 0; b < BLOCKS; ++b) {
-        const int feat = (t.mt * BLOCKS + b) * kBM + q * 32 + lane;
-        if ((t.mt * BLOCKS + b) * kBM >= p.out_feats) break;  // never past the output
+        const int fblock = S::TOKSPLIT ? t.mt : t.mt * BLOCKS + b;  // 128-feature block
+        const int feat = fblock * kBM + q * 32 + lane;
+        if (fblock * kBM >= p.out_feats) break;  // never past the output
         if (MODE == kModeRouter) {
-          float* lp = p.out_f32 + t.kz * p.part_stride + row0 * p.out_ld + feat;
+          // token split: accumulator b holds tokens [b * ACC_N, (b + 1) * ACC_N)
+          const int tok0 = S::TOKSPLIT ? b * S::ACC_N : 0;
+          const int n_b = S::TOKSPLIT ? min(S::ACC_N, t.n_valid - tok0) : t.n_valid;
+          float* lp = p.out_f32 + t.kz * p.part_stride + (row0 + tok0) * p.out_ld + feat;
           const bool keep = feat < p.valid_feats;
-          for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+          for (int c0 = 0; c0 < n_b; c0 += 16) {
             uint32_t ra[16];
-            tmem_ld_x16(taddr + b * BN + c0, ra);
+            tmem_ld_x16(taddr + b * S::ACC_N + c0, ra);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              if (keep && c0 + i < t.n_valid)
+              if (keep && c0 + i < n_b)
                 lp[static_cast<size_t>(c0 + i) * p.out_ld] = __uint_as_float(ra[i]);
           }
         } else if (GU) {
@@ -415,7 +433,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
 using GuCfg = Shape<kModeGateUp, 1, 128>;
 using DnCfg2 = Shape<kModeDown, 2, 128>;
 using DnCfg1 = Shape<kModeDown, 1, 128>;
-using RtCfg = Shape<kModeRouter, 1, 128>;
+using RtCfg = Shape<kModeRouter, 2, 256>;  // 256-token tiles, one accumulator per half
 
 template <typename S, int MODE, int BLOCKS>
 cudaError_t set_smem() {
@@ -431,7 +449,7 @@ cudaError_t gemm_configure_device() {
   if ((e = set_smem<GuCfg, kModeGateUp, 1>()) != cudaSuccess) return e;
   if ((e = set_smem<DnCfg2, kModeDown, 2>()) != cudaSuccess) return e;
   if ((e = set_smem<DnCfg1, kModeDown, 1>()) != cudaSuccess) return e;
-  return set_smem<RtCfg, kModeRouter, 1>();
+  return set_smem<RtCfg, kModeRouter, 2>();
 }
 
 int gemm_down_blocks(int H) { return (H / kBM) % 2 == 0 ? 2 : 1; }
@@ -451,7 +469,7 @@ cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, i
 }
 
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
-  return launch_pdl(grouped_gemm_kernel<kModeRouter, 1, 128>, dim3(grid), dim3(RtCfg::THREADS),
+  return launch_pdl(grouped_gemm_kernel<kModeRouter, 2, 256>, dim3(grid), dim3(RtCfg::THREADS),
                     RtCfg::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 

@@ -398,7 +398,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
     r.valid_feats = E;
     r.out_feats = E;
     r.status = L->status;
-    const int tiles = r.k_parts * r.m_tiles * ((T + moe::kBN - 1) / moe::kBN);
+    const int tiles = r.k_parts * r.m_tiles * ((T + 2 * moe::kBN - 1) / (2 * moe::kBN));  // 256-token tiles
     MOE_CUDA(moe::launch_gemm_router(rt, r, tiles < L->num_sms ? tiles : L->num_sms, st));
     ksplit = moe::kRouterTcParts;
     refine.x = static_cast<const __nv_bfloat16*>(x);
