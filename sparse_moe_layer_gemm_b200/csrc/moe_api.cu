@@ -228,6 +228,7 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
   if (moe::gemm_configure_device() != cudaSuccess ||
       moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
       moe::topk_configure_device() != cudaSuccess ||
+      moe::gather_configure_device() != cudaSuccess ||
       cudaMalloc(&L->w_gu, gu_bytes) != cudaSuccess ||
       cudaMalloc(&L->w_dn, dn_bytes) != cudaSuccess ||
       cudaMalloc(&L->router_w, H * E * sizeof(float)) != cudaSuccess ||
@@ -418,7 +419,8 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
                             chunk_cnt, chunk_base, counts, row_start, tiles_gu, tiles_dn, perm, pos,
                             w_perm, st));
   MOE_CUDA(mark(3));
-  MOE_CUDA(moe::launch_gather(x, xb, perm, w.rows_routed, k, T, H, !xb, x_perm, L->num_sms, st));
+  MOE_CUDA(moe::launch_gather(x, xb, perm, pos, w.rows_routed, k, T, H, !xb, x_perm, L->num_sms,
+                              L->status, st));
   MOE_CUDA(mark(4));
 
   GemmParams p{};

@@ -97,9 +97,10 @@ cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, 
                         int bn_dn, int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
                         int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
                         int* pos, float* w_perm, cudaStream_t st);
-cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_routed, int k, int T,
-                          int H, bool write_shared, __nv_bfloat16* x_perm, int num_sms,
-                          cudaStream_t st);
+// x_perm rows: bf16 x by bulk copies per token (pos), else row by row (perm)
+cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, const int* pos,
+                          int rows_routed, int k, int T, int H, bool write_shared,
+                          __nv_bfloat16* x_perm, int num_sms, int* status, cudaStream_t st);
 // 128-feature weight blocks per down-projection tile for hidden size H.
 int gemm_down_blocks(int H);
 
@@ -152,6 +153,7 @@ cudaError_t gemm_configure_device();
 // also sizes the pair kernels' grid to the co-resident 2-CTA clusters
 cudaError_t gemm_pair_configure_device(int num_sms);
 cudaError_t topk_configure_device();
+cudaError_t gather_configure_device();
 
 
 }  // namespace moe

@@ -244,7 +244,58 @@ __global__ void __launch_bounds__(256) gather_kernel(const TX* __restrict__ x,
   }
 }
 
+// Batches from which the bf16 gather runs per token with bulk copies (below,
+// the row-per-warp form spreads a small batch over more SMs).
+constexpr int kGatherRowsMinTokens = 1024;
+
+// bf16 x: one warp per token at a time, its lane 0 issuing bulk (TMA) copies:
+// the token's row is read into shared memory once and written to its k rows
+// of x_perm (pos[t, j]) by k bulk stores.  Two row buffers per warp, so the
+// next token's load overlaps this token's stores.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const int* __restrict__ pos, int T,
+                                                          int k, int H,
+                                                          __nv_bfloat16* __restrict__ xp,
+                                                          int* status) {
+  extern __shared__ __align__(128) uint8_t gsm[];
+  pdl_wait();  // the previous kernel's results are visible
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int wpb = blockDim.x >> 5;
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2;
+  const uint32_t buf0 = smem_u32(gsm) + static_cast<uint32_t>(warp) * 2 * row_bytes;
+  const uint32_t bar0 = smem_u32(gsm) + static_cast<uint32_t>(wpb) * 2 * row_bytes + warp * 16;
+  if (lane != 0) return;
+  mbar_init(bar0, 1);
+  mbar_init(bar0 + 8, 1);
+  fence_mbar_init();
+  uint32_t i = 0;
+  for (int t = blockIdx.x * wpb + warp; t < T; t += gridDim.x * wpb, ++i) {
+    const uint32_t b = i & 1u;
+    const uint32_t buf = buf0 + b * row_bytes;
+    const uint32_t bar = bar0 + 8 * b;
+    int rows[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < k) rows[j] = pos[static_cast<size_t>(t) * k + j];
+    if (i >= 2) bulk_wait_group_read<1>();  // the stores that read this buffer are done with it
+    mbar_arrive_expect_tx(bar, row_bytes);
+    bulk_load_1d(buf, x + static_cast<size_t>(t) * H, row_bytes, bar);
+    if (!mbar_wait(bar, (i >> 1) & 1u, nullptr, status)) break;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < k) bulk_store_1d(xp + static_cast<size_t>(rows[j]) * H, buf, row_bytes);
+    bulk_commit_group();
+  }
+  bulk_wait_group_all();
+}
+
 }  // namespace
+
+cudaError_t gather_configure_device() {
+  return cudaFuncSetAttribute(gather_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              100 * 1024);
+}
 
 cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn_gu,
                         int bn_dn, int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
@@ -268,9 +319,20 @@ cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, 
                     masks, chunk_base, row_start, perm, pos, w_perm);
 }
 
-cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, int rows_routed, int k, int T,
-                          int H, bool write_shared, __nv_bfloat16* x_perm, int num_sms,
-                          cudaStream_t st) {
+cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, const int* pos,
+                          int rows_routed, int k, int T, int H, bool write_shared,
+                          __nv_bfloat16* x_perm, int num_sms, int* status, cudaStream_t st) {
+  if (x_bf16 && !write_shared && T >= kGatherRowsMinTokens) {
+    // rows of up to 96 KB of buffers per block: 6 warps at H = 4096
+    const int row_bytes = H * 2;
+    int wpb = (96 * 1024) / (2 * row_bytes);
+    wpb = wpb < 1 ? 1 : (wpb > 8 ? 8 : wpb);
+    const int want = (T + wpb - 1) / wpb;
+    const int blocks = max(1, min(want, num_sms * 2));
+    const size_t smem = static_cast<size_t>(wpb) * (2 * row_bytes + 16);
+    return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(32 * wpb), smem, st,
+                      static_cast<const __nv_bfloat16*>(x), pos, T, k, H, x_perm, status);
+  }
   const int nrows = rows_routed + (write_shared ? T : 0);
   const int want = (nrows + 7) / 8;
   const int blocks = max(1, min(want, num_sms * 8));
