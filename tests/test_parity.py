@@ -68,6 +68,18 @@ SMALL = {
     "large_odd_hidden": replace(WORKLOADS["tiny"], name="lo", T=2048, hidden=384,
                                 num_experts=12, top_k=3, intermediate=128,
                                 shared_intermediate=128, act_dtype="bf16", weight_dtype="bf16"),
+    # fp32 x on CTA pairs: CUDA-core router, row gather with the shared rows
+    # in x_perm, pair GEMMs reading them; some experts with a handful of rows
+    "large_fp32_x": replace(WORKLOADS["tiny"], name="lf", T=2304, hidden=512, num_experts=24,
+                            top_k=4, intermediate=256, shared_intermediate=256,
+                            act_dtype="f32", weight_dtype="bf16", swiglu_limit=0.9,
+                            swiglu_limit_shared=1.1, expert_std=0.08),
+    # tensor-core router with the warp-per-token top-k (from 8192 tokens) on a
+    # small layer
+    "many_tokens_small_layer": replace(WORKLOADS["tiny"], name="mt", T=8448, hidden=256,
+                                       num_experts=40, top_k=6, intermediate=128,
+                                       shared_intermediate=128, act_dtype="bf16",
+                                       weight_dtype="bf16", x_dist="rmsnorm_normal"),
 }
 
 
