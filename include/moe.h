@@ -141,6 +141,16 @@ int moe_forward_host(moe_layer_t* layer, const void* x_host, int T, void* out_ho
  * MOE_ERR_DEVICE_TIMEOUT when the word was non-zero. */
 int moe_get_device_error(moe_layer_t* layer, int* device_err);
 
+/* Self-check of the bounded waits every kernel uses (fault detection
+ * without a fault): launches one CTA on the current device whose wait on a
+ * barrier that nothing signals gives up after `limit_us` microseconds
+ * (1 .. 10,000,000), sets the timeout bit (1) of a device status word and
+ * returns.  Synchronises the device.  *device_status (if not NULL) receives
+ * the word.  Returns MOE_OK when the wait gave up and reported exactly the
+ * timeout bit, MOE_ERR_INVALID_ARG for a bad limit, MOE_ERR_CUDA otherwise.
+ * Allocates and frees 4 bytes of device memory. */
+int moe_check_wait_timeout(int limit_us, int* device_status);
+
 /* Static description of a status code. */
 const char* moe_status_string(int status);
 

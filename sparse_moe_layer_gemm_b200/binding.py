@@ -32,6 +32,7 @@ EXPORTS = (
     "moe_forward", "moe_workspace_size_host", "moe_forward_host", "moe_get_device_error",
     "moe_status_string", "moe_destroy", "moe_forward_oneshot", "moe_kernel_launches",
     "moe_set_stage_timing", "moe_get_stage_times", "moe_route_static",
+    "moe_check_wait_timeout",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -102,6 +103,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_kernel_launches.argtypes = [vp, i]
     lib.moe_set_stage_timing.argtypes = [vp, i]
     lib.moe_route_static.argtypes = [vp, i, vp, vp, i, i, i, i, i, f, vp, vp, vp]
+    lib.moe_check_wait_timeout.argtypes = [i, ctypes.POINTER(i)]
     lib.moe_get_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i,
                                         ctypes.POINTER(i)]
     for name in EXPORTS:
@@ -353,3 +355,11 @@ class MoeLayer:
             self.close()
         except Exception:
             pass
+
+
+def moe_check_wait_timeout(limit_us: int):
+    """Runs the bounded-wait self-check (see include/moe.h); returns
+    (status code, device status word)."""
+    word = ctypes.c_int(-1)
+    r = load_library().moe_check_wait_timeout(limit_us, ctypes.byref(word))
+    return r, word.value

@@ -70,9 +70,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Waits for the phase of `bar` with the given parity to complete.  Returns
 // false (without waiting further) once *abort is set by another role of the
-// CTA, or after kWaitLimitNs, in which case it sets *abort and the status bit.
+// CTA, or after limit_ns (default kWaitLimitNs), in which case it sets *abort
+// and the status bit.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
@@ -80,7 +81,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       if (abort != nullptr) *abort = 1;
       atomicOr(status, kDevErrTimeout);
       return false;

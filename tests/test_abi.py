@@ -101,3 +101,9 @@ def test_oneshot_rejects_bad_config_before_cuda(lib):
     r = lib.moe_forward_oneshot(*([None] * 9), 64, 4096, 288, 0, 1280, 3.0, 0.0, 0.0,
                                 B.MOE_BF16, B.MOE_BF16, None, None)
     assert r == B.MOE_ERR_INVALID_ARG
+
+
+def test_wait_self_check_rejects_bad_limits_without_cuda(lib):
+    from sparse_moe_layer_gemm_b200 import binding as B
+    assert B.moe_check_wait_timeout(0)[0] == B.MOE_ERR_INVALID_ARG
+    assert B.moe_check_wait_timeout(20_000_000)[0] == B.MOE_ERR_INVALID_ARG
