@@ -23,7 +23,7 @@ it, written out step by step in float64 (inputs are upcast exactly):
   moe_router_scaling_factor 3, use_moe_router_bias true, need_fp32_gate true,
   swiglu_limits / swiglu_limits_shared).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent (each listed with the design notes):
 
 * the bias is added to the sigmoid scores (not to the logits) to form the
   selection score;
@@ -67,6 +67,9 @@ __all__ = [
     "moe_forward_rows",
     "moe_forward_dense_masked",
     "near_tie_gaps",
+    "decode_e4m3",
+    "dequantize_e4m3",
+    "DequantizedExperts",
 ]
 
 
@@ -347,8 +350,54 @@ def moe_forward_dense_masked(x, router_w, router_bias, w_gate, w_up, w_down,
     return out + swiglu_expert(x64, sh_gate, sh_up, sh_down, swiglu_limit_shared)
 
 
+def decode_e4m3(codes) -> np.ndarray:
+    """Values of FP8 E4M3 codes (the OCP "E4M3FN" encoding), in float64.
+
+    Bit 7 is the sign, bits 6-3 the exponent e (bias 7), bits 2-0 the
+    mantissa m: e = 0 gives the subnormals m * 2^-9; e = 1..15 gives
+    (1 + m/8) * 2^(e-7), except e = 15, m = 7, which is NaN (there are no
+    infinities; the largest finite magnitude is 448).  The pages list FP8
+    official weights for the model (sglang-jax issue #1367, section "Model
+    configuration", the "Official weights" bullet) without stating a format;
+    E4M3FN with one power-of-two scale per output feature is the reading
+    taken.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequantize_e4m3(codes, scale) -> np.ndarray:
+    """Weights from FP8 E4M3 codes [..., K, N] (x @ W layout: N output
+    features) and one scale per output feature [..., N]:
+    w[..., k, n] = value(codes[..., k, n]) * scale[..., n]."""
+    v = decode_e4m3(codes)
+    return v * np.asarray(scale, dtype=np.float64)[..., None, :]
+
+
+class DequantizedExperts:
+    """``view[e]`` -> expert e's dequantized matrix (float64) from codes
+    [E, K, N] and scales [E, N] (torch tensors or arrays; fetched per expert
+    so large weight sets are walked one expert at a time)."""
+
+    def __init__(self, codes, scales):
+        self.codes = codes
+        self.scales = scales
+
+    def __getitem__(self, e: int) -> np.ndarray:
+        return dequantize_e4m3(as_numpy(self.codes[e]), as_numpy(self.scales[e]))
+
+    def __len__(self):
+        return len(self.codes)
+
+
 def as_numpy(t: Any) -> np.ndarray:
-    """Exact host float32 copy of a torch tensor (bf16 widened exactly) or array."""
+    """Exact host copy of a torch tensor (bf16 widened exactly to float32;
+    integer codes kept as they are) or array."""
     if hasattr(t, "detach"):
         import torch  # local: the oracle itself needs only NumPy
         t = t.detach()

@@ -34,7 +34,7 @@ class Workload:
     intermediate: int
     shared_intermediate: int
     act_dtype: str                 # "f32" or "bf16"
-    weight_dtype: str              # "f32" or "bf16"
+    weight_dtype: str              # "f32", "bf16" or "fp8" (E4M3 codes + scales)
     x_dist: str                    # "normal" or "rmsnorm_normal"
     router_std: float
     expert_std: float
@@ -50,7 +50,7 @@ class Workload:
 
     @property
     def weight_bytes_per_expert(self) -> int:
-        el = 2 if self.weight_dtype == "bf16" else 4
+        el = {"fp8": 1, "bf16": 2, "f32": 4}[self.weight_dtype]
         return 3 * self.hidden * self.intermediate * el
 
 
@@ -91,7 +91,23 @@ def _gen(device: torch.device, seed: int, stream: int) -> torch.Generator:
 
 
 def _torch_dtype(name: str) -> torch.dtype:
-    return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
+    # fp8 weights are drawn in fp32, then quantised (quantize_e4m3)
+    return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float32}[name]
+
+
+def quantize_e4m3(w: torch.Tensor):
+    """Input preparation for FP8 weight workloads: ``w`` [..., K, N] (x @ W
+    layout, N output features) -> (codes uint8 [..., K, N], scale fp32
+    [..., N]).  Each output feature gets the power of two
+    scale = 2^ceil(log2(amax / 448)) (1 for an all-zero feature), so w / scale
+    lies within the E4M3FN range, and the codes are torch's round-to-nearest
+    float8_e4m3fn conversion of w / scale."""
+    wf = w.float()
+    amax = wf.abs().amax(dim=-2)
+    e = torch.ceil(torch.log2(torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))))
+    scale = torch.exp2(e)
+    codes = (wf / scale.unsqueeze(-2)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, scale.to(torch.float32)
 
 
 def draw_x(wl: Workload, device="cpu") -> torch.Tensor:
@@ -148,7 +164,10 @@ def draw_shared(wl: Workload, device="cpu"):
 def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
     """All tensors of a workload, in the ABI's layouts:
     x [T, H]; router_w [H, E] f32; router_bias [E] f32;
-    w_gate, w_up [E, H, I]; w_down [E, I, H]; sh_gate, sh_up [H, Is]; sh_down [Is, H]."""
+    w_gate, w_up [E, H, I]; w_down [E, I, H]; sh_gate, sh_up [H, Is]; sh_down [Is, H].
+    FP8 weights: the six weight tensors hold E4M3FN codes (uint8) and
+    s_w_gate, s_w_up [E, I], s_w_down [E, H], s_sh_gate, s_sh_up [Is],
+    s_sh_down [H] their per-output-feature scales (fp32)."""
     dev = torch.device(device)
     x = draw_x(wl, dev)
     rw, rb = draw_router(wl, dev)
@@ -163,8 +182,13 @@ def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
         w_up[e].copy_(wu)
         w_down[e].copy_(wd)
     sg, su, sd = draw_shared(wl, dev)
-    return dict(x=x, router_w=rw, router_bias=rb, w_gate=w_gate, w_up=w_up,
-                w_down=w_down, sh_gate=sg, sh_up=su, sh_down=sd)
+    out = dict(x=x, router_w=rw, router_bias=rb, w_gate=w_gate, w_up=w_up,
+               w_down=w_down, sh_gate=sg, sh_up=su, sh_down=sd)
+    if wl.weight_dtype == "fp8":
+        # codes replace the fp32 draws; scales s_<name> [E, N] / [N]
+        for name in ("w_gate", "w_up", "w_down", "sh_gate", "sh_up", "sh_down"):
+            out[name], out["s_" + name] = quantize_e4m3(out[name])
+    return out
 
 
 class HostExpertView:

@@ -7,6 +7,7 @@ float64 operations.  The mutation tests at the end plant plausible mistakes in
 the oracle (on the CPU) and check that some pin fails.
 """
 import os
+from dataclasses import replace
 
 import numpy as np
 import pytest
@@ -449,3 +450,81 @@ def test_mutant_transposed_down(monkeypatch):
     monkeypatch.setattr(om, "swiglu_expert",
                         lambda rows, wg, wu, wd, limit: orig(rows, wg, wu, np.asarray(wd).T, limit))
     assert _fails([pin_closed_form_identical_experts, pin_clamp_branches])
+
+
+# ---------------------------------------------------------------- FP8 E4M3 weights
+
+def test_e4m3_decode_closed_forms():
+    """Values fixed by the encoding's definition (sign, 4-bit exponent with
+    bias 7, 3-bit mantissa, subnormals below exponent 1, NaN at S.1111.111)."""
+    d = om.decode_e4m3
+    assert d([0x00])[0] == 0.0 and np.signbit(d([0x80])[0])
+    assert d([0x01])[0] == 2.0 ** -9                 # smallest subnormal
+    assert d([0x07])[0] == 7 * 2.0 ** -9             # largest subnormal
+    assert d([0x08])[0] == 2.0 ** -6                 # smallest normal
+    assert d([0x38])[0] == 1.0
+    assert d([0x3C])[0] == 1.5
+    assert d([0x40])[0] == 2.0
+    assert d([0x7E])[0] == 448.0                     # largest finite
+    assert np.isnan(d([0x7F])[0]) and np.isnan(d([0xFF])[0])
+    assert d([0xB8])[0] == -1.0
+
+
+def test_e4m3_decode_structure():
+    """Sign symmetry, strict monotonicity over the finite positive codes, and
+    every value an integer multiple of the smallest subnormal."""
+    v = om.decode_e4m3(np.arange(256))
+    pos = v[:0x7F]
+    assert np.all(np.diff(pos) > 0)
+    assert np.array_equal(v[0x80:0xFF], -pos)
+    k = pos * 2.0 ** 9
+    assert np.array_equal(k, np.round(k))
+
+
+def test_e4m3_decode_matches_torch():
+    """Special case that reduces to a library routine: torch's float8_e4m3fn
+    (CPU) decodes the same 256 codes to the same values."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = om.decode_e4m3(codes.numpy())
+    both_nan = np.isnan(ref) & np.isnan(got)
+    assert np.array_equal(np.where(both_nan, 0, ref), np.where(both_nan, 0, got))
+    assert np.array_equal(np.isnan(ref), np.isnan(got))
+
+
+def test_dequantize_scales_columns():
+    """Scales apply per output feature (column of the x @ W matrix)."""
+    codes = np.array([[0x38, 0x40], [0xB8, 0x3C]], dtype=np.uint8)   # [[1, 2], [-1, 1.5]]
+    w = om.dequantize_e4m3(codes, np.array([0.5, 4.0]))
+    assert np.array_equal(w, [[0.5, 8.0], [-0.5, 6.0]])
+
+
+def test_mutant_e4m3_wrong_bias(monkeypatch):
+    """A planted mistake (exponent bias 8 instead of 7) fails the pins."""
+    real = om.decode_e4m3
+
+    def bad(codes):
+        return real(codes) * 0.5
+    monkeypatch.setattr(om, "decode_e4m3", bad)
+    with pytest.raises(AssertionError):
+        test_e4m3_decode_closed_forms()
+
+
+def test_fp8_workload_quantisation_bound():
+    """The FP8 inputs: power-of-two scales, no code out of the finite range,
+    and every dequantized weight within half an E4M3 step of the fp32 draw
+    (relative 2^-4 for normal values, absolute 2^-10 * scale below them)."""
+    wl = replace(WORKLOADS["tiny"], weight_dtype="fp8")
+    q = make_inputs(wl, "cpu")
+    ref = make_inputs(WORKLOADS["tiny"], "cpu")
+    for name in ("w_gate", "w_down", "sh_up"):
+        codes, sc = q[name].numpy(), q["s_" + name].numpy().astype(np.float64)
+        assert codes.dtype == np.uint8 and not np.any((codes & 0x7F) == 0x7F)
+        assert np.array_equal(np.exp2(np.round(np.log2(sc))), sc)
+        w = ref[name].double().numpy()
+        dq = om.dequantize_e4m3(codes, sc)
+        bound = np.maximum(np.abs(w) * 2.0 ** -4, 2.0 ** -10 * sc[..., None, :])
+        assert np.all(np.abs(dq - w) <= bound)
+    view = om.DequantizedExperts(q["w_up"], q["s_w_up"])
+    assert len(view) == wl.num_experts
+    assert np.array_equal(view[3], om.dequantize_e4m3(q["w_up"][3].numpy(), q["s_w_up"][3].numpy()))
