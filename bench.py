@@ -41,7 +41,7 @@ def _args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode")
-    ap.add_argument("--secondary", default="prefill,zipf_prefill,clamp_ragged,tiny",
+    ap.add_argument("--secondary", default="prefill,zipf_prefill,clamp_ragged,tiny,decode_fp8",
                     help="comma-separated further workloads measured in the same run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -267,7 +267,12 @@ def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step):
         rl = {"bound": "tensor", "achieved": ach, "peak": peaks["tc"], "unit": "TFLOP/s",
               "frac": ach / peaks["tc"]}
     # from 2048 tokens the library runs the expert GEMMs on CTA pairs
-    kname = "grouped_gemm_pair_kernel<gate_up>" if wl.T >= 2048 else "grouped_gemm_kernel<gate_up>"
+    # (FP8 weights: one-SM tiles with converter warps at every size)
+    if wl.weight_dtype == "fp8":
+        kname = "grouped_gemm_kernel<gate_up, fp8>"
+    else:
+        kname = ("grouped_gemm_pair_kernel<gate_up>" if wl.T >= 2048
+                 else "grouped_gemm_kernel<gate_up>")
     rl.update({"kernel": kname, "kernel_ms": gu_ms,
                "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
                "peak_source": (f"{peaks['source']} (MEASURED_PEAKS.json; "
@@ -397,6 +402,9 @@ def run_ours(a):
         entry = {"workload": wl2.name, "T": wl2.T, "value": job_throughput(wl2.T, world, ms2),
                  "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
                  "layer_roofline": lr2, "stage_ms": st2}
+        if wl2.weight_dtype != "bf16":
+            entry["weights"] = {"fp8": "fp8_e4m3 codes + fp32 per-feature scales (bf16 MMA)",
+                                "f32": "fp32 (rounded to bf16 at load)"}[wl2.weight_dtype]
         if wl2.name == "tiny":
             entry["l2"] = "L2-resident (16 KB experts): launch latency, not a roofline case"
         secondary.append(entry)

@@ -53,13 +53,20 @@ typedef enum {
   MOE_ERR_NOT_LOADED = 6       /* moe_forward before moe_load_weights */
 } moe_status_t;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+/* MOE_FP8_E4M3: expert weights only (weight_dtype), loaded with
+ * moe_load_weights_fp8.  The pages list FP8 official weights for the model
+ * (sglang-jax issue #1367, section "Model configuration", "Official weights")
+ * without a format; the one taken here is E4M3FN codes (sign, 4-bit exponent
+ * with bias 7, 3-bit mantissa, no infinities, S.1111.111 = NaN) with one fp32
+ * scale per output feature: w[k][n] = value(code[k][n]) * scale[n]. */
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_FP8_E4M3 = 2 } moe_dtype_t;
 
 /* Layer configuration.  Field names follow the model's config fields
  * (llm-atlas "Step-3.5-Flash", "Raw config fields").
  * Supported: hidden % 128 == 0, 1 <= hidden <= 16384; 1 <= num_experts <= 1024;
  * 1 <= top_k <= min(num_experts, 32); 1 <= intermediate <= 8192;
- * shared_intermediate == intermediate; act_dtype, weight_dtype in {F32, BF16};
+ * shared_intermediate == intermediate; act_dtype in {F32, BF16}; weight_dtype
+ * in {F32, BF16, FP8_E4M3};
  * routed_scaling_factor finite; swiglu limits >= 0 (0 = no clamp). */
 typedef struct {
   int hidden;                  /* H: hidden_size, 4096 */
@@ -98,20 +105,49 @@ typedef struct {
 int moe_config_check(const moe_config_t* cfg);
 
 /* Creates a layer on the current CUDA device.  Allocates the packed weight
- * copy (3 * (E + 1) * H * round_up(I, 128) bf16 plus the router) and a small
- * device status word.  *out receives the handle (NULL on error). */
+ * copy (3 * (E + 1) * H * round_up(I, 128) bf16, or for FP8 weights as many
+ * bytes plus (E + 1) * (2 * round_up(I, 128) + H) fp32 scales, plus the
+ * router) and a small device status word.  *out receives the handle (NULL on
+ * error). */
 int moe_create(const moe_config_t* cfg, moe_layer_t** out);
 
 /* Copies the weights into the layer's packed bf16 layout on `stream`
  * (K-major weight rows; gate and up interleaved in blocks of 128 rows; fp32
  * expert weights are rounded to bf16).  router_w [H, E] and router_bias [E]
  * are fp32 and kept fp32; router_bias may be NULL (zero bias).  The expert
- * pointers have the config's weight_dtype.  The caller's buffers may be
- * freed once `stream` has passed this call. */
+ * pointers have the config's weight_dtype (F32 or BF16; a layer created with
+ * MOE_FP8_E4M3 weights returns MOE_ERR_INVALID_ARG: it loads through
+ * moe_load_weights_fp8).  The caller's buffers may be freed once `stream` has
+ * passed this call. */
 int moe_load_weights(moe_layer_t* layer, const float* router_w, const float* router_bias,
                      const void* w_gate, const void* w_up, const void* w_down,
                      const void* sh_gate, const void* sh_up, const void* sh_down,
                      void* stream);
+
+/* FP8 expert weights (layer created with weight_dtype MOE_FP8_E4M3): the
+ * codes in the layouts of moe_load_weights, one uint8 E4M3FN code per weight
+ * (w_gate / w_up [E, H, I], w_down [E, I, H], sh_gate / sh_up [H, I],
+ * sh_down [I, H]), and their fp32 scales per output feature: s_gate / s_up
+ * [E, I], s_down [E, H], sh_s_gate / sh_s_up [I], sh_s_down [H].  NaN codes
+ * (0x7F, 0xFF) are not valid weights.  The codes are kept as bytes (no bf16
+ * copy); the expert GEMMs expand them to bf16 in shared memory, exactly, and
+ * multiply each output feature's accumulator by its scale.  Router as in
+ * moe_load_weights.  Returns MOE_ERR_INVALID_ARG for a NULL pointer or a
+ * layer whose weight_dtype is not MOE_FP8_E4M3.  Device pointers, caller
+ * owned, free once `stream` has passed this call. */
+int moe_load_weights_fp8(moe_layer_t* layer, const float* router_w, const float* router_bias,
+                         const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
+                         const float* s_gate, const float* s_up, const float* s_down,
+                         const uint8_t* sh_gate, const uint8_t* sh_up, const uint8_t* sh_down,
+                         const float* sh_s_gate, const float* sh_s_up, const float* sh_s_down,
+                         void* stream);
+
+/* E4M3FN codes -> bf16 values (uint16 bit patterns) on `stream`, through the
+ * same routine the FP8 expert GEMMs expand their weights with (every finite
+ * code is exactly a bf16 value; NaN codes give +-480, see
+ * moe_load_weights_fp8).  codes and out are device pointers, 16-byte
+ * aligned; n % 4 == 0 (MOE_ERR_INVALID_ARG otherwise); n = 0 is a no-op. */
+int moe_decode_e4m3(const uint8_t* codes, size_t n, uint16_t* out, void* stream);
 
 /* Device workspace bytes moe_forward needs for T tokens (caller allocates,
  * 256-byte aligned).  Host-only. */
@@ -182,7 +218,9 @@ int moe_get_stage_times(moe_layer_t* layer, float* ms, int n_stages, int* n_forw
 /* One call with the layer's argument list: creates a layer, loads the
  * weights, allocates a workspace, runs the forward on `stream`, synchronises
  * and frees everything.  Convenient for a single forward; for repeated calls
- * use create / load / forward.  Allocates device memory (cudaMalloc). */
+ * use create / load / forward.  Allocates device memory (cudaMalloc).
+ * weight_dtype MOE_FP8_E4M3 returns MOE_ERR_UNSUPPORTED (this argument list
+ * has no scales; use create / moe_load_weights_fp8 / forward). */
 int moe_forward_oneshot(const void* x, const float* router_w, const float* router_bias,
                         const void* w_gate, const void* w_up, const void* w_down,
                         const void* sh_gate, const void* sh_up, const void* sh_down,

@@ -25,6 +25,7 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_NOT_LOADED = 6
 MOE_F32 = 0
 MOE_BF16 = 1
+MOE_FP8_E4M3 = 2
 
 # every symbol include/moe.h declares
 EXPORTS = (
@@ -32,7 +33,7 @@ EXPORTS = (
     "moe_forward", "moe_workspace_size_host", "moe_forward_host", "moe_get_device_error",
     "moe_status_string", "moe_destroy", "moe_forward_oneshot", "moe_kernel_launches",
     "moe_set_stage_timing", "moe_get_stage_times", "moe_route_static",
-    "moe_check_wait_timeout",
+    "moe_check_wait_timeout", "moe_load_weights_fp8", "moe_decode_e4m3",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -104,6 +105,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_set_stage_timing.argtypes = [vp, i]
     lib.moe_route_static.argtypes = [vp, i, vp, vp, i, i, i, i, i, f, vp, vp, vp]
     lib.moe_check_wait_timeout.argtypes = [i, ctypes.POINTER(i)]
+    lib.moe_load_weights_fp8.argtypes = [vp] * 16
+    lib.moe_decode_e4m3.argtypes = [vp, sz, vp, vp]
     lib.moe_get_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i,
                                         ctypes.POINTER(i)]
     for name in EXPORTS:
@@ -138,7 +141,7 @@ def make_config(hidden, num_experts, top_k, intermediate, shared_intermediate=No
 
 
 def config_from_workload(wl) -> moe_config_t:
-    dt = {"f32": MOE_F32, "bf16": MOE_BF16}
+    dt = {"f32": MOE_F32, "bf16": MOE_BF16, "fp8": MOE_FP8_E4M3}
     return make_config(wl.hidden, wl.num_experts, wl.top_k, wl.intermediate,
                        wl.shared_intermediate, routed_scaling_factor=wl.scale,
                        swiglu_limit=wl.swiglu_limit, swiglu_limit_shared=wl.swiglu_limit_shared,
@@ -190,6 +193,26 @@ def moe_load_weights(handle, router_w, router_bias, w_gate, w_up, w_down, sh_gat
         ctypes.c_void_p(handle), _ptr(router_w), _ptr(router_bias), _ptr(w_gate), _ptr(w_up),
         _ptr(w_down), _ptr(sh_gate), _ptr(sh_up), _ptr(sh_down), _stream(stream)),
         "moe_load_weights")
+
+
+def moe_load_weights_fp8(handle, router_w, router_bias, w_gate, w_up, w_down, s_gate, s_up,
+                         s_down, sh_gate, sh_up, sh_down, sh_s_gate, sh_s_up, sh_s_down,
+                         stream=None) -> None:
+    _check(load_library().moe_load_weights_fp8(
+        ctypes.c_void_p(handle), _ptr(router_w), _ptr(router_bias), _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), _ptr(s_gate), _ptr(s_up), _ptr(s_down), _ptr(sh_gate), _ptr(sh_up),
+        _ptr(sh_down), _ptr(sh_s_gate), _ptr(sh_s_up), _ptr(sh_s_down), _stream(stream)),
+        "moe_load_weights_fp8")
+
+
+def moe_decode_e4m3(codes: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """E4M3FN codes (uint8, CUDA) -> bf16 through the library's converter."""
+    if out is None:
+        out = torch.empty(codes.shape, dtype=torch.bfloat16, device=codes.device)
+    _check(load_library().moe_decode_e4m3(_ptr(codes), codes.numel(), _ptr(out),
+                                          _stream(stream)), "moe_decode_e4m3")
+    return out
 
 
 def moe_forward(handle, x, T, out, workspace, ws_bytes, stream=None, routing=None) -> int:
@@ -292,7 +315,36 @@ class MoeLayer:
         moe_load_weights(self.handle, router_w, router_bias, w_gate, w_up, w_down, sh_gate,
                          sh_up, sh_down)
 
+    def load_weights_fp8(self, router_w, router_bias, w_gate, w_up, w_down, s_gate, s_up, s_down,
+                         sh_gate, sh_up, sh_down, sh_s_gate, sh_s_up, sh_s_down):
+        """E4M3FN codes (uint8) in the layouts of load_weights plus their fp32
+        scales per output feature."""
+        c = self.cfg
+        H, E, I, Is = c.hidden, c.num_experts, c.intermediate, c.shared_intermediate
+        self._need(router_w, "router_w", torch.float32, (H, E))
+        if router_bias is not None:
+            self._need(router_bias, "router_bias", torch.float32, (E,))
+        u8, f32 = torch.uint8, torch.float32
+        for t, name, dt, shape in ((w_gate, "w_gate", u8, (E, H, I)), (w_up, "w_up", u8, (E, H, I)),
+                                   (w_down, "w_down", u8, (E, I, H)),
+                                   (s_gate, "s_gate", f32, (E, I)), (s_up, "s_up", f32, (E, I)),
+                                   (s_down, "s_down", f32, (E, H)),
+                                   (sh_gate, "sh_gate", u8, (H, Is)), (sh_up, "sh_up", u8, (H, Is)),
+                                   (sh_down, "sh_down", u8, (Is, H)),
+                                   (sh_s_gate, "sh_s_gate", f32, (Is,)),
+                                   (sh_s_up, "sh_s_up", f32, (Is,)),
+                                   (sh_s_down, "sh_s_down", f32, (H,))):
+            self._need(t, name, dt, shape)
+        moe_load_weights_fp8(self.handle, router_w, router_bias, w_gate, w_up, w_down, s_gate,
+                             s_up, s_down, sh_gate, sh_up, sh_down, sh_s_gate, sh_s_up, sh_s_down)
+
     def load_inputs(self, inp: Dict[str, torch.Tensor]):
+        if self.cfg.weight_dtype == MOE_FP8_E4M3:
+            self.load_weights_fp8(inp["router_w"], inp["router_bias"], inp["w_gate"], inp["w_up"],
+                                  inp["w_down"], inp["s_w_gate"], inp["s_w_up"], inp["s_w_down"],
+                                  inp["sh_gate"], inp["sh_up"], inp["sh_down"], inp["s_sh_gate"],
+                                  inp["s_sh_up"], inp["s_sh_down"])
+            return
         self.load_weights(inp["router_w"], inp["router_bias"], inp["w_gate"], inp["w_up"],
                           inp["w_down"], inp["sh_gate"], inp["sh_up"], inp["sh_down"])
 

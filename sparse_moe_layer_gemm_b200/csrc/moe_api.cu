@@ -21,8 +21,11 @@ struct moe_layer {
   int device;
   int num_sms;
   int I_pad;
-  __nv_bfloat16* w_gu;  // [(E+1) * 2 * I_pad, H]
-  __nv_bfloat16* w_dn;  // [(E+1) * H, I_pad]
+  int fp8;              // expert weights are E4M3 codes (one byte each) + scales
+  void* w_gu;           // [(E+1) * 2 * I_pad, H] bf16 or E4M3 codes
+  void* w_dn;           // [(E+1) * H, I_pad] bf16 or E4M3 codes
+  float* sc_gu;         // FP8: scale of each packed gate|up row [(E+1) * 2 * I_pad]
+  float* sc_dn;         // FP8: scale of each packed down row [(E+1) * H]
   float* router_w;      // [H, E]
   float* router_b;      // [E]
   __nv_bfloat16* router_tc;  // [E_pad, 3H]: bf16 three-term split of router_w^T
@@ -133,6 +136,24 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   return r == CUDA_SUCCESS;
 }
 
+// bf16 [rows, cols] row-major seen as 3-D (64 columns, rows, cols / 64
+// column blocks), box 64 x box_rows x 2 column blocks, 128B swizzle: the FP8
+// GEMMs' token rows for two k-steps in one load (smem: k-block-major).
+bool encode_bf16_kpair(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(moe::kBK), rows, cols / moe::kBK};
+  cuuint64_t strides[2] = {cols * 2, static_cast<cuuint64_t>(moe::kBK) * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::kBK), box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // bf16 [rows, cols] row-major, box 32 columns x 16 rows, no swizzle: the
 // expert GEMM epilogues' TMA stores of h and y.
 bool encode_bf16_store(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols) {
@@ -172,6 +193,9 @@ struct DeviceGuard {
     if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
+// The router part of both weight loaders (defined below).
+int load_router(moe_layer* L, const float* router_w, const float* router_bias, cudaStream_t st);
+
 }  // namespace
 
 extern "C" {
@@ -195,7 +219,8 @@ int moe_config_check(const moe_config_t* c) {
       c->shared_intermediate <= 0)
     return MOE_ERR_INVALID_ARG;
   if ((c->act_dtype != MOE_F32 && c->act_dtype != MOE_BF16) ||
-      (c->weight_dtype != MOE_F32 && c->weight_dtype != MOE_BF16))
+      (c->weight_dtype != MOE_F32 && c->weight_dtype != MOE_BF16 &&
+       c->weight_dtype != MOE_FP8_E4M3))
     return MOE_ERR_INVALID_ARG;
   if (!isfinite(c->routed_scaling_factor) || !isfinite(c->swiglu_limit) ||
       !isfinite(c->swiglu_limit_shared) || c->swiglu_limit < 0.f || c->swiglu_limit_shared < 0.f)
@@ -215,6 +240,7 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
   moe_layer* L = new (std::nothrow) moe_layer();
   if (L == nullptr) return MOE_ERR_CUDA;
   L->cfg = *cfg;
+  L->fp8 = cfg->weight_dtype == MOE_FP8_E4M3 ? 1 : 0;
   L->I_pad = (cfg->intermediate + 127) / 128 * 128;
   L->E_pad = (cfg->num_experts + 127) / 128 * 128;
   if (cudaGetDevice(&L->device) != cudaSuccess ||
@@ -224,8 +250,10 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
     return MOE_ERR_CUDA;
   }
   const size_t H = cfg->hidden, E = cfg->num_experts, Ip = L->I_pad;
-  const size_t gu_bytes = (E + 1) * 2 * Ip * H * 2, dn_bytes = (E + 1) * H * Ip * 2;
+  const size_t el = L->fp8 ? 1 : 2;
+  const size_t gu_bytes = (E + 1) * 2 * Ip * H * el, dn_bytes = (E + 1) * H * Ip * el;
   if (moe::gemm_configure_device() != cudaSuccess ||
+      moe::gemm_fp8_configure_device() != cudaSuccess ||
       moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
       moe::topk_configure_device() != cudaSuccess ||
       moe::gather_configure_device() != cudaSuccess ||
@@ -236,14 +264,18 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
       cudaMalloc(&L->router_tc, static_cast<size_t>(L->E_pad) * 3 * H * 2) != cudaSuccess ||
       cudaMalloc(&L->router_t, E * H * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
-      cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess) {
+      cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess ||
+      (L->fp8 && (cudaMalloc(&L->sc_gu, (E + 1) * 2 * Ip * sizeof(float)) != cudaSuccess ||
+                  cudaMalloc(&L->sc_dn, (E + 1) * H * sizeof(float)) != cudaSuccess))) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
   }
-  if (!encode_bf16_2d(&L->tm_gu, L->w_gu, (E + 1) * 2 * Ip, H, 2 * moe::kBM) ||
-      !encode_bf16_2d(&L->tm_gu64, L->w_gu, (E + 1) * 2 * Ip, H, 64) ||
-      !encode_bf16_2d(&L->tm_dn, L->w_dn, (E + 1) * H, Ip, moe::kBM) ||
-      !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM)) {
+  // (FP8 codes are read with plain bulk copies: no tensor maps)
+  const bool maps_ok =
+      L->fp8 || (encode_bf16_2d(&L->tm_gu, L->w_gu, (E + 1) * 2 * Ip, H, 2 * moe::kBM) &&
+                 encode_bf16_2d(&L->tm_gu64, L->w_gu, (E + 1) * 2 * Ip, H, 64) &&
+                 encode_bf16_2d(&L->tm_dn, L->w_dn, (E + 1) * H, Ip, moe::kBM));
+  if (!maps_ok || !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM)) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
   }
@@ -257,6 +289,7 @@ int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_
   if (L == nullptr || router_w == nullptr || w_gate == nullptr || w_up == nullptr ||
       w_down == nullptr || sh_gate == nullptr || sh_up == nullptr || sh_down == nullptr)
     return MOE_ERR_INVALID_ARG;
+  if (L->fp8) return MOE_ERR_INVALID_ARG;  // codes need their scales: moe_load_weights_fp8
   DeviceGuard dg(L->device);
   if (!dg.ok) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -264,14 +297,80 @@ int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_
   const int H = c.hidden, E = c.num_experts, I = c.intermediate, Ip = L->I_pad;
   const bool wb = c.weight_dtype == MOE_BF16;
   const size_t gu_group = static_cast<size_t>(2) * Ip * H, dn_group = static_cast<size_t>(H) * Ip;
-  MOE_CUDA(cudaMemsetAsync(L->w_gu, 0, (E + 1) * gu_group * 2, st));
-  MOE_CUDA(cudaMemsetAsync(L->w_dn, 0, (E + 1) * dn_group * 2, st));
-  MOE_CUDA(moe::launch_pack_gate_up(w_gate, wb, E, H, I, Ip, 0, L->w_gu, st));
-  MOE_CUDA(moe::launch_pack_gate_up(w_up, wb, E, H, I, Ip, 1, L->w_gu, st));
-  MOE_CUDA(moe::launch_pack_gate_up(sh_gate, wb, 1, H, I, Ip, 0, L->w_gu + E * gu_group, st));
-  MOE_CUDA(moe::launch_pack_gate_up(sh_up, wb, 1, H, I, Ip, 1, L->w_gu + E * gu_group, st));
-  MOE_CUDA(moe::launch_pack_down(w_down, wb, E, H, I, Ip, L->w_dn, st));
-  MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, L->w_dn + E * dn_group, st));
+  __nv_bfloat16* gu = static_cast<__nv_bfloat16*>(L->w_gu);
+  __nv_bfloat16* dn = static_cast<__nv_bfloat16*>(L->w_dn);
+  MOE_CUDA(cudaMemsetAsync(gu, 0, (E + 1) * gu_group * 2, st));
+  MOE_CUDA(cudaMemsetAsync(dn, 0, (E + 1) * dn_group * 2, st));
+  MOE_CUDA(moe::launch_pack_gate_up(w_gate, wb, E, H, I, Ip, 0, gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up(w_up, wb, E, H, I, Ip, 1, gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up(sh_gate, wb, 1, H, I, Ip, 0, gu + E * gu_group, st));
+  MOE_CUDA(moe::launch_pack_gate_up(sh_up, wb, 1, H, I, Ip, 1, gu + E * gu_group, st));
+  MOE_CUDA(moe::launch_pack_down(w_down, wb, E, H, I, Ip, dn, st));
+  MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, dn + E * dn_group, st));
+  return load_router(L, router_w, router_bias, st);
+}
+
+int moe_load_weights_fp8(moe_layer_t* L, const float* router_w, const float* router_bias,
+                         const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
+                         const float* s_gate, const float* s_up, const float* s_down,
+                         const uint8_t* sh_gate, const uint8_t* sh_up, const uint8_t* sh_down,
+                         const float* sh_s_gate, const float* sh_s_up, const float* sh_s_down,
+                         void* stream) {
+  if (L == nullptr || router_w == nullptr || w_gate == nullptr || w_up == nullptr ||
+      w_down == nullptr || s_gate == nullptr || s_up == nullptr || s_down == nullptr ||
+      sh_gate == nullptr || sh_up == nullptr || sh_down == nullptr || sh_s_gate == nullptr ||
+      sh_s_up == nullptr || sh_s_down == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (!L->fp8) return MOE_ERR_INVALID_ARG;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const moe_config_t& c = L->cfg;
+  const int H = c.hidden, E = c.num_experts, I = c.intermediate, Ip = L->I_pad;
+  const size_t gu_group = static_cast<size_t>(2) * Ip * H, dn_group = static_cast<size_t>(H) * Ip;
+  uint8_t* gu = static_cast<uint8_t*>(L->w_gu);
+  uint8_t* dn = static_cast<uint8_t*>(L->w_dn);
+  // padded rows and columns: code 0 (value 0), scale 0
+  MOE_CUDA(cudaMemsetAsync(gu, 0, (E + 1) * gu_group, st));
+  MOE_CUDA(cudaMemsetAsync(dn, 0, (E + 1) * dn_group, st));
+  MOE_CUDA(cudaMemsetAsync(L->sc_gu, 0, (E + 1) * 2 * Ip * sizeof(float), st));
+  MOE_CUDA(moe::launch_pack_codes_gate_up(w_gate, E, H, I, Ip, 0, gu, st));
+  MOE_CUDA(moe::launch_pack_codes_gate_up(w_up, E, H, I, Ip, 1, gu, st));
+  MOE_CUDA(moe::launch_pack_codes_gate_up(sh_gate, 1, H, I, Ip, 0, gu + E * gu_group, st));
+  MOE_CUDA(moe::launch_pack_codes_gate_up(sh_up, 1, H, I, Ip, 1, gu + E * gu_group, st));
+  const int dn_rows = moe::kBM * moe::gemm_down_blocks(H);  // the down GEMM's tile rows
+  MOE_CUDA(moe::launch_pack_codes_down(w_down, E, H, I, Ip, dn_rows, dn, st));
+  MOE_CUDA(moe::launch_pack_codes_down(sh_down, 1, H, I, Ip, dn_rows, dn + E * dn_group, st));
+  float* sgu_sh = L->sc_gu + static_cast<size_t>(E) * 2 * Ip;
+  MOE_CUDA(moe::launch_pack_gate_up_scales(s_gate, E, I, Ip, 0, L->sc_gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up_scales(s_up, E, I, Ip, 1, L->sc_gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up_scales(sh_s_gate, 1, I, Ip, 0, sgu_sh, st));
+  MOE_CUDA(moe::launch_pack_gate_up_scales(sh_s_up, 1, I, Ip, 1, sgu_sh, st));
+  MOE_CUDA(cudaMemcpyAsync(L->sc_dn, s_down, static_cast<size_t>(E) * H * sizeof(float),
+                           cudaMemcpyDeviceToDevice, st));
+  MOE_CUDA(cudaMemcpyAsync(L->sc_dn + static_cast<size_t>(E) * H, sh_s_down, H * sizeof(float),
+                           cudaMemcpyDeviceToDevice, st));
+  return load_router(L, router_w, router_bias, st);
+}
+
+int moe_decode_e4m3(const uint8_t* codes, size_t n, uint16_t* out, void* stream) {
+  if (n == 0) return MOE_OK;
+  if (codes == nullptr || out == nullptr || n % 4 != 0 || !aligned(codes, 16) || !aligned(out, 16))
+    return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(moe::launch_decode_e4m3(codes, n, reinterpret_cast<__nv_bfloat16*>(out),
+                                   static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// The router weight and bias: kept fp32, plus the tensor-core router's bf16
+// three-term split and the fp32 transpose.
+int load_router(moe_layer* L, const float* router_w, const float* router_bias, cudaStream_t st) {
+  const moe_config_t& c = L->cfg;
+  const int H = c.hidden, E = c.num_experts;
   MOE_CUDA(cudaMemcpyAsync(L->router_w, router_w, static_cast<size_t>(H) * E * sizeof(float),
                            cudaMemcpyDeviceToDevice, st));
   MOE_CUDA(moe::launch_pack_router(router_w, H, E, L->E_pad, L->router_tc, L->router_t, st));
@@ -282,6 +381,10 @@ int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_
   L->loaded = 1;
   return MOE_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 int moe_workspace_size(const moe_layer_t* L, int T, size_t* bytes) {
   if (L == nullptr || bytes == nullptr || T < 0) return MOE_ERR_INVALID_ARG;
@@ -339,18 +442,19 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   // expert-GEMM tiles: on one SM, 128 tokens x gate|up one 128-feature block
   // (down one or two); on CTA pairs (large T), 256 tokens x gate|up 128
   // features (down 256)
-  const bool pair_gu = T >= moe::kPairMinTokens;
-  const bool pair_dn = T >= moe::kPairMinTokens && (H / moe::kBM) % 2 == 0;
+  // (FP8 weights: always the one-SM tiles, which expand the codes)
+  const bool pair_gu = !L->fp8 && T >= moe::kPairMinTokens;
+  const bool pair_dn = !L->fp8 && T >= moe::kPairMinTokens && (H / moe::kBM) % 2 == 0;
   const int dn_blocks = moe::gemm_down_blocks(H);
-  const int bn_gu = pair_gu ? 2 * moe::kBN : moe::kBN;
-  const int bn_dn = pair_dn ? 2 * moe::kBN : moe::kBN;
+  const int bn_gu = L->fp8 ? moe::kFp8BN : pair_gu ? 2 * moe::kBN : moe::kBN;
+  const int bn_dn = L->fp8 ? moe::kFp8BN : pair_dn ? 2 * moe::kBN : moe::kBN;
   const int mt_gu = Ip / moe::kBM;
   const int mt_dn = pair_dn ? H / (2 * moe::kBM) : H / moe::kBM / dn_blocks;
 
   // Token-row operands, each with kBBoxRows- and kBN-row boxes: x_perm (or x
   // for the shared expert) for K5 and the router, h for K6.
   moe::GemmMaps gu{}, dn{}, rt{};
-  gu.a = pair_gu ? L->tm_gu64 : L->tm_gu;
+  gu.a = pair_gu ? L->tm_gu64 : L->tm_gu;  // (unused with FP8 weights)
   dn.a = L->tm_dn;
   rt.a = L->tm_router;
   if (!encode_bf16_2d(&gu.b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
@@ -373,6 +477,17 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   }
   dn.bsh = dn.b;
   dn.bshw = dn.bw;
+  moe::GemmMaps gu8{}, dn8{};  // FP8 GEMMs: token rows as k-pair maps
+  if (L->fp8) {
+    gu8.out = gu.out;
+    dn8.out = dn.out;
+    if (!encode_bf16_kpair(&gu8.b, x_perm, w.rows_xperm, H, moe::kFp8BN) ||
+        !encode_bf16_kpair(&dn8.b, hbuf, w.rows_all, Ip, moe::kFp8BN) ||
+        (xb && !encode_bf16_kpair(&gu8.bsh, x, T, H, moe::kFp8BN)))
+      return MOE_ERR_CUDA;
+    if (!xb) gu8.bsh = gu8.b;
+    dn8.bsh = dn8.b;
+  }
 
   cudaEvent_t* ev = nullptr;
   if (L->timing_capacity > 0 && L->timing_recorded < L->timing_capacity)
@@ -441,8 +556,11 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.out_ld = Ip;
   p.out_feats = Ip;
   p.w_perm = nullptr;
-  MOE_CUDA(pair_gu ? moe::launch_gemm_gate_up_pair(gu, p, st)
-                : moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
+  p.a_scale = L->fp8 ? L->sc_gu : nullptr;
+  p.a_codes = L->fp8 ? static_cast<const uint8_t*>(L->w_gu) : nullptr;
+  MOE_CUDA(L->fp8    ? moe::launch_gemm_gate_up_fp8(gu8, p, L->num_sms, st)
+           : pair_gu ? moe::launch_gemm_gate_up_pair(gu, p, st)
+                     : moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
   MOE_CUDA(mark(5));
 
   p.tile_start = tiles_dn;
@@ -454,8 +572,11 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.out_ld = H;
   p.out_feats = H;
   p.w_perm = w_perm;
-  MOE_CUDA(pair_dn ? moe::launch_gemm_down_pair(dn, p, st)
-                : moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
+  p.a_scale = L->fp8 ? L->sc_dn : nullptr;
+  p.a_codes = L->fp8 ? static_cast<const uint8_t*>(L->w_dn) : nullptr;
+  MOE_CUDA(L->fp8    ? moe::launch_gemm_down_fp8(dn8, p, L->num_sms, dn_blocks, st)
+           : pair_dn ? moe::launch_gemm_down_pair(dn, p, st)
+                     : moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
   MOE_CUDA(mark(6));
   MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, out, st));
   MOE_CUDA(mark(7));
@@ -582,6 +703,8 @@ void moe_destroy(moe_layer_t* L) {
     free_events(L);
     cudaFree(L->w_gu);
     cudaFree(L->w_dn);
+    cudaFree(L->sc_gu);
+    cudaFree(L->sc_dn);
     cudaFree(L->router_w);
     cudaFree(L->router_b);
     cudaFree(L->router_tc);
@@ -612,6 +735,7 @@ int moe_forward_oneshot(const void* x, const float* router_w, const float* route
   c.weight_dtype = weight_dtype;
   int r = moe_config_check(&c);
   if (r != MOE_OK) return r;
+  if (weight_dtype == MOE_FP8_E4M3) return MOE_ERR_UNSUPPORTED;  // no scales in this list
   if (T < 0) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   moe_layer_t* L = nullptr;

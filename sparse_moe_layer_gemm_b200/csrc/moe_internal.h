@@ -37,6 +37,11 @@ constexpr int kModeRouter = 2;  // logits = acc, fp32, features < valid_feats
 // 256-token tiles; needs an even number of 128-feature blocks in H).
 constexpr int kPairMinTokens = 2048;
 
+// FP8-weight expert GEMMs: tokens per tile (two accumulator buffers of up to
+// two 128 x kFp8BN chains fill half of tensor memory; the expanded weight
+// operands take the other half).
+constexpr int kFp8BN = 64;
+
 // Token count from which the router runs on the tensor cores (bf16 x only),
 // and the K parts of its reduction (the three bf16 terms of W_r).
 constexpr int kTcRouterMinTokens = 512;
@@ -58,6 +63,9 @@ struct GemmParams {
   int out_ld;
   int out_feats;          // output features (columns) that exist; larger ones are not stored
   const float* w_perm;    // down: gate weight of each row (1 for shared rows)
+  const float* a_scale;   // FP8 weights: scale of each packed weight row (A is
+                          // E4M3 codes); nullptr: A is bf16
+  const uint8_t* a_codes; // FP8 weights: the blocked code layout (see pack.cu)
   float limit;            // gate/up clamp of routed experts (<= 0: none)
   float limit_shared;     // gate/up clamp of the shared expert
   int* status;            // device status word
@@ -121,6 +129,15 @@ cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid,
 // = I_pad / 128 (gate|up) or H / 256 (down).
 cudaError_t launch_gemm_gate_up_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st);
 cudaError_t launch_gemm_down_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st);
+// FP8 E4M3 weights (grouped_gemm_fp8.cu): p.a_codes the tile-major code
+// layout (tiles of 256 rows for gate|up, 128 * gemm_down_blocks(H) for down;
+// see pack.cu), p.a_scale the packed rows' scales; m.b / m.bsh the token rows
+// as 3-D maps (64 columns x kFp8BN rows x 2 K-blocks boxes, see
+// encode_bf16_kpair); one-SM tiles of kFp8BN tokens at every T.
+cudaError_t launch_gemm_gate_up_fp8(const GemmMaps& m, const GemmParams& p, int grid,
+                                    cudaStream_t st);
+cudaError_t launch_gemm_down_fp8(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
+                                 cudaStream_t st);
 cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
                                float* dst_t, cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k, int H, bool out_bf16,
@@ -129,6 +146,17 @@ cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, i
                                 int half, __nv_bfloat16* dst, cudaStream_t st);
 cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
                              __nv_bfloat16* dst, cudaStream_t st);
+// FP8 E4M3 weights: the same packing, one byte per code, and the gate|up
+// rows' scales (down's scales need no reordering: row g * H + n)
+cudaError_t launch_pack_codes_gate_up(const uint8_t* w, int groups, int H, int I, int I_pad,
+                                      int half, uint8_t* dst, cudaStream_t st);
+cudaError_t launch_pack_codes_down(const uint8_t* w, int groups, int H, int I, int I_pad,
+                                   int tile_rows, uint8_t* dst, cudaStream_t st);
+cudaError_t launch_pack_gate_up_scales(const float* s, int groups, int I, int I_pad, int half,
+                                       float* dst, cudaStream_t st);
+// n E4M3 codes (n % 4 == 0, 4-byte aligned) -> n bf16 values
+cudaError_t launch_decode_e4m3(const uint8_t* codes, size_t n, __nv_bfloat16* out,
+                               cudaStream_t st);
 
 // Launches `kernel` on `st` with programmatic stream serialization, so it may
 // start (up to its pdl_wait) while the previous kernel of the stream ends.
@@ -150,6 +178,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t gemm_configure_device();
+cudaError_t gemm_fp8_configure_device();
 // also sizes the pair kernels' grid to the co-resident 2-CTA clusters
 cudaError_t gemm_pair_configure_device(int num_sms);
 cudaError_t topk_configure_device();

@@ -6,6 +6,19 @@
 //   down       [G][I][H]  ->  rows g * H + n, columns i (ld I_pad).
 // Rows and columns past I (up to I_pad, a multiple of 128) stay zero, so the
 // padded features compute silu(0) * 0 = 0 and add nothing in the down GEMM.
+// FP8 E4M3 weights use the same packed rows, one byte per code, with one fp32
+// scale per packed row (the row's output feature; zero for padded rows), but
+// stored tile-major for the FP8 GEMM: for each tile of TR packed rows (the
+// GEMM's weight rows per tile) and each 128-wide K slice (one pipeline
+// stage), one contiguous TR x 128 run, ordered (64-code half h, 128-row block
+// b, row r, code): byte ((tile * K / 128 + k / 128) * TR * 128 + h * TR * 64
+// + b * 8192 + r * 64 + chunk position * 16 + k % 16).  Inside a row the
+// 16-code chunk c sits at position c ^ ((r / 2) % 4) (a 64-byte swizzle), so
+// that a warp reading one chunk of 32 consecutive rows hits every
+// shared-memory bank evenly.  A pipeline stage then reads one contiguous
+// TR x 128-byte run with one bulk copy instead of 64-byte pieces of rows
+// K bytes apart.
+#include "fp8.cuh"
 #include "moe_internal.h"
 
 namespace moe {
@@ -77,7 +90,102 @@ __global__ void __launch_bounds__(256) pack_router_kernel(const float* __restric
   }
 }
 
+// Byte offset of packed row `row`, reduction index k, in the tile-major FP8
+// layout (K codes per packed row, tiles of TR rows).
+__device__ __forceinline__ size_t fp8_tiled_offset(size_t row, int k, int K, int TR) {
+  const size_t tile = row / TR;
+  const int rt = static_cast<int>(row % TR), b = rt / 128, r = rt % 128;
+  const int h = (k % 128) / 64, kk = k % 64;
+  return (tile * (K / 128) + k / 128) * static_cast<size_t>(TR) * 128 +
+         static_cast<size_t>(h) * TR * 64 + b * 8192 + r * 64 +
+         ((((kk >> 4) ^ ((r >> 1) & 3))) << 4) + (kk & 15);
+}
+
+// Byte transpose of the [R][C] code matrix of group blockIdx.z (FP8 weights),
+// rows placed as in pack_kernel, bytes in the tile-major layout (K = dst_ld,
+// tiles of TR rows).
+template <bool GU>
+__global__ void __launch_bounds__(256) pack_codes_kernel(const uint8_t* __restrict__ src, int R,
+                                                         int C, uint8_t* __restrict__ dst,
+                                                         int dst_ld, int I_pad, int H, int half,
+                                                         int TR) {
+  __shared__ uint8_t tile[32][33];
+  const int g = blockIdx.z;
+  const uint8_t* s = src + static_cast<size_t>(g) * R * C;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < R && c < C) ? s[static_cast<size_t>(r) * C + c] : 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < C && r < R) {
+      size_t drow;
+      if (GU)
+        drow = static_cast<size_t>(g) * 2 * I_pad + (c / 128) * 256 + half * 128 + (c % 128);
+      else
+        drow = static_cast<size_t>(g) * H + c;
+      dst[fp8_tiled_offset(drow, r, dst_ld, TR)] = tile[threadIdx.x][i];
+    }
+  }
+}
+
+// gate / up scales [G][I] -> the packed gate|up rows' scales.
+__global__ void pack_gate_up_scales_kernel(const float* __restrict__ s, int groups, int I,
+                                           int I_pad, int half, float* __restrict__ dst) {
+  const size_t n = static_cast<size_t>(groups) * I;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int g = static_cast<int>(i / I), f = static_cast<int>(i % I);
+    dst[static_cast<size_t>(g) * 2 * I_pad + (f / 128) * 256 + half * 128 + (f % 128)] = s[i];
+  }
+}
+
+// E4M3 codes -> bf16 through the expert GEMMs' converter routine (4 codes per
+// thread step; n % 4 == 0).
+__global__ void decode_e4m3_kernel(const uint32_t* __restrict__ codes, size_t n4,
+                                   uint2* __restrict__ out) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    uint2 o;
+    e4m3x4_to_bf16x4(codes[i], o.x, o.y);
+    out[i] = o;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_pack_codes_gate_up(const uint8_t* w, int groups, int H, int I, int I_pad,
+                                      int half, uint8_t* dst, cudaStream_t st) {
+  dim3 grid((I + 31) / 32, (H + 31) / 32, groups), block(32, 8);
+  pack_codes_kernel<true><<<grid, block, 0, st>>>(w, H, I, dst, H, I_pad, H, half, 256);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_codes_down(const uint8_t* w, int groups, int H, int I, int I_pad,
+                                   int tile_rows, uint8_t* dst, cudaStream_t st) {
+  dim3 grid((H + 31) / 32, (I + 31) / 32, groups), block(32, 8);
+  pack_codes_kernel<false><<<grid, block, 0, st>>>(w, I, H, dst, I_pad, I_pad, H, 0, tile_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_gate_up_scales(const float* s, int groups, int I, int I_pad, int half,
+                                       float* dst, cudaStream_t st) {
+  pack_gate_up_scales_kernel<<<(groups * I + 255) / 256 < 1024 ? (groups * I + 255) / 256 : 1024,
+                               256, 0, st>>>(s, groups, I, I_pad, half, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_e4m3(const uint8_t* codes, size_t n, __nv_bfloat16* out,
+                               cudaStream_t st) {
+  const size_t n4 = n / 4;
+  const size_t blocks = (n4 + 255) / 256;
+  decode_e4m3_kernel<<<static_cast<unsigned>(blocks < 4096 ? (blocks > 0 ? blocks : 1) : 4096),
+                       256, 0, st>>>(reinterpret_cast<const uint32_t*>(codes), n4,
+                                     reinterpret_cast<uint2*>(out));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
                                float* dst_t, cudaStream_t st) {

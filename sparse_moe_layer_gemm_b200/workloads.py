@@ -73,6 +73,10 @@ WORKLOADS: Dict[str, Workload] = {
     "zipf_prefill": Workload(
         name="zipf_prefill", T=16384, expert_std=0.02, bias="zipf",
         description="load-imbalanced prefill T=16384, Zipf router bias", **_STEP35),
+    "decode_fp8": Workload(
+        name="decode_fp8", T=64, expert_std=0.02, bias="normal0.1",
+        description="decode shape T=64 with FP8 E4M3 expert weights (per-feature scales)",
+        **dict(_STEP35, weight_dtype="fp8")),
     "clamp_ragged": Workload(
         name="clamp_ragged", T=3001, expert_std=0.05, bias="normal0.1",
         swiglu_limit=7.0, swiglu_limit_shared=7.0,

@@ -74,6 +74,36 @@ def output_errors(gpu_out: np.ndarray, ref_out: np.ndarray):
     return rel, mx
 
 
+def expert_views(inp: dict) -> dict:
+    """Lazy per-expert float views of a workload's expert weights (bf16 / fp32
+    tensors widened exactly, FP8 codes dequantized by the oracle), for the
+    ``experts`` argument of :func:`compare`."""
+    if "s_w_gate" in inp:
+        return dict(w_gate=om.DequantizedExperts(inp["w_gate"], inp["s_w_gate"]),
+                    w_up=om.DequantizedExperts(inp["w_up"], inp["s_w_up"]),
+                    w_down=om.DequantizedExperts(inp["w_down"], inp["s_w_down"]),
+                    sh_gate=om.dequantize_e4m3(om.as_numpy(inp["sh_gate"]),
+                                               om.as_numpy(inp["s_sh_gate"])),
+                    sh_up=om.dequantize_e4m3(om.as_numpy(inp["sh_up"]),
+                                             om.as_numpy(inp["s_sh_up"])),
+                    sh_down=om.dequantize_e4m3(om.as_numpy(inp["sh_down"]),
+                                               om.as_numpy(inp["s_sh_down"])))
+    return dict(w_gate=_Widened(inp["w_gate"]), w_up=_Widened(inp["w_up"]),
+                w_down=_Widened(inp["w_down"]), sh_gate=om.as_numpy(inp["sh_gate"]),
+                sh_up=om.as_numpy(inp["sh_up"]), sh_down=om.as_numpy(inp["sh_down"]))
+
+
+class _Widened:
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, e):
+        return om.as_numpy(self.t[e])
+
+    def __len__(self):
+        return len(self.t)
+
+
 def compare(inp_host: dict, wl, gpu_out: np.ndarray, gpu_rt: dict,
             rows: Optional[np.ndarray] = None, experts=None) -> ParityReport:
     """inp_host: exact fp32 host copies of x, router_w, router_bias (and, when

@@ -107,3 +107,18 @@ def test_wait_self_check_rejects_bad_limits_without_cuda(lib):
     from sparse_moe_layer_gemm_b200 import binding as B
     assert B.moe_check_wait_timeout(0)[0] == B.MOE_ERR_INVALID_ARG
     assert B.moe_check_wait_timeout(20_000_000)[0] == B.MOE_ERR_INVALID_ARG
+
+
+def test_fp8_weights_host_checks(lib):
+    assert B.moe_config_check(_cfg(weight_dtype=B.MOE_FP8_E4M3)) == B.MOE_OK
+    assert B.moe_config_check(_cfg(act_dtype=B.MOE_FP8_E4M3)) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_load_weights_fp8(*([None] * 16)) == B.MOE_ERR_INVALID_ARG
+    # the one-shot list has no scales
+    r = lib.moe_forward_oneshot(*([None] * 9), 64, 4096, 288, 8, 1280, 3.0, 0.0, 0.0,
+                                B.MOE_BF16, B.MOE_FP8_E4M3, None, None)
+    assert r == B.MOE_ERR_UNSUPPORTED
+    # decode: n = 0 is a no-op, n % 4 != 0 and NULL pointers are rejected
+    assert lib.moe_decode_e4m3(None, 0, None, None) == B.MOE_OK
+    assert lib.moe_decode_e4m3(None, 8, None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_e4m3(ctypes.c_void_p(256), 6, ctypes.c_void_p(512), None) == \
+        B.MOE_ERR_INVALID_ARG

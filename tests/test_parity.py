@@ -15,7 +15,7 @@ import torch
 from sparse_moe_layer_gemm_b200 import binding as B
 from sparse_moe_layer_gemm_b200.workloads import (WORKLOADS, HostExpertView, draw_router,
                                                   draw_x, host_f32, make_inputs)
-from tests.parity import compare
+from tests.parity import compare, expert_views
 
 pytestmark = pytest.mark.gpu
 
@@ -25,14 +25,15 @@ def _routing_np(rt):
 
 
 def _run_small(wl):
-    inp = {k: v.cuda() for k, v in make_inputs(wl, "cpu").items()}
+    cpu = make_inputs(wl, "cpu")
+    inp = {k: v.cuda() for k, v in cpu.items()}
     layer = B.MoeLayer.from_workload(wl)
     layer.load_inputs(inp)
     out, rt = layer.forward(inp["x"], routing=True)
     torch.cuda.synchronize()
     assert layer.device_error() == 0
-    host = {k: host_f32(v) for k, v in inp.items()}
-    rep = compare(host, wl, host_f32(out), _routing_np(rt))
+    host = {k: host_f32(cpu[k]) for k in ("x", "router_w", "router_bias")}
+    rep = compare(host, wl, host_f32(out), _routing_np(rt), experts=expert_views(cpu))
     layer.close()
     return rep
 
@@ -80,7 +81,41 @@ SMALL = {
                                        num_experts=40, top_k=6, intermediate=128,
                                        shared_intermediate=128, act_dtype="bf16",
                                        weight_dtype="bf16", x_dist="rmsnorm_normal"),
+    # FP8 E4M3 expert weights (codes + per-feature scales), one-SM tiles with
+    # converter warps at every size: padded I (320 -> 384) with two-block down
+    # tiles; odd H (one-block down tiles) with fp32 x; many rows per expert
+    # with the clamp; one token
+    "fp8_multi_tile_ragged": replace(WORKLOADS["tiny"], name="f8m", T=777, hidden=512,
+                                     num_experts=32, top_k=4, intermediate=320,
+                                     shared_intermediate=320, act_dtype="bf16",
+                                     weight_dtype="fp8", x_dist="rmsnorm_normal"),
+    "fp8_odd_hidden_fp32_x": replace(WORKLOADS["tiny"], name="f8o", T=300, hidden=384,
+                                     num_experts=12, top_k=3, intermediate=128,
+                                     shared_intermediate=128, weight_dtype="fp8"),
+    "fp8_clamped_many_rows": replace(WORKLOADS["tiny"], name="f8c", T=2100, hidden=512,
+                                     num_experts=16, top_k=4, intermediate=256,
+                                     shared_intermediate=256, act_dtype="bf16",
+                                     weight_dtype="fp8", x_dist="rmsnorm_normal",
+                                     swiglu_limit=0.9, swiglu_limit_shared=1.3,
+                                     expert_std=0.08),
+    "fp8_single_token": replace(WORKLOADS["tiny"], name="f81", T=1, act_dtype="bf16",
+                                weight_dtype="fp8"),
 }
+
+
+@pytest.mark.timeout(120)
+def test_fp8_decode_every_code():
+    """The GEMMs' E4M3 -> bf16 converter on all 256 codes: every finite code
+    gives the oracle's value exactly (bf16 holds them all), subnormals
+    included; the two NaN codes give +-480 (the format excludes them)."""
+    import oracle.moe_oracle as om
+    codes = torch.arange(256, dtype=torch.uint8, device="cuda")
+    got = B.moe_decode_e4m3(codes).float().cpu().numpy().astype(np.float64)
+    want = om.decode_e4m3(np.arange(256))
+    fin = ~np.isnan(want)
+    assert np.array_equal(got[fin], want[fin])
+    assert got[0x7F] == 480.0 and got[0xFF] == -480.0
+    assert np.signbit(got[0x80])
 
 
 @pytest.mark.timeout(300)
@@ -203,5 +238,26 @@ def test_full_size_clamp_ragged():
     inp = make_inputs(wl, "cuda")
     layer = B.MoeLayer.from_workload(wl)
     rep = _full(wl, inp, layer)
+    layer.close()
+    assert rep.ok(), rep
+
+
+@pytest.mark.timeout(900)
+def test_full_size_fp8_decode():
+    """The decode workload with FP8 E4M3 expert weights (the fp32 draws
+    quantised per output feature), at full size, sampled rows."""
+    wl = replace(WORKLOADS["decode"], name="decode_fp8", weight_dtype="fp8")
+    inp = make_inputs(wl, "cuda")
+    layer = B.MoeLayer.from_workload(wl)
+    layer.load_inputs(inp)
+    out, rt = layer.forward(inp["x"], routing=True)
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    host = {k: host_f32(inp[k]) for k in ("x", "router_w", "router_bias")}
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 24)]))
+    rep = compare(host, wl, host_f32(out), _routing_np(rt), rows=rows,
+                  experts=expert_views(inp))
+    print(wl.name, rep)
     layer.close()
     assert rep.ok(), rep
