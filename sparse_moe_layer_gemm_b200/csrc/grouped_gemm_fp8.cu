@@ -20,14 +20,20 @@
 //                   registers; RB token-row slots, each the tile's rows for
 //                   both k-steps (B, bf16, 128-byte swizzle, one 3-D TMA
 //                   box), freed by the MMA commits (the MMA reads B there);
-//   tensor memory   columns [0, 256): two accumulator buffers; [256, 512): SA
+//   tensor memory   the partial accumulators (chain x stage parity, BN columns
+//                   each; two buffers when they fit in 256 columns), then SA
 //                   stages of expanded weights, 64 columns (128 bf16 of K) per
-//                   128-row accumulator operand, lane = weight row.
+//                   128-row accumulator operand, lane = weight row; smaller
+//                   token tiles leave room for more stages.
 // Warps:
 //   0         code producer (one bulk copy per stage);
 //   1         token-row producer (one TMA load per stage);
-//   2..1+NI   tcgen05.mma issuers, one accumulator chain each (gate and up,
-//             or two weight blocks); warp 2 allocates TMEM;
+//   next 2*NI tcgen05.mma issuers: per accumulator chain (gate and up, or
+//             two weight blocks) two warps taking alternate stages into two
+//             partial accumulators that the epilogue adds (each MMA costs
+//             the issuing thread about a hundred cycles at these shapes, so
+//             one issuer per chain could not keep up with the codes); the
+//             first allocates TMEM;
 //   next 8    converters, two groups of four taking alternate stages: thread
 //             = one weight row of every chain, 64-byte-swizzled code reads
 //             without bank conflicts, E4M3 -> bf16 in registers, tcgen05.st
@@ -57,11 +63,12 @@ struct F8Shape {
   static constexpr int KS = 2;                               // k-steps per pipeline stage
   static constexpr int ROW = BK * 2;                         // bf16 bytes per B row
   static constexpr int ACCS = BLOCKS * (GU ? 2 : 1);         // 128-row accumulators
-  static constexpr int NI = ACCS;                            // one issuer per chain
+  static constexpr int NI = ACCS;                            // accumulator chains
+  static constexpr int NISS = 2 * NI;                        // issuers: chain x stage parity
   static constexpr int GROUPS = 2;                           // converter groups (4 warps each)
   static constexpr int CONV = 4 * GROUPS;
   static constexpr int W_ISS = 2;
-  static constexpr int W_CONV = W_ISS + NI;
+  static constexpr int W_CONV = W_ISS + NISS;
   static constexpr int W_EPI = W_CONV + CONV;
   static constexpr int THREADS = 32 * (W_EPI + 4);
   static constexpr int A_ROWS = kBM * ACCS;
@@ -73,8 +80,9 @@ struct F8Shape {
   static constexpr int RC_FIT = (200 * 1024 - RB * BSLOT) / CSLOT;
   static constexpr int RC = RC_FIT < 8 ? RC_FIT : 8;
   static constexpr int OFF_B = RC * CSLOT;
-  static constexpr int ACC_COLS = ACCS * BN;                 // TMEM columns per buffer
-  static constexpr int A_COL0 = 256;                         // first operand-stage column
+  static constexpr int ACC_COLS = ACCS * 2 * BN;             // TMEM columns per buffer
+  static constexpr int NBUF = 2 * ACC_COLS <= 256 ? 2 : 1;   // accumulator buffers
+  static constexpr int A_COL0 = NBUF * ACC_COLS;             // first operand-stage column
   static constexpr int CHAIN_COLS = KS * BK / 2;             // bf16 pairs of a stage's K
   static constexpr int A_STAGE_COLS = ACCS * CHAIN_COLS;
   static constexpr int SA = (512 - A_COL0) / A_STAGE_COLS;   // operand stages in TMEM
@@ -88,8 +96,11 @@ struct F8Shape {
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(TAB_OFFSET) + kTabBytes;
   static_assert(MODE == kModeGateUp || MODE == kModeDown, "expert GEMMs");
   static_assert(ACCS == 1 || ACCS == 2, "one or two accumulator chains");
-  static_assert(2 * ACC_COLS <= A_COL0, "two accumulator buffers below the operand stages");
-  static_assert(SA % GROUPS == 0, "each converter group owns whole operand stages");
+  static_assert(SA >= 2 && A_COL0 + SA * A_STAGE_COLS <= 512, "tensor memory");
+  // each converter group must wait on every phase of its stages' barriers in
+  // order (a parity wait is ambiguous two phases apart): the groups own
+  // disjoint sets of stages
+  static_assert(SA % GROUPS == 0, "operand stages per converter group");
   static_assert(RC >= 3, "code ring depth");
   static_assert(NBARS * 8 + 8 <= BAR_BYTES, "barrier area");
   static_assert(CSLOT % 1024 == 0 && B_BYTES % 1024 == 0, "slots stay 1024-byte aligned");
@@ -174,10 +185,10 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
       mbar_init(aempty0 + 8 * s, 1); // that chain's MMA commit
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull0 + 8 * b, S::NI);
+      mbar_init(tfull0 + 8 * b, S::NISS);
       mbar_init(tempty0 + 8 * b, 4);
     }
-    mbar_init(drain, S::NI);
+    mbar_init(drain, S::NISS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -272,7 +283,8 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
   } else if (warp < S::W_CONV) {
     // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
-      const int me = warp - S::W_ISS;  // this warp's accumulator chain
+      const int me = (warp - S::W_ISS) % S::NI;                             // chain
+      const uint32_t par = static_cast<uint32_t>((warp - S::W_ISS) / S::NI);  // stage parity
       const uint64_t desc0 = sdesc_k_sw<S::ROW>(smem_u32(smem));
       uint32_t it = 0, tc = 0;
       for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -280,13 +292,18 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
         const Tile t = decode_tile<BN>(gp, w);
         const int n_mma = (t.n_valid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kBM, n_mma);
-        const uint32_t buf = tc & 1u;
-        const uint32_t tph = (tc >> 1) & 1u;
+        const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
+        const uint32_t tph = (S::NBUF == 2 ? (tc >> 1) : tc) & 1u;
         if (!mbar_wait(tempty0 + 8 * buf, tph ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + buf * S::ACC_COLS + me * BN;
-        bool ok = true;
+        // this warp's partial accumulator: stages with it % 2 == par
+        const uint32_t d = tmem_base + buf * S::ACC_COLS + (me * 2 + par) * BN;
+        bool ok = true, first = true;
         for (int st = 0; st < nstage; ++st) {
+          if ((it & 1u) != par) {
+            ++it;
+            continue;
+          }
           const uint32_t rb = it % S::RB, sa = it % S::SA;
           const uint32_t ab = (sa * S::NI + me) * 8;
           // the converters waited for the stage's token rows (and codes)
@@ -302,9 +319,10 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
           for (int kk = 0; kk < S::KS * BK / 16; ++kk)
             mma_issue_ts(d, a_t + kk * 8,
                          bd + static_cast<uint64_t>(((kk / 4) * S::B_BYTES + (kk % 4) * 32) >> 4),
-                         idesc, (st != 0 || kk != 0) ? 1u : 0u);
+                         idesc, (!first || kk != 0) ? 1u : 0u);
           tc_commit(aempty0 + ab);           // the operand stage is free again
           tc_commit(bempty0 + 8 * rb);       // and (both chains) the token rows
+          first = false;
           ++it;
         }
         if (!ok) break;
@@ -319,8 +337,8 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
   } else if (warp < S::W_EPI) {
     // ------------------------------------------------------------ converters
     // Two groups of four warps take alternate stages (group g: stages with
-    // it % 2 == g, always its own operand stages), so one group's barrier
-    // waits overlap the other's expansion.  Warp -> TMEM lane quadrant
+    // it % 2 == g), so one group's barrier waits overlap the other's
+    // expansion.  Warp -> TMEM lane quadrant
     // q = warp % 4 (the only lanes it may write); thread -> weight row
     // q * 32 + lane of every chain: per stage it expands KS x 64 codes per
     // chain, read as 16-byte chunks from the blocks (chunk c of row r stored
@@ -412,8 +430,8 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
     uint32_t tc = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       const Tile t = decode_tile<BN>(gp, w);
-      const uint32_t buf = tc & 1u;
-      const uint32_t tph = (tc >> 1) & 1u;
+      const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
+      const uint32_t tph = (S::NBUF == 2 ? (tc >> 1) : tc) & 1u;
       const size_t row0 = static_cast<size_t>(group_row0(gp, t.g)) + static_cast<size_t>(t.nc) * BN;
       // this lane's feature scale of each chain: weight rows
       // a_row0 + j * 128 + q * 32 + lane
@@ -421,21 +439,27 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
                           static_cast<size_t>(t.mt) * S::A_ROWS + q * 32 + lane;
       const float sc0 = __ldg(p.a_scale + srow);
       const float sc1 = S::ACCS > 1 ? __ldg(p.a_scale + srow + kBM) : 0.f;
-      float wl[BN / 32];
+      constexpr int WL = (BN + 31) / 32;
+      float wl[WL];
       if (MODE == kModeDown) {
 #pragma unroll
-        for (int m = 0; m < BN / 32; ++m)
+        for (int m = 0; m < WL; ++m)
           wl[m] = lane + 32 * m < t.n_valid ? __ldg(p.w_perm + row0 + lane + 32 * m) : 0.f;
       }
       if (!warp_wait(tfull0 + 8 * buf, tph, abort_flag, p.status)) break;
       tc_fence_after();
       if (MODE == kModeDown) {
 #pragma unroll
-        for (int m = 0; m < BN / 32; ++m) wbuf[lane + 32 * m] = wl[m];
+        for (int m = 0; m < WL; ++m)
+          if (lane + 32 * m < BN) wbuf[lane + 32 * m] = wl[m];
         __syncwarp();
       }
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * S::ACC_COLS;
+      // partial accumulators: the one of the tile's first stage parity, plus
+      // the other one when the tile has more than one stage
+      const uint32_t p0 = (static_cast<uint32_t>(tc) * static_cast<uint32_t>(nstage)) & 1u;
+      const bool both = nstage > 1;
 #pragma unroll 1
       for (int b = 0; b < BLOCKS; ++b) {
         const int fblock = t.mt * BLOCKS + b;
@@ -444,17 +468,34 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
         __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
         if (GU) {
           const float L = (t.g == p.E) ? p.limit_shared : p.limit;
-          const uint32_t tg = taddr + (2 * b) * BN, tu = taddr + (2 * b + 1) * BN;
+          // chain 2b (gate) and 2b + 1 (up), partial p at (chain * 2 + p) * BN
+          const uint32_t tg = taddr + (4 * b) * BN, tu = taddr + (4 * b + 2) * BN;
           for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
             uint32_t ra[16], rb[16];
-            tmem_ld_x16(tg + c0, ra);
-            tmem_ld_x16(tu + c0, rb);
+            float ga[16], ua[16];
+            tmem_ld_x16(tg + p0 * BN + c0, ra);
+            tmem_ld_x16(tu + p0 * BN + c0, rb);
             tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              ga[i] = __uint_as_float(ra[i]);
+              ua[i] = __uint_as_float(rb[i]);
+            }
+            if (both) {
+              tmem_ld_x16(tg + (p0 ^ 1u) * BN + c0, ra);
+              tmem_ld_x16(tu + (p0 ^ 1u) * BN + c0, rb);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                ga[i] += __uint_as_float(ra[i]);
+                ua[i] += __uint_as_float(rb[i]);
+              }
+            }
             float hv[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float a = __uint_as_float(ra[i]) * sc0;
-              float u = __uint_as_float(rb[i]) * sc1;
+              float a = ga[i] * sc0;
+              float u = ua[i] * sc1;
               if (L > 0.f) {
                 a = fminf(a, L);
                 u = fminf(fmaxf(u, -L), L);
@@ -465,13 +506,17 @@ __global__ void __launch_bounds__(F8Shape<MODE, BLOCKS>::THREADS, 1)
           }
         } else {
           const float scb = b == 0 ? sc0 : sc1;
+          const uint32_t tb = taddr + (2 * b) * BN;  // chain b's partials
           for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
-            uint32_t ra[16];
-            tmem_ld_x16(taddr + b * BN + c0, ra);
+            uint32_t ra[16], rc[16];
+            tmem_ld_x16(tb + p0 * BN + c0, ra);
+            if (both) tmem_ld_x16(tb + (p0 ^ 1u) * BN + c0, rc);
             tmem_ld_wait();
             float yv[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) yv[i] = __uint_as_float(ra[i]) * scb * wbuf[c0 + i];
+            for (int i = 0; i < 16; ++i)
+              yv[i] = (__uint_as_float(ra[i]) + (both ? __uint_as_float(rc[i]) : 0.f)) * scb *
+                      wbuf[c0 + i];
             store_chunk(yv, c0, t.n_valid, row0, feat, outp);
           }
         }

@@ -37,10 +37,10 @@ constexpr int kModeRouter = 2;  // logits = acc, fp32, features < valid_feats
 // 256-token tiles; needs an even number of 128-feature blocks in H).
 constexpr int kPairMinTokens = 2048;
 
-// FP8-weight expert GEMMs: tokens per tile (two accumulator buffers of up to
-// two 128 x kFp8BN chains fill half of tensor memory; the expanded weight
-// operands take the other half).
-constexpr int kFp8BN = 64;
+// FP8-weight expert GEMMs: tokens per tile (two buffers of up to four
+// 128 x kFp8BN partial accumulators fill half of tensor memory; the expanded
+// weight operands take the other half).
+constexpr int kFp8BN = 32;
 
 // Token count from which the router runs on the tensor cores (bf16 x only),
 // and the K parts of its reduction (the three bf16 terms of W_r).

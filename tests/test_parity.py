@@ -100,6 +100,13 @@ SMALL = {
                                      expert_std=0.08),
     "fp8_single_token": replace(WORKLOADS["tiny"], name="f81", T=1, act_dtype="bf16",
                                 weight_dtype="fp8"),
+    # an odd number of pipeline stages per gate|up tile (H = 384: three) and
+    # many tiles per CTA, so the issuers' stage parity alternates from tile
+    # to tile
+    "fp8_odd_stages_many_tiles": replace(WORKLOADS["tiny"], name="f8s", T=1500, hidden=384,
+                                         num_experts=12, top_k=3, intermediate=192,
+                                         shared_intermediate=192, act_dtype="bf16",
+                                         weight_dtype="fp8", x_dist="rmsnorm_normal"),
 }
 
 
