@@ -41,7 +41,8 @@ def _args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode")
-    ap.add_argument("--secondary", default="prefill,zipf_prefill,clamp_ragged,tiny,decode_fp8",
+    ap.add_argument("--secondary",
+                    default="prefill,zipf_prefill,clamp_ragged,tiny,decode_fp8,dense_decode,dense_prefill",
                     help="comma-separated further workloads measured in the same run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -288,13 +289,65 @@ def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step):
     return rl, layer
 
 
+def _dense_secondary(wl, a, dev, world, rank, stream, peaks):
+    """Times the dense SwiGLU MLP layer (K5 + K6 with one group of all T
+    rows) on its own seeded inputs; roofline of the whole layer (HBM bytes of
+    the weights + x + out, or flops on the sustained bf16 peak)."""
+    import torch
+    from sparse_moe_layer_gemm_b200 import binding as B
+    from sparse_moe_layer_gemm_b200.replicas import job_throughput, max_over_ranks
+    from sparse_moe_layer_gemm_b200.workloads import make_dense_inputs
+    from dataclasses import replace as _replace
+    inp = make_dense_inputs(_replace(wl, seed=wl.seed + rank), dev)
+    layer = B.DenseMLP.from_workload(wl)
+    layer.load_inputs(inp)
+    x = inp["x"]
+    steps, warm = max(3, a.steps // 10), max(3, a.warmup)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            layer.forward(x)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            layer.forward(x)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
+    if layer.device_error() != 0:
+        raise RuntimeError(f"device status word ({wl.name})")
+    el_w = 2 if wl.weight_dtype == "bf16" else 4
+    el_x = 2 if wl.act_dtype == "bf16" else 4
+    H, I, T = wl.hidden, wl.intermediate, wl.T
+    nbytes = 3 * H * I * el_w + 2 * T * H * el_x
+    flops = 6 * T * H * I
+    t_b, t_f = nbytes / (peaks["hbm"] * 1e9), flops / (peaks["tc"] * 1e12)
+    if t_b >= t_f:
+        rl = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peaks["hbm"],
+              "unit": "GB/s"}
+    else:
+        rl = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peaks["tc"],
+              "unit": "TFLOP/s"}
+    rl["frac"] = rl["achieved"] / rl["peak"]
+    rl.update({"scope": "whole dense layer (gate|up + down GEMMs)", "algorithmic_bytes": nbytes,
+               "algorithmic_flops": flops})
+    layer.close()
+    del inp, x
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "T": T, "value": job_throughput(T, world, ms), "unit": "tokens/s",
+            "ms_per_step": ms, "roofline": rl,
+            "layer": f"dense SwiGLU MLP, H={H}, I={I} (the first three decoder layers)"}
+
+
 def run_ours(a):
     import torch
     import torch.distributed as dist
     from sparse_moe_layer_gemm_b200 import binding as B
     from sparse_moe_layer_gemm_b200.replicas import (job_throughput, max_over_ranks,
                                                      rank_batch_workload)
-    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS, draw_x, make_inputs
+    from sparse_moe_layer_gemm_b200.workloads import (DENSE_WORKLOADS, WORKLOADS, draw_x,
+                                                      make_inputs)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -375,6 +428,11 @@ def run_ours(a):
 
     secondary = []
     for name2 in [n for n in (a.secondary or "").split(",") if n and n != "none" and n != a.workload]:
+        if name2 in DENSE_WORKLOADS:  # the dense MLP layer (no routing)
+            barrier()
+            secondary.append(_dense_secondary(DENSE_WORKLOADS[name2], a, dev, world, rank, stream,
+                                              peaks))
+            continue
         wl2 = WORKLOADS[name2]
         same_experts = (wl2.expert_std == wl.expert_std and wl2.weight_dtype == wl.weight_dtype
                         and wl2.hidden == wl.hidden and wl2.num_experts == wl.num_experts

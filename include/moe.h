@@ -261,6 +261,59 @@ int moe_route_static(const void* x, int act_dtype, const float* router_w,
                      int norm_expert_weight, float routed_scaling_factor,
                      int32_t* topk_idx, float* topk_w, void* stream);
 
+/* ---------------------------------------------------------------- dense MLP
+ * The dense SwiGLU MLP of the model's first three decoder layers
+ * (sglang-jax issue #1367, section "Model configuration", MLP bullet: the
+ * first 3 layers are dense, intermediate 11264; llm-atlas "Step-3.5-Flash",
+ * table "Raw config fields", intermediate_size 11264):
+ *
+ *   out = (silu(min(x.W_gate, L)) * clip(x.W_up, -L, L)) . W_down
+ *
+ * (L = 0: no clamp), computed by the MoE layer's expert GEMMs with one group
+ * of all T rows.  Same conventions as the MoE entry points: device pointers,
+ * caller-owned; x [T, H] and out [T, H] in act_dtype; w_gate, w_up [H, I],
+ * w_down [I, H] in weight_dtype (fp32 weights are rounded to bf16 at load);
+ * stream-ordered, no host synchronisation in the forward; every argument is
+ * checked on the host and nothing is enqueued on error. */
+typedef struct moe_dense moe_dense_t;
+
+/* Supported: hidden % 128 == 0, hidden <= 16384; 1 <= intermediate <=
+ * 32768; act_dtype in {F32, BF16}; weight_dtype in {F32, BF16}
+ * (MOE_FP8_E4M3 returns MOE_ERR_UNSUPPORTED); swiglu_limit finite, >= 0. */
+typedef struct {
+  int hidden;          /* H: hidden_size, 4096 */
+  int intermediate;    /* I: intermediate_size, 11264 */
+  float swiglu_limit;  /* clamp, 0 = none */
+  int act_dtype;       /* moe_dtype_t of x and out */
+  int weight_dtype;    /* moe_dtype_t of the weights passed to load */
+} moe_dense_config_t;
+
+/* Host-only check of a configuration; no CUDA call. */
+int moe_dense_config_check(const moe_dense_config_t* cfg);
+
+/* Creates the layer on the current device: packed bf16 weights
+ * (3 * H * round_up(I, 128) elements) and a device status word. */
+int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out);
+
+/* Copies the weights into the packed layout on `stream` (the caller's
+ * buffers may be freed once `stream` has passed this call). */
+int moe_dense_load_weights(moe_dense_t* layer, const void* w_gate, const void* w_up,
+                           const void* w_down, void* stream);
+
+/* Device workspace bytes moe_dense_forward needs for T tokens (256-byte
+ * aligned, caller-allocated).  Host-only. */
+int moe_dense_workspace_size(const moe_dense_t* layer, int T, size_t* bytes);
+
+/* out [T, H] from x [T, H]; x and out must not alias; T = 0 is a no-op. */
+int moe_dense_forward(moe_dense_t* layer, const void* x, int T, void* out,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* As moe_get_device_error, for the dense layer's status word. */
+int moe_dense_get_device_error(moe_dense_t* layer, int* device_err);
+
+/* Frees the layer (synchronises the device first).  NULL is ignored. */
+void moe_dense_destroy(moe_dense_t* layer);
+
 #ifdef __cplusplus
 }
 #endif

@@ -67,6 +67,7 @@ __all__ = [
     "moe_forward_rows",
     "moe_forward_dense_masked",
     "near_tie_gaps",
+    "dense_mlp",
     "decode_e4m3",
     "dequantize_e4m3",
     "DequantizedExperts",
@@ -348,6 +349,19 @@ def moe_forward_dense_masked(x, router_w, router_bias, w_gate, w_up, w_down,
                   for e in range(E)])                      # [E, T, H]
     out = np.einsum("te,eth->th", M, Y)
     return out + swiglu_expert(x64, sh_gate, sh_up, sh_down, swiglu_limit_shared)
+
+
+def dense_mlp(x, w_gate, w_up, w_down, swiglu_limit: float = 0.0) -> np.ndarray:
+    """The model's dense SwiGLU MLP (the first three decoder layers): the same
+    expert function applied to every token, without routing.
+
+    sglang-jax issue #1367, section "Model configuration", MLP bullet (the
+    first 3 layers are dense, intermediate 11264; layers 3-44 are MoE);
+    llm-atlas "Step-3.5-Flash", table "Raw config fields" (intermediate_size
+    11264).  x [T, H]; w_gate, w_up [H, I]; w_down [I, H]; the clamp as in
+    the experts (L <= 0: none).
+    """
+    return swiglu_expert(_f64(x), w_gate, w_up, w_down, swiglu_limit)
 
 
 def decode_e4m3(codes) -> np.ndarray:

@@ -34,6 +34,9 @@ EXPORTS = (
     "moe_status_string", "moe_destroy", "moe_forward_oneshot", "moe_kernel_launches",
     "moe_set_stage_timing", "moe_get_stage_times", "moe_route_static",
     "moe_check_wait_timeout", "moe_load_weights_fp8", "moe_decode_e4m3",
+    "moe_dense_config_check", "moe_dense_create", "moe_dense_load_weights",
+    "moe_dense_workspace_size", "moe_dense_forward", "moe_dense_get_device_error",
+    "moe_dense_destroy",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -51,6 +54,16 @@ class moe_config_t(ctypes.Structure):
         ("use_router_bias", ctypes.c_int),
         ("swiglu_limit", ctypes.c_float),
         ("swiglu_limit_shared", ctypes.c_float),
+        ("act_dtype", ctypes.c_int),
+        ("weight_dtype", ctypes.c_int),
+    ]
+
+
+class moe_dense_config_t(ctypes.Structure):
+    _fields_ = [
+        ("hidden", ctypes.c_int),
+        ("intermediate", ctypes.c_int),
+        ("swiglu_limit", ctypes.c_float),
         ("act_dtype", ctypes.c_int),
         ("weight_dtype", ctypes.c_int),
     ]
@@ -107,10 +120,18 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_check_wait_timeout.argtypes = [i, ctypes.POINTER(i)]
     lib.moe_load_weights_fp8.argtypes = [vp] * 16
     lib.moe_decode_e4m3.argtypes = [vp, sz, vp, vp]
+    lib.moe_dense_config_check.argtypes = [ctypes.POINTER(moe_dense_config_t)]
+    lib.moe_dense_create.argtypes = [ctypes.POINTER(moe_dense_config_t), ctypes.POINTER(vp)]
+    lib.moe_dense_load_weights.argtypes = [vp, vp, vp, vp, vp]
+    lib.moe_dense_workspace_size.argtypes = [vp, i, ctypes.POINTER(sz)]
+    lib.moe_dense_forward.argtypes = [vp, vp, i, vp, vp, sz, vp]
+    lib.moe_dense_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
+    lib.moe_dense_destroy.argtypes = [vp]
+    lib.moe_dense_destroy.restype = None
     lib.moe_get_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i,
                                         ctypes.POINTER(i)]
     for name in EXPORTS:
-        if name not in ("moe_status_string", "moe_destroy"):
+        if name not in ("moe_status_string", "moe_destroy", "moe_dense_destroy"):
             getattr(lib, name).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -415,3 +436,97 @@ def moe_check_wait_timeout(limit_us: int):
     word = ctypes.c_int(-1)
     r = load_library().moe_check_wait_timeout(limit_us, ctypes.byref(word))
     return r, word.value
+
+
+# ----------------------------------------------------------------- dense MLP
+_DT_CODE = {"f32": MOE_F32, "bf16": MOE_BF16, "fp8": MOE_FP8_E4M3}
+
+
+def make_dense_config(hidden, intermediate, swiglu_limit=0.0, act_dtype=MOE_BF16,
+                      weight_dtype=MOE_BF16) -> moe_dense_config_t:
+    return moe_dense_config_t(int(hidden), int(intermediate), float(swiglu_limit),
+                              int(act_dtype), int(weight_dtype))
+
+
+def dense_config_from_workload(wl) -> moe_dense_config_t:
+    return make_dense_config(wl.hidden, wl.intermediate, wl.swiglu_limit,
+                             _DT_CODE[wl.act_dtype], _DT_CODE[wl.weight_dtype])
+
+
+def moe_dense_config_check(cfg: moe_dense_config_t) -> int:
+    return load_library().moe_dense_config_check(ctypes.byref(cfg))
+
+
+class DenseMLP:
+    """The dense SwiGLU MLP layer on the current CUDA device (owns the library
+    handle and a cached workspace)."""
+
+    def __init__(self, cfg: moe_dense_config_t):
+        if not torch.cuda.is_available():
+            raise RuntimeError("DenseMLP needs a CUDA device")
+        self.cfg = cfg
+        self.device = torch.device("cuda", torch.cuda.current_device())
+        h = ctypes.c_void_p()
+        _check(load_library().moe_dense_create(ctypes.byref(cfg), ctypes.byref(h)),
+               "moe_dense_create")
+        self.handle = h.value
+        self._ws: Optional[torch.Tensor] = None
+
+    @classmethod
+    def from_workload(cls, wl) -> "DenseMLP":
+        return cls(dense_config_from_workload(wl))
+
+    def load_weights(self, w_gate, w_up, w_down):
+        c = self.cfg
+        dt = _TORCH_DT[c.weight_dtype]
+        for t, name, shape in ((w_gate, "w_gate", (c.hidden, c.intermediate)),
+                               (w_up, "w_up", (c.hidden, c.intermediate)),
+                               (w_down, "w_down", (c.intermediate, c.hidden))):
+            if t.device != self.device or t.dtype != dt or not t.is_contiguous() \
+                    or tuple(t.shape) != shape:
+                raise ValueError(f"{name}: want contiguous {dt} {shape} on {self.device}")
+        _check(load_library().moe_dense_load_weights(ctypes.c_void_p(self.handle), _ptr(w_gate),
+                                                     _ptr(w_up), _ptr(w_down), _stream(None)),
+               "moe_dense_load_weights")
+
+    def load_inputs(self, inp: Dict[str, torch.Tensor]):
+        self.load_weights(inp["w_gate"], inp["w_up"], inp["w_down"])
+
+    def workspace(self, T: int) -> torch.Tensor:
+        n = ctypes.c_size_t()
+        _check(load_library().moe_dense_workspace_size(ctypes.c_void_p(self.handle), T,
+                                                       ctypes.byref(n)),
+               "moe_dense_workspace_size")
+        if self._ws is None or self._ws.numel() < n.value:
+            self._ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):
+        T = x.shape[0]
+        adt = _TORCH_DT[self.cfg.act_dtype]
+        if x.device != self.device or x.dtype != adt or not x.is_contiguous() \
+                or tuple(x.shape) != (T, self.cfg.hidden):
+            raise ValueError(f"x: want contiguous {adt} (T, {self.cfg.hidden}) on {self.device}")
+        if out is None:
+            out = torch.empty_like(x)
+        ws = self.workspace(T)
+        _check(load_library().moe_dense_forward(ctypes.c_void_p(self.handle), x.data_ptr(), T,
+                                                out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                _stream(stream)), "moe_dense_forward")
+        return out
+
+    def device_error(self) -> int:
+        v = ctypes.c_int()
+        load_library().moe_dense_get_device_error(ctypes.c_void_p(self.handle), ctypes.byref(v))
+        return v.value
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load_library().moe_dense_destroy(ctypes.c_void_p(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

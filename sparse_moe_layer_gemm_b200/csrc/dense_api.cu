@@ -1,0 +1,270 @@
+// The dense SwiGLU MLP of the model's first three decoder layers
+// (sglang-jax issue #1367 "Support Step 3.5 Flash", section "Model
+// configuration", MLP bullet: the first 3 layers are dense with intermediate
+// 11264; llm-atlas "Step-3.5-Flash", table "Raw config fields",
+// intermediate_size 11264), on the MoE layer's expert GEMMs run with one
+// group of all T rows:
+//   h   = silu(min(x.W_gate, L)) * clip(x.W_up, -L, L)   K5 (gate|up + SwiGLU)
+//   out = h . W_down                                       K6 (down, weight 1)
+// Declared in include/moe.h (moe_dense_*).
+#include <math.h>
+#include <string.h>
+
+#include <new>
+
+#include "api_util.h"
+#include "moe_internal.h"
+
+struct moe_dense {
+  moe_dense_config_t cfg;
+  int device;
+  int num_sms;
+  int I_pad;
+  __nv_bfloat16* w_gu;  // [2 * I_pad, H]: blocks of 128 gate rows then 128 up rows
+  __nv_bfloat16* w_dn;  // [H, I_pad]
+  int* status;
+  int loaded;
+  CUtensorMap tm_gu;    // box 64 x 256 (one CTA per tile)
+  CUtensorMap tm_gu64;  // box 64 x 64 (CTA pairs)
+  CUtensorMap tm_dn;    // box 64 x 128
+};
+
+namespace {
+
+constexpr int kMaxTokens = 1 << 20;
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+__global__ void cast_f32_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y,
+                                     size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = __float2bfloat16_rn(x[i]);
+}
+
+__global__ void cast_bf16_f32_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ y,
+                                     size_t n) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    y[i] = __bfloat162float(x[i]);
+}
+
+__global__ void fill_f32_kernel(float* __restrict__ p, float v, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = v;
+}
+
+unsigned grid_for(size_t n, int num_sms) {
+  const size_t blocks = (n + 255) / 256;
+  const size_t cap = static_cast<size_t>(num_sms) * 8;
+  return static_cast<unsigned>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+struct DenseWs {
+  size_t xb, h, y, ones, total;
+};
+
+DenseWs dense_ws(const moe_dense* L, int T) {
+  const size_t H = L->cfg.hidden;
+  DenseWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  const bool xf = L->cfg.act_dtype == MOE_F32;
+  w.xb = xf ? take(static_cast<size_t>(T) * H * 2) : 0;    // bf16 copy of fp32 x
+  w.h = take(static_cast<size_t>(T) * L->I_pad * 2);
+  w.y = xf ? take(static_cast<size_t>(T) * H * 2) : 0;     // bf16 result before widening
+  w.ones = take(static_cast<size_t>(T) * sizeof(float));  // the down GEMM's row weights
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_dense_config_check(const moe_dense_config_t* c) {
+  if (c == nullptr) return MOE_ERR_INVALID_ARG;
+  if (c->hidden <= 0 || c->intermediate <= 0) return MOE_ERR_INVALID_ARG;
+  if ((c->act_dtype != MOE_F32 && c->act_dtype != MOE_BF16) ||
+      (c->weight_dtype != MOE_F32 && c->weight_dtype != MOE_BF16 &&
+       c->weight_dtype != MOE_FP8_E4M3))
+    return MOE_ERR_INVALID_ARG;
+  if (!isfinite(c->swiglu_limit) || c->swiglu_limit < 0.f) return MOE_ERR_INVALID_ARG;
+  if (c->weight_dtype == MOE_FP8_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (c->hidden % 128 != 0 || c->hidden > 16384 || c->intermediate > 32768)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out) {
+  if (out == nullptr) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const int chk = moe_dense_config_check(cfg);
+  if (chk != MOE_OK) return chk;
+  moe_dense* L = new (std::nothrow) moe_dense();
+  if (L == nullptr) return MOE_ERR_CUDA;
+  L->cfg = *cfg;
+  L->I_pad = (cfg->intermediate + 127) / 128 * 128;
+  if (cudaGetDevice(&L->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) !=
+          cudaSuccess) {
+    delete L;
+    return MOE_ERR_CUDA;
+  }
+  const size_t H = cfg->hidden, Ip = L->I_pad;
+  if (moe::gemm_configure_device() != cudaSuccess ||
+      moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
+      cudaMalloc(&L->w_gu, 2 * Ip * H * 2) != cudaSuccess ||
+      cudaMalloc(&L->w_dn, H * Ip * 2) != cudaSuccess ||
+      cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
+      cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess ||
+      !moe::encode_bf16_2d(&L->tm_gu, L->w_gu, 2 * Ip, H, 2 * moe::kBM) ||
+      !moe::encode_bf16_2d(&L->tm_gu64, L->w_gu, 2 * Ip, H, 64) ||
+      !moe::encode_bf16_2d(&L->tm_dn, L->w_dn, H, Ip, moe::kBM)) {
+    moe_dense_destroy(L);
+    return MOE_ERR_CUDA;
+  }
+  *out = L;
+  return MOE_OK;
+}
+
+int moe_dense_load_weights(moe_dense_t* L, const void* w_gate, const void* w_up,
+                           const void* w_down, void* stream) {
+  if (L == nullptr || w_gate == nullptr || w_up == nullptr || w_down == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  moe::DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = L->cfg.hidden, I = L->cfg.intermediate, Ip = L->I_pad;
+  const bool wb = L->cfg.weight_dtype == MOE_BF16;
+  MOE_CUDA(cudaMemsetAsync(L->w_gu, 0, static_cast<size_t>(2) * Ip * H * 2, st));
+  MOE_CUDA(cudaMemsetAsync(L->w_dn, 0, static_cast<size_t>(H) * Ip * 2, st));
+  MOE_CUDA(moe::launch_pack_gate_up(w_gate, wb, 1, H, I, Ip, 0, L->w_gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up(w_up, wb, 1, H, I, Ip, 1, L->w_gu, st));
+  MOE_CUDA(moe::launch_pack_down(w_down, wb, 1, H, I, Ip, L->w_dn, st));
+  L->loaded = 1;
+  return MOE_OK;
+}
+
+int moe_dense_workspace_size(const moe_dense_t* L, int T, size_t* bytes) {
+  if (L == nullptr || bytes == nullptr || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > kMaxTokens) return MOE_ERR_UNSUPPORTED;
+  *bytes = T == 0 ? 0 : dense_ws(L, T).total;
+  return MOE_OK;
+}
+
+int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* workspace,
+                      size_t ws_bytes, void* stream) {
+  if (L == nullptr || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T > kMaxTokens) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (x == nullptr || out == nullptr || x == out) return MOE_ERR_INVALID_ARG;
+  if (!moe::aligned(x, 16) || !moe::aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  const DenseWs w = dense_ws(L, T);
+  if (workspace == nullptr || ws_bytes < w.total || !moe::aligned(workspace, 256))
+    return MOE_ERR_WORKSPACE;
+  moe::DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = L->cfg.hidden, Ip = L->I_pad;
+  const bool xf = L->cfg.act_dtype == MOE_F32;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t n = static_cast<size_t>(T) * H;
+  // bf16 operand rows (x itself when bf16)
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (xf) {
+    __nv_bfloat16* xc = reinterpret_cast<__nv_bfloat16*>(ws + w.xb);
+    cast_f32_bf16_kernel<<<grid_for(n, L->num_sms), 256, 0, st>>>(static_cast<const float*>(x),
+                                                                    xc, n);
+    MOE_CUDA(cudaGetLastError());
+    xb = xc;
+  }
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + w.h);
+  __nv_bfloat16* y = xf ? reinterpret_cast<__nv_bfloat16*>(ws + w.y)
+                        : static_cast<__nv_bfloat16*>(out);
+  float* ones = reinterpret_cast<float*>(ws + w.ones);
+  fill_f32_kernel<<<grid_for(static_cast<size_t>(T), L->num_sms), 256, 0, st>>>(ones, 1.f, T);
+  MOE_CUDA(cudaGetLastError());
+
+  // one group of all T rows; CTA pairs (256-token tiles) from kPairMinTokens
+  const bool pair = T >= moe::kPairMinTokens;
+  const bool pair_dn = pair && (H / moe::kBM) % 2 == 0;
+  const int dn_blocks = moe::gemm_down_blocks(H);
+  moe::GemmMaps gu{}, dn{};
+  gu.a = pair ? L->tm_gu64 : L->tm_gu;
+  dn.a = L->tm_dn;
+  if (!moe::encode_bf16_2d(&gu.b, xb, T, H, moe::kBBoxRows) ||
+      !moe::encode_bf16_2d(&gu.bw, xb, T, H, moe::kBN) ||
+      !moe::encode_bf16_store(&gu.out, h, T, Ip) ||
+      !moe::encode_bf16_2d(&dn.b, h, T, Ip, moe::kBBoxRows) ||
+      !moe::encode_bf16_2d(&dn.bw, h, T, Ip, moe::kBN) ||
+      !moe::encode_bf16_store(&dn.out, y, T, H))
+    return MOE_ERR_CUDA;
+  gu.bsh = gu.b;
+  gu.bshw = gu.bw;
+  dn.bsh = dn.b;
+  dn.bshw = dn.bw;
+
+  moe::GemmParams p{};
+  p.single_rows = T;
+  p.G = 1;
+  p.E = -1;  // no shared group
+  p.k_parts = 1;
+  p.status = L->status;
+  p.limit = L->cfg.swiglu_limit;
+  p.limit_shared = L->cfg.swiglu_limit;
+  p.num_kb = H / (pair ? 2 * moe::kBK : moe::kBK);
+  p.m_tiles = Ip / moe::kBM;
+  p.a_rows_per_group = 2 * Ip;
+  p.out = h;
+  p.out_ld = Ip;
+  p.out_feats = Ip;
+  MOE_CUDA(pair ? moe::launch_gemm_gate_up_pair(gu, p, st)
+                : moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
+
+  p.num_kb = Ip / (pair_dn ? 2 * moe::kBK : moe::kBK);
+  p.m_tiles = pair_dn ? H / (2 * moe::kBM) : H / moe::kBM / dn_blocks;
+  p.a_rows_per_group = H;
+  p.out = y;
+  p.out_ld = H;
+  p.out_feats = H;
+  p.w_perm = ones;
+  MOE_CUDA(pair_dn ? moe::launch_gemm_down_pair(dn, p, st)
+                   : moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
+  if (xf) {
+    cast_bf16_f32_kernel<<<grid_for(n, L->num_sms), 256, 0, st>>>(y, static_cast<float*>(out), n);
+    MOE_CUDA(cudaGetLastError());
+  }
+  return MOE_OK;
+}
+
+int moe_dense_get_device_error(moe_dense_t* L, int* device_err) {
+  if (L == nullptr || device_err == nullptr) return MOE_ERR_INVALID_ARG;
+  moe::DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  int v = 0;
+  MOE_CUDA(cudaDeviceSynchronize());
+  MOE_CUDA(cudaMemcpy(&v, L->status, sizeof(int), cudaMemcpyDeviceToHost));
+  MOE_CUDA(cudaMemset(L->status, 0, sizeof(int)));
+  *device_err = v;
+  return v == 0 ? MOE_OK : MOE_ERR_DEVICE_TIMEOUT;
+}
+
+void moe_dense_destroy(moe_dense_t* L) {
+  if (L == nullptr) return;
+  {
+    moe::DeviceGuard dg(L->device);
+    cudaDeviceSynchronize();
+    cudaFree(L->w_gu);
+    cudaFree(L->w_dn);
+    cudaFree(L->status);
+  }
+  delete L;
+}
+
+}  // extern "C"

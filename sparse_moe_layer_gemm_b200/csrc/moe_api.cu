@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "../../include/moe.h"
+#include "api_util.h"
 #include "moe_internal.h"
 
 using moe::GemmParams;
@@ -44,67 +45,7 @@ struct moe_layer {
   int timing_recorded;
 };
 
-namespace {
-
-constexpr int kMaxTokens = 1 << 20;
-constexpr size_t kAlign = 1024;
-
-size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-struct WsLayout {
-  size_t partial, topk_idx, topk_w, masks, chunk_cnt, chunk_base, counts, row_start, tiles_gu,
-      tiles_dn, perm, pos, w_perm, x_perm, h, y, total;
-  int ksplit, nch, rows_routed, rows_xperm, rows_all;
-};
-
-// K splits of the CUDA-core router: fixed 128-wide K chunks, so a token's
-// logits do not depend on the batch it arrives in; halved (or dropped to one)
-// only if the partial logits would exceed 64 MB.
-int router_ksplit(int T, int H, int E) {
-  constexpr size_t kMaxPartialFloats = static_cast<size_t>(16) << 20;
-  int s = H / 128;
-  while (s > 1 && static_cast<size_t>(T) * E * s > kMaxPartialFloats) s = (s % 2 == 0) ? s / 2 : 1;
-  return s;
-}
-
-WsLayout ws_layout(const moe_layer* L, int T) {
-  const moe_config_t& c = L->cfg;
-  const int H = c.hidden, E = c.num_experts, k = c.top_k, G = E + 1;
-  WsLayout w{};
-  w.ksplit = router_ksplit(T, H, E);
-  w.nch = (T + moe::kSortChunk - 1) / moe::kSortChunk;
-  w.rows_routed = T * k;
-  w.rows_xperm = T * k + (c.act_dtype == MOE_F32 ? T : 0);
-  w.rows_all = T * k + T;
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t at = off;
-    off = align_up(off + bytes, kAlign);
-    return at;
-  };
-  // partial logits: the CUDA-core router's K splits, or the tensor-core
-  // router's three parts
-  const bool tc_router = c.act_dtype == MOE_BF16 && T >= moe::kTcRouterMinTokens;
-  const int parts = tc_router ? moe::kRouterTcParts : w.ksplit;
-  w.partial = take(static_cast<size_t>(parts) * T * E * sizeof(float));
-  w.topk_idx = take(static_cast<size_t>(T) * k * sizeof(int));
-  w.topk_w = take(static_cast<size_t>(T) * k * sizeof(float));
-  w.masks = take(static_cast<size_t>(w.nch) * E * 4 * sizeof(uint32_t));
-  w.chunk_cnt = take(static_cast<size_t>(w.nch) * E * sizeof(int));
-  w.chunk_base = take(static_cast<size_t>(w.nch) * E * sizeof(int));
-  w.counts = take(static_cast<size_t>(G) * sizeof(int));
-  w.row_start = take(static_cast<size_t>(G + 1) * sizeof(int));
-  w.tiles_gu = take(static_cast<size_t>(G + 1) * sizeof(int));
-  w.tiles_dn = take(static_cast<size_t>(G + 1) * sizeof(int));
-  w.perm = take(static_cast<size_t>(T) * k * sizeof(int));
-  w.pos = take(static_cast<size_t>(T) * k * sizeof(int));
-  w.w_perm = take(static_cast<size_t>(w.rows_all) * sizeof(float));
-  w.x_perm = take(static_cast<size_t>(w.rows_xperm) * H * 2);
-  w.h = take(static_cast<size_t>(w.rows_all) * L->I_pad * 2);
-  w.y = take(static_cast<size_t>(w.rows_all) * H * 2);
-  w.total = off;
-  return w;
-}
+namespace moe {
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -169,29 +110,75 @@ bool encode_bf16_store(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols)
   return r == CUDA_SUCCESS;
 }
 
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+}  // namespace moe
 
-// Makes the layer's device current for the lifetime of the guard.
-struct DeviceGuard {
-  int prev = -1;
-  bool ok = true;
-  explicit DeviceGuard(int dev) {
-    if (cudaGetDevice(&prev) != cudaSuccess) {
-      ok = false;
-      return;
-    }
-    if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
-  }
-  ~DeviceGuard() {
-    int cur = -1;
-    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
-  }
+using moe::aligned;
+using moe::DeviceGuard;
+using moe::encode_bf16_2d;
+using moe::encode_bf16_kpair;
+using moe::encode_bf16_store;
+
+namespace {
+
+constexpr int kMaxTokens = 1 << 20;
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t partial, topk_idx, topk_w, masks, chunk_cnt, chunk_base, counts, row_start, tiles_gu,
+      tiles_dn, perm, pos, w_perm, x_perm, h, y, total;
+  int ksplit, nch, rows_routed, rows_xperm, rows_all;
 };
 
-#define MOE_CUDA(call)                          \
-  do {                                          \
-    if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
-  } while (0)
+// K splits of the CUDA-core router: fixed 128-wide K chunks, so a token's
+// logits do not depend on the batch it arrives in; halved (or dropped to one)
+// only if the partial logits would exceed 64 MB.
+int router_ksplit(int T, int H, int E) {
+  constexpr size_t kMaxPartialFloats = static_cast<size_t>(16) << 20;
+  int s = H / 128;
+  while (s > 1 && static_cast<size_t>(T) * E * s > kMaxPartialFloats) s = (s % 2 == 0) ? s / 2 : 1;
+  return s;
+}
+
+WsLayout ws_layout(const moe_layer* L, int T) {
+  const moe_config_t& c = L->cfg;
+  const int H = c.hidden, E = c.num_experts, k = c.top_k, G = E + 1;
+  WsLayout w{};
+  w.ksplit = router_ksplit(T, H, E);
+  w.nch = (T + moe::kSortChunk - 1) / moe::kSortChunk;
+  w.rows_routed = T * k;
+  w.rows_xperm = T * k + (c.act_dtype == MOE_F32 ? T : 0);
+  w.rows_all = T * k + T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  // partial logits: the CUDA-core router's K splits, or the tensor-core
+  // router's three parts
+  const bool tc_router = c.act_dtype == MOE_BF16 && T >= moe::kTcRouterMinTokens;
+  const int parts = tc_router ? moe::kRouterTcParts : w.ksplit;
+  w.partial = take(static_cast<size_t>(parts) * T * E * sizeof(float));
+  w.topk_idx = take(static_cast<size_t>(T) * k * sizeof(int));
+  w.topk_w = take(static_cast<size_t>(T) * k * sizeof(float));
+  w.masks = take(static_cast<size_t>(w.nch) * E * 4 * sizeof(uint32_t));
+  w.chunk_cnt = take(static_cast<size_t>(w.nch) * E * sizeof(int));
+  w.chunk_base = take(static_cast<size_t>(w.nch) * E * sizeof(int));
+  w.counts = take(static_cast<size_t>(G) * sizeof(int));
+  w.row_start = take(static_cast<size_t>(G + 1) * sizeof(int));
+  w.tiles_gu = take(static_cast<size_t>(G + 1) * sizeof(int));
+  w.tiles_dn = take(static_cast<size_t>(G + 1) * sizeof(int));
+  w.perm = take(static_cast<size_t>(T) * k * sizeof(int));
+  w.pos = take(static_cast<size_t>(T) * k * sizeof(int));
+  w.w_perm = take(static_cast<size_t>(w.rows_all) * sizeof(float));
+  w.x_perm = take(static_cast<size_t>(w.rows_xperm) * H * 2);
+  w.h = take(static_cast<size_t>(w.rows_all) * L->I_pad * 2);
+  w.y = take(static_cast<size_t>(w.rows_all) * H * 2);
+  w.total = off;
+  return w;
+}
 
 // The router part of both weight loaders (defined below).
 int load_router(moe_layer* L, const float* router_w, const float* router_bias, cudaStream_t st);

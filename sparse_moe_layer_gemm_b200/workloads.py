@@ -212,3 +212,60 @@ class HostExpertView:
 def host_f32(t: torch.Tensor):
     """Exact float32 host copy (bf16 widens exactly)."""
     return t.detach().float().cpu().numpy()
+
+
+# ---------------------------------------------------------------- dense MLP
+
+@dataclass(frozen=True)
+class DenseWorkload:
+    """The dense SwiGLU MLP of the first three decoder layers (no routing):
+    x [T, H] -> out [T, H] through w_gate, w_up [H, I] and w_down [I, H]."""
+    name: str
+    T: int
+    hidden: int
+    intermediate: int
+    act_dtype: str                 # "f32" or "bf16"
+    weight_dtype: str              # "f32" or "bf16"
+    x_dist: str                    # "normal" or "rmsnorm_normal"
+    weight_std: float
+    swiglu_limit: float = 0.0
+    seed: int = 0
+    description: str = ""
+
+    def with_T(self, T: int) -> "DenseWorkload":
+        return replace(self, T=T)
+
+
+# stream ids of the dense MLP's tensors (disjoint from the MoE layer's)
+_S_DENSE = 500
+
+DENSE_WORKLOADS: Dict[str, DenseWorkload] = {
+    "dense_tiny": DenseWorkload(
+        name="dense_tiny", T=96, hidden=256, intermediate=320, act_dtype="f32",
+        weight_dtype="f32", x_dist="normal", weight_std=0.05,
+        description="T=96, H=256, I=320 (padded to 384), fp32"),
+    "dense_decode": DenseWorkload(
+        name="dense_decode", T=64, hidden=4096, intermediate=11264, act_dtype="bf16",
+        weight_dtype="bf16", x_dist="rmsnorm_normal", weight_std=0.02,
+        description="Step-3.5-Flash dense MLP layer (intermediate 11264), T=64"),
+    "dense_prefill": DenseWorkload(
+        name="dense_prefill", T=4096, hidden=4096, intermediate=11264, act_dtype="bf16",
+        weight_dtype="bf16", x_dist="rmsnorm_normal", weight_std=0.02,
+        description="Step-3.5-Flash dense MLP layer (intermediate 11264), T=4096"),
+}
+
+
+def make_dense_inputs(wl: DenseWorkload, device="cpu") -> Dict[str, torch.Tensor]:
+    """x [T, H] (act dtype); w_gate, w_up [H, I]; w_down [I, H] (weight dtype)."""
+    dev = torch.device(device)
+    x = torch.randn(wl.T, wl.hidden, generator=_gen(dev, wl.seed, _S_DENSE),
+                    device=dev, dtype=torch.float32)
+    if wl.x_dist == "rmsnorm_normal":
+        x = x / torch.sqrt(torch.mean(x * x, dim=1, keepdim=True))
+    g = _gen(dev, wl.seed, _S_DENSE + 1)
+    H, I = wl.hidden, wl.intermediate
+    dt = _torch_dtype(wl.weight_dtype)
+    wg = (torch.randn(H, I, generator=g, device=dev) * wl.weight_std).to(dt)
+    wu = (torch.randn(H, I, generator=g, device=dev) * wl.weight_std).to(dt)
+    wd = (torch.randn(I, H, generator=g, device=dev) * wl.weight_std).to(dt)
+    return dict(x=x.to(_torch_dtype(wl.act_dtype)), w_gate=wg, w_up=wu, w_down=wd)

@@ -122,3 +122,28 @@ def test_fp8_weights_host_checks(lib):
     assert lib.moe_decode_e4m3(None, 8, None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_decode_e4m3(ctypes.c_void_p(256), 6, ctypes.c_void_p(512), None) == \
         B.MOE_ERR_INVALID_ARG
+
+
+def test_dense_host_checks(lib):
+    ok = B.make_dense_config(4096, 11264)
+    assert B.moe_dense_config_check(ok) == B.MOE_OK
+    assert B.moe_dense_config_check(B.make_dense_config(256, 320, act_dtype=B.MOE_F32,
+                                                        weight_dtype=B.MOE_F32)) == B.MOE_OK
+    for cfg, want in ((B.make_dense_config(0, 64), B.MOE_ERR_INVALID_ARG),
+                      (B.make_dense_config(256, 0), B.MOE_ERR_INVALID_ARG),
+                      (B.make_dense_config(256, 64, swiglu_limit=-1.0), B.MOE_ERR_INVALID_ARG),
+                      (B.make_dense_config(256, 64, act_dtype=B.MOE_FP8_E4M3), B.MOE_ERR_INVALID_ARG),
+                      (B.make_dense_config(200, 64), B.MOE_ERR_UNSUPPORTED),
+                      (B.make_dense_config(256, 40000), B.MOE_ERR_UNSUPPORTED),
+                      (B.make_dense_config(256, 64, weight_dtype=B.MOE_FP8_E4M3),
+                       B.MOE_ERR_UNSUPPORTED)):
+        assert B.moe_dense_config_check(cfg) == want
+    assert lib.moe_dense_config_check(None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_dense_create(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_dense_load_weights(None, None, None, None, None) == B.MOE_ERR_INVALID_ARG
+    n = ctypes.c_size_t()
+    assert lib.moe_dense_workspace_size(None, 8, ctypes.byref(n)) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_dense_forward(None, None, 8, None, None, 0, None) == B.MOE_ERR_INVALID_ARG
+    v = ctypes.c_int()
+    assert lib.moe_dense_get_device_error(None, ctypes.byref(v)) == B.MOE_ERR_INVALID_ARG
+    lib.moe_dense_destroy(None)

@@ -1,0 +1,81 @@
+"""GPU parity of the dense SwiGLU MLP (the first three decoder layers) with
+the CPU oracle: small shapes compared on every row (several weight tiles,
+padded I, ragged T, both tile schedules), the full-size decode and prefill
+shapes on sampled rows."""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as om
+from sparse_moe_layer_gemm_b200 import binding as B
+from sparse_moe_layer_gemm_b200.workloads import DENSE_WORKLOADS, host_f32, make_dense_inputs
+from tests.parity import MAX_ABS_OVER_RMS, REL_FRO, output_errors
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny_fp32": DENSE_WORKLOADS["dense_tiny"],
+    "bf16_clamped_ragged": replace(DENSE_WORKLOADS["dense_tiny"], name="dc", T=333, hidden=512,
+                                   intermediate=700, act_dtype="bf16", weight_dtype="bf16",
+                                   x_dist="rmsnorm_normal", swiglu_limit=0.8),
+    "one_token": replace(DENSE_WORKLOADS["dense_tiny"], name="d1", T=1, act_dtype="bf16",
+                         weight_dtype="bf16"),
+    # from 2048 tokens: CTA pairs, 256-token tiles, and a ragged last tile
+    "pairs_ragged": replace(DENSE_WORKLOADS["dense_tiny"], name="dp", T=2100, hidden=512,
+                            intermediate=384, act_dtype="bf16", weight_dtype="bf16",
+                            x_dist="rmsnorm_normal"),
+    # odd H / 128: down tiles of one 128-feature block
+    "odd_hidden_fp32": replace(DENSE_WORKLOADS["dense_tiny"], name="do", T=150, hidden=384,
+                               intermediate=256),
+}
+
+
+def _run(wl, rows=None):
+    cpu_or_dev = "cpu" if wl.hidden * wl.intermediate < (1 << 24) else "cuda"
+    inp = {k: v.cuda() for k, v in make_dense_inputs(wl, cpu_or_dev).items()}
+    layer = B.DenseMLP.from_workload(wl)
+    layer.load_inputs(inp)
+    out = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    rows = np.arange(wl.T) if rows is None else rows
+    x = host_f32(inp["x"])[rows]
+    ref = om.dense_mlp(x, host_f32(inp["w_gate"]), host_f32(inp["w_up"]),
+                       host_f32(inp["w_down"]), wl.swiglu_limit)
+    rel, mx = output_errors(host_f32(out)[rows], ref)
+    layer.close()
+    return rel, mx
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("name", list(SMALL))
+def test_dense_small_parity(name):
+    rel, mx = _run(SMALL[name])
+    assert rel <= REL_FRO and mx <= MAX_ABS_OVER_RMS, (rel, mx)
+
+
+@pytest.mark.timeout(600)
+@pytest.mark.parametrize("name", ["dense_decode", "dense_prefill"])
+def test_dense_full_size_parity(name):
+    wl = DENSE_WORKLOADS[name]
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 24)]))
+    rel, mx = _run(wl, rows)
+    assert rel <= REL_FRO and mx <= MAX_ABS_OVER_RMS, (rel, mx)
+
+
+@pytest.mark.timeout(120)
+def test_dense_deterministic_and_batch_independent():
+    wl = SMALL["bf16_clamped_ragged"]
+    inp = {k: v.cuda() for k, v in make_dense_inputs(wl, "cpu").items()}
+    layer = B.DenseMLP.from_workload(wl)
+    layer.load_inputs(inp)
+    a = layer.forward(inp["x"]).clone()
+    b = layer.forward(inp["x"]).clone()
+    part = layer.forward(inp["x"][100:250].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert torch.equal(part, a[100:250])
+    layer.close()

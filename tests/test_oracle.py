@@ -528,3 +528,38 @@ def test_fp8_workload_quantisation_bound():
     view = om.DequantizedExperts(q["w_up"], q["s_w_up"])
     assert len(view) == wl.num_experts
     assert np.array_equal(view[3], om.dequantize_e4m3(q["w_up"][3].numpy(), q["s_w_up"][3].numpy()))
+
+
+# ---------------------------------------------------------------- dense MLP
+
+def test_dense_mlp_diagonal_closed_form():
+    """Diagonal weights (H = I): out_i = silu(a_i x_i) * (b_i x_i) * c_i per
+    element, written with scalar math.exp; with a clamp L the gate is
+    min(., L) and up clip(., -L, L) before the product."""
+    import math
+    rng = np.random.default_rng(11)
+    n = 7
+    x = rng.normal(size=(3, n))
+    a, b, c = rng.normal(size=n) * 2, rng.normal(size=n) * 2, rng.normal(size=n)
+    for L in (0.0, 0.7):
+        got = om.dense_mlp(x, np.diag(a), np.diag(b), np.diag(c), L)
+        for t in range(3):
+            for i in range(n):
+                g, u = a[i] * x[t, i], b[i] * x[t, i]
+                if L > 0:
+                    g, u = min(g, L), min(max(u, -L), L)
+                want = g / (1.0 + math.exp(-g)) * u * c[i]
+                assert abs(got[t, i] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_dense_mlp_row_independence_and_linearity_in_down():
+    """Each row depends only on its own input (to BLAS summation order);
+    scaling W_down by a power of two scales the output exactly."""
+    rng = np.random.default_rng(12)
+    x = rng.normal(size=(5, 16))
+    wg, wu, wd = (rng.normal(size=s) * 0.3 for s in ((16, 24), (16, 24), (24, 16)))
+    full = om.dense_mlp(x, wg, wu, wd)
+    for t in range(5):
+        np.testing.assert_allclose(om.dense_mlp(x[t:t + 1], wg, wu, wd)[0], full[t],
+                                   rtol=1e-12, atol=1e-12)
+    assert np.array_equal(om.dense_mlp(x, wg, wu, 4.0 * wd), 4.0 * full)
