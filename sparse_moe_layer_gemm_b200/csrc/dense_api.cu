@@ -6,7 +6,10 @@
 // group of all T rows:
 //   h   = silu(min(x.W_gate, L)) * clip(x.W_up, -L, L)   K5 (gate|up + SwiGLU)
 //   out = h . W_down                                       K6 (down, weight 1)
-// Declared in include/moe.h (moe_dense_*).
+// When the tiles of one token block cannot fill the GPU (decode-sized T),
+// both GEMMs split K instead: each part writes raw fp32 accumulators and a
+// reduction kernel sums the parts in fixed order (then applies the SwiGLU, or
+// writes out).  Declared in include/moe.h (moe_dense_*).
 #include <math.h>
 #include <string.h>
 
@@ -25,6 +28,7 @@ struct moe_dense {
   int* status;
   int loaded;
   CUtensorMap tm_gu;    // box 64 x 256 (one CTA per tile)
+  CUtensorMap tm_gu128; // box 64 x 128 (split-K partial tiles)
   CUtensorMap tm_gu64;  // box 64 x 64 (CTA pairs)
   CUtensorMap tm_dn;    // box 64 x 128
 };
@@ -54,6 +58,66 @@ __global__ void fill_f32_kernel(float* __restrict__ p, float v, int n) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = v;
 }
 
+// h[t][f] = silu(min(a, L)) * clip(u, -L, L) with a, u the sums over the S
+// split-K parts (in order) of packed rows (f / 128) * 256 + f % 128 (gate)
+// and that + 128 (up); parts [S][T][2 * I_pad] fp32.
+__global__ void swiglu_parts_kernel(const float* __restrict__ parts, int S, size_t part_stride,
+                                    int T, int I_pad, float L, __nv_bfloat16* __restrict__ h) {
+  const size_t n = static_cast<size_t>(T) * I_pad;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t t = i / I_pad;
+    const int f = static_cast<int>(i % I_pad);
+    const size_t gr = t * 2 * static_cast<size_t>(I_pad) + (f / 128) * 256 + f % 128;
+    float a = 0.f, u = 0.f;
+    for (int z = 0; z < S; ++z) {
+      a += parts[z * part_stride + gr];
+      u += parts[z * part_stride + gr + 128];
+    }
+    if (L > 0.f) {
+      a = fminf(a, L);
+      u = fminf(fmaxf(u, -L), L);
+    }
+    h[i] = __float2bfloat16_rn(a / (1.0f + __expf(-a)) * u);
+  }
+}
+
+// out[i] = sum over the S parts (in order) of parts[z][i].
+template <typename TO>
+__global__ void sum_parts_kernel(const float* __restrict__ parts, int S, size_t part_stride,
+                                 size_t n, TO* __restrict__ out) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float v = 0.f;
+    for (int z = 0; z < S; ++z) v += parts[z * part_stride + i];
+    if constexpr (sizeof(TO) == 2)
+      out[i] = __float2bfloat16_rn(v);
+    else
+      out[i] = v;
+  }
+}
+
+// Split-K parts for a GEMM whose tiles (one token block) are too few for the
+// GPU: the smallest divisor S of the k-block count (up to 16) that fills the
+// SMs' waves to >= 85 %, else the best filling one; 1 when the tiles already
+// fill the GPU.
+int choose_parts(int tiles, int num_kb, int num_sms) {
+  if (tiles >= num_sms) return 1;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int S = 1; S <= 16; ++S) {
+    if (num_kb % S != 0 || num_kb / S < 2) continue;
+    const int n = tiles * S;
+    const double eff = static_cast<double>(n) / (((n + num_sms - 1) / num_sms) * num_sms);
+    if (eff >= 0.85) return S;
+    if (eff > best_eff + 1e-9) {
+      best = S;
+      best_eff = eff;
+    }
+  }
+  return best;
+}
+
 unsigned grid_for(size_t n, int num_sms) {
   const size_t blocks = (n + 255) / 256;
   const size_t cap = static_cast<size_t>(num_sms) * 8;
@@ -61,7 +125,8 @@ unsigned grid_for(size_t n, int num_sms) {
 }
 
 struct DenseWs {
-  size_t xb, h, y, ones, total;
+  size_t xb, h, y, ones, parts, total;
+  int s_gu, s_dn;  // split-K parts of the two GEMMs (1: no split)
 };
 
 DenseWs dense_ws(const moe_dense* L, int T) {
@@ -78,6 +143,19 @@ DenseWs dense_ws(const moe_dense* L, int T) {
   w.h = take(static_cast<size_t>(T) * L->I_pad * 2);
   w.y = xf ? take(static_cast<size_t>(T) * H * 2) : 0;     // bf16 result before widening
   w.ones = take(static_cast<size_t>(T) * sizeof(float));  // the down GEMM's row weights
+  // split-K only below the CTA-pair range (one token block of tiles)
+  const int Ip = L->I_pad;
+  const int tok_blocks = (T + moe::kBN - 1) / moe::kBN;
+  const bool small = T < moe::kPairMinTokens && (L->cfg.hidden / moe::kBM) % 2 == 0;
+  w.s_gu = small ? choose_parts((Ip / moe::kBM) * tok_blocks, L->cfg.hidden / moe::kBK,
+                                L->num_sms)
+                 : 1;
+  w.s_dn = small ? choose_parts((L->cfg.hidden / (2 * moe::kBM)) * tok_blocks, Ip / moe::kBK,
+                                L->num_sms)
+                 : 1;
+  const size_t gu_parts = w.s_gu > 1 ? static_cast<size_t>(w.s_gu) * T * 2 * Ip : 0;
+  const size_t dn_parts = w.s_dn > 1 ? static_cast<size_t>(w.s_dn) * T * H : 0;
+  w.parts = take((gu_parts > dn_parts ? gu_parts : dn_parts) * sizeof(float));
   w.total = off;
   return w;
 }
@@ -123,6 +201,7 @@ int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out) {
       cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
       cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess ||
       !moe::encode_bf16_2d(&L->tm_gu, L->w_gu, 2 * Ip, H, 2 * moe::kBM) ||
+      !moe::encode_bf16_2d(&L->tm_gu128, L->w_gu, 2 * Ip, H, moe::kBM) ||
       !moe::encode_bf16_2d(&L->tm_gu64, L->w_gu, 2 * Ip, H, 64) ||
       !moe::encode_bf16_2d(&L->tm_dn, L->w_dn, H, Ip, moe::kBM)) {
     moe_dense_destroy(L);
@@ -188,8 +267,10 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
   __nv_bfloat16* y = xf ? reinterpret_cast<__nv_bfloat16*>(ws + w.y)
                         : static_cast<__nv_bfloat16*>(out);
   float* ones = reinterpret_cast<float*>(ws + w.ones);
-  fill_f32_kernel<<<grid_for(static_cast<size_t>(T), L->num_sms), 256, 0, st>>>(ones, 1.f, T);
-  MOE_CUDA(cudaGetLastError());
+  if (w.s_dn <= 1) {  // the unsplit down GEMM's row weights
+    fill_f32_kernel<<<grid_for(static_cast<size_t>(T), L->num_sms), 256, 0, st>>>(ones, 1.f, T);
+    MOE_CUDA(cudaGetLastError());
+  }
 
   // one group of all T rows; CTA pairs (256-token tiles) from kPairMinTokens
   const bool pair = T >= moe::kPairMinTokens;
@@ -218,6 +299,74 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
   p.status = L->status;
   p.limit = L->cfg.swiglu_limit;
   p.limit_shared = L->cfg.swiglu_limit;
+  float* parts = reinterpret_cast<float*>(ws + w.parts);
+  const int sgrid = L->num_sms;
+
+  if (w.s_gu > 1) {
+    // gate|up in S parts of K: raw accumulators of all 2 * I_pad packed rows
+    moe::GemmMaps pg = gu;
+    pg.a = L->tm_gu128;
+    p.k_parts = w.s_gu;
+    p.num_kb = H / moe::kBK / w.s_gu;
+    p.m_tiles = 2 * Ip / (2 * moe::kBM);
+    p.a_rows_per_group = 2 * Ip;
+    p.out_f32 = parts;
+    p.out_ld = 2 * Ip;
+    p.out_feats = 2 * Ip;
+    p.part_stride = static_cast<size_t>(T) * 2 * Ip;
+    MOE_CUDA(moe::launch_gemm_partial(pg, p, sgrid, st));
+    swiglu_parts_kernel<<<grid_for(static_cast<size_t>(T) * Ip, L->num_sms), 256, 0, st>>>(
+        parts, w.s_gu, p.part_stride, T, Ip, L->cfg.swiglu_limit, h);
+    MOE_CUDA(cudaGetLastError());
+  }
+  if (w.s_dn > 1) {
+    if (w.s_gu <= 1) {  // gate|up unsplit
+      p.k_parts = 1;
+      p.num_kb = H / moe::kBK;
+      p.m_tiles = Ip / moe::kBM;
+      p.a_rows_per_group = 2 * Ip;
+      p.out = h;
+      p.out_ld = Ip;
+      p.out_feats = Ip;
+      MOE_CUDA(moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
+    }
+    // down in S parts of K, then the sum in order
+    p.k_parts = w.s_dn;
+    p.num_kb = Ip / moe::kBK / w.s_dn;
+    p.m_tiles = H / (2 * moe::kBM);
+    p.a_rows_per_group = H;
+    p.out_f32 = parts;
+    p.out_ld = H;
+    p.out_feats = H;
+    p.part_stride = static_cast<size_t>(T) * H;
+    MOE_CUDA(moe::launch_gemm_partial(dn, p, sgrid, st));
+    if (xf)
+      sum_parts_kernel<float><<<grid_for(n, L->num_sms), 256, 0, st>>>(
+          parts, w.s_dn, p.part_stride, n, static_cast<float*>(out));
+    else
+      sum_parts_kernel<__nv_bfloat16><<<grid_for(n, L->num_sms), 256, 0, st>>>(
+          parts, w.s_dn, p.part_stride, n, static_cast<__nv_bfloat16*>(out));
+    MOE_CUDA(cudaGetLastError());
+    return MOE_OK;
+  }
+  if (w.s_gu > 1) {  // down unsplit after a split gate|up
+    p.k_parts = 1;
+    p.num_kb = Ip / moe::kBK;
+    p.m_tiles = H / moe::kBM / dn_blocks;
+    p.a_rows_per_group = H;
+    p.out = y;
+    p.out_ld = H;
+    p.out_feats = H;
+    p.w_perm = ones;
+    MOE_CUDA(moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
+    if (xf) {
+      cast_bf16_f32_kernel<<<grid_for(n, L->num_sms), 256, 0, st>>>(y, static_cast<float*>(out),
+                                                                     n);
+      MOE_CUDA(cudaGetLastError());
+    }
+    return MOE_OK;
+  }
+
   p.num_kb = H / (pair ? 2 * moe::kBK : moe::kBK);
   p.m_tiles = Ip / moe::kBM;
   p.a_rows_per_group = 2 * Ip;

@@ -6,6 +6,9 @@
 //                  h = silu(gate) * up, stored bf16.
 //   K6 (down):     y = (h_g . Wd_g) * w_row, the row's gate weight (1 for the
 //                  shared rows), stored bf16.
+//   split-K partials (dense MLP at small T): part z of a single group's
+//                  product over K slice z, raw fp32 accumulators per packed
+//                  weight row; a reduction kernel finishes the layer.
 //   K1 (router, large T):  logits = x . W_r on the bf16 tensor cores: W_r =
 //                  W1 + W2 + W3 split into three bf16 terms concatenated along
 //                  K; the tiles of part z accumulate x . Wz (each bf16 x bf16
@@ -59,6 +62,8 @@ struct Shape {
   // router with BLOCKS = 2: one weight block, the tile's tokens split into two
   // halves, one accumulator (and issuer) each
   static constexpr bool TOKSPLIT = MODE == kModeRouter && BLOCKS == 2;
+  // fp32 outputs straight from the accumulators (no tables, no TMA stores)
+  static constexpr bool F32OUT = MODE == kModeRouter || MODE == kModePartial;
   static constexpr int BN = BN_;
   static constexpr int BK = kBK;
   static constexpr int ROW = BK * 2;                        // bytes per operand row in SMEM
@@ -82,10 +87,10 @@ struct Shape {
   // bf16 staging buffers for TMA stores of h or y
   // (down: plus per warp the tile's BN gate weights, fp32)
   static constexpr int EPI_STAGE_BYTES =
-      MODE != kModeRouter ? 4 * 2 * kEpiRows * 32 * 2 + (MODE == kModeDown ? 4 * BN * 4 : 0) : 0;
+      !F32OUT ? 4 * 2 * kEpiRows * 32 * 2 + (MODE == kModeDown ? 4 * BN * 4 : 0) : 0;
   // group tables (tile_start, counts, row_start) copied to shared memory
   static constexpr int TAB_OFFSET = STAGES * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES;
-  static constexpr int TAB_BYTES = MODE != kModeRouter ? kTabBytes : 0;
+  static constexpr int TAB_BYTES = !F32OUT ? kTabBytes : 0;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(TAB_OFFSET) + TAB_BYTES;
   static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
   static_assert(NBUF * ACC_COLS <= 512, "TMEM capacity");
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
   pdl_wait();
   // group tables in shared memory (visible after the __syncthreads below)
   const GemmParams gp =
-      MODE != kModeRouter ? stage_group_tables(p, reinterpret_cast<int*>(smem + S::TAB_OFFSET)) : p;
+      !S::F32OUT ? stage_group_tables(p, reinterpret_cast<int*>(smem + S::TAB_OFFSET)) : p;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -203,6 +208,9 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
         const uint32_t bytes = S::A_BYTES + (wide ? nbox * kBN * S::ROW : S::B_BOX_BYTES);
         const uint64_t pol_a = t.nch > 1 ? pol_normal : pol_first;
         const int a_k0 = t.kz * p.num_kb * BK;  // K part of a split-K tile
+        // router: every part multiplies the same token rows (the parts are
+        // terms of W_r); split-K partials: the token rows' own K slice
+        const int b_k0 = MODE == kModePartial ? a_k0 : 0;
         bool ok = true;
         for (int kb = 0; kb < p.num_kb; ++kb) {
           const uint32_t s = it % S::STAGES;
@@ -219,7 +227,8 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
             tma_load_2d(sa + i * S::A_BOX * S::ROW, &tmA, fb, a_k0 + kb * BK, a_row + i * S::A_BOX,
                         pol_a);
           for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sa + S::A_BYTES + i * kBN * S::ROW, mb, fb, kb * BK, b_row + i * kBN, pol_b);
+            tma_load_2d(sa + S::A_BYTES + i * kBN * S::ROW, mb, fb, b_k0 + kb * BK,
+                        b_row + i * kBN, pol_b);
           ++it;
         }
         if (!ok) break;
@@ -302,7 +311,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
                                            4 * 2 * kEpiRows * 32 * 2) +
                   (warp - (1 + S::NI)) * BN;
     uint32_t chunks = 0;  // TMA-store chunks this warp has issued
-    if (MODE != kModeRouter && lane == 0) prefetch_tmap(&tmOut);
+    if (!S::F32OUT && lane == 0) prefetch_tmap(&tmOut);
     // Writes rows [c0, c0 + 16) of this lane's output feature.  A chunk whose
     // 16 rows all belong to the tile goes through a staging buffer and one
     // TMA store of 16 x 32 values; a ragged one is stored directly, so no row
@@ -359,7 +368,19 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
         const int fblock = S::TOKSPLIT ? t.mt : t.mt * BLOCKS + b;  // 128-feature block
         const int feat = fblock * kBM + q * 32 + lane;
         if (fblock * kBM >= p.out_feats) break;  // never past the output
-        if (MODE == kModeRouter) {
+        if (MODE == kModePartial) {
+          // raw accumulators of packed weight row prow for the tile's tokens
+          const int prow = fblock * kBM + q * 32 + lane;
+          float* pp = p.out_f32 + t.kz * p.part_stride + row0 * p.out_ld + prow;
+          for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t ra[16];
+            tmem_ld_x16(taddr + b * BN + c0, ra);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c0 + i < t.n_valid) pp[static_cast<size_t>(c0 + i) * p.out_ld] = __uint_as_float(ra[i]);
+          }
+        } else if (MODE == kModeRouter) {
           // token split: accumulator b holds tokens [b * ACC_N, (b + 1) * ACC_N)
           const int tok0 = S::TOKSPLIT ? b * S::ACC_N : 0;
           const int n_b = S::TOKSPLIT ? min(S::ACC_N, t.n_valid - tok0) : t.n_valid;
@@ -414,7 +435,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
       if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
       ++tc;
     }
-    if (MODE != kModeRouter && lane == 0) bulk_wait_group_all();  // h / y fully written
+    if (!S::F32OUT && lane == 0) bulk_wait_group_all();  // h / y fully written
   }
 
   tc_fence_before();
@@ -434,6 +455,7 @@ using GuCfg = Shape<kModeGateUp, 1, 128>;
 using DnCfg2 = Shape<kModeDown, 2, 128>;
 using DnCfg1 = Shape<kModeDown, 1, 128>;
 using RtCfg = Shape<kModeRouter, 2, 256>;  // 256-token tiles, one accumulator per half
+using PtCfg = Shape<kModePartial, 2, 128>;  // two 128-row blocks, 128-token tiles
 
 template <typename S, int MODE, int BLOCKS>
 cudaError_t set_smem() {
@@ -449,6 +471,7 @@ cudaError_t gemm_configure_device() {
   if ((e = set_smem<GuCfg, kModeGateUp, 1>()) != cudaSuccess) return e;
   if ((e = set_smem<DnCfg2, kModeDown, 2>()) != cudaSuccess) return e;
   if ((e = set_smem<DnCfg1, kModeDown, 1>()) != cudaSuccess) return e;
+  if ((e = set_smem<PtCfg, kModePartial, 2>()) != cudaSuccess) return e;
   return set_smem<RtCfg, kModeRouter, 2>();
 }
 
@@ -471,6 +494,15 @@ cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, i
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
   return launch_pdl(grouped_gemm_kernel<kModeRouter, 2, 256>, dim3(grid), dim3(RtCfg::THREADS),
                     RtCfg::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
+}
+
+}  // namespace moe
+
+namespace moe {
+
+cudaError_t launch_gemm_partial(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
+  return launch_pdl(grouped_gemm_kernel<kModePartial, 2, 128>, dim3(grid), dim3(PtCfg::THREADS),
+                    PtCfg::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 
 }  // namespace moe

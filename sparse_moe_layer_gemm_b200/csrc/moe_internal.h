@@ -32,6 +32,8 @@ constexpr int kSortChunk = 128;
 constexpr int kModeGateUp = 0;  // h = silu(clamp(gate)) * clamp(up), bf16
 constexpr int kModeDown = 1;    // y = acc * w_perm[row], bf16
 constexpr int kModeRouter = 2;  // logits = acc, fp32, features < valid_feats
+constexpr int kModePartial = 3; // split-K part z of one group: raw fp32 accumulators of
+                                // every packed weight row, at out_f32 + z * part_stride
 
 // Token count from which the expert GEMMs run on CTA pairs (2-SM UMMA,
 // 256-token tiles; needs an even number of 128-feature blocks in H).
@@ -124,6 +126,10 @@ cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid
 cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
                              cudaStream_t st);
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
+// Split-K partial products of one group (single_rows, k_parts parts of num_kb
+// k-blocks; A and B both offset by the part's K): m.a with 128-row boxes, two
+// 128-row weight blocks per tile; fp32 [T, out_ld] per part.
+cudaError_t launch_gemm_partial(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
 // CTA-pair versions (grouped_gemm_pair.cu): m.a has 64-row boxes for gate|up
 // and 128-row boxes for down; tiles of 256 tokens; num_kb = K / 128; m_tiles
 // = I_pad / 128 (gate|up) or H / 256 (down).
