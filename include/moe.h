@@ -111,6 +111,22 @@ int moe_config_check(const moe_config_t* cfg);
  * error). */
 int moe_create(const moe_config_t* cfg, moe_layer_t** out);
 
+/* Expert parallelism: a layer holding only the routed experts
+ * [expert_first, expert_first + expert_count) of the configuration's E (and
+ * the shared expert if with_shared is 1).  Routing still covers all E
+ * experts (the router weight is loaded whole); moe_forward then computes only
+ * this shard's experts for the pairs that selected them (and the shared
+ * expert if held) and writes their weighted sum to out: summed over shards
+ * that cover every expert once (and the shared expert once), e.g. by an
+ * all-reduce across the GPUs that hold them, it is the layer's output.  The
+ * load entry points take the full [E, ...] expert tensors and pick the
+ * shard's slice.  With a shard, moe_routing_t's counts [expert_count] and
+ * offsets [expert_count + 1] are the shard's, perm lists its pairs first.
+ * Returns MOE_ERR_INVALID_ARG for an empty or out-of-range expert range or
+ * with_shared not 0/1.  moe_create(cfg) is moe_create_shard(cfg, 0, E, 1). */
+int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count,
+                     int with_shared, moe_layer_t** out);
+
 /* Copies the weights into the layer's packed bf16 layout on `stream`
  * (K-major weight rows; gate and up interleaved in blocks of 128 rows; fp32
  * expert weights are rounded to bf16).  router_w [H, E] and router_bias [E]

@@ -36,7 +36,7 @@ EXPORTS = (
     "moe_check_wait_timeout", "moe_load_weights_fp8", "moe_decode_e4m3",
     "moe_dense_config_check", "moe_dense_create", "moe_dense_load_weights",
     "moe_dense_workspace_size", "moe_dense_forward", "moe_dense_get_device_error",
-    "moe_dense_destroy",
+    "moe_dense_destroy", "moe_create_shard",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -103,6 +103,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
     lib.moe_config_check.argtypes = [ctypes.POINTER(moe_config_t)]
     lib.moe_create.argtypes = [ctypes.POINTER(moe_config_t), ctypes.POINTER(vp)]
+    lib.moe_create_shard.argtypes = [ctypes.POINTER(moe_config_t), i, i, i, ctypes.POINTER(vp)]
     lib.moe_load_weights.argtypes = [vp] * 9 + [vp]
     lib.moe_workspace_size.argtypes = [vp, i, ctypes.POINTER(sz)]
     lib.moe_workspace_size_host.argtypes = [vp, i, ctypes.POINTER(sz)]
@@ -177,6 +178,15 @@ def moe_config_check(cfg: moe_config_t) -> int:
 def moe_create(cfg: moe_config_t) -> int:
     h = ctypes.c_void_p()
     _check(load_library().moe_create(ctypes.byref(cfg), ctypes.byref(h)), "moe_create")
+    return h.value
+
+
+def moe_create_shard(cfg: moe_config_t, expert_first: int, expert_count: int,
+                     with_shared: bool) -> int:
+    h = ctypes.c_void_p()
+    _check(load_library().moe_create_shard(ctypes.byref(cfg), int(expert_first), int(expert_count),
+                                           int(bool(with_shared)), ctypes.byref(h)),
+           "moe_create_shard")
     return h.value
 
 
@@ -298,17 +308,19 @@ class MoeLayer:
     """One layer on the current CUDA device: owns the library handle (and its
     packed weights) and a cached device workspace."""
 
-    def __init__(self, cfg: moe_config_t):
+    def __init__(self, cfg: moe_config_t, shard: Optional[tuple] = None):
+        """shard: (expert_first, expert_count, with_shared) for an expert
+        shard (see moe_create_shard), else the whole layer."""
         if not torch.cuda.is_available():
             raise RuntimeError("MoeLayer needs a CUDA device")
         self.cfg = cfg
         self.device = torch.device("cuda", torch.cuda.current_device())
-        self.handle = moe_create(cfg)
+        self.handle = moe_create(cfg) if shard is None else moe_create_shard(cfg, *shard)
         self._ws: Optional[torch.Tensor] = None
 
     @classmethod
-    def from_workload(cls, wl) -> "MoeLayer":
-        return cls(config_from_workload(wl))
+    def from_workload(cls, wl, shard: Optional[tuple] = None) -> "MoeLayer":
+        return cls(config_from_workload(wl), shard)
 
     @property
     def act_dtype(self) -> torch.dtype:

@@ -23,6 +23,9 @@ struct moe_layer {
   int num_sms;
   int I_pad;
   int fp8;              // expert weights are E4M3 codes (one byte each) + scales
+  int first;            // expert shard: the layer holds experts [first, first + E_loc)
+  int E_loc;            //   (E_loc = E: all of them)
+  int with_shared;      //   and the shared expert if set
   void* w_gu;           // [(E+1) * 2 * I_pad, H] bf16 or E4M3 codes
   void* w_dn;           // [(E+1) * H, I_pad] bf16 or E4M3 codes
   float* sc_gu;         // FP8: scale of each packed gate|up row [(E+1) * 2 * I_pad]
@@ -127,7 +130,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
   size_t partial, topk_idx, topk_w, masks, chunk_cnt, chunk_base, counts, row_start, tiles_gu,
-      tiles_dn, perm, pos, w_perm, x_perm, h, y, total;
+      tiles_dn, perm, pos, w_perm, x_perm, h, y, local_idx, total;
   int ksplit, nch, rows_routed, rows_xperm, rows_all;
 };
 
@@ -176,6 +179,9 @@ WsLayout ws_layout(const moe_layer* L, int T) {
   w.x_perm = take(static_cast<size_t>(w.rows_xperm) * H * 2);
   w.h = take(static_cast<size_t>(w.rows_all) * L->I_pad * 2);
   w.y = take(static_cast<size_t>(w.rows_all) * H * 2);
+  // expert shard: the selection in local expert ids (-1: another shard's)
+  const bool shard = L->E_loc != E || L->first != 0;
+  w.local_idx = shard ? take(static_cast<size_t>(T) * k * sizeof(int)) : 0;
   w.total = off;
   return w;
 }
@@ -220,13 +226,28 @@ int moe_config_check(const moe_config_t* c) {
 }
 
 int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
+  if (cfg == nullptr) {
+    if (out != nullptr) *out = nullptr;
+    return MOE_ERR_INVALID_ARG;
+  }
+  return moe_create_shard(cfg, 0, cfg->num_experts, 1, out);
+}
+
+int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count,
+                     int with_shared, moe_layer_t** out) {
   if (out == nullptr) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   const int chk = moe_config_check(cfg);
   if (chk != MOE_OK) return chk;
+  if (expert_first < 0 || expert_count < 1 || expert_first + expert_count > cfg->num_experts ||
+      (with_shared != 0 && with_shared != 1))
+    return MOE_ERR_INVALID_ARG;
   moe_layer* L = new (std::nothrow) moe_layer();
   if (L == nullptr) return MOE_ERR_CUDA;
   L->cfg = *cfg;
+  L->first = expert_first;
+  L->E_loc = expert_count;
+  L->with_shared = with_shared;
   L->fp8 = cfg->weight_dtype == MOE_FP8_E4M3 ? 1 : 0;
   L->I_pad = (cfg->intermediate + 127) / 128 * 128;
   L->E_pad = (cfg->num_experts + 127) / 128 * 128;
@@ -236,9 +257,11 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
     delete L;
     return MOE_ERR_CUDA;
   }
-  const size_t H = cfg->hidden, E = cfg->num_experts, Ip = L->I_pad;
+  // expert weights: the shard's experts + the shared expert (group E_loc);
+  // the router covers all experts
+  const size_t H = cfg->hidden, E = cfg->num_experts, Ip = L->I_pad, El = L->E_loc;
   const size_t el = L->fp8 ? 1 : 2;
-  const size_t gu_bytes = (E + 1) * 2 * Ip * H * el, dn_bytes = (E + 1) * H * Ip * el;
+  const size_t gu_bytes = (El + 1) * 2 * Ip * H * el, dn_bytes = (El + 1) * H * Ip * el;
   if (moe::gemm_configure_device() != cudaSuccess ||
       moe::gemm_fp8_configure_device() != cudaSuccess ||
       moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
@@ -252,16 +275,16 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out) {
       cudaMalloc(&L->router_t, E * H * sizeof(float)) != cudaSuccess ||
       cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
       cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess ||
-      (L->fp8 && (cudaMalloc(&L->sc_gu, (E + 1) * 2 * Ip * sizeof(float)) != cudaSuccess ||
-                  cudaMalloc(&L->sc_dn, (E + 1) * H * sizeof(float)) != cudaSuccess))) {
+      (L->fp8 && (cudaMalloc(&L->sc_gu, (El + 1) * 2 * Ip * sizeof(float)) != cudaSuccess ||
+                  cudaMalloc(&L->sc_dn, (El + 1) * H * sizeof(float)) != cudaSuccess))) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
   }
   // (FP8 codes are read with plain bulk copies: no tensor maps)
   const bool maps_ok =
-      L->fp8 || (encode_bf16_2d(&L->tm_gu, L->w_gu, (E + 1) * 2 * Ip, H, 2 * moe::kBM) &&
-                 encode_bf16_2d(&L->tm_gu64, L->w_gu, (E + 1) * 2 * Ip, H, 64) &&
-                 encode_bf16_2d(&L->tm_dn, L->w_dn, (E + 1) * H, Ip, moe::kBM));
+      L->fp8 || (encode_bf16_2d(&L->tm_gu, L->w_gu, (El + 1) * 2 * Ip, H, 2 * moe::kBM) &&
+                 encode_bf16_2d(&L->tm_gu64, L->w_gu, (El + 1) * 2 * Ip, H, 64) &&
+                 encode_bf16_2d(&L->tm_dn, L->w_dn, (El + 1) * H, Ip, moe::kBM));
   if (!maps_ok || !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM)) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
@@ -281,19 +304,26 @@ int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_
   if (!dg.ok) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const moe_config_t& c = L->cfg;
-  const int H = c.hidden, E = c.num_experts, I = c.intermediate, Ip = L->I_pad;
+  const int H = c.hidden, El = L->E_loc, I = c.intermediate, Ip = L->I_pad;
   const bool wb = c.weight_dtype == MOE_BF16;
   const size_t gu_group = static_cast<size_t>(2) * Ip * H, dn_group = static_cast<size_t>(H) * Ip;
   __nv_bfloat16* gu = static_cast<__nv_bfloat16*>(L->w_gu);
   __nv_bfloat16* dn = static_cast<__nv_bfloat16*>(L->w_dn);
-  MOE_CUDA(cudaMemsetAsync(gu, 0, (E + 1) * gu_group * 2, st));
-  MOE_CUDA(cudaMemsetAsync(dn, 0, (E + 1) * dn_group * 2, st));
-  MOE_CUDA(moe::launch_pack_gate_up(w_gate, wb, E, H, I, Ip, 0, gu, st));
-  MOE_CUDA(moe::launch_pack_gate_up(w_up, wb, E, H, I, Ip, 1, gu, st));
-  MOE_CUDA(moe::launch_pack_gate_up(sh_gate, wb, 1, H, I, Ip, 0, gu + E * gu_group, st));
-  MOE_CUDA(moe::launch_pack_gate_up(sh_up, wb, 1, H, I, Ip, 1, gu + E * gu_group, st));
-  MOE_CUDA(moe::launch_pack_down(w_down, wb, E, H, I, Ip, dn, st));
-  MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, dn + E * dn_group, st));
+  // the shard's experts start `first` experts into the caller's tensors
+  const size_t off = static_cast<size_t>(L->first) * H * I * (wb ? 2 : 4);
+  const uint8_t* wg = static_cast<const uint8_t*>(w_gate) + off;
+  const uint8_t* wu = static_cast<const uint8_t*>(w_up) + off;
+  const uint8_t* wd = static_cast<const uint8_t*>(w_down) + off;
+  MOE_CUDA(cudaMemsetAsync(gu, 0, (El + 1) * gu_group * 2, st));
+  MOE_CUDA(cudaMemsetAsync(dn, 0, (El + 1) * dn_group * 2, st));
+  MOE_CUDA(moe::launch_pack_gate_up(wg, wb, El, H, I, Ip, 0, gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up(wu, wb, El, H, I, Ip, 1, gu, st));
+  MOE_CUDA(moe::launch_pack_down(wd, wb, El, H, I, Ip, dn, st));
+  if (L->with_shared) {
+    MOE_CUDA(moe::launch_pack_gate_up(sh_gate, wb, 1, H, I, Ip, 0, gu + El * gu_group, st));
+    MOE_CUDA(moe::launch_pack_gate_up(sh_up, wb, 1, H, I, Ip, 1, gu + El * gu_group, st));
+    MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, dn + El * dn_group, st));
+  }
   return load_router(L, router_w, router_bias, st);
 }
 
@@ -313,30 +343,36 @@ int moe_load_weights_fp8(moe_layer_t* L, const float* router_w, const float* rou
   if (!dg.ok) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const moe_config_t& c = L->cfg;
-  const int H = c.hidden, E = c.num_experts, I = c.intermediate, Ip = L->I_pad;
+  const int H = c.hidden, El = L->E_loc, I = c.intermediate, Ip = L->I_pad;
   const size_t gu_group = static_cast<size_t>(2) * Ip * H, dn_group = static_cast<size_t>(H) * Ip;
   uint8_t* gu = static_cast<uint8_t*>(L->w_gu);
   uint8_t* dn = static_cast<uint8_t*>(L->w_dn);
+  // the shard's experts start `first` experts into the caller's tensors
+  const size_t f = static_cast<size_t>(L->first);
+  const size_t off = f * H * I;
   // padded rows and columns: code 0 (value 0), scale 0
-  MOE_CUDA(cudaMemsetAsync(gu, 0, (E + 1) * gu_group, st));
-  MOE_CUDA(cudaMemsetAsync(dn, 0, (E + 1) * dn_group, st));
-  MOE_CUDA(cudaMemsetAsync(L->sc_gu, 0, (E + 1) * 2 * Ip * sizeof(float), st));
-  MOE_CUDA(moe::launch_pack_codes_gate_up(w_gate, E, H, I, Ip, 0, gu, st));
-  MOE_CUDA(moe::launch_pack_codes_gate_up(w_up, E, H, I, Ip, 1, gu, st));
-  MOE_CUDA(moe::launch_pack_codes_gate_up(sh_gate, 1, H, I, Ip, 0, gu + E * gu_group, st));
-  MOE_CUDA(moe::launch_pack_codes_gate_up(sh_up, 1, H, I, Ip, 1, gu + E * gu_group, st));
+  MOE_CUDA(cudaMemsetAsync(gu, 0, (El + 1) * gu_group, st));
+  MOE_CUDA(cudaMemsetAsync(dn, 0, (El + 1) * dn_group, st));
+  MOE_CUDA(cudaMemsetAsync(L->sc_gu, 0, (El + 1) * 2 * Ip * sizeof(float), st));
+  MOE_CUDA(cudaMemsetAsync(L->sc_dn, 0, (El + 1) * H * sizeof(float), st));
+  MOE_CUDA(moe::launch_pack_codes_gate_up(w_gate + off, El, H, I, Ip, 0, gu, st));
+  MOE_CUDA(moe::launch_pack_codes_gate_up(w_up + off, El, H, I, Ip, 1, gu, st));
   const int dn_rows = moe::kBM * moe::gemm_down_blocks(H);  // the down GEMM's tile rows
-  MOE_CUDA(moe::launch_pack_codes_down(w_down, E, H, I, Ip, dn_rows, dn, st));
-  MOE_CUDA(moe::launch_pack_codes_down(sh_down, 1, H, I, Ip, dn_rows, dn + E * dn_group, st));
-  float* sgu_sh = L->sc_gu + static_cast<size_t>(E) * 2 * Ip;
-  MOE_CUDA(moe::launch_pack_gate_up_scales(s_gate, E, I, Ip, 0, L->sc_gu, st));
-  MOE_CUDA(moe::launch_pack_gate_up_scales(s_up, E, I, Ip, 1, L->sc_gu, st));
-  MOE_CUDA(moe::launch_pack_gate_up_scales(sh_s_gate, 1, I, Ip, 0, sgu_sh, st));
-  MOE_CUDA(moe::launch_pack_gate_up_scales(sh_s_up, 1, I, Ip, 1, sgu_sh, st));
-  MOE_CUDA(cudaMemcpyAsync(L->sc_dn, s_down, static_cast<size_t>(E) * H * sizeof(float),
+  MOE_CUDA(moe::launch_pack_codes_down(w_down + off, El, H, I, Ip, dn_rows, dn, st));
+  MOE_CUDA(moe::launch_pack_gate_up_scales(s_gate + f * I, El, I, Ip, 0, L->sc_gu, st));
+  MOE_CUDA(moe::launch_pack_gate_up_scales(s_up + f * I, El, I, Ip, 1, L->sc_gu, st));
+  MOE_CUDA(cudaMemcpyAsync(L->sc_dn, s_down + f * H, static_cast<size_t>(El) * H * sizeof(float),
                            cudaMemcpyDeviceToDevice, st));
-  MOE_CUDA(cudaMemcpyAsync(L->sc_dn + static_cast<size_t>(E) * H, sh_s_down, H * sizeof(float),
-                           cudaMemcpyDeviceToDevice, st));
+  if (L->with_shared) {
+    float* sgu_sh = L->sc_gu + static_cast<size_t>(El) * 2 * Ip;
+    MOE_CUDA(moe::launch_pack_codes_gate_up(sh_gate, 1, H, I, Ip, 0, gu + El * gu_group, st));
+    MOE_CUDA(moe::launch_pack_codes_gate_up(sh_up, 1, H, I, Ip, 1, gu + El * gu_group, st));
+    MOE_CUDA(moe::launch_pack_codes_down(sh_down, 1, H, I, Ip, dn_rows, dn + El * dn_group, st));
+    MOE_CUDA(moe::launch_pack_gate_up_scales(sh_s_gate, 1, I, Ip, 0, sgu_sh, st));
+    MOE_CUDA(moe::launch_pack_gate_up_scales(sh_s_up, 1, I, Ip, 1, sgu_sh, st));
+    MOE_CUDA(cudaMemcpyAsync(L->sc_dn + static_cast<size_t>(El) * H, sh_s_down,
+                             H * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  }
   return load_router(L, router_w, router_bias, st);
 }
 
@@ -405,7 +441,11 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   if (!dg.ok) return MOE_ERR_CUDA;
 
   const moe_config_t& c = L->cfg;
-  const int H = c.hidden, E = c.num_experts, k = c.top_k, G = E + 1, Ip = L->I_pad;
+  // E: all experts (router, selection); El: this layer's experts (a shard
+  // holds [first, first + El)); G: its groups (the shared expert is group El)
+  const int H = c.hidden, E = c.num_experts, k = c.top_k, Ip = L->I_pad;
+  const int El = L->E_loc, G = El + 1;
+  const bool shard = El != E || L->first != 0;
   const bool xb = c.act_dtype == MOE_BF16;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -517,9 +557,15 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
                             st, routing != nullptr ? routing->logits : nullptr,
                             tc_router ? &refine : nullptr));
   MOE_CUDA(mark(2));
-  MOE_CUDA(moe::launch_sort(topk_idx, topk_w, T, k, E, bn_gu, bn_dn, mt_gu, mt_dn, masks,
-                            chunk_cnt, chunk_base, counts, row_start, tiles_gu, tiles_dn, perm, pos,
-                            w_perm, st));
+  const int* sel = topk_idx;  // the selection in this layer's expert ids
+  if (shard) {
+    int* local_idx = reinterpret_cast<int*>(ws + w.local_idx);
+    MOE_CUDA(moe::launch_localize(topk_idx, T * k, L->first, El, local_idx, st));
+    sel = local_idx;
+  }
+  MOE_CUDA(moe::launch_sort(sel, topk_w, T, k, El, L->with_shared ? T : 0, bn_gu, bn_dn, mt_gu,
+                            mt_dn, masks, chunk_cnt, chunk_base, counts, row_start, tiles_gu,
+                            tiles_dn, perm, pos, w_perm, st));
   MOE_CUDA(mark(3));
   MOE_CUDA(moe::launch_gather(x, xb, perm, pos, w.rows_routed, k, T, H, !xb, x_perm, L->num_sms,
                               L->status, st));
@@ -529,7 +575,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.counts = counts;
   p.row_start = row_start;
   p.G = G;
-  p.E = E;
+  p.E = El;
   p.status = L->status;
   p.limit = c.swiglu_limit;
   p.limit_shared = c.swiglu_limit_shared;
@@ -565,7 +611,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
            : pair_dn ? moe::launch_gemm_down_pair(dn, p, st)
                      : moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
   MOE_CUDA(mark(6));
-  MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, out, st));
+  MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, L->with_shared != 0, out, st));
   MOE_CUDA(mark(7));
 
   if (routing != nullptr) {
@@ -574,11 +620,12 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
       MOE_CUDA(cudaMemcpyAsync(routing->topk_idx, topk_idx, tk * 4, cudaMemcpyDeviceToDevice, st));
     if (routing->topk_w)
       MOE_CUDA(cudaMemcpyAsync(routing->topk_w, topk_w, tk * 4, cudaMemcpyDeviceToDevice, st));
+    // (a shard: counts and offsets of its own El experts)
     if (routing->counts)
-      MOE_CUDA(cudaMemcpyAsync(routing->counts, counts, E * 4, cudaMemcpyDeviceToDevice, st));
+      MOE_CUDA(cudaMemcpyAsync(routing->counts, counts, El * 4, cudaMemcpyDeviceToDevice, st));
     if (routing->offsets)
       MOE_CUDA(
-          cudaMemcpyAsync(routing->offsets, row_start, (E + 1) * 4, cudaMemcpyDeviceToDevice, st));
+          cudaMemcpyAsync(routing->offsets, row_start, (El + 1) * 4, cudaMemcpyDeviceToDevice, st));
     if (routing->perm)
       MOE_CUDA(cudaMemcpyAsync(routing->perm, perm, tk * 4, cudaMemcpyDeviceToDevice, st));
   }
@@ -627,8 +674,10 @@ int moe_get_device_error(moe_layer_t* L, int* device_err) {
 int moe_kernel_launches(const moe_layer_t* L, int T) {
   if (L == nullptr || T <= 0) return 0;
   // router, top-k, counting sort (one kernel up to kSortChunk tokens, else
-  // three), gather, gate|up GEMM, down GEMM, combine
-  return T <= moe::kSortChunk ? 7 : 9;
+  // three), gather, gate|up GEMM, down GEMM, combine; a shard also maps the
+  // selection to its own expert ids
+  const bool shard = L->E_loc != L->cfg.num_experts || L->first != 0;
+  return (T <= moe::kSortChunk ? 7 : 9) + (shard ? 1 : 0);
 }
 
 namespace {

@@ -103,10 +103,16 @@ cudaError_t launch_router_logits(const void* x, bool x_bf16, const float* router
 cudaError_t launch_topk(const float* partial, int ksplit, int T, int E, int k, const float* bias,
                         bool norm, float scale, int* topk_idx, float* topk_w, cudaStream_t st,
                         float* logits_out = nullptr, const TopkRefine* refine = nullptr);
-cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn_gu,
-                        int bn_dn, int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
-                        int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
-                        int* pos, float* w_perm, cudaStream_t st);
+// shared_rows: T, or 0 for an expert shard without the shared expert; ids
+// outside [0, E) are another shard's experts (pos -1)
+cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E,
+                        int shared_rows, int bn_gu, int bn_dn, int m_tiles_gu, int m_tiles_dn,
+                        uint32_t* masks, int* chunk_cnt, int* chunk_base, int* counts,
+                        int* row_start, int* tiles_gu, int* tiles_dn, int* perm, int* pos,
+                        float* w_perm, cudaStream_t st);
+// expert shard: local_idx = topk_idx - first inside [first, first + count), else -1
+cudaError_t launch_localize(const int* topk_idx, int n, int first, int count, int* local_idx,
+                            cudaStream_t st);
 // x_perm rows: bf16 x by bulk copies per token (pos), else row by row (perm)
 cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, const int* pos,
                           int rows_routed, int k, int T, int H, bool write_shared,
@@ -147,7 +153,7 @@ cudaError_t launch_gemm_down_fp8(const GemmMaps& m, const GemmParams& p, int gri
 cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfloat16* dst,
                                float* dst_t, cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k, int H, bool out_bf16,
-                           void* out, cudaStream_t st);
+                           bool with_shared, void* out, cudaStream_t st);
 cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
                                 int half, __nv_bfloat16* dst, cudaStream_t st);
 cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,

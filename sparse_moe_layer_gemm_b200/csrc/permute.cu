@@ -6,7 +6,11 @@
 // strategy") needs each expert's rows contiguous.  Definition kept here:
 // perm lists the pair ids t * k + j of expert 0, then expert 1, ..., each in
 // ascending t; pos[t * k + j] is the pair's slot in perm.  The shared expert
-// is group E with the T identity rows [T*k, T*k + T).
+// is group E with the T identity rows [T*k, T*k + T) (or no rows).
+//
+// Expert shards: the caller passes local expert ids (another shard's expert
+// is -1); such pairs get pos = -1 and no slot, the routed rows then end
+// before T*k, and the shared group still starts at row T*k.
 //
 // No order-dependent atomics: each block owns kSortChunk tokens and records,
 // per expert, a 128-bit mask of its tokens that chose that expert (atomicOr
@@ -52,10 +56,11 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const int* __restrict__ 
 // Warp-wide exclusive prefix over the G = E + 1 groups of the row counts and
 // of the GEMM tile counts (ceil(rows / bn) token tiles x m_tiles weight
 // tiles, with each GEMM's own bn).  Called by one full warp; cnt_s holds
-// the G row counts.  When
+// the G row counts; the last group (the shared expert) starts at row
+// shared_row0 (T*k: equal to the prefix unless a shard dropped pairs).  When
 // start_s is given, the row starts are also left there for the caller.
 __device__ void scan_groups(const int* cnt_s, int G, int bn_gu, int bn_dn, int mt_gu, int mt_dn,
-                            int* __restrict__ counts,
+                            int shared_row0, int* __restrict__ counts,
                             int* __restrict__ row_start, int* __restrict__ tiles_gu,
                             int* __restrict__ tiles_dn, int* start_s) {
   const int lane = threadIdx.x & 31;
@@ -84,8 +89,8 @@ __device__ void scan_groups(const int* cnt_s, int G, int bn_gu, int bn_dn, int m
   for (int g = g0; g < g1; ++g) {
     const int n = cnt_s[g];
     counts[g] = n;
-    row_start[g] = b_rows;
-    if (start_s != nullptr) start_s[g] = b_rows;
+    row_start[g] = g == G - 1 ? shared_row0 : b_rows;
+    if (start_s != nullptr) start_s[g] = row_start[g];
     tiles_gu[g] = b_gu;
     tiles_dn[g] = b_dn;
     b_rows += n;
@@ -93,7 +98,7 @@ __device__ void scan_groups(const int* cnt_s, int G, int bn_gu, int bn_dn, int m
     b_dn += (n + bn_dn - 1) / bn_dn * mt_dn;
   }
   if (lane == 31) {
-    row_start[G] = i_rows;
+    row_start[G] = shared_row0 + cnt_s[G - 1];
     tiles_gu[G] = i_gu;
     tiles_dn[G] = i_dn;
   }
@@ -102,9 +107,9 @@ __device__ void scan_groups(const int* cnt_s, int G, int bn_gu, int bn_dn, int m
 // One block.  Per expert: running offsets of the chunks; then warp 0 forms
 // the prefixes over the groups.
 __global__ void __launch_bounds__(1024) sort_scan_kernel(
-    const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int bn_gu, int bn_dn, int mt_gu, int mt_dn,
-    int* __restrict__ chunk_base, int* __restrict__ counts, int* __restrict__ row_start,
-    int* __restrict__ tiles_gu, int* __restrict__ tiles_dn) {
+    const int* __restrict__ chunk_cnt, int nch, int T, int k, int E, int shared_rows, int bn_gu,
+    int bn_dn, int mt_gu, int mt_dn, int* __restrict__ chunk_base, int* __restrict__ counts,
+    int* __restrict__ row_start, int* __restrict__ tiles_gu, int* __restrict__ tiles_dn) {
   pdl_wait();  // the previous kernel's results are visible
   __shared__ int cnt_s[1025];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -115,10 +120,11 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(
     }
     cnt_s[e] = run;
   }
-  if (threadIdx.x == 0) cnt_s[E] = T;
+  if (threadIdx.x == 0) cnt_s[E] = shared_rows;
   __syncthreads();
   if (threadIdx.x < 32)
-    scan_groups(cnt_s, E + 1, bn_gu, bn_dn, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, nullptr);
+    scan_groups(cnt_s, E + 1, bn_gu, bn_dn, mt_gu, mt_dn, T * k, counts, row_start, tiles_gu,
+                tiles_dn, nullptr);
 }
 
 // Rank of token tl among the tokens of this chunk that chose the expert whose
@@ -133,7 +139,8 @@ __device__ __forceinline__ int chunk_rank(const uint32_t* m, int tl) {
 // T <= kSortChunk (decode): histogram, prefixes and stable scatter in one block.
 __global__ void __launch_bounds__(1024) sort_small_kernel(
     const int* __restrict__ topk_idx, const float* __restrict__ topk_w, int T, int k, int E,
-    int bn_gu, int bn_dn, int mt_gu, int mt_dn, int* __restrict__ counts, int* __restrict__ row_start,
+    int shared_rows, int bn_gu, int bn_dn, int mt_gu, int mt_dn, int* __restrict__ counts,
+    int* __restrict__ row_start,
     int* __restrict__ tiles_gu, int* __restrict__ tiles_dn, int* __restrict__ perm,
     int* __restrict__ pos, float* __restrict__ w_perm) {
   pdl_wait();  // the previous kernel's results are visible
@@ -156,15 +163,19 @@ __global__ void __launch_bounds__(1024) sort_small_kernel(
     for (int q = 0; q < kMaskWords; ++q) n += __popc(masks[e * kMaskWords + q]);
     cnt_s[e] = n;
   }
-  if (threadIdx.x == 0) cnt_s[E] = T;
+  if (threadIdx.x == 0) cnt_s[E] = shared_rows;
   __syncthreads();
   if (threadIdx.x < 32)
-    scan_groups(cnt_s, E + 1, bn_gu, bn_dn, mt_gu, mt_dn, counts, row_start, tiles_gu, tiles_dn, start_s);
+    scan_groups(cnt_s, E + 1, bn_gu, bn_dn, mt_gu, mt_dn, T * k, counts, row_start, tiles_gu,
+                tiles_dn, start_s);
   __syncthreads();
   for (int p = threadIdx.x; p < T * k; p += blockDim.x) {
     const int tl = p / k;
     const int e = topk_idx[p];
-    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) continue;
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {  // another shard's expert
+      pos[p] = -1;
+      continue;
+    }
     const int slot = start_s[e] + chunk_rank(masks + e * kMaskWords, tl);
     perm[slot] = p;
     pos[p] = slot;
@@ -190,7 +201,10 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(
     const int tl = p / k;
     const size_t pair = static_cast<size_t>(t0) * k + p;
     const int e = topk_idx[pair];
-    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) continue;
+    if (static_cast<unsigned>(e) >= static_cast<unsigned>(E)) {  // another shard's expert
+      pos[pair] = -1;
+      continue;
+    }
     const int slot = row_start[e] + chunk_base[static_cast<size_t>(c) * E + e] +
                      chunk_rank(sm + e * kMaskWords, tl);
     perm[slot] = static_cast<int>(pair);
@@ -283,37 +297,57 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
     bulk_load_1d(buf, x + static_cast<size_t>(t) * H, row_bytes, bar);
     if (!mbar_wait(bar, (i >> 1) & 1u, nullptr, status)) break;
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < k) bulk_store_1d(xp + static_cast<size_t>(rows[j]) * H, buf, row_bytes);
+    for (int j = 0; j < 32; ++j)  // (pos -1: another shard's expert, no row)
+      if (j < k && rows[j] >= 0) bulk_store_1d(xp + static_cast<size_t>(rows[j]) * H, buf, row_bytes);
     bulk_commit_group();
   }
   bulk_wait_group_all();
 }
 
+// Expert shard: global expert ids -> local ids (e - first for the shard's
+// experts [first, first + count), else -1).
+__global__ void localize_kernel(const int* __restrict__ topk_idx, int n, int first, int count,
+                                int* __restrict__ local_idx) {
+  pdl_wait();  // the previous kernel's results are visible
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int e = topk_idx[i] - first;
+    local_idx[i] = static_cast<unsigned>(e) < static_cast<unsigned>(count) ? e : -1;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_localize(const int* topk_idx, int n, int first, int count, int* local_idx,
+                            cudaStream_t st) {
+  const int blocks = max(1, min((n + 255) / 256, 1024));
+  return launch_pdl(localize_kernel, dim3(blocks), dim3(256), 0, st, topk_idx, n, first, count,
+                    local_idx);
+}
 
 cudaError_t gather_configure_device() {
   return cudaFuncSetAttribute(gather_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               100 * 1024);
 }
 
-cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E, int bn_gu,
-                        int bn_dn, int m_tiles_gu, int m_tiles_dn, uint32_t* masks, int* chunk_cnt, int* chunk_base,
-                        int* counts, int* row_start, int* tiles_gu, int* tiles_dn, int* perm,
-                        int* pos, float* w_perm, cudaStream_t st) {
+cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, int E,
+                        int shared_rows, int bn_gu, int bn_dn, int m_tiles_gu, int m_tiles_dn,
+                        uint32_t* masks, int* chunk_cnt, int* chunk_base, int* counts,
+                        int* row_start, int* tiles_gu, int* tiles_dn, int* perm, int* pos,
+                        float* w_perm, cudaStream_t st) {
   const int nch = (T + kSortChunk - 1) / kSortChunk;
   const size_t smem = static_cast<size_t>(E) * kMaskWords * sizeof(uint32_t);
   if (nch == 1) {
     const size_t smem1 = smem + 2 * static_cast<size_t>(E + 1) * sizeof(int);
     return launch_pdl(sort_small_kernel, dim3(1), dim3(1024), smem1, st, topk_idx, topk_w, T, k, E,
-                      bn_gu, bn_dn, m_tiles_gu, m_tiles_dn, counts, row_start, tiles_gu, tiles_dn,
-                      perm, pos, w_perm);
+                      shared_rows, bn_gu, bn_dn, m_tiles_gu, m_tiles_dn, counts, row_start,
+                      tiles_gu, tiles_dn, perm, pos, w_perm);
   }
   cudaError_t err = launch_pdl(sort_hist_kernel, dim3(nch), dim3(256), smem, st, topk_idx, T, k, E,
                                masks, chunk_cnt);
   if (err != cudaSuccess) return err;
-  err = launch_pdl(sort_scan_kernel, dim3(1), dim3(1024), 0, st, chunk_cnt, nch, T, k, E, bn_gu,
-                   bn_dn, m_tiles_gu, m_tiles_dn, chunk_base, counts, row_start, tiles_gu, tiles_dn);
+  err = launch_pdl(sort_scan_kernel, dim3(1), dim3(1024), 0, st, chunk_cnt, nch, T, k, E,
+                   shared_rows, bn_gu, bn_dn, m_tiles_gu, m_tiles_dn, chunk_base, counts,
+                   row_start, tiles_gu, tiles_dn);
   if (err != cudaSuccess) return err;
   return launch_pdl(sort_scatter_kernel, dim3(nch), dim3(256), smem, st, topk_idx, topk_w, T, k, E,
                     masks, chunk_base, row_start, perm, pos, w_perm);

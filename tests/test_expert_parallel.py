@@ -1,0 +1,136 @@
+"""Expert parallelism.  CPU (gloo, world size 2): the shard split covers
+every expert once and the summed partial outputs equal the whole layer, with
+the oracle standing in for each rank's kernels.  GPU (one device): shard
+layers run one after another on the same GPU, and their partial outputs sum
+to the oracle's output; the shard's routing counts are its own experts'."""
+import os
+import socket
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle.moe_oracle as om
+from sparse_moe_layer_gemm_b200.expert_parallel import (holds_shared, reduce_partials,
+                                                        shard_range)
+from sparse_moe_layer_gemm_b200.workloads import WORKLOADS, host_f32, make_inputs
+
+
+@pytest.mark.parametrize("E,world", [(288, 8), (288, 7), (16, 2), (5, 5), (13, 4)])
+def test_shard_ranges_cover_once(E, world):
+    seen = []
+    for r in range(world):
+        f, c = shard_range(E, world, r)
+        assert c >= 1 and abs(c - E // world) <= 1
+        seen.extend(range(f, f + c))
+    assert seen == list(range(E))
+    assert sum(holds_shared(r) for r in range(world)) == 1
+
+
+def test_shard_range_rejects_bad_splits():
+    with pytest.raises(ValueError):
+        shard_range(3, 4, 0)
+    with pytest.raises(ValueError):
+        shard_range(16, 2, 2)
+
+
+def _partial_oracle(inp, wl, first, count, with_shared):
+    """The oracle's layer output restricted to one shard: the other experts'
+    weights (and the shared expert's, if not held) set to zero, so their
+    SwiGLU terms vanish while the routing (which does not read them) is the
+    whole layer's."""
+    keep = np.zeros(wl.num_experts, bool)
+    keep[first:first + count] = True
+    z = lambda a: np.where(keep[:, None, None], a, 0.0)
+    sh = 1.0 if with_shared else 0.0
+    return om.moe_forward(inp["x"], inp["router_w"], inp["router_bias"], z(inp["w_gate"]),
+                          z(inp["w_up"]), z(inp["w_down"]), sh * inp["sh_gate"],
+                          sh * inp["sh_up"], sh * inp["sh_down"], top_k=wl.top_k,
+                          scale=wl.scale).out
+
+
+def _port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    wl = WORKLOADS["tiny"]
+    inp = {k: host_f32(v).astype(np.float64) for k, v in make_inputs(wl, "cpu").items()}
+    first, count = shard_range(wl.num_experts, world, rank)
+    part = torch.from_numpy(_partial_oracle(inp, wl, first, count, holds_shared(rank)))
+    total = reduce_partials(part.clone())
+    full = om.moe_forward(inp["x"], inp["router_w"], inp["router_bias"], inp["w_gate"],
+                          inp["w_up"], inp["w_down"], inp["sh_gate"], inp["sh_up"],
+                          inp["sh_down"], top_k=wl.top_k, scale=wl.scale).out
+    q.put((rank, float(np.max(np.abs(total.numpy() - full))), float(np.max(np.abs(full))),
+           float(np.max(np.abs(part.numpy() - full)))))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_two_rank_partials_sum_to_layer_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=150) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err, scale, part_err in res:
+        assert err <= 1e-12 * scale          # fp64 sums of two partials
+        assert part_err > 1e-3 * scale       # a partial alone is not the layer
+
+
+@pytest.mark.gpu
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("case", ["two_shards", "three_uneven_fp32_x", "prefill_shape"])
+def test_gpu_shards_sum_to_oracle(case):
+    from sparse_moe_layer_gemm_b200 import binding as B
+    from tests.parity import MAX_ABS_OVER_RMS, REL_FRO, output_errors
+    if case == "two_shards":
+        wl = replace(WORKLOADS["tiny"], name="ep2", T=200, act_dtype="bf16", weight_dtype="bf16")
+        splits = [(0, 8, True), (8, 8, False)]
+    elif case == "three_uneven_fp32_x":
+        wl = replace(WORKLOADS["tiny"], name="ep3", T=300, num_experts=13, top_k=3)
+        splits = [(0, 4, False), (4, 5, True), (9, 4, False)]
+    else:  # bulk-copy gather (bf16, >= 1024 tokens) and CTA pairs (>= 2048)
+        wl = replace(WORKLOADS["tiny"], name="epp", T=2100, hidden=512, num_experts=16, top_k=4,
+                     intermediate=256, shared_intermediate=256, act_dtype="bf16",
+                     weight_dtype="bf16", x_dist="rmsnorm_normal")
+        splits = [(0, 6, False), (6, 10, True)]
+    cpu = make_inputs(wl, "cpu")
+    inp = {k: v.cuda() for k, v in cpu.items()}
+    total = None
+    for first, count, sh in splits:
+        layer = B.MoeLayer.from_workload(wl, (first, count, sh))
+        layer.load_inputs(inp)
+        out, rt = layer.forward(inp["x"], routing=True)
+        torch.cuda.synchronize()
+        assert layer.device_error() == 0
+        sel = rt["topk_idx"].cpu().numpy()
+        want = np.bincount(sel.ravel(), minlength=wl.num_experts)[first:first + count]
+        assert np.array_equal(rt["counts"].cpu().numpy()[:count], want)
+        part = out.float().cpu()
+        total = part if total is None else total + part
+        layer.close()
+    host = {k: host_f32(cpu[k]) for k in cpu}
+    ref = om.moe_forward(host["x"], host["router_w"], host["router_bias"], host["w_gate"],
+                         host["w_up"], host["w_down"], host["sh_gate"], host["sh_up"],
+                         host["sh_down"], top_k=wl.top_k, scale=wl.scale).out
+    rel, mx = output_errors(total.numpy(), ref)
+    assert rel <= REL_FRO and mx <= MAX_ABS_OVER_RMS, (rel, mx)
