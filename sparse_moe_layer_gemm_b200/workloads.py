@@ -77,6 +77,10 @@ WORKLOADS: Dict[str, Workload] = {
         name="decode_fp8", T=64, expert_std=0.02, bias="normal0.1",
         description="decode shape T=64 with FP8 E4M3 expert weights (per-feature scales)",
         **dict(_STEP35, weight_dtype="fp8")),
+    "prefill_fp8": Workload(
+        name="prefill_fp8", T=4096, expert_std=0.02, bias="normal0.1",
+        description="prefill shape T=4096 with FP8 E4M3 expert weights (per-feature scales)",
+        **dict(_STEP35, weight_dtype="fp8")),
     "clamp_ragged": Workload(
         name="clamp_ragged", T=3001, expert_std=0.05, bias="normal0.1",
         swiglu_limit=7.0, swiglu_limit_shared=7.0,

@@ -98,7 +98,8 @@ def test_two_rank_partials_sum_to_layer_gloo():
 
 @pytest.mark.gpu
 @pytest.mark.timeout(300)
-@pytest.mark.parametrize("case", ["two_shards", "three_uneven_fp32_x", "prefill_shape"])
+@pytest.mark.parametrize("case", ["two_shards", "three_uneven_fp32_x", "prefill_shape",
+                                  "fp8_two_shards"])
 def test_gpu_shards_sum_to_oracle(case):
     from sparse_moe_layer_gemm_b200 import binding as B
     from tests.parity import MAX_ABS_OVER_RMS, REL_FRO, output_errors
@@ -108,6 +109,11 @@ def test_gpu_shards_sum_to_oracle(case):
     elif case == "three_uneven_fp32_x":
         wl = replace(WORKLOADS["tiny"], name="ep3", T=300, num_experts=13, top_k=3)
         splits = [(0, 4, False), (4, 5, True), (9, 4, False)]
+    elif case == "fp8_two_shards":  # FP8 codes and scales sliced per shard
+        wl = replace(WORKLOADS["tiny"], name="ep8", T=150, hidden=512, num_experts=12, top_k=3,
+                     intermediate=256, shared_intermediate=256, act_dtype="bf16",
+                     weight_dtype="fp8", x_dist="rmsnorm_normal")
+        splits = [(0, 5, False), (5, 7, True)]
     else:  # bulk-copy gather (bf16, >= 1024 tokens) and CTA pairs (>= 2048)
         wl = replace(WORKLOADS["tiny"], name="epp", T=2100, hidden=512, num_experts=16, top_k=4,
                      intermediate=256, shared_intermediate=256, act_dtype="bf16",
@@ -128,9 +134,11 @@ def test_gpu_shards_sum_to_oracle(case):
         part = out.float().cpu()
         total = part if total is None else total + part
         layer.close()
-    host = {k: host_f32(cpu[k]) for k in cpu}
-    ref = om.moe_forward(host["x"], host["router_w"], host["router_bias"], host["w_gate"],
-                         host["w_up"], host["w_down"], host["sh_gate"], host["sh_up"],
-                         host["sh_down"], top_k=wl.top_k, scale=wl.scale).out
+    from tests.parity import expert_views
+    host = {k: host_f32(cpu[k]) for k in ("x", "router_w", "router_bias")}
+    ev = expert_views(cpu)
+    ref = om.moe_forward(host["x"], host["router_w"], host["router_bias"], ev["w_gate"],
+                         ev["w_up"], ev["w_down"], ev["sh_gate"], ev["sh_up"], ev["sh_down"],
+                         top_k=wl.top_k, scale=wl.scale).out
     rel, mx = output_errors(total.numpy(), ref)
     assert rel <= REL_FRO and mx <= MAX_ABS_OVER_RMS, (rel, mx)
