@@ -7,9 +7,9 @@
 // pages list FP8 official weights in the same bullet list, without a format).
 //
 // Every finite E4M3 code is exactly a bf16 value, so the codes are expanded to
-// bf16 in shared memory and multiplied on the same bf16 x bf16 -> fp32
-// tensor-core path; the epilogue multiplies each accumulator row (one output
-// feature) by its scale.  HBM moves one byte per weight instead of two.
+// bf16 (into tensor memory, below) and multiplied on the same bf16 x bf16 ->
+// fp32 tensor-core path; the epilogue multiplies each accumulator row (one
+// output feature) by its scale.  HBM moves one byte per weight instead of two.
 //
 // Swap-AB tiles as in the bf16 kernel (128 weight rows per MMA on M, up to
 // kFp8BN tokens on N), one persistent CTA per SM.  The expanded weights never
@@ -30,10 +30,10 @@
 //   1         token-row producer (one TMA load per stage);
 //   next 2*NI tcgen05.mma issuers: per accumulator chain (gate and up, or
 //             two weight blocks) two warps taking alternate stages into two
-//             partial accumulators that the epilogue adds (each MMA costs
-//             the issuing thread about a hundred cycles at these shapes, so
-//             one issuer per chain could not keep up with the codes); the
-//             first allocates TMEM;
+//             partial accumulators that the epilogue adds, so that each
+//             issuer (about a hundred cycles per MMA at these shapes) has
+//             two stages of time for one stage's MMAs; the first allocates
+//             TMEM;
 //   next 8    converters, two groups of four taking alternate stages: thread
 //             = one weight row of every chain, 64-byte-swizzled code reads
 //             without bank conflicts, E4M3 -> bf16 in registers, tcgen05.st
