@@ -51,6 +51,10 @@ def _args():
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling case: override the number of routed experts "
                          "(smaller device footprint for ncu captures)")
+    ap.add_argument("--intermediate", type=int, default=0,
+                    help="profiling case: override the experts' intermediate size I (the "
+                         "routing stages see the same inputs; smaller device footprint "
+                         "for ncu captures of them)")
     return ap.parse_args()
 
 
@@ -359,10 +363,14 @@ def run_ours(a):
     torch.cuda.set_device(dev)
     B.load_library()
     wl = WORKLOADS[a.workload]
-    if a.experts or a.tokens:
+    if a.experts or a.tokens or a.intermediate:
         from dataclasses import replace as _replace
+        I = a.intermediate or wl.intermediate
+        Is = a.intermediate or wl.shared_intermediate
         wl = _replace(wl, num_experts=a.experts or wl.num_experts, T=a.tokens or wl.T,
-                      name=f"{wl.name}_e{a.experts or wl.num_experts}_t{a.tokens or wl.T}")
+                      intermediate=I, shared_intermediate=Is,
+                      name=f"{wl.name}_e{a.experts or wl.num_experts}_t{a.tokens or wl.T}"
+                           + (f"_i{I}" if a.intermediate else ""))
     peaks = _peaks()
 
     inp = make_inputs(wl, dev)                          # weights replicated on every rank

@@ -174,6 +174,44 @@ __device__ __forceinline__ void warp_select(const float* s_sc, const float* s_be
   }
 }
 
+// Unsigned key with the order of the float (no NaN): -0 is taken as +0.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// The k-th largest of the warp's values (lane l holds v[i] for slot l + 32 i;
+// equal values count separately, so it is the k-th selection score of any
+// ordering by value), 1 <= k <= the number of slots.  Each round takes one
+// largest remaining value: a lane-local maximum, a warp max-reduction of its
+// key, and the lowest lane holding it retires one copy.
+template <int MPL>
+__device__ __forceinline__ float warp_kth_largest(const float (&v)[MPL], int k) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[MPL];
+#pragma unroll
+  for (int i = 0; i < MPL; ++i) key[i] = order_key(v[i]);
+  uint32_t taken = 0, best = 0;
+  for (int j = 0; j < k; ++j) {
+    uint32_t m = 0;  // below every key: a lane with nothing left never wins
+    int mi = 0;
+#pragma unroll
+    for (int i = 0; i < MPL; ++i) {
+      const bool better = !((taken >> i) & 1u) && key[i] > m;
+      m = better ? key[i] : m;
+      mi = better ? i : mi;
+    }
+    best = __reduce_max_sync(0xffffffffu, m);
+    const uint32_t holders = __ballot_sync(0xffffffffu, m == best);
+    if (lane == __ffs(holders) - 1) taken |= 1u << mi;
+  }
+  return key_value(best);
+}
+
 // Block-per-token form (small and medium batches: more threads per token,
 // so the latency of one token's work is shorter).  Thread e sums the ksplit partial logits of expert e
 // (independent loads, fixed order), forms the fp32 sigmoid score s and the
@@ -202,6 +240,8 @@ __global__ void __launch_bounds__(1024) topk_block_kernel(const float* __restric
   __shared__ float s_sc[32 * MPL];
   __shared__ float s_be[32 * MPL];
   __shared__ int s_cand[32 * MPL];
+  __shared__ float s_cb[32];     // selection scores of the first 32 candidates
+  __shared__ int s_rank_e[32];   // the candidates by rank
   __shared__ int s_ncand;
   __shared__ float s_kth;
   const int t = blockIdx.x;
@@ -229,10 +269,13 @@ __global__ void __launch_bounds__(1024) topk_block_kernel(const float* __restric
   int my_idx = 0;
   float my_s = 0.f, kth, next;
   if (rf.band > 0.f) {
-    if (warp == 0) {
-      warp_select<MPL>(s_sc, s_be, E, k, my_idx, my_s, kth, next);
+    if (warp == 0) {  // only the k-th approximate selection score is needed here
+      float v[MPL];
+#pragma unroll
+      for (int i = 0; i < MPL; ++i) v[i] = lane + 32 * i < E ? s_be[lane + 32 * i] : -INFINITY;
+      const float kth_approx = warp_kth_largest<MPL>(v, k);
       if (lane == 0) {
-        s_kth = kth;
+        s_kth = kth_approx;
         s_ncand = 0;
       }
     }
@@ -290,29 +333,25 @@ __global__ void __launch_bounds__(1024) topk_block_kernel(const float* __restric
     if (n <= 32) {
       // order the candidates by rank: lane c holds candidate c; its rank is
       // the number of candidates ahead of it (higher score, or equal score
-      // and lower index); lane with rank j supplies the j-th pick
+      // and lower index); the lane with rank j supplies the j-th pick.  The
+      // candidates' scores are listed beside them so the rank loop's loads
+      // are independent.
       if (warp == 0) {
         const int e = lane < n ? s_cand[lane] : 0x7fffffff;
         const float b = lane < n ? s_be[e] : -INFINITY;
+        if (lane < n) s_cb[lane] = b;
+        __syncwarp();
         int rank = 0;
+#pragma unroll 4
         for (int c = 0; c < n; ++c) {
-          const float bc = __shfl_sync(0xffffffffu, b, c);
-          const int ec = __shfl_sync(0xffffffffu, e, c);
+          const float bc = s_cb[c];
+          const int ec = s_cand[c];
           rank += (bc > b || (bc == b && ec < e)) ? 1 : 0;
         }
-        // lane j gathers the candidate of rank j
-        int pick_e = 0;
-        float pick_s = 0.f;
-        for (int c = 0; c < n; ++c) {
-          const int rc = __shfl_sync(0xffffffffu, rank, c);
-          const int ec = __shfl_sync(0xffffffffu, e, c);
-          if (rc == lane) {
-            pick_e = ec;
-            pick_s = s_sc[ec];
-          }
-        }
-        my_idx = pick_e;
-        my_s = pick_s;
+        if (lane < n) s_rank_e[rank] = e;  // ranks are distinct
+        __syncwarp();
+        my_idx = lane < n ? s_rank_e[lane] : 0;
+        my_s = lane < n ? s_sc[my_idx] : 0.f;
       }
     } else if (warp == 0) {
       warp_select<MPL>(s_sc, s_be, E, k, my_idx, my_s, kth, next);
@@ -524,7 +563,10 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(
   }
   int my_idx = 0;
   float my_s = 0.f, kth;
-  warp_select_regs<MPL>(sc, be, E, k, my_idx, my_s, kth);
+  if (rf.band > 0.f)
+    kth = warp_kth_largest<MPL>(be, k);  // the picks come from the refined scores below
+  else
+    warp_select_regs<MPL>(sc, be, E, k, my_idx, my_s, kth);
   int c_e = 0x7fffffff;  // after the refinement: lane c's candidate and its fp32 logit
   float c_l = 0.f;
   if (rf.band > 0.f) {

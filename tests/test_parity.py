@@ -75,6 +75,15 @@ SMALL = {
                             top_k=4, intermediate=256, shared_intermediate=256,
                             act_dtype="f32", weight_dtype="bf16", swiglu_limit=0.9,
                             swiglu_limit_shared=1.1, expert_std=0.08),
+    # CTA pairs with mostly narrow tiles (a median of ~12 rows per expert,
+    # 80 of 96 experts at most 128): MMAs of 16-144 columns next to the shared
+    # expert's full 256-token tiles in one CTA's sequence; down with an odd
+    # number of K stages (I = 384: three)
+    "pair_narrow_tiles": replace(WORKLOADS["tiny"], name="pn", T=2048, hidden=512,
+                                 num_experts=96, top_k=4, intermediate=384,
+                                 shared_intermediate=384, act_dtype="bf16",
+                                 weight_dtype="bf16", x_dist="rmsnorm_normal",
+                                 swiglu_limit=0.9, swiglu_limit_shared=1.2, expert_std=0.08),
     # tensor-core router with the warp-per-token top-k (from 8192 tokens) on a
     # small layer
     "many_tokens_small_layer": replace(WORKLOADS["tiny"], name="mt", T=8448, hidden=256,
