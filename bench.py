@@ -93,17 +93,65 @@ def _traffic_record(kernel: str, workload: str, groups: int):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling in the background."""
+    """SM clock and throttle-reason sampling around the timed region.  NVML
+    (read-only queries) in a background thread every 10 ms; the nvidia-smi
+    ``-lms`` loop is the fallback (its first sample comes only after its
+    start-up, so a short region may get one or none).  ``stop()`` returns
+    None when neither source gave a sample."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clocks-event reason bits
+    REASON_BITS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+                   ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+    PERIOD_S = 0.01
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, nvml=None):
         self.idx = gpu_index
         self.proc = None
+        self._nvml = nvml          # a module with the pynvml interface (tests pass a fake)
+        self._thread = None
+        self._stop = None
+        self._samples = []         # (sm MHz, reason bits)
+        self._max = None
+
+    def _start_nvml(self) -> bool:
+        import threading
+        try:
+            nv = self._nvml
+            if nv is None:
+                import pynvml as nv
+            nv.nvmlInit()
+            if str(self.idx).startswith("GPU-"):
+                h = nv.nvmlDeviceGetHandleByUUID(str(self.idx))
+            else:
+                h = nv.nvmlDeviceGetHandleByIndex(int(self.idx))
+            self._max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            # one trial sample: an NVML without these queries falls back now
+            self._samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                  int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+        except Exception:
+            self._samples = []
+            return False
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self._samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                          int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                except Exception:
+                    pass
+                self._stop.wait(self.PERIOD_S)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+        return True
 
     def start(self):
+        if self._start_nvml():
+            return
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
@@ -112,7 +160,20 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    @staticmethod
+    def _summary(sm, mx, reasons, source):
+        if not sm:
+            return None
+        busy = [v for v in sm if mx is None or v > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "source": source}
+
     def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            reasons = {n for n, bit in self.REASON_BITS for _, r in self._samples if r & bit}
+            return self._summary([v for v, _ in self._samples], self._max, reasons, "nvml")
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -122,7 +183,7 @@ class ClockSampler:
             self.proc.kill()
             out, _ = self.proc.communicate()
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        names = [n for n, _ in self.REASON_BITS]
         for line in out.splitlines():
             f = [c.strip() for c in line.split(",")]
             if len(f) < 9:
@@ -135,11 +196,7 @@ class ClockSampler:
             for n, v in zip(names, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
-        if not sm:
-            return None
-        busy = [s for s in sm if mx is None or s > 0.5 * mx] or sm
-        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return self._summary(sm, mx, reasons, "nvidia-smi")
 
 
 # ---------------------------------------------------------------- CPU oracle arm
