@@ -420,6 +420,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
 
 using GuPair = PairShape<kModeGateUp, 2>;
 using DnPair = PairShape<kModeDown, 2>;
+// The host sets GemmParams::num_kb of these launches to K / (2 * kBK).
+static_assert(GuPair::BK == 2 * kBK && DnPair::BK == 2 * kBK,
+              "the host's stage count assumes two 64-deep sub-blocks per stage");
 
 int g_pair_grid = 0;  // CTAs per launch: twice the co-resident clusters
 

@@ -581,7 +581,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.limit_shared = c.swiglu_limit_shared;
 
   p.tile_start = tiles_gu;
-  p.num_kb = H / (pair_gu ? 2 * moe::kBK : moe::kBK);
+  p.num_kb = H / (pair_gu ? 2 * moe::kBK : moe::kBK);  // CTA pairs: 128-deep stages
   p.m_tiles = mt_gu;
   p.a_rows_per_group = 2 * Ip;
   p.shared_b_row0 = xb ? 0 : T * k;
