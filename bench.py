@@ -44,6 +44,9 @@ def _args():
     ap.add_argument("--secondary",
                     default="prefill,zipf_prefill,clamp_ragged,tiny,decode_fp8,dense_decode,dense_prefill",
                     help="comma-separated further workloads measured in the same run")
+    ap.add_argument("--detail", default="",
+                    help="write the full record (per-stage times, every workload's rooflines) "
+                         "to this JSON file; the printed line stays compact")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
@@ -62,12 +65,42 @@ def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        # the tensor peak is the sustained figure: the K forwards of a timed
-        # region run back to back under the 1 kW power cap (the layer's own
-        # clocks under load: ~1.5 GHz at T=4096, ~1.4 GHz at T=16384)
-        return dict(hbm=d["hbm_gbs"], tc=d.get("bf16_tflops_sustained") or d["bf16_tflops"],
-                    tc_burst=d["bf16_tflops"], source="measured")
-    return dict(hbm=6650.0, tc=1400.0, tc_burst=1590.0, source="fallback")
+        return dict(hbm=d["hbm_gbs"], tc_burst=d["bf16_tflops"],
+                    tc_sustained=d.get("bf16_tflops_sustained") or d["bf16_tflops"],
+                    source="measured")
+    return dict(hbm=6650.0, tc_burst=1590.0, tc_sustained=1400.0, source="fallback")
+
+
+# A timed region shorter than this runs at the burst clocks; a longer one
+# settles at the power-capped sustained clocks.
+SUSTAINED_REGION_MS = 1000.0
+
+
+def _tc_peak(peaks, region_ms):
+    """The bf16 tensor peak that applies to a timed region of region_ms:
+    (TFLOP/s, label)."""
+    if region_ms >= SUSTAINED_REGION_MS:
+        return peaks["tc_sustained"], "sustained"
+    return peaks["tc_burst"], "burst"
+
+
+def _sig(v, n=4):
+    """v rounded to n significant digits, as an int when that is whole (keeps
+    the printed line short)."""
+    if v is None or isinstance(v, (bool, int)) or v == 0:
+        return v
+    from math import floor, log10
+    nd = n - 1 - int(floor(log10(abs(v))))
+    r = round(v, nd)
+    return int(r) if nd <= 0 else r
+
+
+def _config(wl, world):
+    """The config dict both arms print (identical for the same workload)."""
+    return {"workload": wl.name, "T": wl.T, "hidden": wl.hidden, "experts": wl.num_experts,
+            "top_k": wl.top_k, "intermediate": wl.intermediate, "shared_experts": 1,
+            "parallelism": f"replicas x{world} (weak)",
+            "l2": "inputs > L2: weights streamed from HBM each step"}
 
 
 def _traffic_record(kernel: str, workload: str, groups: int):
@@ -262,9 +295,7 @@ def run_reference(a):
         "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
         "ms_per_step": 1e3 * total / a.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "T": wl.T, "hidden": wl.hidden,
-                   "experts": wl.num_experts, "top_k": wl.top_k,
-                   "intermediate": wl.intermediate},
+        "config": _config(wl, a.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{sample} of {wl.T} tokens per step ({touched} routed experts "
                                    f"+ shared, weights drawn on the host, in RAM before timing)"},
@@ -312,42 +343,53 @@ def _routing_stats(layer, x):
     return int((counts > 0).sum()), int(counts.max())
 
 
-def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step):
+def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step, steps):
+    """Roofline of the dominant kernel (K5 gate|up) and of the whole layer.
+    The tensor peak is the burst figure for timed regions under a second (the
+    kernel at its burst clocks), the sustained one for longer regions."""
     from sparse_moe_layer_gemm_b200.roofline import (algorithmic_bytes, algorithmic_flops,
                                                      gate_up_bytes, gate_up_flops)
     gu_ms = stages_ms["gate_up"]
+    tc, tc_kind = _tc_peak(peaks, ms_step * steps)
     gu_bytes = gate_up_bytes(wl, touched)
     gu_flops = gate_up_flops(wl)
     t_bytes = gu_bytes / (peaks["hbm"] * 1e9)
-    t_flops = gu_flops / (peaks["tc"] * 1e12)
+    t_flops = gu_flops / (tc * 1e12)
     if t_bytes >= t_flops:
         ach = gu_bytes / (gu_ms * 1e-3) / 1e9
         rl = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
               "frac": ach / peaks["hbm"]}
     else:
         ach = gu_flops / (gu_ms * 1e-3) / 1e12
-        rl = {"bound": "tensor", "achieved": ach, "peak": peaks["tc"], "unit": "TFLOP/s",
-              "frac": ach / peaks["tc"]}
+        rl = {"bound": "tensor", "achieved": ach, "peak": tc, "unit": "TFLOP/s",
+              "frac": ach / tc}
     # from 2048 tokens the library runs the expert GEMMs on CTA pairs
     # (FP8 weights: one-SM tiles with converter warps at every size)
     if wl.weight_dtype == "fp8":
-        kname = "grouped_gemm_kernel<gate_up, fp8>"
+        kname = "K5 gate_up fp8"
     else:
-        kname = ("grouped_gemm_pair_kernel<gate_up>" if wl.T >= 2048
-                 else "grouped_gemm_kernel<gate_up>")
+        kname = "K5 gate_up pairs" if wl.T >= 2048 else "K5 gate_up"
     rl.update({"kernel": kname, "kernel_ms": gu_ms,
                "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
-               "peak_source": (f"{peaks['source']} (MEASURED_PEAKS.json; "
-                               "tensor: bf16_tflops_sustained)")
-               if peaks["source"] == "measured" else "fallback (tensor: sustained)",
+               "peak_source": f"{peaks['source']}: hbm_gbs, bf16 {tc_kind}",
                "traffic": _traffic_record("gate_up", wl.name, touched + 1)})
     lb = algorithmic_bytes(wl, touched)
     lf = algorithmic_flops(wl)
-    t_layer = max(lb / (peaks["hbm"] * 1e9), lf / (peaks["tc"] * 1e12))
-    layer = {"bound": "hbm" if lb / peaks["hbm"] >= lf / (peaks["tc"] * 1e3) else "tensor",
+    t_layer = max(lb / (peaks["hbm"] * 1e9), lf / (tc * 1e12))
+    layer = {"bound": "hbm" if lb / peaks["hbm"] >= lf / (tc * 1e3) else "tensor",
              "roofline_ms": 1e3 * t_layer, "frac": 1e3 * t_layer / ms_step,
-             "bytes": lb, "flops": lf, "touched_experts": touched}
+             "bytes": lb, "flops": lf, "touched_experts": touched, "tensor_peak": tc_kind}
     return rl, layer
+
+
+def _compact_roofline(rl):
+    """The roofline object of the printed line (the contract's keys, short)."""
+    out = {k: _sig(rl[k]) if isinstance(rl[k], float) else rl[k]
+           for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    out["kernel"] = rl.get("kernel", rl.get("scope", ""))
+    if "kernel_ms" in rl:
+        out["kernel_ms"] = _sig(rl["kernel_ms"])
+    return out
 
 
 def _dense_secondary(wl, a, dev, world, rank, stream, peaks):
@@ -363,7 +405,7 @@ def _dense_secondary(wl, a, dev, world, rank, stream, peaks):
     layer = B.DenseMLP.from_workload(wl)
     layer.load_inputs(inp)
     x = inp["x"]
-    steps, warm = max(3, a.steps // 10), max(3, a.warmup)
+    steps, warm = a.steps, max(3, a.warmup)
     with torch.cuda.stream(stream):
         for _ in range(warm):
             layer.forward(x)
@@ -383,21 +425,24 @@ def _dense_secondary(wl, a, dev, world, rank, stream, peaks):
     H, I, T = wl.hidden, wl.intermediate, wl.T
     nbytes = 3 * H * I * el_w + 2 * T * H * el_x
     flops = 6 * T * H * I
-    t_b, t_f = nbytes / (peaks["hbm"] * 1e9), flops / (peaks["tc"] * 1e12)
+    tc, tc_kind = _tc_peak(peaks, ms * steps)
+    t_b, t_f = nbytes / (peaks["hbm"] * 1e9), flops / (tc * 1e12)
     if t_b >= t_f:
         rl = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peaks["hbm"],
               "unit": "GB/s"}
     else:
-        rl = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peaks["tc"],
+        rl = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tc,
               "unit": "TFLOP/s"}
     rl["frac"] = rl["achieved"] / rl["peak"]
     rl.update({"scope": "whole dense layer (gate|up + down GEMMs)", "algorithmic_bytes": nbytes,
-               "algorithmic_flops": flops})
+               "algorithmic_flops": flops, "traffic": None,
+               "peak_source": f"{peaks['source']}: hbm_gbs, bf16 {tc_kind}"})
     layer.close()
     del inp, x
     torch.cuda.empty_cache()
     return {"workload": wl.name, "T": T, "value": job_throughput(T, world, ms), "unit": "tokens/s",
-            "ms_per_step": ms, "roofline": rl,
+            "ms_per_step": ms, "roofline": rl, "layer_roofline": {"frac": rl["frac"],
+                                                                  "bound": rl["bound"]},
             "layer": f"dense SwiGLU MLP, H={H}, I={I} (the first three decoder layers)"}
 
 
@@ -467,7 +512,7 @@ def run_ours(a):
     if err != 0:
         raise RuntimeError(f"device status word {err}")
     value = job_throughput(wl.T, world, ms)
-    kr, lr = _kernel_roofline(wl, touched, stages, peaks, ms)
+    kr, lr = _kernel_roofline(wl, touched, stages, peaks, ms, a.steps)
 
     e2e = None
     if not a.no_e2e:
@@ -515,13 +560,12 @@ def run_ours(a):
         x2 = draw_x(rank_batch_workload(wl2, rank), dev)
         touched2, _ = _routing_stats(layer2, x2)
         barrier()
-        ms2, _ = _measure(layer2, x2, max(3, a.steps // 10), max(3, a.warmup), stream,
-                          record_stages=False)
+        ms2, _ = _measure(layer2, x2, a.steps, max(3, a.warmup), stream, record_stages=False)
         ms2 = max_over_ranks(ms2, dev)
-        _, st2 = _measure(layer2, x2, max(3, a.steps // 10), 0, stream)
+        _, st2 = _measure(layer2, x2, a.steps, 0, stream)
         if layer2.device_error() != 0:
             raise RuntimeError(f"device status word {layer2.device_error()} ({wl2.name})")
-        kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2)
+        kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2, a.steps)
         entry = {"workload": wl2.name, "T": wl2.T, "value": job_throughput(wl2.T, world, ms2),
                  "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
                  "layer_roofline": lr2, "stage_ms": st2}
@@ -543,27 +587,68 @@ def run_ours(a):
 
     launches = B.moe_kernel_launches(layer.handle, wl.T) * a.steps
     if rank == 0:
-        line = {
+        full = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "T": wl.T, "hidden": wl.hidden,
-                       "experts": wl.num_experts, "top_k": wl.top_k,
-                       "intermediate": wl.intermediate, "shared_experts": 1,
-                       "parallelism": f"replicas x{world} (weak)",
-                       "l2": "inputs larger than L2: touched expert weights streamed from HBM "
-                             "every step"},
-            "roofline": kr, "layer_roofline": lr, "stage_ms": stages,
+            "config": _config(wl, world), "roofline": kr, "layer_roofline": lr,
+            "stage_ms": stages,
             "routing": {"touched_experts": touched, "max_rows_per_expert": max_rows},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
             "secondary": secondary,
         }
-        print(json.dumps(line), flush=True)
+        if a.detail:
+            with open(a.detail, "w") as f:
+                json.dump(full, f, indent=1)
+        print(json.dumps(_compact_line(full), separators=(",", ":")), flush=True)
     layer.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def _compact_line(full):
+    """The one printed JSON line, kept under 1500 characters: the contract's
+    keys with short values, the headline's layer roofline fraction, then the
+    other workloads as [tokens/s, layer roofline fraction] and, last, the
+    prefill (T=4096) half of the metric in full; per-stage tables and every
+    workload's kernel rooflines stay in the --detail file."""
+    line = {k: full[k] for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup",
+                                 "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
+                                 "dtype", "data", "config")}
+    line["value"] = _sig(line["value"], 6)
+    line["ms_per_step"] = _sig(line["ms_per_step"], 5)
+    line["roofline"] = _compact_roofline(full["roofline"])
+    line["layer_roofline"] = {"bound": full["layer_roofline"]["bound"],
+                              "frac": _sig(full["layer_roofline"]["frac"])}
+    cpu = full["cpu_baseline"]
+    if cpu is not None:
+        cpu = {"value": _sig(cpu["value"]), "unit": cpu["unit"], "cores": cpu["cores"],
+               "kind": cpu["kind"], "sample": cpu["short"]}
+    line["cpu_baseline"] = cpu
+    e2e = full["e2e"]
+    if e2e is not None:
+        e2e = {k: (_sig(v, 6) if k == "value" else v) for k, v in e2e.items() if k != "path"}
+    line["e2e"] = e2e
+    line["gpu_launches"] = full["gpu_launches"]
+    c = full["clocks"]
+    line["clocks"] = None if c is None else {"sm_mhz": c["sm_mhz"], "sm_max_mhz": c["sm_max_mhz"],
+                                             "reasons": c["reasons"]}
+    others, pre = {}, None
+    for e in full["secondary"]:
+        if e["workload"] == "prefill" and pre is None:
+            pre = {"T": e["T"], "value": _sig(e["value"], 6),
+                   "ms_per_step": _sig(e["ms_per_step"], 5),
+                   "layer_roofline": {"bound": e["layer_roofline"]["bound"],
+                                      "frac": _sig(e["layer_roofline"]["frac"])},
+                   "roofline": _compact_roofline(e["roofline"])}
+        else:
+            others[e["workload"]] = [_sig(e["value"], 3), _sig(e["layer_roofline"]["frac"], 3)]
+    line["others"] = others
+    if pre is not None:
+        line["prefill"] = pre
+    return line
 
 
 def _cpu_baseline_from_device(wl, inp, x):
@@ -586,6 +671,7 @@ def _cpu_baseline_from_device(wl, inp, x):
             "kind": "oracle",
             "sample": f"{sample} of {wl.T} tokens of the same batch, {touched} routed experts "
                       f"+ shared, fp64 NumPy, weights in host RAM before timing",
+            "short": f"{sample}/{wl.T} tokens, {touched} experts + shared, fp64",
             "seconds": secs}
 
 

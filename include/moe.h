@@ -264,14 +264,18 @@ int moe_forward_oneshot(const void* x, const float* router_w, const float* route
  * differ only on tokens whose k-th and (k+1)-th scores are within ~1e-6).
  *
  * Scratch: a 4 MiB static device array inside the library (1,048,576 fp32
- * partial logits), held on every GPU that loads the library until the
- * process exits.  T * E must not exceed 1,048,576 (MOE_ERR_UNSUPPORTED
- * otherwise).  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call uses the same array, so calls that
- * may overlap on the GPU (different streams, or different host threads) race
- * and must be serialised by the caller.  No cudaMalloc, cudaFree or other
- * allocating routine is called. */
+ * partial logits), held on a GPU from the first call on that device (module
+ * loading may be lazy) until the process exits.  T * E must not exceed
+ * 1,048,576 (MOE_ERR_UNSUPPORTED otherwise).  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  The
+ * address is kept per device together with the id of the context it was
+ * taken in; a call whose current context differs (for instance after a
+ * cudaDeviceReset) looks it up again, so that call, too, should come before
+ * any capture.  Every call uses the same array, so calls that may overlap on
+ * the GPU (different streams, or different host threads) race and must be
+ * serialised by the caller.  No cudaMalloc, cudaFree or other allocating
+ * routine is called. */
 int moe_route_static(const void* x, int act_dtype, const float* router_w,
                      const float* router_bias, int T, int H, int E, int k,
                      int norm_expert_weight, float routed_scaling_factor,

@@ -248,21 +248,22 @@ def _route(x, router_w, router_bias, top_k, scale, norm, use_bias, forced_idx):
         idx = np.asarray(forced_idx, dtype=np.int32).reshape(-1, top_k)
     s_sel = np.take_along_axis(s32, idx.astype(np.int64), axis=1)
     w = gate_weights(s_sel, scale, norm)
-    return logits, beta32, idx, w
+    return logits, s32, beta32, idx, w
 
 
 def moe_routing(x, router_w, router_bias, *, top_k: int, scale: float = 3.0,
                 norm: bool = True, use_bias: bool = True):
-    """Routing of every token without the expert FFNs: (topk_idx, topk_w,
-    counts, offsets, perm, pos, beta32, tie_gap).  Same steps as
+    """Routing of every token without the expert FFNs: a dict of topk_idx,
+    topk_w, counts, offsets, perm, pos, logits, s32 (the fp32 bias-free
+    scores), beta32 (the fp32 selection scores) and tie_gap.  Same steps as
     :func:`moe_forward` (sglang-jax issue #1367, "Key difficulties" item 1)."""
     x64 = _f64(x)
     E = np.asarray(router_w).shape[1]
-    logits, beta32, idx, w = _route(x64, router_w, router_bias, top_k, scale, norm, use_bias,
-                                    None)
+    logits, s32, beta32, idx, w = _route(x64, router_w, router_bias, top_k, scale, norm,
+                                         use_bias, None)
     counts, offsets, perm, pos = expert_permutation(idx, E)
     return dict(topk_idx=idx, topk_w=w, counts=counts, offsets=offsets, perm=perm, pos=pos,
-                beta32=beta32, tie_gap=near_tie_gaps(beta32, top_k), logits=logits)
+                s32=s32, beta32=beta32, tie_gap=near_tie_gaps(beta32, top_k), logits=logits)
 
 
 def moe_forward(x, router_w, router_bias, w_gate, w_up, w_down,
@@ -286,8 +287,8 @@ def moe_forward(x, router_w, router_bias, w_gate, w_up, w_down,
     x64 = _f64(x)
     T, H = x64.shape
     E = np.asarray(router_w).shape[1]
-    logits, beta32, idx, w = _route(x64, router_w, router_bias, top_k, scale,
-                                    norm, use_bias, forced_idx)
+    logits, _, beta32, idx, w = _route(x64, router_w, router_bias, top_k, scale,
+                                       norm, use_bias, forced_idx)
     counts, offsets, perm, pos = expert_permutation(idx, E)
     out = swiglu_expert(x64, sh_gate, sh_up, sh_down, swiglu_limit_shared)
     for e in range(E):
@@ -339,8 +340,8 @@ def moe_forward_dense_masked(x, router_w, router_bias, w_gate, w_up, w_down,
     x64 = _f64(x)
     T, H = x64.shape
     E = np.asarray(router_w).shape[1]
-    _, _, idx, w = _route(x64, router_w, router_bias, top_k, scale, norm,
-                          use_bias, None)
+    _, _, _, idx, w = _route(x64, router_w, router_bias, top_k, scale, norm,
+                             use_bias, None)
     M = np.zeros((T, E))
     for t in range(T):
         for j in range(top_k):

@@ -10,10 +10,14 @@
 // handle whose creation allocates; this entry point needs neither.
 //
 // Its only scratch, the split-K partial logits, lives in the file-scope array
-// below.  Every GPU that loads the library holds it until the process exits.
-// In host code `g_route_scratch` is a host-side stand-in, not a device
-// address, so its device address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+// below.  A GPU holds it from the first call on that device (module loading
+// may be lazy) until the process exits.  In host code `g_route_scratch` is a
+// host-side stand-in, not a device address, so its device address is looked
+// up with cudaGetSymbolAddress (with that device current) when a device is
+// first seen, and again whenever the device's current CUDA context is not
+// the one the address was taken in (after a cudaDeviceReset the module may
+// be loaded at another address), then passed to the kernels.
+#include <cudaTypedefs.h>
 #include <math.h>
 
 #include <mutex>
@@ -28,23 +32,61 @@ constexpr size_t kRouteScratchFloats = static_cast<size_t>(1) << 20;
 __device__ __align__(256) float g_route_scratch[kRouteScratchFloats];
 
 constexpr int kMaxDevices = 64;
-float* g_scratch_dev[kMaxDevices] = {};
+struct ScratchSlot {
+  float* ptr;                 // device address of g_route_scratch
+  unsigned long long ctx_id;  // the context it was taken in (0: unknown)
+};
+ScratchSlot g_scratch_dev[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (looked up the
-// first time this device is seen).
+// The unique id of the calling thread's current CUDA context (cuCtxGetId, a
+// per-process counter that is never reused), through the driver entry points
+// the runtime exposes; false if there is no current context or no entry point.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {  // (under g_scratch_mu)
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    looked_up = true;
+  }
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array on the current device: looked up the
+// first time the device is seen and whenever its current context has changed
+// since (or cannot be identified).
 int scratch_for_current_device(float** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_dev[dev] == nullptr) {
+  ScratchSlot& slot = g_scratch_dev[dev];
+  unsigned long long id = 0;
+  const bool known = current_context_id(&id);
+  if (slot.ptr == nullptr || !known || id != slot.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
       return MOE_ERR_CUDA;
-    g_scratch_dev[dev] = static_cast<float*>(p);
+    // the lookup has made the device's primary context current if none was
+    unsigned long long now = 0;
+    slot.ptr = static_cast<float*>(p);
+    slot.ctx_id = current_context_id(&now) ? now : 0;
   }
-  *out = g_scratch_dev[dev];
+  *out = slot.ptr;
   return MOE_OK;
 }
 

@@ -4,8 +4,14 @@ by the smoke check).
 Bar (element by element):
 * top-k indices bit-exact, except tokens whose oracle k-th and (k+1)-th fp32
   selection scores differ by less than TIE_BAND (several selections are then
-  correct); those are counted, and their outputs are re-checked against the
-  oracle evaluated on the GPU's selection;
+  correct).  Such a token's GPU selection must still be one of the correct
+  ones: k distinct experts that differ from the oracle's only in experts whose
+  oracle score lies within TIE_BAND of the oracle's k-th score, listed in
+  descending oracle score (within TIE_BAND), with the weights the oracle
+  gives that selection.  Those tokens are counted, and their outputs are
+  re-checked against the oracle evaluated on the GPU's selection;
+* ``strict=True`` (inputs built with exact ties, which both sides must break
+  to the lower index) allows no exception at all;
 * counts, offsets and the permutation bit-exact given the selection;
 * gate weights within fp32 rounding (rtol 1e-5);
 * router logits of the selected experts within LOGIT_TOL of the fp64 logits
@@ -45,16 +51,58 @@ class ParityReport:
         return self.rel_fro <= REL_FRO and self.max_abs_over_rms <= MAX_ABS_OVER_RMS
 
 
-def check_routing(gpu_rt: dict, ref: dict, top_k: int, E: int):
-    """Selection, weights and grouping.  Returns (mismatched-row mask, near-tie mask)."""
-    gidx = gpu_rt["topk_idx"]
+def check_tied_row(gidx_row, ref: dict, t: int, top_k: int, E: int):
+    """A near-tied token whose GPU selection differs from the oracle's: assert
+    it is another correct selection (see the module docstring)."""
+    beta = ref["beta32"][t].astype(np.float64)
+    oidx = ref["topk_idx"][t]
+    kth = beta[oidx[top_k - 1]]
+    g = [int(e) for e in gidx_row]
+    assert all(0 <= e < E for e in g), f"token {t}: expert id out of range {g}"
+    assert len(set(g)) == top_k, f"token {t}: repeated expert {g}"
+    added = set(g) - set(int(e) for e in oidx)
+    dropped = set(int(e) for e in oidx) - set(g)
+    for e in added:
+        assert beta[e] >= kth - TIE_BAND, \
+            f"token {t}: expert {e} (score {beta[e]!r}) is below the k-th score {kth!r}"
+    for e in dropped:
+        assert beta[e] <= kth + TIE_BAND, \
+            f"token {t}: dropped expert {e} (score {beta[e]!r}) is above the k-th {kth!r}"
+    for j in range(top_k - 1):
+        a, b = beta[g[j]], beta[g[j + 1]]
+        assert a >= b - TIE_BAND, f"token {t}: order not descending at slot {j}: {g}"
+
+
+def check_selection(gidx: np.ndarray, gw: np.ndarray, ref: dict, top_k: int, E: int,
+                    scale: float = 3.0, strict: bool = False):
+    """Top-k indices and gate weights against the oracle's routing ``ref``.
+    Returns (mismatched-row mask, near-tie mask)."""
     tie = ref["tie_gap"] < TIE_BAND
     mism = (gidx != ref["topk_idx"]).any(axis=1)
+    if strict:
+        bad = np.nonzero(mism)[0]
+        assert bad.size == 0, f"top-k differs on {bad.size} exactly-tied tokens, first {bad[:8]}"
     bad = np.nonzero(mism & ~tie)[0]
     assert bad.size == 0, f"top-k differs on {bad.size} non-tied tokens, first {bad[:8]}"
-    # weights: the bias-free scores of the (same) selection, renormalised, scaled
+    for t in np.nonzero(mism)[0]:
+        check_tied_row(gidx[t], ref, int(t), top_k, E)
+    # weights: the bias-free scores of the selection, renormalised, scaled --
+    # the oracle's own for matching rows, the oracle's for the GPU's selection
+    # on the others
     ok = ~mism
-    np.testing.assert_allclose(gpu_rt["topk_w"][ok], ref["topk_w"][ok], rtol=W_RTOL, atol=1e-7)
+    np.testing.assert_allclose(gw[ok], ref["topk_w"][ok], rtol=W_RTOL, atol=1e-7)
+    if mism.any():
+        s_sel = np.take_along_axis(ref["s32"][mism], gidx[mism].astype(np.int64), axis=1)
+        want = om.gate_weights(s_sel, scale, True)
+        np.testing.assert_allclose(gw[mism], want, rtol=W_RTOL, atol=1e-7)
+    return mism, tie
+
+
+def check_routing(gpu_rt: dict, ref: dict, top_k: int, E: int, wl=None, strict: bool = False):
+    """Selection, weights and grouping.  Returns (mismatched-row mask, near-tie mask)."""
+    gidx = gpu_rt["topk_idx"]
+    mism, tie = check_selection(gidx, gpu_rt["topk_w"], ref, top_k, E,
+                                scale=3.0 if wl is None else wl.scale, strict=strict)
     # grouping: the permutation of the GPU's own selection is unique
     counts, offsets, perm, _ = om.expert_permutation(gidx, E)
     assert np.array_equal(gpu_rt["counts"], counts)
@@ -105,7 +153,8 @@ class _Widened:
 
 
 def compare(inp_host: dict, wl, gpu_out: np.ndarray, gpu_rt: dict,
-            rows: Optional[np.ndarray] = None, experts=None) -> ParityReport:
+            rows: Optional[np.ndarray] = None, experts=None,
+            strict: bool = False) -> ParityReport:
     """inp_host: exact fp32 host copies of x, router_w, router_bias (and, when
     ``experts`` is None, of all weights); ``experts`` may supply lazy
     per-expert views (w_gate, w_up, w_down, sh_gate, sh_up, sh_down)."""
@@ -113,7 +162,7 @@ def compare(inp_host: dict, wl, gpu_out: np.ndarray, gpu_rt: dict,
     x = inp_host["x"]
     ref = om.moe_routing(x, inp_host["router_w"], inp_host["router_bias"], top_k=k,
                          scale=wl.scale)
-    mism, tie = check_routing(gpu_rt, ref, k, E)
+    mism, tie = check_routing(gpu_rt, ref, k, E, wl=wl, strict=strict)
     logit_err = 0.0
     if "logits" in gpu_rt:
         d = np.abs(gpu_rt["logits"].astype(np.float64) - ref["logits"])

@@ -117,3 +117,69 @@ def test_committed_traffic_records_match_the_sources():
             assert os.path.exists(os.path.join(bench.ROOT, src)), src
         keys.append(f[0])
     assert keys, "no records"
+
+
+def _fake_full(n_secondary=6):
+    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS
+    peaks = bench._peaks()
+    wl, wp = WORKLOADS["decode"], WORKLOADS["prefill"]
+    kr, lr = bench._kernel_roofline(wl, 131, {"gate_up": 0.4021234}, peaks, 0.62099, 200)
+    kr2, lr2 = bench._kernel_roofline(wp, 201, {"gate_up": 1.0712345}, peaks, 1.7131, 200)
+    kr2["traffic"] = 4533671234
+    sec = [{"workload": n, "T": 1, "value": 12345678.91, "ms_per_step": 1.0,
+            "roofline": kr2, "layer_roofline": lr2}
+           for n in ["zipf_prefill", "clamp_ragged", "tiny", "decode_fp8", "dense_decode",
+                     "dense_prefill"][:n_secondary]]
+    sec.insert(1, {"workload": "prefill", "T": 4096, "value": 2391694.123,
+                   "ms_per_step": 1.7131234, "roofline": kr2, "layer_roofline": lr2})
+    return {"metric": bench.METRIC, "value": 103059.849, "unit": "tokens/s", "n_gpus": 8,
+            "steps": 200, "warmup": 5, "ms_per_step": 0.62099838, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": bench._config(wl, 8), "roofline": kr, "layer_roofline": lr,
+            "stage_ms": {}, "routing": {},
+            "cpu_baseline": {"value": 9.4835962, "unit": "tokens/s", "cores": 128,
+                             "kind": "oracle", "short": "8/64 tokens, 148 experts + shared, fp64"},
+            "e2e": {"value": 91327.955, "unit": "tokens/s", "h2d_bytes_per_step": 524288,
+                    "d2h_bytes_per_step": 524288, "path": "p"},
+            "gpu_launches": 1400,
+            "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0,
+                       "reasons": ["sw_power_cap", "hw_slowdown"], "samples": 9,
+                       "source": "nvml"},
+            "secondary": sec}
+
+
+def test_compact_line_fits_the_tail_and_ends_with_prefill():
+    """The printed line stays under 1500 characters (the part of stdout the
+    round's record keeps) and ends with the T=4096 half of the metric."""
+    import json
+    line = bench._compact_line(_fake_full())
+    s = json.dumps(line, separators=(",", ":"))
+    assert len(s) < 1500, len(s)
+    assert list(line)[-1] == "prefill"
+    pre = line["prefill"]
+    assert pre["T"] == 4096 and pre["roofline"]["traffic"] == 4533671234
+    for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert k in line["roofline"] and k in pre["roofline"]
+    assert set(line["others"]) == {"zipf_prefill", "clamp_ragged", "tiny", "decode_fp8",
+                                   "dense_decode", "dense_prefill"}
+
+
+def test_tensor_peak_follows_the_timed_region():
+    peaks = bench._peaks()
+    assert bench._tc_peak(peaks, 999.0) == (peaks["tc_burst"], "burst")
+    assert bench._tc_peak(peaks, 1000.0) == (peaks["tc_sustained"], "sustained")
+    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS
+    wl = WORKLOADS["zipf_prefill"]
+    # a 20-step region of 4 ms steps is short: burst peak
+    kr, lr = bench._kernel_roofline(wl, 28, {"gate_up": 2.5}, peaks, 4.0, 20)
+    assert kr["bound"] == "tensor" and kr["peak"] == peaks["tc_burst"]
+    assert lr["tensor_peak"] == "burst"
+    kr, lr = bench._kernel_roofline(wl, 28, {"gate_up": 2.5}, peaks, 4.0, 500)
+    assert kr["peak"] == peaks["tc_sustained"] and lr["tensor_peak"] == "sustained"
+
+
+def test_both_arms_print_the_same_config():
+    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS
+    wl = WORKLOADS["decode"]
+    assert bench._config(wl, 4) == _fake_full()["config"] or bench._config(wl, 8) == \
+        _fake_full()["config"]

@@ -240,10 +240,42 @@ def pin_clamp_off():
     assert not np.allclose(a.out, c.out)
 
 
+def pin_routing_fields():
+    """moe_routing (the routing half alone, which the GPU checks compare with)
+    equals moe_forward's routing fields field by field, and its score arrays
+    equal an independent torch recomputation: the fp64 logits rounded once to
+    fp32, the fp32 rounding of the float64 sigmoid, plus the bias in fp32;
+    tie_gap is the gap between the k-th and (k+1)-th of a full sort."""
+    for kw in ({}, dict(swiglu_limit=0.3, swiglu_limit_shared=0.5, T=48, top_k=3)):
+        wl, inp = _tiny(**kw)
+        f = _fwd(inp, wl)
+        r = om.moe_routing(inp["x"], inp["router_w"], inp["router_bias"], top_k=wl.top_k,
+                           scale=wl.scale)
+        for name in ("topk_idx", "topk_w", "counts", "offsets", "perm", "pos", "beta32",
+                     "tie_gap", "logits"):
+            assert np.array_equal(np.asarray(r[name]), np.asarray(getattr(f, name))), name
+        lt = (torch.as_tensor(inp["x"], dtype=torch.float64)
+              @ torch.as_tensor(inp["router_w"], dtype=torch.float64))
+        s = torch.sigmoid(lt.float().double()).float()
+        beta = s + torch.as_tensor(inp["router_bias"], dtype=torch.float32)
+        assert np.array_equal(r["s32"], s.numpy())
+        assert np.array_equal(r["beta32"], beta.numpy())
+        srt = torch.sort(beta.double(), dim=1, descending=True).values
+        gap = (srt[:, wl.top_k - 1] - srt[:, wl.top_k]).numpy()
+        assert np.array_equal(r["tie_gap"], gap)
+        T, k = wl.T, wl.top_k
+        assert np.array_equal(r["perm"][r["pos"].reshape(-1)], np.arange(T * k))
+        sel = torch.as_tensor(r["topk_idx"].astype(np.int64))
+        ssel = torch.gather(s.double(), 1, sel)
+        assert np.allclose(r["topk_w"], (3.0 * ssel / ssel.sum(1, keepdim=True)).numpy(),
+                           rtol=1e-15, atol=0)
+
+
 PINS = [pin_topk_brute_force, pin_weights_sum_to_scale, pin_bias_selects_only,
         pin_closed_form_identical_experts, pin_single_expert_is_dense_mlp,
         pin_all_experts_mixture, pin_grouped_equals_dense_masked,
-        pin_row_independence, pin_permutation, pin_clamp_branches, pin_clamp_off]
+        pin_row_independence, pin_permutation, pin_clamp_branches, pin_clamp_off,
+        pin_routing_fields]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -450,6 +482,21 @@ def test_mutant_transposed_down(monkeypatch):
     monkeypatch.setattr(om, "swiglu_expert",
                         lambda rows, wg, wu, wd, limit: orig(rows, wg, wu, np.asarray(wd).T, limit))
     assert _fails([pin_closed_form_identical_experts, pin_clamp_branches])
+
+
+def test_mutant_routing_ignores_bias(monkeypatch):
+    orig = om.moe_routing
+
+    def no_bias(x, router_w, router_bias, **kw):
+        return orig(x, router_w, None, **kw)
+    monkeypatch.setattr(om, "moe_routing", no_bias)
+    assert _fails([pin_routing_fields])
+
+
+def test_mutant_routing_gap_of_wrong_slots(monkeypatch):
+    orig = om.near_tie_gaps
+    monkeypatch.setattr(om, "near_tie_gaps", lambda beta, k: orig(beta, k + 1))
+    assert _fails([pin_routing_fields])
 
 
 # ---------------------------------------------------------------- FP8 E4M3 weights

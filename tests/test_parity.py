@@ -24,8 +24,9 @@ def _routing_np(rt):
     return {k: v.cpu().numpy() for k, v in rt.items()}
 
 
-def _run_small(wl):
-    cpu = make_inputs(wl, "cpu")
+def _run_small(wl, cpu=None, strict=False):
+    if cpu is None:
+        cpu = make_inputs(wl, "cpu")
     inp = {k: v.cuda() for k, v in cpu.items()}
     layer = B.MoeLayer.from_workload(wl)
     layer.load_inputs(inp)
@@ -33,9 +34,10 @@ def _run_small(wl):
     torch.cuda.synchronize()
     assert layer.device_error() == 0
     host = {k: host_f32(cpu[k]) for k in ("x", "router_w", "router_bias")}
-    rep = compare(host, wl, host_f32(out), _routing_np(rt), experts=expert_views(cpu))
+    rt_np = _routing_np(rt)
+    rep = compare(host, wl, host_f32(out), rt_np, experts=expert_views(cpu), strict=strict)
     layer.close()
-    return rep
+    return rep, rt_np, host_f32(out)
 
 
 SMALL = {
@@ -137,8 +139,99 @@ def test_fp8_decode_every_code():
 @pytest.mark.timeout(300)
 @pytest.mark.parametrize("name", list(SMALL))
 def test_small_parity(name):
-    rep = _run_small(SMALL[name])
+    rep, _, _ = _run_small(SMALL[name])
     assert rep.ok(), rep
+
+
+# ------------------------------------------------------------ exact ties
+# The reading of the pages (sglang-jax issue #1367, "Key difficulties" item 1:
+# top-k of the biased fp32 scores; the order of equal scores is not stated):
+# equal selection scores go to the lower expert index.  These inputs make both
+# sides compute bit-identical scores for several experts, so the tie rule
+# itself decides, and the comparison allows no near-tie exception.
+
+TIES = {
+    # CUDA-core router; k odd, so the k-th and (k+1)-th are an exactly tied pair
+    "dup_columns_cuda_core": replace(WORKLOADS["tiny"], name="d1", T=64, top_k=3,
+                                     act_dtype="bf16", weight_dtype="bf16"),
+    # tensor-core router (>= 512 bf16 tokens) with the candidate recomputation
+    "dup_columns_tensor_core": replace(WORKLOADS["tiny"], name="d2", T=1024, hidden=512,
+                                       num_experts=32, top_k=5, intermediate=128,
+                                       shared_intermediate=128, act_dtype="bf16",
+                                       weight_dtype="bf16", x_dist="rmsnorm_normal"),
+    # warp-per-token top-k (from 8192 tokens)
+    "dup_columns_warp_topk": replace(WORKLOADS["tiny"], name="d3", T=8448, hidden=256,
+                                     num_experts=40, top_k=5, intermediate=128,
+                                     shared_intermediate=128, act_dtype="bf16",
+                                     weight_dtype="bf16", x_dist="rmsnorm_normal"),
+}
+
+
+def _dup_columns(wl):
+    """Router columns 2j+1 copied from 2j, with equal biases."""
+    cpu = make_inputs(wl, "cpu")
+    rw = cpu["router_w"].clone()
+    rb = cpu["router_bias"].clone()
+    rw[:, 1::2] = rw[:, 0::2]
+    rb[1::2] = rb[0::2]
+    cpu["router_w"], cpu["router_bias"] = rw, rb
+    return cpu
+
+
+@pytest.mark.timeout(600)
+@pytest.mark.parametrize("name", list(TIES))
+def test_exact_ties_duplicated_router_columns(name):
+    import oracle.moe_oracle as om
+    wl = TIES[name]
+    cpu = _dup_columns(wl)
+    host = {k: host_f32(cpu[k]) for k in ("x", "router_w", "router_bias")}
+    ref = om.moe_routing(host["x"], host["router_w"], host["router_bias"], top_k=wl.top_k,
+                         scale=wl.scale)
+    # precondition: the oracle's scores tie exactly in pairs, and many tokens
+    # have a tied pair straddling the k-th slot
+    assert np.array_equal(ref["beta32"][:, 0::2], ref["beta32"][:, 1::2])
+    assert (ref["tie_gap"] == 0).mean() > 0.5
+    rep, rt, _ = _run_small(wl, cpu=cpu, strict=True)
+    assert rep.ok(), rep
+    assert rep.idx_mismatch_rows == 0
+    idx = rt["topk_idx"]
+    # within every selected pair the lower index comes first
+    for t in range(0, wl.T, max(1, wl.T // 64)):
+        row = list(idx[t])
+        for j, e in enumerate(row):
+            if e % 2 == 1:
+                assert e - 1 in row[:j], (t, row)
+
+
+ZERO_ROWS = {
+    "cuda_core": replace(WORKLOADS["tiny"], name="z1", T=96, bias="zero", act_dtype="bf16",
+                         weight_dtype="bf16"),
+    # tensor-core router: every expert of a zero row is a candidate (more
+    # than 32 of them)
+    "tensor_core": replace(WORKLOADS["tiny"], name="z2", T=640, hidden=256, num_experts=40,
+                           top_k=6, intermediate=128, shared_intermediate=128, bias="zero",
+                           act_dtype="bf16", weight_dtype="bf16", x_dist="rmsnorm_normal"),
+}
+
+
+@pytest.mark.timeout(600)
+@pytest.mark.parametrize("name", list(ZERO_ROWS))
+def test_exact_ties_zero_rows(name):
+    """An all-zero input row with zero bias: every logit is 0 and every score
+    0.5, so the selection must be experts 0..k-1 with weights 3/k, and the
+    output row is f_shared(0) + sum of f_e(0) = 0."""
+    wl = ZERO_ROWS[name]
+    cpu = make_inputs(wl, "cpu")
+    zero = [0, 1, wl.T // 2, wl.T - 1]
+    x = cpu["x"].clone()
+    x[zero] = 0
+    cpu["x"] = x
+    rep, rt, out = _run_small(wl, cpu=cpu, strict=True)
+    assert rep.ok(), rep
+    for t in zero:
+        assert list(rt["topk_idx"][t]) == list(range(wl.top_k))
+        assert np.all(rt["topk_w"][t] == np.float32(wl.scale / wl.top_k))
+        assert np.all(out[t] == 0)
 
 
 @pytest.mark.timeout(300)
@@ -233,11 +326,29 @@ def _full(wl, inp, layer, n_rows=24):
     experts = dict(w_gate=HostExpertView(inp["w_gate"]), w_up=HostExpertView(inp["w_up"]),
                    w_down=HostExpertView(inp["w_down"]), sh_gate=host_f32(inp["sh_gate"]),
                    sh_up=host_f32(inp["sh_up"]), sh_down=host_f32(inp["sh_down"]))
-    rng = np.random.default_rng(0)
-    rows = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, n_rows)]))
-    rep = compare(host, wl, host_f32(out), _routing_np(rt), rows=rows, experts=experts)
+    rt_np = _routing_np(rt)
+    rows = _check_rows(wl, rt_np, n_rows)
+    rep = compare(host, wl, host_f32(out), rt_np, rows=rows, experts=experts)
     print(wl.name, rep)
     return rep
+
+
+def _check_rows(wl, rt_np, n_rows=24, tile=128, groups=5):
+    """Rows compared with the oracle at full size: every row up to 64 tokens;
+    else the first and last, n_rows random ones, and one random row of every
+    128-row token tile (each half of a CTA pair's 256-token tile) of the
+    `groups` largest expert groups."""
+    if wl.T <= 64:
+        return np.arange(wl.T)
+    rng = np.random.default_rng(0)
+    rows = [np.array([0, wl.T - 1]), rng.integers(0, wl.T, n_rows)]
+    counts, offsets, perm = rt_np["counts"], rt_np["offsets"], rt_np["perm"]
+    for e in np.argsort(-counts, kind="stable")[:groups]:
+        for b0 in range(0, int(counts[e]), tile):
+            n = min(tile, int(counts[e]) - b0)
+            pair = perm[int(offsets[e]) + b0 + int(rng.integers(0, n))]
+            rows.append(np.array([pair // wl.top_k]))
+    return np.unique(np.concatenate(rows))
 
 
 @pytest.mark.timeout(900)
@@ -270,9 +381,8 @@ def test_full_size_fp8_decode():
     torch.cuda.synchronize()
     assert layer.device_error() == 0
     host = {k: host_f32(inp[k]) for k in ("x", "router_w", "router_bias")}
-    rng = np.random.default_rng(1)
-    rows = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 24)]))
-    rep = compare(host, wl, host_f32(out), _routing_np(rt), rows=rows,
+    rt_np = _routing_np(rt)
+    rep = compare(host, wl, host_f32(out), rt_np, rows=_check_rows(wl, rt_np),
                   experts=expert_views(inp))
     print(wl.name, rep)
     layer.close()
