@@ -19,6 +19,21 @@
  * Selection order and ties: descending s + b, equal scores to the lower
  * expert index.  The shared expert has no gate and weight 1.
  *
+ * Arithmetic: the router, the scores, the selection and the gate weights are
+ * fp32 on the CUDA cores (from 512 bf16 tokens the logits are first
+ * approximated on the tensor cores and every expert near the selection
+ * boundary is recomputed in fp32).  The expert GEMMs are bf16 x bf16 with
+ * fp32 accumulation: fp32 x and fp32 expert weights (the act_dtype /
+ * weight_dtype MOE_F32 case) are rounded to bf16 (round to nearest even) on
+ * the way in, h = SwiGLU(...) and each expert's weighted output row are
+ * rounded to bf16, and the k + 1 rows of a token are summed in fp32 and
+ * rounded once to the output dtype.  Error budget: each bf16 rounding is a
+ * relative error of at most 2^-9; with independent rounding errors over
+ * K-term sums the output's relative Frobenius error stays near 2^-9 times a
+ * small constant (measured against the fp64 definition: ~5e-3 with fp32
+ * inputs of the tiny shape, ~3e-3 at the full layer), inside the 1e-2 bar.
+ * There is no fp32 or tf32 expert GEMM.
+ *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers unless the name says _host.
  *    They are owned by the caller; the library never frees or keeps them past

@@ -2,8 +2,9 @@
 by the smoke check).
 
 Bar (element by element):
-* top-k indices bit-exact, except tokens whose oracle k-th and (k+1)-th fp32
-  selection scores differ by less than TIE_BAND (several selections are then
+* top-k indices bit-exact, except near-tied tokens: those whose oracle k-th
+  and (k+1)-th fp32 selection scores differ by less than TIE_BAND, or two of
+  whose selected experts do (several selections, or orders, are then
   correct).  Such a token's GPU selection must still be one of the correct
   ones: k distinct experts that differ from the oracle's only in experts whose
   oracle score lies within TIE_BAND of the oracle's k-th score, listed in
@@ -51,6 +52,20 @@ class ParityReport:
         return self.rel_fro <= REL_FRO and self.max_abs_over_rms <= MAX_ABS_OVER_RMS
 
 
+def order_gaps(beta32: np.ndarray, top_k: int) -> np.ndarray:
+    """Per token, the smallest gap between neighbours among the k + 1 largest
+    fp32 selection scores.  Below TIE_BAND the token is near-tied: either the
+    k-th and (k+1)-th (which expert is selected) or two selected experts
+    (their order) are within fp32 rounding of each other, so a GPU whose fp32
+    logits differ from the correctly rounded ones in the last bits may
+    legitimately decide the other way."""
+    b = -np.sort(-np.asarray(beta32, dtype=np.float64), axis=1)
+    n = min(top_k + 1, b.shape[1])
+    if n < 2:
+        return np.full(b.shape[0], np.inf)
+    return (b[:, :n - 1] - b[:, 1:n]).min(axis=1)
+
+
 def check_tied_row(gidx_row, ref: dict, t: int, top_k: int, E: int):
     """A near-tied token whose GPU selection differs from the oracle's: assert
     it is another correct selection (see the module docstring)."""
@@ -77,7 +92,7 @@ def check_selection(gidx: np.ndarray, gw: np.ndarray, ref: dict, top_k: int, E: 
                     scale: float = 3.0, strict: bool = False):
     """Top-k indices and gate weights against the oracle's routing ``ref``.
     Returns (mismatched-row mask, near-tie mask)."""
-    tie = ref["tie_gap"] < TIE_BAND
+    tie = order_gaps(ref["beta32"], top_k) < TIE_BAND
     mism = (gidx != ref["topk_idx"]).any(axis=1)
     if strict:
         bad = np.nonzero(mism)[0]

@@ -112,3 +112,22 @@ def test_non_tied_mismatch_rejected():
     idx[u, wl.top_k - 1] = out[0]
     with pytest.raises(AssertionError):
         check_routing(_gpu(ref, idx, wl), ref, wl.top_k, wl.num_experts, wl=wl)
+
+
+def test_order_swap_of_near_equal_selected_experts():
+    """Two selected experts whose scores are within TIE_BAND may come in
+    either order; with a larger gap the swap is rejected."""
+    wl = WORKLOADS["tiny"]
+    inp = {k: v.float().numpy() for k, v in make_inputs(wl, "cpu").items()}
+    ref = om.moe_routing(inp["x"], inp["router_w"], inp["router_bias"], top_k=wl.top_k,
+                         scale=wl.scale)
+    t = 3
+    e1, e2 = int(ref["topk_idx"][t, 1]), int(ref["topk_idx"][t, 2])
+    idx = ref["topk_idx"].copy()
+    idx[t, [1, 2]] = idx[t, [2, 1]]
+    with pytest.raises(AssertionError):        # a real gap: the order is fixed
+        check_routing(_gpu(ref, idx, wl), ref, wl.top_k, wl.num_experts, wl=wl)
+    ref["beta32"] = ref["beta32"].copy()
+    ref["beta32"][t, e2] = np.nextafter(ref["beta32"][t, e1], np.float32(-1))
+    mism, tie = check_routing(_gpu(ref, idx, wl), ref, wl.top_k, wl.num_experts, wl=wl)
+    assert mism[t] and tie[t]
