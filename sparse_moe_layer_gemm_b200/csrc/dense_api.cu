@@ -29,8 +29,11 @@ struct moe_dense {
   int loaded;
   CUtensorMap tm_gu;    // box 64 x 256 (one CTA per tile)
   CUtensorMap tm_gu128; // box 64 x 128 (split-K partial tiles)
-  CUtensorMap tm_gu64;  // box 64 x 64 (CTA pairs)
+  CUtensorMap tm_gu_pw; // CTA pairs, wide stages: 64 + 64 rows x 2 K blocks
+  CUtensorMap tm_gu_pn; // CTA pairs, narrow stages: 64 + 64 rows x 3 K blocks
   CUtensorMap tm_dn;    // box 64 x 128
+  CUtensorMap tm_dn_pw; // CTA pairs: 128 rows x 2 K blocks
+  CUtensorMap tm_dn_pn; // CTA pairs: 128 rows x 3 K blocks
 };
 
 namespace {
@@ -202,8 +205,11 @@ int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out) {
       cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess ||
       !moe::encode_bf16_2d(&L->tm_gu, L->w_gu, 2 * Ip, H, 2 * moe::kBM) ||
       !moe::encode_bf16_2d(&L->tm_gu128, L->w_gu, 2 * Ip, H, moe::kBM) ||
-      !moe::encode_bf16_2d(&L->tm_gu64, L->w_gu, 2 * Ip, H, 64) ||
-      !moe::encode_bf16_2d(&L->tm_dn, L->w_dn, H, Ip, moe::kBM)) {
+      !moe::encode_bf16_gate_up_pair(&L->tm_gu_pw, L->w_gu, 2 * Ip, H, 2) ||
+      !moe::encode_bf16_gate_up_pair(&L->tm_gu_pn, L->w_gu, 2 * Ip, H, 3) ||
+      !moe::encode_bf16_2d(&L->tm_dn, L->w_dn, H, Ip, moe::kBM) ||
+      !moe::encode_bf16_kblocks(&L->tm_dn_pw, L->w_dn, H, Ip, moe::kBM, 2) ||
+      !moe::encode_bf16_kblocks(&L->tm_dn_pn, L->w_dn, H, Ip, moe::kBM, 3)) {
     moe_dense_destroy(L);
     return MOE_ERR_CUDA;
   }
@@ -277,14 +283,31 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
   const bool pair_dn = pair && (H / moe::kBM) % 2 == 0;
   const int dn_blocks = moe::gemm_down_blocks(H);
   moe::GemmMaps gu{}, dn{};
-  gu.a = pair ? L->tm_gu64 : L->tm_gu;
-  dn.a = L->tm_dn;
-  if (!moe::encode_bf16_2d(&gu.b, xb, T, H, moe::kBBoxRows) ||
-      !moe::encode_bf16_2d(&gu.bw, xb, T, H, moe::kBN) ||
-      !moe::encode_bf16_store(&gu.out, h, T, Ip) ||
-      !moe::encode_bf16_2d(&dn.b, h, T, Ip, moe::kBBoxRows) ||
-      !moe::encode_bf16_2d(&dn.bw, h, T, Ip, moe::kBN) ||
-      !moe::encode_bf16_store(&dn.out, y, T, H))
+  if (pair) {  // CTA pairs: K-block maps (see launch_gemm_gate_up_pair)
+    gu.a = L->tm_gu_pw;
+    gu.a2 = L->tm_gu_pn;
+    if (!moe::encode_bf16_kblocks(&gu.b, xb, T, H, moe::kBBoxRows, 3) ||
+        !moe::encode_bf16_kblocks(&gu.bw, xb, T, H, moe::kBN, 2))
+      return MOE_ERR_CUDA;
+  } else {
+    gu.a = L->tm_gu;
+    if (!moe::encode_bf16_2d(&gu.b, xb, T, H, moe::kBBoxRows) ||
+        !moe::encode_bf16_2d(&gu.bw, xb, T, H, moe::kBN))
+      return MOE_ERR_CUDA;
+  }
+  if (pair_dn) {
+    dn.a = L->tm_dn_pw;
+    dn.a2 = L->tm_dn_pn;
+    if (!moe::encode_bf16_kblocks(&dn.b, h, T, Ip, moe::kBBoxRows, 3) ||
+        !moe::encode_bf16_kblocks(&dn.bw, h, T, Ip, moe::kBN, 2))
+      return MOE_ERR_CUDA;
+  } else {
+    dn.a = L->tm_dn;
+    if (!moe::encode_bf16_2d(&dn.b, h, T, Ip, moe::kBBoxRows) ||
+        !moe::encode_bf16_2d(&dn.bw, h, T, Ip, moe::kBN))
+      return MOE_ERR_CUDA;
+  }
+  if (!moe::encode_bf16_store(&gu.out, h, T, Ip) || !moe::encode_bf16_store(&dn.out, y, T, H))
     return MOE_ERR_CUDA;
   gu.bsh = gu.b;
   gu.bshw = gu.bw;
@@ -367,7 +390,7 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
     return MOE_OK;
   }
 
-  p.num_kb = H / (pair ? 2 * moe::kBK : moe::kBK);
+  p.num_kb = H / moe::kBK;
   p.m_tiles = Ip / moe::kBM;
   p.a_rows_per_group = 2 * Ip;
   p.out = h;
@@ -376,7 +399,7 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
   MOE_CUDA(pair ? moe::launch_gemm_gate_up_pair(gu, p, st)
                 : moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
 
-  p.num_kb = Ip / (pair_dn ? 2 * moe::kBK : moe::kBK);
+  p.num_kb = Ip / moe::kBK;
   p.m_tiles = pair_dn ? H / (2 * moe::kBM) : H / moe::kBM / dn_blocks;
   p.a_rows_per_group = H;
   p.out = y;

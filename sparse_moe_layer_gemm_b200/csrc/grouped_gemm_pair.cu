@@ -16,11 +16,22 @@
 // 128) of the tile and tokens [r N/2, (r + 1) N/2), and holds accumulator rows
 // [128 r, 128 r + 128) x all N tokens in its TMEM.
 //   gate|up: a tile is 128 features of one expert; CTA r loads the gate and the
-//            up rows of features [64 r, 64 r + 64) (two 64-row boxes), so its
+//            up rows of features [64 r, 64 r + 64) (one 4-D box), so its
 //            accumulator holds gate in lanes 0-63 and up in lanes 64-127 for
 //            the same features; the epilogue pairs warp q (gate) with warp
 //            q + 2 (up) through shared memory for the SwiGLU.
 //   down:    a tile is 256 features; CTA r loads features [128 r, 128 r + 128).
+//
+// Pipeline stages (3 slots of 64 KB per CTA) carry several 64-deep K
+// sub-blocks of both operands, each operand brought by ONE TMA load per stage
+// (a 4-D box for the gate|up weights, 3-D boxes whose last dimension walks the
+// K sub-blocks otherwise).  The weight stream is latency-bound at prefill
+// sizes: a slot's round trip is the load's latency plus the issue of its
+// MMAs, and only three slots fit.  So a tile whose token half is at most 32
+// rows (most experts' tiles at prefill) uses a narrow stage: 3 K sub-blocks
+// of weights (48 KB) and 3 of 32 token rows (12 KB), where a wide tile's
+// stage holds 2 sub-blocks of weights and 2 of 128 token rows: 50 % more
+// weight bytes in flight for the same ring.
 //
 // Roles per CTA (6 warps): warp 0 TMA producer (both CTAs: own halves, every
 // load completing on the leader's full barrier); warp 1 TMEM allocation (both)
@@ -41,17 +52,22 @@ using namespace gemm;
 
 constexpr int kPairBN = 256;  // tokens per tile (the pair MMA's N)
 
-template <int MODE, int KSUB>
+template <int MODE>
 struct PairShape {
   static constexpr bool GU = MODE == kModeGateUp;
   static constexpr int BN = kPairBN;
-  static constexpr int BK = kBK * KSUB;                  // K per pipeline stage
   static constexpr int ROW = kBK * 2;                    // bytes per 64-element swizzled row
   static constexpr int SUB_A = kBM * ROW;                // one 64-K sub-block of this CTA's A
-  static constexpr int SUB_B = (BN / 2) * ROW;           // one 64-K sub-block of this CTA's B
-  static constexpr int A_BYTES = KSUB * SUB_A;
-  static constexpr int STAGE_BYTES = KSUB * (SUB_A + SUB_B);
-  static constexpr int STAGES = (192 * 1024 / STAGE_BYTES) < 6 ? (192 * 1024 / STAGE_BYTES) : 6;
+  static constexpr int SUB_BW = (BN / 2) * ROW;          // ... of this CTA's B, wide tile
+  static constexpr int SUB_BN = kBBoxRows * ROW;         // ... of this CTA's B, narrow tile
+  static constexpr int KS_W = 2;                         // K sub-blocks per wide stage
+  static constexpr int KS_N = 3;                         // K sub-blocks per narrow stage
+  static constexpr int B_OFF_W = KS_W * SUB_A;           // B within a wide stage
+  static constexpr int B_OFF_N = KS_N * SUB_A;           // B within a narrow stage
+  static constexpr int BYTES_W = KS_W * (SUB_A + SUB_BW);  // one CTA's bytes per stage
+  static constexpr int BYTES_N = KS_N * (SUB_A + SUB_BN);
+  static constexpr int STAGE_BYTES = 64 * 1024;
+  static constexpr int STAGES = 3;
   static constexpr int THREADS = 32 * 6;
   static constexpr int ACC_COLS = BN;                    // fp32 columns per accumulator buffer
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
@@ -65,13 +81,20 @@ struct PairShape {
   static constexpr int TAB_OFFSET = EPI_OFFSET + EPI_BYTES;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(TAB_OFFSET) + kTabBytes;
   static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
-  static_assert(STAGES >= 2, "pipeline depth");
-  static_assert(STAGE_BYTES % 1024 == 0 && SUB_A % 1024 == 0, "swizzle atoms stay aligned");
+  static_assert(BYTES_W <= STAGE_BYTES && BYTES_N <= STAGE_BYTES, "stage contents fit a slot");
+  static_assert(STAGE_BYTES % 1024 == 0 && SUB_A % 1024 == 0 && SUB_BN % 1024 == 0 &&
+                    SUB_BW % 1024 == 0,
+                "swizzle atoms stay aligned");
   static_assert(1024 + STAGES * STAGE_BYTES + BAR_BYTES <= 256 * 1024, "descriptor range");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   static_assert(TMEM_COLS <= 512, "TMEM capacity");
   static_assert(BN / 2 == kBN, "the wide token-row box is BN / 2 rows");
 };
+
+// A tile is narrow when this CTA's token half of it fits one 32-row box.
+__device__ __forceinline__ bool narrow_tile(int n_valid) {
+  return (((n_valid + 15) & ~15) >> 1) <= kBBoxRows;
+}
 
 // D[tmem of both CTAs] (+)= A[both CTAs' smem] * B[both CTAs' smem]^T.
 __device__ __forceinline__ void mma_issue_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -83,19 +106,41 @@ __device__ __forceinline__ void mma_issue_pair(uint32_t d_tmem, uint64_t a_desc,
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
-// tmA: gate|up weights with 64-row boxes, or down weights with 128-row boxes.
-// tmB / tmBsh (32-row boxes) and tmBw / tmBshw (128-row boxes): token rows
-// (x_perm or h; tmBsh / tmBshw the shared expert's rows of x, gate|up only).
-// tmOut: h or y with 32-feature x 16-row boxes.
-template <int MODE, int KSUB>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB>::THREADS, 1)
-    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+// The MMAs of one stage: KS K sub-blocks (nsub of them inside K) x 4 K steps
+// of 16, unrolled with constant descriptor offsets (the issue loop's own cost
+// adds to every MMA's ~100-cycle issue time).  `first`: the tile's first
+// stage, whose first MMA overwrites the accumulator.
+template <int KS, int SUB_A, int SUB_B>
+__device__ __forceinline__ void issue_stage_pair(uint32_t d, uint64_t ad, uint64_t bd,
+                                                 uint32_t idesc, int nsub, bool first) {
+#pragma unroll
+  for (int h = 0; h < KS; ++h) {
+    if (h == 0 || h < nsub) {
+#pragma unroll
+      for (int kk = 0; kk < kBK / 16; ++kk)
+        mma_issue_pair(d, ad + static_cast<uint64_t>((h * SUB_A + kk * 32) >> 4),
+                       bd + static_cast<uint64_t>((h * SUB_B + kk * 32) >> 4), idesc,
+                       (first && h == 0 && kk == 0) ? 0u : 1u);
+    }
+  }
+}
+
+// tmAw / tmAn: the weights of a wide / narrow stage (gate|up: 4-D boxes of
+// 64 gate + 64 up rows x 2 or 3 K sub-blocks; down: 3-D boxes of 128 rows x 2
+// or 3 K sub-blocks).  tmBw / tmBshw (128 rows x 2 K sub-blocks) and tmB /
+// tmBsh (32 rows x 3 K sub-blocks): token rows (x_perm or h; tmBsh / tmBshw
+// the shared expert's rows of x, gate|up only).  tmOut: h or y with
+// 32-feature x 16-row boxes.  p.num_kb is K / 64 (K sub-blocks).
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE>::THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmAw,
+                             const __grid_constant__ CUtensorMap tmAn,
                              const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmBsh,
                              const __grid_constant__ CUtensorMap tmBw,
                              const __grid_constant__ CUtensorMap tmBshw,
                              const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-  using S = PairShape<MODE, KSUB>;
+  using S = PairShape<MODE>;
   constexpr bool GU = S::GU;
   constexpr int BN = S::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -132,7 +177,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmAw);
+    prefetch_tmap(&tmAn);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmBw);
     if (GU) {
@@ -167,40 +213,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
         if (*abort_flag) break;
         const Tile t = decode_tile<BN>(gp, w);
         const int half = ((t.n_valid + 15) & ~15) >> 1;  // this CTA's token rows of the MMA
-        const bool wide = half > kBBoxRows;
+        const bool narrow = narrow_tile(t.n_valid);
+        const int ks = narrow ? S::KS_N : S::KS_W;
+        const int n_st = (p.num_kb + ks - 1) / ks;
         const bool sh = GU && t.g == p.E;
-        const CUtensorMap* mb = wide ? (sh ? &tmBshw : &tmBw) : (sh ? &tmBsh : &tmB);
+        const CUtensorMap* mb = narrow ? (sh ? &tmBsh : &tmB) : (sh ? &tmBshw : &tmBw);
+        const CUtensorMap* ma = narrow ? &tmAn : &tmAw;
         const int b_row = (sh ? p.shared_b_row0 : group_row0(gp, t.g)) + t.nc * BN +
                           static_cast<int>(rank) * half;
-        // gate|up: rows of features [mt*128 + 64 r, +64) of the gate half, then
-        // of the up half, of the group's [gate 128 | up 128] blocks
+        // gate|up: rows of features [mt*128 + 64 r, +64) of the gate half (and,
+        // 128 rows on, of the up half) of the group's [gate 128 | up 128] blocks
         const int a_row = GU ? t.g * p.a_rows_per_group + t.mt * 2 * kBM + static_cast<int>(rank) * 64
                              : t.g * p.a_rows_per_group + t.mt * 2 * kBM + static_cast<int>(rank) * kBM;
-        const uint32_t cta_bytes = KSUB * (S::SUB_A + (wide ? kBN : kBBoxRows) * S::ROW);
+        const uint32_t cta_bytes = narrow ? S::BYTES_N : S::BYTES_W;
+        const uint32_t b_off = narrow ? S::B_OFF_N : S::B_OFF_W;
         const uint64_t pol_a = t.nch > 1 ? pol_normal : pol_first;
         bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int st = 0; st < n_st; ++st) {
           const uint32_t s = it % S::STAGES;
           const uint32_t ph = (it / S::STAGES) & 1u;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
+          // (a last stage past K reads zeros for the missing sub-blocks; their
+          // bytes still count, and the issuer skips their MMAs)
           if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * cta_bytes);
           const uint32_t fb = full_leader + 8 * s;
           const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
-#pragma unroll
-          for (int h = 0; h < KSUB; ++h) {
-            const int x = kb * S::BK + h * kBK;
-            const uint32_t da = sa + h * S::SUB_A;
-            if (GU) {
-              tma_load_2d_pair(da, &tmA, fb, x, a_row, pol_a);
-              tma_load_2d_pair(da + 64 * S::ROW, &tmA, fb, x, a_row + kBM, pol_a);
-            } else {
-              tma_load_2d_pair(da, &tmA, fb, x, a_row, pol_a);
-            }
-            tma_load_2d_pair(sa + S::A_BYTES + h * S::SUB_B, mb, fb, x, b_row, pol_b);
-          }
+          const int kb0 = st * ks;
+          if (GU)
+            tma_load_4d_pair(sa, ma, fb, 0, a_row, 0, kb0, pol_a);
+          else
+            tma_load_3d_pair(sa, ma, fb, 0, a_row, kb0, pol_a);
+          tma_load_3d_pair(sa + b_off, mb, fb, 0, b_row, kb0, pol_b);
           ++it;
         }
         if (!ok) break;
@@ -230,8 +276,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
         if (!mbar_wait(tempty0 + 8 * buf, tph ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + buf * S::ACC_COLS;
+        const bool narrow = narrow_tile(t.n_valid);
+        const int ks = narrow ? S::KS_N : S::KS_W;
+        const int n_st = (p.num_kb + ks - 1) / ks;
+        const uint32_t b_off = narrow ? S::B_OFF_N : S::B_OFF_W;
         bool ok = true;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int st = 0; st < n_st; ++st) {
           const uint32_t s = it % S::STAGES;
           const uint32_t ph = (it / S::STAGES) & 1u;
           if (!mbar_wait(full0 + 8 * s, ph, abort_flag, p.status)) {
@@ -240,14 +290,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
           }
           tc_fence_after();
           const uint64_t ad = desc0 + static_cast<uint64_t>((s * S::STAGE_BYTES) >> 4);
-          const uint64_t bd = ad + static_cast<uint64_t>(S::A_BYTES >> 4);
-#pragma unroll
-          for (int h = 0; h < KSUB; ++h)
-#pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)
-              mma_issue_pair(d, ad + static_cast<uint64_t>((h * S::SUB_A + kk * 32) >> 4),
-                             bd + static_cast<uint64_t>((h * S::SUB_B + kk * 32) >> 4), idesc,
-                             (kb | h | kk) != 0 ? 1u : 0u);
+          const uint64_t bd = ad + static_cast<uint64_t>(b_off >> 4);
+          const int nsub = min(ks, p.num_kb - st * ks);  // K sub-blocks inside K
+          if (narrow)
+            issue_stage_pair<S::KS_N, S::SUB_A, S::SUB_BN>(d, ad, bd, idesc, nsub, st == 0);
+          else
+            issue_stage_pair<S::KS_W, S::SUB_A, S::SUB_BW>(d, ad, bd, idesc, nsub, st == 0);
           tc_commit_pair_mc(empty0 + 8 * s, 3);  // frees the stage in both CTAs
           ++it;
         }
@@ -418,11 +466,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<MODE, KSUB
   }
 }
 
-using GuPair = PairShape<kModeGateUp, 2>;
-using DnPair = PairShape<kModeDown, 2>;
-// The host sets GemmParams::num_kb of these launches to K / (2 * kBK).
-static_assert(GuPair::BK == 2 * kBK && DnPair::BK == 2 * kBK,
-              "the host's stage count assumes two 64-deep sub-blocks per stage");
+using GuPair = PairShape<kModeGateUp>;
+using DnPair = PairShape<kModeDown>;
 
 int g_pair_grid = 0;  // CTAs per launch: twice the co-resident clusters
 
@@ -430,11 +475,11 @@ int g_pair_grid = 0;  // CTAs per launch: twice the co-resident clusters
 
 cudaError_t gemm_pair_configure_device(int num_sms) {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kModeGateUp, 2>,
+  if ((e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kModeGateUp>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(GuPair::SMEM))) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kModeDown, 2>,
+  if ((e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<kModeDown>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(DnPair::SMEM))) != cudaSuccess)
     return e;
@@ -450,7 +495,7 @@ cudaError_t gemm_pair_configure_device(int num_sms) {
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int clusters = 0;
-  if ((e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<kModeGateUp, 2>,
+  if ((e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<kModeGateUp>,
                                           &cfg)) != cudaSuccess)
     return e;
   g_pair_grid = 2 * (clusters < num_sms / 2 ? clusters : num_sms / 2);
@@ -461,15 +506,16 @@ int gemm_pair_grid() { return g_pair_grid; }
 
 cudaError_t launch_gemm_gate_up_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   if (g_pair_grid <= 0) return cudaErrorInvalidConfiguration;
-  return launch_pdl(grouped_gemm_pair_kernel<kModeGateUp, 2>, dim3(g_pair_grid),
-                    dim3(GuPair::THREADS), GuPair::SMEM, st, m.a, m.b, m.bsh, m.bw, m.bshw, m.out,
-                    p);
+  return launch_pdl(grouped_gemm_pair_kernel<kModeGateUp>, dim3(g_pair_grid),
+                    dim3(GuPair::THREADS), GuPair::SMEM, st, m.a, m.a2, m.b, m.bsh, m.bw, m.bshw,
+                    m.out, p);
 }
 
 cudaError_t launch_gemm_down_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st) {
   if (g_pair_grid <= 0) return cudaErrorInvalidConfiguration;
-  return launch_pdl(grouped_gemm_pair_kernel<kModeDown, 2>, dim3(g_pair_grid),
-                    dim3(DnPair::THREADS), DnPair::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
+  return launch_pdl(grouped_gemm_pair_kernel<kModeDown>, dim3(g_pair_grid),
+                    dim3(DnPair::THREADS), DnPair::SMEM, st, m.a, m.a2, m.b, m.b, m.bw, m.bw, m.out,
+                    p);
 }
 
 }  // namespace moe

@@ -39,8 +39,11 @@ struct moe_layer {
   int* status;          // device status word
   int loaded;
   CUtensorMap tm_gu;    // A operand of K5 (box 64 x 256)
-  CUtensorMap tm_gu64;  // A operand of K5 on CTA pairs (box 64 x 64)
-  CUtensorMap tm_dn;    // A operand of K6 (box 64 x 128)
+  CUtensorMap tm_gu_pw;  // A operand of K5 on CTA pairs, wide stages (64 + 64 rows x 2 K blocks)
+  CUtensorMap tm_gu_pn;  //   narrow stages (64 + 64 rows x 3 K blocks)
+  CUtensorMap tm_dn;     // A operand of K6 (box 64 x 128)
+  CUtensorMap tm_dn_pw;  // A operand of K6 on CTA pairs, wide stages (128 rows x 2 K blocks)
+  CUtensorMap tm_dn_pn;  //   narrow stages (128 rows x 3 K blocks)
   CUtensorMap tm_router;  // A operand of the tensor-core router (box 64 x 128)
   // stage timers: capacity x (MOE_NUM_STAGES + 1) events, filled in order
   std::vector<cudaEvent_t> events;
@@ -81,17 +84,36 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 }
 
 // bf16 [rows, cols] row-major seen as 3-D (64 columns, rows, cols / 64
-// column blocks), box 64 x box_rows x 2 column blocks, 128B swizzle: the FP8
-// GEMMs' token rows for two k-steps in one load (smem: k-block-major).
-bool encode_bf16_kpair(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
-                       uint32_t box_rows) {
+// column blocks), box 64 x box_rows x kblocks column blocks, 128B swizzle:
+// several K blocks of token rows (or weight rows) in one load (smem:
+// k-block-major).
+bool encode_bf16_kblocks(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows, uint32_t kblocks) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(moe::kBK), rows, cols / moe::kBK};
   cuuint64_t strides[2] = {cols * 2, static_cast<cuuint64_t>(moe::kBK) * 2};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::kBK), box_rows, 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(moe::kBK), box_rows, kblocks};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The packed gate|up weights as 4-D (64 columns, rows - 128, 2 halves 128
+// rows apart, cols / 64 column blocks), box 64 x 64 x 2 x kblocks.
+bool encode_bf16_gate_up_pair(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                              uint32_t kblocks) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr || rows < 2 * moe::kBM) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(moe::kBK), rows - moe::kBM, 2, cols / moe::kBK};
+  cuuint64_t strides[3] = {cols * 2, static_cast<cuuint64_t>(moe::kBM) * cols * 2,
+                           static_cast<cuuint64_t>(moe::kBK) * 2};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(moe::kBK), 64, 2, kblocks};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -118,6 +140,8 @@ bool encode_bf16_store(CUtensorMap* m, void* base, uint64_t rows, uint64_t cols)
 using moe::aligned;
 using moe::DeviceGuard;
 using moe::encode_bf16_2d;
+using moe::encode_bf16_gate_up_pair;
+using moe::encode_bf16_kblocks;
 using moe::encode_bf16_kpair;
 using moe::encode_bf16_store;
 
@@ -283,8 +307,11 @@ int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count
   // (FP8 codes are read with plain bulk copies: no tensor maps)
   const bool maps_ok =
       L->fp8 || (encode_bf16_2d(&L->tm_gu, L->w_gu, (El + 1) * 2 * Ip, H, 2 * moe::kBM) &&
-                 encode_bf16_2d(&L->tm_gu64, L->w_gu, (El + 1) * 2 * Ip, H, 64) &&
-                 encode_bf16_2d(&L->tm_dn, L->w_dn, (El + 1) * H, Ip, moe::kBM));
+                 encode_bf16_gate_up_pair(&L->tm_gu_pw, L->w_gu, (El + 1) * 2 * Ip, H, 2) &&
+                 encode_bf16_gate_up_pair(&L->tm_gu_pn, L->w_gu, (El + 1) * 2 * Ip, H, 3) &&
+                 encode_bf16_2d(&L->tm_dn, L->w_dn, (El + 1) * H, Ip, moe::kBM) &&
+                 encode_bf16_kblocks(&L->tm_dn_pw, L->w_dn, (El + 1) * H, Ip, moe::kBM, 2) &&
+                 encode_bf16_kblocks(&L->tm_dn_pn, L->w_dn, (El + 1) * H, Ip, moe::kBM, 3));
   if (!maps_ok || !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM)) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
@@ -479,31 +506,64 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   const int mt_dn = pair_dn ? H / (2 * moe::kBM) : H / moe::kBM / dn_blocks;
 
   // Token-row operands, each with kBBoxRows- and kBN-row boxes: x_perm (or x
-  // for the shared expert) for K5 and the router, h for K6.
+  // for the shared expert) for K5 and the router, h for K6.  The CTA-pair
+  // kernels read them as K-block maps (32 rows x 3 K blocks, 128 rows x 2).
   moe::GemmMaps gu{}, dn{}, rt{};
-  gu.a = pair_gu ? L->tm_gu64 : L->tm_gu;  // (unused with FP8 weights)
-  dn.a = L->tm_dn;
-  rt.a = L->tm_router;
-  if (!encode_bf16_2d(&gu.b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
-      !encode_bf16_2d(&gu.bw, x_perm, w.rows_xperm, H, moe::kBN) ||
-      !encode_bf16_2d(&dn.b, hbuf, w.rows_all, Ip, moe::kBBoxRows) ||
-      !encode_bf16_2d(&dn.bw, hbuf, w.rows_all, Ip, moe::kBN) ||
-      !encode_bf16_store(&gu.out, hbuf, w.rows_all, Ip) ||
-      !encode_bf16_store(&dn.out, ybuf, w.rows_all, H))
-    return MOE_ERR_CUDA;
-  rt.out = dn.out;  // unused by the router
-  if (xb) {
-    if (!encode_bf16_2d(&gu.bsh, x, T, H, moe::kBBoxRows) ||
-        !encode_bf16_2d(&gu.bshw, x, T, H, moe::kBN))
-      return MOE_ERR_CUDA;
-    rt.b = gu.bsh;
-    rt.bw = gu.bshw;
-  } else {
-    gu.bsh = gu.b;
-    gu.bshw = gu.bw;
-  }
-  dn.bsh = dn.b;
-  dn.bshw = dn.bw;
+  const bool maps_ok = [&] {
+    if (pair_gu) {
+      gu.a = L->tm_gu_pw;
+      gu.a2 = L->tm_gu_pn;
+      if (!encode_bf16_kblocks(&gu.b, x_perm, w.rows_xperm, H, moe::kBBoxRows, 3) ||
+          !encode_bf16_kblocks(&gu.bw, x_perm, w.rows_xperm, H, moe::kBN, 2))
+        return false;
+      if (xb) {
+        if (!encode_bf16_kblocks(&gu.bsh, x, T, H, moe::kBBoxRows, 3) ||
+            !encode_bf16_kblocks(&gu.bshw, x, T, H, moe::kBN, 2))
+          return false;
+      } else {
+        gu.bsh = gu.b;
+        gu.bshw = gu.bw;
+      }
+    } else {
+      gu.a = L->tm_gu;  // (unused with FP8 weights)
+      if (!encode_bf16_2d(&gu.b, x_perm, w.rows_xperm, H, moe::kBBoxRows) ||
+          !encode_bf16_2d(&gu.bw, x_perm, w.rows_xperm, H, moe::kBN))
+        return false;
+      if (xb) {
+        if (!encode_bf16_2d(&gu.bsh, x, T, H, moe::kBBoxRows) ||
+            !encode_bf16_2d(&gu.bshw, x, T, H, moe::kBN))
+          return false;
+      } else {
+        gu.bsh = gu.b;
+        gu.bshw = gu.bw;
+      }
+    }
+    if (pair_dn) {
+      dn.a = L->tm_dn_pw;
+      dn.a2 = L->tm_dn_pn;
+      if (!encode_bf16_kblocks(&dn.b, hbuf, w.rows_all, Ip, moe::kBBoxRows, 3) ||
+          !encode_bf16_kblocks(&dn.bw, hbuf, w.rows_all, Ip, moe::kBN, 2))
+        return false;
+    } else {
+      dn.a = L->tm_dn;
+      if (!encode_bf16_2d(&dn.b, hbuf, w.rows_all, Ip, moe::kBBoxRows) ||
+          !encode_bf16_2d(&dn.bw, hbuf, w.rows_all, Ip, moe::kBN))
+        return false;
+    }
+    dn.bsh = dn.b;
+    dn.bshw = dn.bw;
+    if (!encode_bf16_store(&gu.out, hbuf, w.rows_all, Ip) ||
+        !encode_bf16_store(&dn.out, ybuf, w.rows_all, H))
+      return false;
+    // the tensor-core router (bf16 x): the one-SM kernel's 2-D maps of x
+    rt.a = L->tm_router;
+    rt.out = dn.out;  // unused by the router
+    if (xb && (!encode_bf16_2d(&rt.b, x, T, H, moe::kBBoxRows) ||
+               !encode_bf16_2d(&rt.bw, x, T, H, moe::kBN)))
+      return false;
+    return true;
+  }();
+  if (!maps_ok) return MOE_ERR_CUDA;
   moe::GemmMaps gu8{}, dn8{};  // FP8 GEMMs: token rows as k-pair maps
   if (L->fp8) {
     gu8.out = gu.out;
@@ -581,7 +641,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.limit_shared = c.swiglu_limit_shared;
 
   p.tile_start = tiles_gu;
-  p.num_kb = H / (pair_gu ? 2 * moe::kBK : moe::kBK);  // CTA pairs: 128-deep stages
+  p.num_kb = H / moe::kBK;
   p.m_tiles = mt_gu;
   p.a_rows_per_group = 2 * Ip;
   p.shared_b_row0 = xb ? 0 : T * k;
@@ -597,7 +657,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   MOE_CUDA(mark(5));
 
   p.tile_start = tiles_dn;
-  p.num_kb = Ip / (pair_dn ? 2 * moe::kBK : moe::kBK);
+  p.num_kb = Ip / moe::kBK;
   p.m_tiles = mt_dn;
   p.a_rows_per_group = H;
   p.shared_b_row0 = T * k;

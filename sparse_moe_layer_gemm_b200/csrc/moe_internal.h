@@ -123,9 +123,11 @@ int gemm_down_blocks(int H);
 // Tensor maps of one grouped-GEMM launch: the weight operand, the token-row
 // operand with kBBoxRows- and BN-row boxes, the shared expert's token rows
 // (gate|up only) with both box heights, and the output for TMA stores (h or
-// y with 32-feature x 16-row boxes, no swizzle).
+// y with 32-feature x 16-row boxes, no swizzle).  The CTA-pair kernels take
+// a (wide stages) and a2 (narrow stages) for the weights and K-block maps for
+// the token rows (see launch_gemm_gate_up_pair).
 struct GemmMaps {
-  CUtensorMap a, b, bsh, bw, bshw, out;
+  CUtensorMap a, a2, b, bsh, bw, bshw, out;
 };
 
 cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
@@ -136,9 +138,12 @@ cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid,
 // k-blocks; A and B both offset by the part's K): m.a with 128-row boxes, two
 // 128-row weight blocks per tile; fp32 [T, out_ld] per part.
 cudaError_t launch_gemm_partial(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
-// CTA-pair versions (grouped_gemm_pair.cu): m.a has 64-row boxes for gate|up
-// and 128-row boxes for down; tiles of 256 tokens; num_kb = K / 128; m_tiles
-// = I_pad / 128 (gate|up) or H / 256 (down).
+// CTA-pair versions (grouped_gemm_pair.cu), tiles of 256 tokens: m.a / m.a2
+// the weights of wide / narrow stages (gate|up: encode_bf16_gate_up_pair with
+// 2 / 3 K blocks; down: encode_bf16_kblocks, 128 rows, 2 / 3 K blocks); m.bw /
+// m.bshw the token rows with 128-row x 2 K-block boxes, m.b / m.bsh with
+// 32-row x 3 K-block boxes; num_kb = K / 64; m_tiles = I_pad / 128 (gate|up)
+// or H / 256 (down).
 cudaError_t launch_gemm_gate_up_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st);
 cudaError_t launch_gemm_down_pair(const GemmMaps& m, const GemmParams& p, cudaStream_t st);
 // FP8 E4M3 weights (grouped_gemm_fp8.cu): p.a_codes the tile-major code
