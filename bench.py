@@ -44,6 +44,8 @@ def _args():
     ap.add_argument("--secondary",
                     default="prefill,zipf_prefill,clamp_ragged,tiny,decode_fp8,dense_decode,dense_prefill",
                     help="comma-separated further workloads measured in the same run")
+    ap.add_argument("--path", choices=["auto", "multi", "fused"], default="auto",
+                    help="moe_forward's execution path (auto: the library's choice)")
     ap.add_argument("--detail", default="",
                     help="write the full record (per-stage times, every workload's rooflines) "
                          "to this JSON file; the printed line stays compact")
@@ -343,36 +345,46 @@ def _routing_stats(layer, x):
     return int((counts > 0).sum()), int(counts.max())
 
 
-def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step, steps):
-    """Roofline of the dominant kernel (K5 gate|up) and of the whole layer.
-    The tensor peak is the burst figure for timed regions under a second (the
-    kernel at its burst clocks), the sustained one for longer regions."""
+def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step, steps, fused=False):
+    """Roofline of the dominant kernel and of the whole layer.  Multi-launch
+    path: K5 gate|up, timed by its stage events.  Fused path: the one kernel
+    is the whole layer (its time is stage 0).  The tensor peak is the burst
+    figure for timed regions under a second (the kernel at its burst clocks),
+    the sustained one for longer regions."""
     from sparse_moe_layer_gemm_b200.roofline import (algorithmic_bytes, algorithmic_flops,
                                                      gate_up_bytes, gate_up_flops)
-    gu_ms = stages_ms["gate_up"]
     tc, tc_kind = _tc_peak(peaks, ms_step * steps)
-    gu_bytes = gate_up_bytes(wl, touched)
-    gu_flops = gate_up_flops(wl)
-    t_bytes = gu_bytes / (peaks["hbm"] * 1e9)
-    t_flops = gu_flops / (tc * 1e12)
+    if fused:
+        k_ms = stages_ms["router"]
+        k_bytes = algorithmic_bytes(wl, touched)
+        k_flops = algorithmic_flops(wl)
+        kname = "moe_fused_kernel (whole layer)"
+        trec = _traffic_record("fused", wl.name, touched + 1)
+    else:
+        k_ms = stages_ms["gate_up"]
+        k_bytes = gate_up_bytes(wl, touched)
+        k_flops = gate_up_flops(wl)
+        # from 2048 tokens the library runs the expert GEMMs on CTA pairs
+        # (FP8 weights: one-SM tiles with converter warps at every size)
+        if wl.weight_dtype == "fp8":
+            kname = "K5 gate_up fp8"
+        else:
+            kname = "K5 gate_up pairs" if wl.T >= 2048 else "K5 gate_up"
+        trec = _traffic_record("gate_up", wl.name, touched + 1)
+    t_bytes = k_bytes / (peaks["hbm"] * 1e9)
+    t_flops = k_flops / (tc * 1e12)
     if t_bytes >= t_flops:
-        ach = gu_bytes / (gu_ms * 1e-3) / 1e9
+        ach = k_bytes / (k_ms * 1e-3) / 1e9
         rl = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
               "frac": ach / peaks["hbm"]}
     else:
-        ach = gu_flops / (gu_ms * 1e-3) / 1e12
+        ach = k_flops / (k_ms * 1e-3) / 1e12
         rl = {"bound": "tensor", "achieved": ach, "peak": tc, "unit": "TFLOP/s",
               "frac": ach / tc}
-    # from 2048 tokens the library runs the expert GEMMs on CTA pairs
-    # (FP8 weights: one-SM tiles with converter warps at every size)
-    if wl.weight_dtype == "fp8":
-        kname = "K5 gate_up fp8"
-    else:
-        kname = "K5 gate_up pairs" if wl.T >= 2048 else "K5 gate_up"
-    rl.update({"kernel": kname, "kernel_ms": gu_ms,
-               "algorithmic_bytes": gu_bytes, "algorithmic_flops": gu_flops,
+    rl.update({"kernel": kname, "kernel_ms": k_ms,
+               "algorithmic_bytes": k_bytes, "algorithmic_flops": k_flops,
                "peak_source": f"{peaks['source']}: hbm_gbs, bf16 {tc_kind}",
-               "traffic": _traffic_record("gate_up", wl.name, touched + 1)})
+               "traffic": trec})
     lb = algorithmic_bytes(wl, touched)
     lf = algorithmic_flops(wl)
     t_layer = max(lb / (peaks["hbm"] * 1e9), lf / (tc * 1e12))
@@ -478,6 +490,8 @@ def run_ours(a):
     inp = make_inputs(wl, dev)                          # weights replicated on every rank
     x = draw_x(rank_batch_workload(wl, rank), dev)      # each rank its own batch
     layer = B.MoeLayer.from_workload(wl)
+    path = {"auto": B.MOE_PATH_AUTO, "multi": B.MOE_PATH_MULTI, "fused": B.MOE_PATH_FUSED}[a.path]
+    layer.set_path(path)
     layer.load_inputs(inp)
     stream = torch.cuda.Stream(device=dev)
     touched, max_rows = _routing_stats(layer, x)
@@ -512,7 +526,8 @@ def run_ours(a):
     if err != 0:
         raise RuntimeError(f"device status word {err}")
     value = job_throughput(wl.T, world, ms)
-    kr, lr = _kernel_roofline(wl, touched, stages, peaks, ms, a.steps)
+    fused = B.moe_forward_path(layer.handle, wl.T) == B.MOE_PATH_FUSED
+    kr, lr = _kernel_roofline(wl, touched, stages, peaks, ms, a.steps, fused)
 
     e2e = None
     if not a.no_e2e:
@@ -551,6 +566,7 @@ def run_ours(a):
         if not same_experts:  # its own layer and weights (clamped / tiny configs)
             inp2 = make_inputs(wl2, dev)
             layer2 = B.MoeLayer.from_workload(wl2)
+            layer2.set_path(path)
             layer2.load_inputs(inp2)
         elif wl2.bias != wl.bias:  # same experts, another router bias
             from sparse_moe_layer_gemm_b200.workloads import draw_router
@@ -565,10 +581,12 @@ def run_ours(a):
         _, st2 = _measure(layer2, x2, a.steps, 0, stream)
         if layer2.device_error() != 0:
             raise RuntimeError(f"device status word {layer2.device_error()} ({wl2.name})")
-        kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2, a.steps)
+        fused2 = B.moe_forward_path(layer2.handle, wl2.T) == B.MOE_PATH_FUSED
+        kr2, lr2 = _kernel_roofline(wl2, touched2, st2, peaks, ms2, a.steps, fused2)
         entry = {"workload": wl2.name, "T": wl2.T, "value": job_throughput(wl2.T, world, ms2),
                  "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
-                 "layer_roofline": lr2, "stage_ms": st2}
+                 "layer_roofline": lr2, "stage_ms": st2,
+                 "path": "fused" if fused2 else "multi-launch"}
         if wl2.weight_dtype != "bf16":
             entry["weights"] = {"fp8": "fp8_e4m3 codes + fp32 per-feature scales (bf16 MMA)",
                                 "f32": "fp32 (rounded to bf16 at load)"}[wl2.weight_dtype]

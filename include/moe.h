@@ -191,6 +191,54 @@ int moe_forward(moe_layer_t* layer, const void* x, int T, void* out,
                 void* workspace, size_t ws_bytes, void* stream,
                 const moe_routing_t* routing);
 
+/* Execution paths of moe_forward.
+ *  MOE_PATH_MULTI: one kernel per stage (router, top-k, sort, gather,
+ *    gate|up GEMM, down GEMM, combine: 7 to 10 launches).
+ *  MOE_PATH_FUSED: the whole layer in one persistent kernel (the pages'
+ *    FusedEPMoE backend, sglang-jax issue #1367, section "Reuse map" and the
+ *    sub-issue "FusedEPMoE performance backend switch"): routing, sort,
+ *    both expert GEMMs and the combine as phases of one launch, the down
+ *    tiles starting as soon as their token block's gate|up tiles are done,
+ *    the token rows read straight from x (no gathered copy).  Same results,
+ *    bit for bit, as the multi-launch path.  Eligible for bf16 x and bf16
+ *    weights, T >= 2048, hidden / 128 even, num_experts <= 288, a whole layer
+ *    (not a shard); otherwise moe_forward takes the multi-launch path.  Its
+ *    grid-wide barriers need every CTA of the launch resident at once (one
+ *    CTA pair per two SMs): kernels that occupy SMs on other streams for
+ *    seconds make its bounded waits expire (MOE_ERR_DEVICE_TIMEOUT through
+ *    moe_get_device_error) rather than hang.
+ *  MOE_PATH_AUTO (default): the fused path where it is eligible and measured
+ *    faster, else the multi-launch path. */
+#define MOE_PATH_AUTO 0
+#define MOE_PATH_MULTI 1
+#define MOE_PATH_FUSED 2
+
+/* Selects the path of the following forwards (MOE_ERR_INVALID_ARG for an
+ * unknown path).  Host-only. */
+int moe_set_path(moe_layer_t* layer, int path);
+
+/* The path a forward of T tokens takes with the layer's current setting:
+ * MOE_PATH_MULTI or MOE_PATH_FUSED (0 for a NULL layer or T <= 0). */
+int moe_forward_path(const moe_layer_t* layer, int T);
+
+/* Self-check of the fused path's bounded waits (fault detection without a
+ * fault): one fused forward of x [T, H] into out (T, the layer and the
+ * workspace as for moe_forward on the fused path) in which no down-projection
+ * tile can ever become ready, and every bounded wait of the kernel (the
+ * readiness counters, the grid barriers, the mbarriers) gives up after
+ * limit_us microseconds (1 .. 10,000,000).  The down tiles' waits expire,
+ * every role of the kernel winds down and frees its tensor memory, and the
+ * timeout bit is set in the layer's device status word.  Synchronises the
+ * device, reads and clears the word into *device_status (if not NULL).
+ * Returns MOE_OK when exactly the timeout bit (1) was reported,
+ * MOE_ERR_UNSUPPORTED when the fused path does not apply to this layer and T,
+ * MOE_ERR_INVALID_ARG / MOE_ERR_WORKSPACE / MOE_ERR_NOT_LOADED as
+ * moe_forward, MOE_ERR_CUDA otherwise.  out's contents are undefined
+ * afterwards. */
+int moe_check_fused_timeout(moe_layer_t* layer, const void* x, int T, void* out,
+                            void* workspace, size_t ws_bytes, int limit_us,
+                            int* device_status);
+
 /* Workspace bytes for moe_forward_host: moe_workspace_size plus device
  * staging for x and out. */
 int moe_workspace_size_host(const moe_layer_t* layer, int T, size_t* bytes);
@@ -228,7 +276,8 @@ void moe_destroy(moe_layer_t* layer);
 /* Stages of one forward, in launch order, for the stage timers below:
  * 0 router logits, 1 top-k and gate weights, 2 counting sort (3 kernels),
  * 3 gather of the input rows, 4 grouped gate|up GEMM + SwiGLU,
- * 5 grouped down GEMM x gate weight, 6 combine. */
+ * 5 grouped down GEMM x gate weight, 6 combine.  A forward on the fused path
+ * is one kernel: its whole time is recorded as stage 0, the others as 0. */
 #define MOE_NUM_STAGES 7
 
 /* Kernel launches one moe_forward makes for T tokens (0 for T = 0). */

@@ -26,6 +26,9 @@ MOE_ERR_NOT_LOADED = 6
 MOE_F32 = 0
 MOE_BF16 = 1
 MOE_FP8_E4M3 = 2
+MOE_PATH_AUTO = 0
+MOE_PATH_MULTI = 1
+MOE_PATH_FUSED = 2
 
 # every symbol include/moe.h declares
 EXPORTS = (
@@ -36,7 +39,8 @@ EXPORTS = (
     "moe_check_wait_timeout", "moe_load_weights_fp8", "moe_decode_e4m3",
     "moe_dense_config_check", "moe_dense_create", "moe_dense_load_weights",
     "moe_dense_workspace_size", "moe_dense_forward", "moe_dense_get_device_error",
-    "moe_dense_destroy", "moe_create_shard",
+    "moe_dense_destroy", "moe_create_shard", "moe_set_path", "moe_forward_path",
+    "moe_check_fused_timeout",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -131,6 +135,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_dense_destroy.restype = None
     lib.moe_get_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), i,
                                         ctypes.POINTER(i)]
+    lib.moe_set_path.argtypes = [vp, i]
+    lib.moe_check_fused_timeout.argtypes = [vp, vp, i, vp, vp, sz, i, ctypes.POINTER(i)]
+    lib.moe_forward_path.argtypes = [vp, i]
     for name in EXPORTS:
         if name not in ("moe_status_string", "moe_destroy", "moe_dense_destroy"):
             getattr(lib, name).restype = ctypes.c_int
@@ -276,6 +283,24 @@ def moe_kernel_launches(handle, T: int) -> int:
     return load_library().moe_kernel_launches(ctypes.c_void_p(handle), T)
 
 
+def moe_set_path(handle, path: int) -> None:
+    """MOE_PATH_AUTO, MOE_PATH_MULTI or MOE_PATH_FUSED (see include/moe.h)."""
+    _check(load_library().moe_set_path(ctypes.c_void_p(handle), path), "moe_set_path")
+
+
+def moe_forward_path(handle, T: int) -> int:
+    return load_library().moe_forward_path(ctypes.c_void_p(handle), T)
+
+
+def moe_check_fused_timeout(handle, x, T, out, workspace, ws_bytes, limit_us):
+    """-> (status, device status word); see include/moe.h."""
+    word = ctypes.c_int(-1)
+    r = load_library().moe_check_fused_timeout(ctypes.c_void_p(handle), _ptr(x), T, _ptr(out),
+                                               _ptr(workspace), ws_bytes, limit_us,
+                                               ctypes.byref(word))
+    return r, word.value
+
+
 def moe_set_stage_timing(handle, capacity: int) -> None:
     _check(load_library().moe_set_stage_timing(ctypes.c_void_p(handle), capacity),
            "moe_set_stage_timing")
@@ -325,6 +350,12 @@ class MoeLayer:
     @property
     def act_dtype(self) -> torch.dtype:
         return _TORCH_DT[self.cfg.act_dtype]
+
+    def set_path(self, path: int) -> None:
+        moe_set_path(self.handle, path)
+
+    def forward_path(self, T: int) -> int:
+        return moe_forward_path(self.handle, T)
 
     def _need(self, t: torch.Tensor, name: str, dtype: torch.dtype, shape):
         if t.device != self.device or t.dtype != dtype or not t.is_contiguous() \

@@ -1,0 +1,57 @@
+// Device code of the weighted combine (K7), shared by the combine kernel
+// (combine.cu) and the fused persistent MoE kernel (fused_moe.cu):
+// out[t] = sum_j y[pos(t, j)] + y[shared row t], summed in fp32 in the fixed
+// order j = 0..k-1 then the shared row, rounded once to the output dtype.
+#pragma once
+
+#include <cuda_bf16.h>
+
+namespace moe {
+namespace combine {
+
+__device__ __forceinline__ void add8(float (&acc)[8], const __nv_bfloat16* p) {
+  const uint4 q = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
+  }
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
+  uint4 q;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = q;
+}
+
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// Token t's output row, by all threads of the block (threadIdx.x / blockDim.x
+// strides over the row's 8-element vectors); rows_s: k + 1 ints of shared
+// memory.  Ends with a __syncthreads, so rows_s may be reused at once.
+template <typename TO>
+__device__ __forceinline__ void combine_token(int t, const __nv_bfloat16* __restrict__ y,
+                                              const int* __restrict__ pos, int T, int k, int H,
+                                              int with_shared, TO* __restrict__ out, int* rows_s) {
+  if (threadIdx.x < k) rows_s[threadIdx.x] = pos[static_cast<size_t>(t) * k + threadIdx.x];
+  if (threadIdx.x == 0) rows_s[k] = with_shared ? T * k + t : -1;
+  __syncthreads();
+  const int nvec = H / 8;
+  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j <= k; ++j)  // (-1: another shard's expert, or no shared expert here)
+      if (rows_s[j] >= 0) add8(acc, y + static_cast<size_t>(rows_s[j]) * H + v * 8);
+    store8(out + static_cast<size_t>(t) * H + v * 8, acc);
+  }
+  __syncthreads();
+}
+
+}  // namespace combine
+}  // namespace moe

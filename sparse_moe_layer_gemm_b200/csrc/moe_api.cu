@@ -45,6 +45,9 @@ struct moe_layer {
   CUtensorMap tm_dn_pw;  // A operand of K6 on CTA pairs, wide stages (128 rows x 2 K blocks)
   CUtensorMap tm_dn_pn;  //   narrow stages (128 rows x 3 K blocks)
   CUtensorMap tm_router;  // A operand of the tensor-core router (box 64 x 128)
+  CUtensorMap tm_rt_pw;   // the same for the fused kernel's pair MMAs: 128 rows x 2 K blocks
+  CUtensorMap tm_rt_pn;   //   and x 3 K blocks
+  int path;               // MOE_PATH_AUTO / MULTI / FUSED
   // stage timers: capacity x (MOE_NUM_STAGES + 1) events, filled in order
   std::vector<cudaEvent_t> events;
   int timing_capacity;
@@ -154,7 +157,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
   size_t partial, topk_idx, topk_w, masks, chunk_cnt, chunk_base, counts, row_start, tiles_gu,
-      tiles_dn, perm, pos, w_perm, x_perm, h, y, local_idx, total;
+      tiles_dn, perm, pos, w_perm, x_perm, h, y, local_idx, sync, total;
   int ksplit, nch, rows_routed, rows_xperm, rows_all;
 };
 
@@ -206,12 +209,125 @@ WsLayout ws_layout(const moe_layer* L, int T) {
   // expert shard: the selection in local expert ids (-1: another shard's)
   const bool shard = L->E_loc != E || L->first != 0;
   w.local_idx = shard ? take(static_cast<size_t>(T) * k * sizeof(int)) : 0;
+  // fused path: the grid barrier's counter and the token blocks' readiness
+  w.sync = take(moe::fused_sync_words(T, k, G) * sizeof(unsigned int));
   w.total = off;
   return w;
 }
 
 // The router part of both weight loaders (defined below).
 int load_router(moe_layer* L, const float* router_w, const float* router_bias, cudaStream_t st);
+
+// The fused persistent forward's conditions (see MOE_PATH_FUSED in moe.h).
+bool fused_eligible(const moe_layer* L, int T) {
+  const moe_config_t& c = L->cfg;
+  return c.act_dtype == MOE_BF16 && !L->fp8 && T >= moe::kPairMinTokens &&
+         (c.hidden / moe::kBM) % 2 == 0 && c.num_experts <= moe::kFusedMaxExperts &&
+         L->E_loc == c.num_experts && L->first == 0 && L->with_shared != 0;
+}
+
+// The optional routing outputs of a forward, copied from the workspace
+// (a shard: counts and offsets of its own El experts).
+int copy_routing(const moe_routing_t* routing, int T, int k, int El, const int* topk_idx,
+                 const float* topk_w, const int* counts, const int* row_start, const int* perm,
+                 cudaStream_t st) {
+  if (routing == nullptr) return MOE_OK;
+  const size_t tk = static_cast<size_t>(T) * k;
+  if (routing->topk_idx)
+    MOE_CUDA(cudaMemcpyAsync(routing->topk_idx, topk_idx, tk * 4, cudaMemcpyDeviceToDevice, st));
+  if (routing->topk_w)
+    MOE_CUDA(cudaMemcpyAsync(routing->topk_w, topk_w, tk * 4, cudaMemcpyDeviceToDevice, st));
+  if (routing->counts)
+    MOE_CUDA(cudaMemcpyAsync(routing->counts, counts, El * 4, cudaMemcpyDeviceToDevice, st));
+  if (routing->offsets)
+    MOE_CUDA(
+        cudaMemcpyAsync(routing->offsets, row_start, (El + 1) * 4, cudaMemcpyDeviceToDevice, st));
+  if (routing->perm)
+    MOE_CUDA(cudaMemcpyAsync(routing->perm, perm, tk * 4, cudaMemcpyDeviceToDevice, st));
+  return MOE_OK;
+}
+
+// The fused persistent forward (fused_moe.cu) on a checked workspace:
+// zeroes the barrier and readiness counters, encodes the per-call tensor maps
+// and launches the one kernel.  wait_ns / ready_extra: see FusedLaunch.
+int launch_fused_forward(moe_layer* L, const void* x, int T, void* out, uint8_t* ws,
+                         const WsLayout& w, cudaStream_t st, const moe_routing_t* routing,
+                         uint64_t wait_ns, unsigned int ready_extra) {
+  const moe_config_t& c = L->cfg;
+  const int H = c.hidden, E = c.num_experts, k = c.top_k, Ip = L->I_pad, G = E + 1;
+  float* partial = reinterpret_cast<float*>(ws + w.partial);
+  int* topk_idx = reinterpret_cast<int*>(ws + w.topk_idx);
+  float* topk_w = reinterpret_cast<float*>(ws + w.topk_w);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(ws + w.masks);
+  int* chunk_cnt = reinterpret_cast<int*>(ws + w.chunk_cnt);
+  int* chunk_base = reinterpret_cast<int*>(ws + w.chunk_base);
+  int* counts = reinterpret_cast<int*>(ws + w.counts);
+  int* row_start = reinterpret_cast<int*>(ws + w.row_start);
+  int* tiles_gu = reinterpret_cast<int*>(ws + w.tiles_gu);
+  int* tiles_dn = reinterpret_cast<int*>(ws + w.tiles_dn);
+  int* perm = reinterpret_cast<int*>(ws + w.perm);
+  int* pos = reinterpret_cast<int*>(ws + w.pos);
+  float* w_perm = reinterpret_cast<float*>(ws + w.w_perm);
+  __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + w.h);
+  __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(ws + w.y);
+  moe::FusedLaunch f{};
+  f.rt_w = L->tm_rt_pw;
+  f.rt_n = L->tm_rt_pn;
+  f.gu_w = L->tm_gu_pw;
+  f.gu_n = L->tm_gu_pn;
+  f.dn_w = L->tm_dn_pw;
+  f.dn_n = L->tm_dn_pn;
+  if (!encode_bf16_kblocks(&f.x_w, x, T, H, moe::kBN, 2) ||
+      !encode_bf16_kblocks(&f.x_n, x, T, H, moe::kBBoxRows, 3) ||
+      !encode_bf16_kblocks(&f.h_w, hbuf, w.rows_all, Ip, moe::kBN, 2) ||
+      !encode_bf16_kblocks(&f.h_n, hbuf, w.rows_all, Ip, moe::kBBoxRows, 3) ||
+      !encode_bf16_store(&f.st_h, hbuf, w.rows_all, Ip) ||
+      !encode_bf16_store(&f.st_y, ybuf, w.rows_all, H))
+    return MOE_ERR_CUDA;
+  f.x = static_cast<const __nv_bfloat16*>(x);
+  f.out = static_cast<__nv_bfloat16*>(out);
+  f.T = T;
+  f.H = H;
+  f.E = E;
+  f.k = k;
+  f.I_pad = Ip;
+  f.bias = L->has_bias ? L->router_b : nullptr;
+  f.router_t = L->router_t;
+  f.band = moe::router_refine_band(H);
+  f.norm = c.norm_expert_weight != 0;
+  f.scale = c.routed_scaling_factor;
+  f.rt_mtiles = (L->E_pad + 2 * moe::kBM - 1) / (2 * moe::kBM);
+  f.logits_out = routing != nullptr ? routing->logits : nullptr;
+  f.partial = partial;
+  f.topk_idx = topk_idx;
+  f.topk_w = topk_w;
+  f.masks = masks;
+  f.chunk_cnt = chunk_cnt;
+  f.chunk_base = chunk_base;
+  f.counts = counts;
+  f.row_start = row_start;
+  f.tiles_gu = tiles_gu;
+  f.tiles_dn = tiles_dn;
+  f.perm = perm;
+  f.pos = pos;
+  f.w_perm = w_perm;
+  f.h = hbuf;
+  f.y = ybuf;
+  f.sync = reinterpret_cast<unsigned int*>(ws + w.sync);
+  f.limit = c.swiglu_limit;
+  f.limit_shared = c.swiglu_limit_shared;
+  f.status = L->status;
+  f.wait_ns = wait_ns;
+  f.ready_extra = ready_extra;
+  MOE_CUDA(cudaMemsetAsync(f.sync, 0, moe::fused_sync_words(T, k, G) * sizeof(unsigned int), st));
+  MOE_CUDA(moe::launch_fused(f, st));
+  return MOE_OK;
+}
+
+int forward_path(const moe_layer* L, int T) {
+  if (L->path == MOE_PATH_FUSED && fused_eligible(L, T)) return MOE_PATH_FUSED;
+  return MOE_PATH_MULTI;
+}
 
 }  // namespace
 
@@ -289,6 +405,7 @@ int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count
   if (moe::gemm_configure_device() != cudaSuccess ||
       moe::gemm_fp8_configure_device() != cudaSuccess ||
       moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
+      moe::fused_configure_device(L->num_sms) != cudaSuccess ||
       moe::topk_configure_device() != cudaSuccess ||
       moe::gather_configure_device() != cudaSuccess ||
       cudaMalloc(&L->w_gu, gu_bytes) != cudaSuccess ||
@@ -312,7 +429,9 @@ int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count
                  encode_bf16_2d(&L->tm_dn, L->w_dn, (El + 1) * H, Ip, moe::kBM) &&
                  encode_bf16_kblocks(&L->tm_dn_pw, L->w_dn, (El + 1) * H, Ip, moe::kBM, 2) &&
                  encode_bf16_kblocks(&L->tm_dn_pn, L->w_dn, (El + 1) * H, Ip, moe::kBM, 3));
-  if (!maps_ok || !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM)) {
+  if (!maps_ok || !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM) ||
+      !encode_bf16_kblocks(&L->tm_rt_pw, L->router_tc, L->E_pad, 3 * H, moe::kBM, 2) ||
+      !encode_bf16_kblocks(&L->tm_rt_pn, L->router_tc, L->E_pad, 3 * H, moe::kBM, 3)) {
     moe_destroy(L);
     return MOE_ERR_CUDA;
   }
@@ -493,6 +612,20 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + w.h);
   __nv_bfloat16* ybuf = reinterpret_cast<__nv_bfloat16*>(ws + w.y);
 
+  cudaEvent_t* ev = nullptr;
+  if (L->timing_capacity > 0 && L->timing_recorded < L->timing_capacity)
+    ev = &L->events[static_cast<size_t>(L->timing_recorded++) * (MOE_NUM_STAGES + 1)];
+  auto mark = [&](int i) { return ev == nullptr ? cudaSuccess : cudaEventRecord(ev[i], st); };
+
+  if (forward_path(L, T) == MOE_PATH_FUSED) {
+    // one persistent kernel (fused_moe.cu); the whole forward is stage 0
+    MOE_CUDA(mark(0));
+    const int r = launch_fused_forward(L, x, T, out, ws, w, st, routing, 0, 0);
+    if (r != MOE_OK) return r;
+    for (int i = 1; i <= MOE_NUM_STAGES; ++i) MOE_CUDA(mark(i));
+    return copy_routing(routing, T, k, El, topk_idx, topk_w, counts, row_start, perm, st);
+  }
+
   // expert-GEMM tiles: on one SM, 128 tokens x gate|up one 128-feature block
   // (down one or two); on CTA pairs (large T), 256 tokens x gate|up 128
   // features (down 256)
@@ -575,11 +708,6 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
     if (!xb) gu8.bsh = gu8.b;
     dn8.bsh = dn8.b;
   }
-
-  cudaEvent_t* ev = nullptr;
-  if (L->timing_capacity > 0 && L->timing_recorded < L->timing_capacity)
-    ev = &L->events[static_cast<size_t>(L->timing_recorded++) * (MOE_NUM_STAGES + 1)];
-  auto mark = [&](int i) { return ev == nullptr ? cudaSuccess : cudaEventRecord(ev[i], st); };
 
   MOE_CUDA(mark(0));
   int ksplit = w.ksplit;
@@ -674,22 +802,7 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, L->with_shared != 0, out, st));
   MOE_CUDA(mark(7));
 
-  if (routing != nullptr) {
-    const size_t tk = static_cast<size_t>(T) * k;
-    if (routing->topk_idx)
-      MOE_CUDA(cudaMemcpyAsync(routing->topk_idx, topk_idx, tk * 4, cudaMemcpyDeviceToDevice, st));
-    if (routing->topk_w)
-      MOE_CUDA(cudaMemcpyAsync(routing->topk_w, topk_w, tk * 4, cudaMemcpyDeviceToDevice, st));
-    // (a shard: counts and offsets of its own El experts)
-    if (routing->counts)
-      MOE_CUDA(cudaMemcpyAsync(routing->counts, counts, El * 4, cudaMemcpyDeviceToDevice, st));
-    if (routing->offsets)
-      MOE_CUDA(
-          cudaMemcpyAsync(routing->offsets, row_start, (El + 1) * 4, cudaMemcpyDeviceToDevice, st));
-    if (routing->perm)
-      MOE_CUDA(cudaMemcpyAsync(routing->perm, perm, tk * 4, cudaMemcpyDeviceToDevice, st));
-  }
-  return MOE_OK;
+  return copy_routing(routing, T, k, El, topk_idx, topk_w, counts, row_start, perm, st);
 }
 
 int moe_forward_host(moe_layer_t* L, const void* x_host, int T, void* out_host, void* workspace,
@@ -731,8 +844,46 @@ int moe_get_device_error(moe_layer_t* L, int* device_err) {
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE_TIMEOUT;
 }
 
+int moe_check_fused_timeout(moe_layer_t* L, const void* x, int T, void* out, void* workspace,
+                            size_t ws_bytes, int limit_us, int* device_status) {
+  if (L == nullptr || x == nullptr || out == nullptr || x == out || limit_us <= 0 ||
+      limit_us > 10000000)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  if (T <= 0 || T > kMaxTokens || !fused_eligible(L, T)) return MOE_ERR_UNSUPPORTED;
+  const WsLayout w = ws_layout(L, T);
+  if (workspace == nullptr || ws_bytes < w.total || !aligned(workspace, 256))
+    return MOE_ERR_WORKSPACE;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  MOE_CUDA(cudaDeviceSynchronize());
+  MOE_CUDA(cudaMemset(L->status, 0, sizeof(int)));
+  const int r = launch_fused_forward(L, x, T, out, static_cast<uint8_t*>(workspace), w, nullptr,
+                                     nullptr, static_cast<uint64_t>(limit_us) * 1000ull, 1u);
+  if (r != MOE_OK) return r;
+  int v = 0;
+  MOE_CUDA(cudaDeviceSynchronize());
+  MOE_CUDA(cudaMemcpy(&v, L->status, sizeof(int), cudaMemcpyDeviceToHost));
+  MOE_CUDA(cudaMemset(L->status, 0, sizeof(int)));
+  if (device_status != nullptr) *device_status = v;
+  return v == 1 ? MOE_OK : MOE_ERR_CUDA;  // exactly the timeout bit
+}
+
+int moe_set_path(moe_layer_t* L, int path) {
+  if (L == nullptr || path < MOE_PATH_AUTO || path > MOE_PATH_FUSED) return MOE_ERR_INVALID_ARG;
+  L->path = path;
+  return MOE_OK;
+}
+
+int moe_forward_path(const moe_layer_t* L, int T) {
+  if (L == nullptr || T <= 0) return 0;
+  return forward_path(L, T);
+}
+
 int moe_kernel_launches(const moe_layer_t* L, int T) {
   if (L == nullptr || T <= 0) return 0;
+  if (forward_path(L, T) == MOE_PATH_FUSED) return 1;
   // router, top-k, counting sort (one kernel up to kSortChunk tokens, else
   // three), gather, gate|up GEMM, down GEMM, combine; a shard also maps the
   // selection to its own expert ids

@@ -175,6 +175,51 @@ cudaError_t launch_pack_gate_up_scales(const float* s, int groups, int I, int I_
 cudaError_t launch_decode_e4m3(const uint8_t* codes, size_t n, __nv_bfloat16* out,
                                cudaStream_t st);
 
+// The fused persistent forward (fused_moe.cu): bf16 x and weights, from
+// kPairMinTokens tokens, H / 128 even, E <= kFusedMaxExperts (the top-k's
+// experts per lane, kFusedMPL, is fixed).
+constexpr int kFusedMaxExperts = 288;
+constexpr int kFusedMPL = 9;
+
+struct FusedLaunch {
+  // tensor maps: weights of wide / narrow stages (router: encode_bf16_kblocks
+  // of the packed three-term split, 128 rows; gate|up: encode_bf16_gate_up_pair;
+  // down: encode_bf16_kblocks, 128 rows), token rows of x and h (128 rows x 2
+  // and 32 rows x 3 K blocks), and the TMA stores of h and y
+  CUtensorMap rt_w, rt_n, gu_w, gu_n, dn_w, dn_n, x_w, x_n, h_w, h_n, st_h, st_y;
+  const __nv_bfloat16* x;
+  __nv_bfloat16* out;
+  int T, H, E, k, I_pad;
+  const float* bias;      // [E] or nullptr
+  const float* router_t;  // [E, H]
+  float band;
+  int norm;
+  float scale;
+  int rt_mtiles;          // ceil(E_pad / 256)
+  float* logits_out;      // optional [T, E]
+  float* partial;         // [3, T, E]
+  int *topk_idx;
+  float* topk_w;
+  uint32_t* masks;
+  int *chunk_cnt, *chunk_base, *counts, *row_start, *tiles_gu, *tiles_dn, *perm, *pos;
+  float* w_perm;
+  __nv_bfloat16 *h, *y;
+  unsigned int* sync;     // zeroed before the launch: [0] grid barrier, [1 + b] token block b
+  float limit, limit_shared;
+  int* status;
+  uint64_t wait_ns;       // limit of every bounded wait (0: the default, 2 s)
+  unsigned int ready_extra;  // self-check only: unreachable readiness target (0 in a forward)
+};
+
+// Readiness counters of the fused forward for T tokens and G groups: one per
+// 256-token block of every group's rows, plus the grid barrier's.
+inline size_t fused_sync_words(int T, int k, int G) {
+  return 1 + static_cast<size_t>(T) * (k + 1) / 256 + static_cast<size_t>(G) + 1;
+}
+
+cudaError_t fused_configure_device(int num_sms);
+cudaError_t launch_fused(const FusedLaunch& f, cudaStream_t st);
+
 // Launches `kernel` on `st` with programmatic stream serialization, so it may
 // start (up to its pdl_wait) while the previous kernel of the stream ends.
 template <typename... KArgs, typename... Args>

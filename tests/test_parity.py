@@ -387,3 +387,40 @@ def test_full_size_fp8_decode():
     print(wl.name, rep)
     layer.close()
     assert rep.ok(), rep
+
+
+@pytest.mark.timeout(900)
+@pytest.mark.parametrize("name", ["prefill", "zipf_prefill"])
+def test_full_size_fused(step35, name):
+    """The fused persistent forward (one launch) at full size: bit-identical
+    to the multi-launch path, and against the oracle on the sampled rows."""
+    _, inp, layer = step35
+    wl = WORKLOADS[name]
+    rw, rb = draw_router(wl, "cuda")
+    layer.load_weights(inp["router_w"], rb, inp["w_gate"], inp["w_up"], inp["w_down"],
+                       inp["sh_gate"], inp["sh_up"], inp["sh_down"])
+    x = draw_x(wl, "cuda")
+    try:
+        layer.set_path(B.MOE_PATH_MULTI)
+        out_m, rt_m = layer.forward(x, routing=True)
+        out_m = out_m.clone()
+        rt_m = {k: v.clone() for k, v in rt_m.items()}
+        layer.set_path(B.MOE_PATH_FUSED)
+        assert layer.forward_path(wl.T) == B.MOE_PATH_FUSED
+        out_f, rt_f = layer.forward(x, routing=True)
+        torch.cuda.synchronize()
+        assert layer.device_error() == 0
+    finally:
+        layer.set_path(B.MOE_PATH_AUTO)
+    for n in ("topk_idx", "topk_w", "counts", "offsets", "perm"):
+        assert torch.equal(rt_f[n], rt_m[n]), n
+    assert torch.equal(out_f, out_m)
+    host = dict(x=host_f32(x), router_w=host_f32(inp["router_w"]), router_bias=host_f32(rb))
+    experts = dict(w_gate=HostExpertView(inp["w_gate"]), w_up=HostExpertView(inp["w_up"]),
+                   w_down=HostExpertView(inp["w_down"]), sh_gate=host_f32(inp["sh_gate"]),
+                   sh_up=host_f32(inp["sh_up"]), sh_down=host_f32(inp["sh_down"]))
+    rt_np = _routing_np(rt_f)
+    rep = compare(host, wl, host_f32(out_f), rt_np, rows=_check_rows(wl, rt_np, n_rows=8),
+                  experts=experts)
+    print(wl.name, "fused", rep)
+    assert rep.ok(), rep
