@@ -44,6 +44,10 @@ def _args():
     ap.add_argument("--secondary",
                     default="prefill,zipf_prefill,clamp_ragged,tiny,decode_fp8,dense_decode,dense_prefill",
                     help="comma-separated further workloads measured in the same run")
+    ap.add_argument("--parallel", choices=["auto", "ep", "replicas"], default="auto",
+                    help="N > 1: expert parallelism (ep, the default: each rank holds 1/N of "
+                         "the experts, all ranks route the same tokens, an NCCL all-reduce "
+                         "sums the partial outputs) or independent replicas")
     ap.add_argument("--path", choices=["auto", "multi", "fused"], default="auto",
                     help="moe_forward's execution path (auto: the library's choice)")
     ap.add_argument("--detail", default="",
@@ -626,6 +630,171 @@ def run_ours(a):
     return 0
 
 
+def ep_plan(num_experts: int, world: int, rank: int) -> dict:
+    """This rank's part of the expert-parallel layer: its contiguous shard of
+    the routed experts and whether it holds the shared expert."""
+    from sparse_moe_layer_gemm_b200.expert_parallel import holds_shared, shard_range
+    first, count = shard_range(num_experts, world, rank)
+    return {"first": first, "count": count, "with_shared": holds_shared(rank)}
+
+
+def ep_config(wl, world: int) -> dict:
+    cfg = _config(wl, world)
+    cfg["parallelism"] = f"ep{world}: experts sharded, all-reduce of the partial outputs"
+    return cfg
+
+
+def run_ep(a):
+    """N > 1, expert parallelism: every rank routes the same T tokens over all
+    experts, computes the pairs of its own shard (rank 0 also the shared
+    expert) and an NCCL all-reduce sums the bf16 partial outputs; each rank
+    draws and loads only its shard's expert tensors.  One step = the forward
+    plus the all-reduce; the job processes T tokens per step (strong scaling:
+    the work per step is fixed, the experts per GPU shrink with N)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from sparse_moe_layer_gemm_b200 import binding as B
+    from sparse_moe_layer_gemm_b200.replicas import max_over_ranks
+    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS, draw_router, draw_x, \
+        make_shard_inputs
+
+    world = int(os.environ["WORLD_SIZE"])
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    B.load_library()
+    peaks = _peaks()
+    stream = torch.cuda.Stream(device=dev)
+    path = {"auto": B.MOE_PATH_AUTO, "multi": B.MOE_PATH_MULTI, "fused": B.MOE_PATH_FUSED}[a.path]
+
+    def step(layer, x, out):
+        layer.forward(x, out)
+        dist.all_reduce(out, op=dist.ReduceOp.SUM)
+
+    def timed(layer, x, out, steps, warmup):
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                step(layer, x, out)
+            torch.cuda.synchronize()
+            dist.barrier()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                step(layer, x, out)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        dist.barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+
+    def measure(wl, layer, inp):
+        x = inp["x"]
+        out = torch.empty_like(x)
+        _, rt = layer.forward(x, routing=True)
+        torch.cuda.synchronize()
+        touched_local = int((rt["counts"][:plan["count"]] > 0).sum())  # the shard's experts
+        t = torch.tensor([touched_local], device=dev)
+        dist.all_reduce(t)                     # routed experts touched by the whole job
+        ms = timed(layer, x, out, a.steps, a.warmup)
+        B.moe_set_stage_timing(layer.handle, a.steps)
+        with torch.cuda.stream(stream):
+            for _ in range(a.steps):
+                layer.forward(x, out)
+        torch.cuda.synchronize()
+        tot, n = B.moe_get_stage_times(layer.handle)
+        B.moe_set_stage_timing(layer.handle, 0)
+        stages = {k: v / max(n, 1) for k, v in tot.items()}
+        if layer.device_error() != 0:
+            raise RuntimeError(f"device status word ({wl.name})")
+        fused = B.moe_forward_path(layer.handle, wl.T) == B.MOE_PATH_FUSED
+        # the dominant kernel on this rank (its own touched experts); the
+        # layer against the whole job's HBM bandwidth (N GPUs)
+        kr, _ = _kernel_roofline(wl, touched_local, stages, peaks, ms, a.steps, fused)
+        job = dict(peaks, hbm=peaks["hbm"] * world, tc_burst=peaks["tc_burst"] * world,
+                   tc_sustained=peaks["tc_sustained"] * world)
+        _, lr = _kernel_roofline(wl, int(t.item()), stages, job, ms, a.steps, fused)
+        return ms, stages, kr, lr, x, out
+
+    wl = WORKLOADS[a.workload]
+    plan = ep_plan(wl.num_experts, world, rank)
+    shard = (plan["first"], plan["count"], 1 if plan["with_shared"] else 0)
+    inp = make_shard_inputs(wl, plan["first"], plan["count"], plan["with_shared"], dev)
+    layer = B.MoeLayer.from_workload(wl, shard)
+    layer.set_path(path)
+    layer.load_shard_weights(inp["router_w"], inp["router_bias"], inp["w_gate"], inp["w_up"],
+                             inp["w_down"], inp.get("sh_gate"), inp.get("sh_up"),
+                             inp.get("sh_down"))
+    sampler = ClockSampler(str(local))
+    sampler.start()
+    ms, stages, kr, lr, x, out = measure(wl, layer, inp)
+    clocks = sampler.stop()
+    value = wl.T / (ms * 1e-3)
+
+    e2e = None
+    if not a.no_e2e:
+        xh = x.cpu().pin_memory()
+        oh = torch.empty_like(xh).pin_memory()
+        xd = torch.empty_like(x)
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, a.warmup)):
+                xd.copy_(xh, non_blocking=True)
+                step(layer, xd, out)
+                oh.copy_(out, non_blocking=True)
+            torch.cuda.synchronize()
+            dist.barrier()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(a.steps):
+                xd.copy_(xh, non_blocking=True)
+                step(layer, xd, out)
+                oh.copy_(out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        et = max_over_ranks(e0.elapsed_time(e1) / a.steps, dev)
+        io = wl.T * wl.hidden * (2 if wl.act_dtype == "bf16" else 4)
+        e2e = {"value": wl.T / (et * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": world * io, "d2h_bytes_per_step": world * io,
+               "path": "every rank: pinned x in, forward + all-reduce, out back to the host"}
+
+    secondary = []
+    for name2 in [n for n in (a.secondary or "").split(",") if n and n != "none"]:
+        if name2 not in ("prefill", "zipf_prefill") or name2 == a.workload:
+            continue  # the same experts, another batch and router bias
+        wl2 = WORKLOADS[name2]
+        _, rb2 = draw_router(wl2, dev)
+        layer.load_shard_weights(inp["router_w"], rb2, inp["w_gate"], inp["w_up"], inp["w_down"],
+                                 inp.get("sh_gate"), inp.get("sh_up"), inp.get("sh_down"))
+        inp2 = dict(inp, x=draw_x(wl2, dev))
+        ms2, st2, kr2, lr2, _, _ = measure(wl2, layer, inp2)
+        secondary.append({"workload": wl2.name, "T": wl2.T, "value": wl2.T / (ms2 * 1e-3),
+                          "unit": "tokens/s", "ms_per_step": ms2, "roofline": kr2,
+                          "layer_roofline": lr2, "stage_ms": st2})
+        del inp2
+    launches = B.moe_kernel_launches(layer.handle, wl.T) * a.steps
+    if rank == 0:
+        full = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": ep_config(wl, world), "roofline": kr, "layer_roofline": lr,
+            "stage_ms": stages, "routing": {}, "cpu_baseline": None, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks, "secondary": secondary,
+        }
+        if a.detail:
+            with open(a.detail, "w") as f:
+                json.dump(full, f, indent=1)
+        print(json.dumps(_compact_line(full), separators=(",", ":")), flush=True)
+    layer.close()
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 def _compact_line(full):
     """The one printed JSON line, kept under 1500 characters: the contract's
     keys with short values, the headline's layer roofline fraction, then the
@@ -697,6 +866,8 @@ def main():
     a = _args()
     if a.impl == "reference":
         return run_reference(a)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and a.parallel != "replicas":
+        return run_ep(a)
     return run_ours(a)
 
 

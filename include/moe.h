@@ -155,6 +155,20 @@ int moe_load_weights(moe_layer_t* layer, const float* router_w, const float* rou
                      const void* sh_gate, const void* sh_up, const void* sh_down,
                      void* stream);
 
+/* moe_load_weights for an expert shard (moe_create_shard) whose caller holds
+ * only the shard's own experts: w_gate, w_up [expert_count, H, I] and w_down
+ * [expert_count, I, H] start at the shard's first expert (moe_load_weights
+ * takes the whole [E, ...] tensors and skips to it).  sh_gate / sh_up /
+ * sh_down may be NULL when the shard holds no shared expert.  router_w and
+ * router_bias are the whole layer's (every shard routes over all experts).
+ * Lets each rank of an expert-parallel layer load 1/N of the expert bytes.
+ * bf16 / fp32 weights (a layer created with MOE_FP8_E4M3 returns
+ * MOE_ERR_INVALID_ARG). */
+int moe_load_shard_weights(moe_layer_t* layer, const float* router_w, const float* router_bias,
+                           const void* w_gate, const void* w_up, const void* w_down,
+                           const void* sh_gate, const void* sh_up, const void* sh_down,
+                           void* stream);
+
 /* FP8 expert weights (layer created with weight_dtype MOE_FP8_E4M3): the
  * codes in the layouts of moe_load_weights, one uint8 E4M3FN code per weight
  * (w_gate / w_up [E, H, I], w_down [E, I, H], sh_gate / sh_up [H, I],

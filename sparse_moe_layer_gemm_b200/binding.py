@@ -40,7 +40,7 @@ EXPORTS = (
     "moe_dense_config_check", "moe_dense_create", "moe_dense_load_weights",
     "moe_dense_workspace_size", "moe_dense_forward", "moe_dense_get_device_error",
     "moe_dense_destroy", "moe_create_shard", "moe_set_path", "moe_forward_path",
-    "moe_check_fused_timeout",
+    "moe_check_fused_timeout", "moe_load_shard_weights",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -109,6 +109,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_create.argtypes = [ctypes.POINTER(moe_config_t), ctypes.POINTER(vp)]
     lib.moe_create_shard.argtypes = [ctypes.POINTER(moe_config_t), i, i, i, ctypes.POINTER(vp)]
     lib.moe_load_weights.argtypes = [vp] * 9 + [vp]
+    lib.moe_load_shard_weights.argtypes = [vp] * 9 + [vp]
     lib.moe_workspace_size.argtypes = [vp, i, ctypes.POINTER(sz)]
     lib.moe_workspace_size_host.argtypes = [vp, i, ctypes.POINTER(sz)]
     lib.moe_forward.argtypes = [vp, vp, i, vp, vp, sz, vp, ctypes.POINTER(moe_routing_t)]
@@ -233,6 +234,14 @@ def moe_load_weights(handle, router_w, router_bias, w_gate, w_up, w_down, sh_gat
         "moe_load_weights")
 
 
+def moe_load_shard_weights(handle, router_w, router_bias, w_gate, w_up, w_down, sh_gate, sh_up,
+                           sh_down, stream=None) -> None:
+    _check(load_library().moe_load_shard_weights(
+        ctypes.c_void_p(handle), _ptr(router_w), _ptr(router_bias), _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), _ptr(sh_gate), _ptr(sh_up), _ptr(sh_down), _stream(stream)),
+        "moe_load_shard_weights")
+
+
 def moe_load_weights_fp8(handle, router_w, router_bias, w_gate, w_up, w_down, s_gate, s_up,
                          s_down, sh_gate, sh_up, sh_down, sh_s_gate, sh_s_up, sh_s_down,
                          stream=None) -> None:
@@ -339,6 +348,7 @@ class MoeLayer:
         if not torch.cuda.is_available():
             raise RuntimeError("MoeLayer needs a CUDA device")
         self.cfg = cfg
+        self.shard = shard
         self.device = torch.device("cuda", torch.cuda.current_device())
         self.handle = moe_create(cfg) if shard is None else moe_create_shard(cfg, *shard)
         self._ws: Optional[torch.Tensor] = None
@@ -378,6 +388,27 @@ class MoeLayer:
         self._need(sh_down, "sh_down", wdt, (Is, H))
         moe_load_weights(self.handle, router_w, router_bias, w_gate, w_up, w_down, sh_gate,
                          sh_up, sh_down)
+
+    def load_shard_weights(self, router_w, router_bias, w_gate, w_up, w_down, sh_gate=None,
+                           sh_up=None, sh_down=None):
+        """An expert shard's own experts only: w_gate, w_up [count, H, I],
+        w_down [count, I, H] (see moe_load_shard_weights)."""
+        c = self.cfg
+        H, E, I, Is = c.hidden, c.num_experts, c.intermediate, c.shared_intermediate
+        first, count, with_shared = self.shard if self.shard is not None else (0, E, 1)
+        wdt = _TORCH_DT[c.weight_dtype]
+        self._need(router_w, "router_w", torch.float32, (H, E))
+        if router_bias is not None:
+            self._need(router_bias, "router_bias", torch.float32, (E,))
+        self._need(w_gate, "w_gate", wdt, (count, H, I))
+        self._need(w_up, "w_up", wdt, (count, H, I))
+        self._need(w_down, "w_down", wdt, (count, I, H))
+        if with_shared:
+            self._need(sh_gate, "sh_gate", wdt, (H, Is))
+            self._need(sh_up, "sh_up", wdt, (H, Is))
+            self._need(sh_down, "sh_down", wdt, (Is, H))
+        moe_load_shard_weights(self.handle, router_w, router_bias, w_gate, w_up, w_down,
+                               sh_gate, sh_up, sh_down)
 
     def load_weights_fp8(self, router_w, router_bias, w_gate, w_up, w_down, s_gate, s_up, s_down,
                          sh_gate, sh_up, sh_down, sh_s_gate, sh_s_up, sh_s_down):

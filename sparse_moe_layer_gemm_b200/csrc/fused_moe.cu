@@ -70,8 +70,7 @@ struct FusedShape : PairStage {
   static constexpr int XCH_OFFSET = EPI_OFFSET + 4 * 2 * STG_BYTES;
   static constexpr int OKX_OFFSET = XCH_OFFSET + 2 * XCH_BYTES;
   static constexpr int WB_OFFSET = OKX_OFFSET + 64;       // down: per warp BN gate weights
-  static constexpr int TOK_OFFSET = WB_OFFSET + 4 * BN * 4;  // gather: this CTA's token ids
-  static constexpr int TAB_OFFSET = TOK_OFFSET + (BN / 2) * 4;
+  static constexpr int TAB_OFFSET = WB_OFFSET + 4 * BN * 4;
   // tiles_gu, tiles_dn, counts, row_start of up to kFusedGroups groups
   static constexpr int TAB_BYTES = 4 * (kFusedGroups + 1) * 4;
   static constexpr size_t SMEM = 1024 + static_cast<size_t>(TAB_OFFSET) + TAB_BYTES;
@@ -330,7 +329,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
   const uint32_t full_leader = mapa_shared(full0, 0);
   const uint32_t tempty_leader = mapa_shared(tempty0, 0);
   const uint64_t desc0 = sdesc_k_sw<128>(smem_u32(smem));
-  int* tok_s = reinterpret_cast<int*>(smem + S::TOK_OFFSET);
 
   // ------------------------------------------------------------------ roles
   // Every role walks the same tiles (w = pair, pair + n_pairs, ...) of a phase.
@@ -401,13 +399,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
       }
     } else if (warp >= kGatherWarp0) {
       // ---------------------------------------------------- token-row gather
-      // Gather warp wg owns the tile's rows i = wg, wg + 2, ... of this CTA's
-      // token half: it looks their tokens up once per tile (perm), then per
-      // stage copies their 128-byte K chunks with cp.async into the
-      // 128B-swizzled B slot (chunk c of row i at (c ^ (i % 8)) * 16).  Rows
-      // past the group are left as they are: their MMA columns are never
-      // stored.  The two warps never wait for each other.
-      const int wg = warp - kGatherWarp0;
+      // Thread g (0..63) of the two gather warps copies chunk c = g % 8 (16
+      // bytes) of rows r = g / 8 + 8 j of this CTA's token half: per tile it
+      // looks its rows' tokens up in perm once and keeps their source
+      // pointers; per stage and K sub-block each copy is one cp.async to the
+      // 128B-swizzled slot (chunk c of row r at (c ^ r % 8) * 16, and r % 8 =
+      // g / 8 for every j).  Eight consecutive threads cover one row's 128
+      // bytes.  Rows past the group are not copied: their MMA columns are
+      // never stored.  The two warps never wait for each other.
+      constexpr int kRowsPerThread = (kPairBN / 2) / 8;  // 16
+      const int g = threadIdx.x - kGatherWarp0 * 32;
+      const int c = g & 7, rg = g >> 3;
+      const uint32_t swz = static_cast<uint32_t>((c ^ rg) << 4);
+      const __nv_bfloat16* src[kRowsPerThread];
       for (int w = pair; w < n_tiles; w += n_pairs) {
         if (*abort_flag) return;
         const FTile t = tile_of(w);
@@ -416,17 +420,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
         const int ks = narrow ? S::KS_N : S::KS_W;
         const int num_kb = num_kb_of[t.kind];
         const int n_st = (num_kb + ks - 1) / ks;
-        const int nrows = (half - wg + 1) / 2;  // this warp's rows (half >= 8)
         if (t.gather) {
           const int cnt = gpu.counts[t.g];
-          const int r0 = gpu.row_start[t.g];
-          __syncwarp();  // this warp's previous ids are read
-          for (int rr = lane; rr < nrows; rr += 32) {
-            const int i = wg + 2 * rr;
-            const int r = t.nc * BN + static_cast<int>(rank) * half + i;
-            tok_s[i] = r < cnt ? p.perm[r0 + r] / p.k : -1;  // (written in this launch)
+          const int* pg = p.perm + gpu.row_start[t.g];  // (written in this launch: plain loads)
+          const int rbase = t.nc * BN + static_cast<int>(rank) * half;
+#pragma unroll
+          for (int j = 0; j < kRowsPerThread; ++j) {
+            const int r = rg + 8 * j;
+            src[j] = nullptr;
+            if (r < half && rbase + r < cnt)
+              src[j] = p.x + static_cast<size_t>(pg[rbase + r] / p.k) * p.H + c * 8;
           }
-          __syncwarp();
         }
         const uint32_t b_off = narrow ? S::B_OFF_N : S::B_OFF_W;
         const uint32_t sub_b = narrow ? S::SUB_BN : S::SUB_BW;
@@ -438,19 +442,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) return;
           if (t.gather) {
-            const uint32_t sb = smem_u32(smem + s * S::STAGE_BYTES) + b_off;
+            const uint32_t sb = smem_u32(smem + s * S::STAGE_BYTES) + b_off + rg * 128 + swz;
             const int kb0 = st * ks;
             const int nsub = min(ks, num_kb - kb0);
-            const int items = nrows * nsub * 8;  // 16-byte chunks of this warp's rows
-            for (int q = lane; q < items; q += 32) {
-              const int c = q & 7;                  // chunk of the 128-byte row
-              const int rr = (q >> 3) % nrows;
-              const int hh = (q >> 3) / nrows;      // K sub-block
-              const int i = wg + 2 * rr;            // token row
-              const int tk = tok_s[i];
-              if (tk < 0) continue;
-              const uint32_t dst = sb + hh * sub_b + i * 128 + ((c ^ (i & 7)) << 4);
-              cp_async_16(dst, p.x + static_cast<size_t>(tk) * p.H + (kb0 + hh) * kBK + c * 8);
+            for (int hh = 0; hh < nsub; ++hh) {
+              const uint32_t dh = sb + hh * sub_b;
+              const int ko = (kb0 + hh) * kBK;
+#pragma unroll
+              for (int j = 0; j < kRowsPerThread; ++j)
+                if (src[j] != nullptr) cp_async_16(dh + j * 8 * 128, src[j] + ko);
             }
             cp_async_arrive_noinc(gfull0 + 8 * s);
           } else {
@@ -765,9 +765,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
 
   // ------------------------------------------------------------ C: combine
   {
-    int* rows_s = reinterpret_cast<int*>(scratch);
-    for (int t = blockIdx.x; t < p.T; t += gridDim.x)
-      combine::combine_token<__nv_bfloat16>(t, p.y, p.pos, p.T, p.k, p.H, 1, p.out, rows_s);
+    // one (token, 8-element vector) item per thread at a time, over the whole
+    // grid (many independent row loads in flight); the same fixed order as
+    // the combine kernel: j = 0..k-1, then the shared row
+    const int nvec = p.H / 8;
+    const size_t items = static_cast<size_t>(p.T) * nvec;
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < items;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+      const int t = static_cast<int>(i / nvec);
+      const int v = static_cast<int>(i - static_cast<size_t>(t) * nvec);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const int* pt = p.pos + static_cast<size_t>(t) * p.k;
+      for (int j = 0; j < p.k; ++j)
+        combine::add8(acc, p.y + static_cast<size_t>(pt[j]) * p.H + v * 8);
+      combine::add8(acc, p.y + (static_cast<size_t>(p.T) * p.k + t) * p.H + v * 8);
+      combine::store8(p.out + static_cast<size_t>(t) * p.H + v * 8, acc);
+    }
   }
 
 teardown:

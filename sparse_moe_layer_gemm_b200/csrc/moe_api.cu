@@ -439,24 +439,24 @@ int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count
   return MOE_OK;
 }
 
-int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_bias,
-                     const void* w_gate, const void* w_up, const void* w_down, const void* sh_gate,
-                     const void* sh_up, const void* sh_down, void* stream) {
-  if (L == nullptr || router_w == nullptr || w_gate == nullptr || w_up == nullptr ||
-      w_down == nullptr || sh_gate == nullptr || sh_up == nullptr || sh_down == nullptr)
-    return MOE_ERR_INVALID_ARG;
-  if (L->fp8) return MOE_ERR_INVALID_ARG;  // codes need their scales: moe_load_weights_fp8
-  DeviceGuard dg(L->device);
-  if (!dg.ok) return MOE_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+}  // extern "C"
+
+namespace {
+
+// Packs the bf16 / fp32 expert weights: the layer's E_loc routed experts start
+// first_in_tensor experts into the caller's tensors (the shard's own first
+// expert for moe_load_weights, 0 for moe_load_shard_weights), then the shared
+// expert if the layer holds it, then the router.
+int load_bf16(moe_layer* L, const float* router_w, const float* router_bias, const void* w_gate,
+              const void* w_up, const void* w_down, const void* sh_gate, const void* sh_up,
+              const void* sh_down, size_t first_in_tensor, cudaStream_t st) {
   const moe_config_t& c = L->cfg;
   const int H = c.hidden, El = L->E_loc, I = c.intermediate, Ip = L->I_pad;
   const bool wb = c.weight_dtype == MOE_BF16;
   const size_t gu_group = static_cast<size_t>(2) * Ip * H, dn_group = static_cast<size_t>(H) * Ip;
   __nv_bfloat16* gu = static_cast<__nv_bfloat16*>(L->w_gu);
   __nv_bfloat16* dn = static_cast<__nv_bfloat16*>(L->w_dn);
-  // the shard's experts start `first` experts into the caller's tensors
-  const size_t off = static_cast<size_t>(L->first) * H * I * (wb ? 2 : 4);
+  const size_t off = first_in_tensor * H * I * (wb ? 2 : 4);
   const uint8_t* wg = static_cast<const uint8_t*>(w_gate) + off;
   const uint8_t* wu = static_cast<const uint8_t*>(w_up) + off;
   const uint8_t* wd = static_cast<const uint8_t*>(w_down) + off;
@@ -471,6 +471,40 @@ int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_
     MOE_CUDA(moe::launch_pack_down(sh_down, wb, 1, H, I, Ip, dn + El * dn_group, st));
   }
   return load_router(L, router_w, router_bias, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_load_weights(moe_layer_t* L, const float* router_w, const float* router_bias,
+                     const void* w_gate, const void* w_up, const void* w_down, const void* sh_gate,
+                     const void* sh_up, const void* sh_down, void* stream) {
+  if (L == nullptr || router_w == nullptr || w_gate == nullptr || w_up == nullptr ||
+      w_down == nullptr || sh_gate == nullptr || sh_up == nullptr || sh_down == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (L->fp8) return MOE_ERR_INVALID_ARG;  // codes need their scales: moe_load_weights_fp8
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  // the shard's experts start `first` experts into the caller's tensors
+  return load_bf16(L, router_w, router_bias, w_gate, w_up, w_down, sh_gate, sh_up, sh_down,
+                   static_cast<size_t>(L->first), static_cast<cudaStream_t>(stream));
+}
+
+int moe_load_shard_weights(moe_layer_t* L, const float* router_w, const float* router_bias,
+                           const void* w_gate, const void* w_up, const void* w_down,
+                           const void* sh_gate, const void* sh_up, const void* sh_down,
+                           void* stream) {
+  if (L == nullptr || router_w == nullptr || w_gate == nullptr || w_up == nullptr ||
+      w_down == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (L->with_shared && (sh_gate == nullptr || sh_up == nullptr || sh_down == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (L->fp8) return MOE_ERR_INVALID_ARG;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  return load_bf16(L, router_w, router_bias, w_gate, w_up, w_down, sh_gate, sh_up, sh_down, 0,
+                   static_cast<cudaStream_t>(stream));
 }
 
 int moe_load_weights_fp8(moe_layer_t* L, const float* router_w, const float* router_bias,

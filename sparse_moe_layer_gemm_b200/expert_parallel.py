@@ -57,6 +57,13 @@ class ExpertParallelMoE:
         only this rank's slice."""
         self.layer.load_inputs(inp)
 
+    def load_shard_inputs(self, inp: Dict[str, torch.Tensor]):
+        """This rank's experts only ([count, ...], e.g. from
+        workloads.make_shard_inputs): a rank holds 1/N of the expert bytes."""
+        self.layer.load_shard_weights(inp["router_w"], inp["router_bias"], inp["w_gate"],
+                                      inp["w_up"], inp["w_down"], inp.get("sh_gate"),
+                                      inp.get("sh_up"), inp.get("sh_down"))
+
     def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
         return reduce_partials(self.layer.forward(x, out), self.group)
 

@@ -199,6 +199,31 @@ def make_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
     return out
 
 
+def make_shard_inputs(wl: Workload, first: int, count: int, with_shared: bool,
+                      device="cpu") -> Dict[str, torch.Tensor]:
+    """The tensors an expert shard loads (moe_load_shard_weights): x, the
+    whole router, experts [first, first + count) only ([count, ...]), and the
+    shared expert if the shard holds it.  Each expert comes from its own
+    generator, so these equal the matching slices of make_inputs."""
+    dev = torch.device(device)
+    x = draw_x(wl, dev)
+    rw, rb = draw_router(wl, dev)
+    H, I = wl.hidden, wl.intermediate
+    dt = _torch_dtype(wl.weight_dtype)
+    w_gate = torch.empty(count, H, I, dtype=dt, device=dev)
+    w_up = torch.empty(count, H, I, dtype=dt, device=dev)
+    w_down = torch.empty(count, I, H, dtype=dt, device=dev)
+    for i in range(count):
+        wg, wu, wd = draw_expert(wl, first + i, dev)
+        w_gate[i].copy_(wg)
+        w_up[i].copy_(wu)
+        w_down[i].copy_(wd)
+    out = dict(x=x, router_w=rw, router_bias=rb, w_gate=w_gate, w_up=w_up, w_down=w_down)
+    if with_shared:
+        out["sh_gate"], out["sh_up"], out["sh_down"] = draw_shared(wl, dev)
+    return out
+
+
 class HostExpertView:
     """``view[e]`` -> exact float32 host copy of expert e's matrix of a device
     tensor [E, ...]; lets the oracle walk a 9 GB weight set expert by expert."""

@@ -142,3 +142,112 @@ def test_gpu_shards_sum_to_oracle(case):
                          top_k=wl.top_k, scale=wl.scale).out
     rel, mx = output_errors(total.numpy(), ref)
     assert rel <= REL_FRO and mx <= MAX_ABS_OVER_RMS, (rel, mx)
+
+
+def test_shard_inputs_are_slices_of_the_layer():
+    """What a rank of the expert-parallel bench draws (its experts only)
+    equals the matching slices of the whole layer's tensors."""
+    from sparse_moe_layer_gemm_b200.workloads import make_shard_inputs
+    wl = WORKLOADS["tiny"]
+    full = make_inputs(wl, "cpu")
+    for first, count, sh in ((0, 5, True), (5, 11, False)):
+        part = make_shard_inputs(wl, first, count, sh, "cpu")
+        for n in ("x", "router_w", "router_bias"):
+            assert torch.equal(part[n], full[n])
+        for n in ("w_gate", "w_up", "w_down"):
+            assert torch.equal(part[n], full[n][first:first + count])
+        assert ("sh_gate" in part) == sh
+        if sh:
+            for n in ("sh_gate", "sh_up", "sh_down"):
+                assert torch.equal(part[n], full[n])
+
+
+def test_bench_ep_plan_covers_experts_once():
+    import bench
+    for E, world in ((288, 8), (288, 2), (16, 3)):
+        seen, shared = [], 0
+        for r in range(world):
+            pl = bench.ep_plan(E, world, r)
+            seen.extend(range(pl["first"], pl["first"] + pl["count"]))
+            shared += pl["with_shared"]
+        assert seen == list(range(E)) and shared == 1
+    cfg = bench.ep_config(WORKLOADS["decode"], 8)
+    assert cfg["parallelism"].startswith("ep8") and cfg["workload"] == "decode"
+
+
+def _ep_bench_worker(rank, world, port, q):
+    """One rank of the bench's expert-parallel step on the CPU: its own
+    shard's tensors only, its partial output (the oracle standing in for the
+    kernels), then the all-reduce the bench runs after every forward."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    import bench
+    from sparse_moe_layer_gemm_b200.workloads import make_shard_inputs
+    wl = WORKLOADS["tiny"]
+    pl = bench.ep_plan(wl.num_experts, world, rank)
+    part_in = {k: host_f32(v).astype(np.float64)
+               for k, v in make_shard_inputs(wl, pl["first"], pl["count"], pl["with_shared"],
+                                             "cpu").items()}
+    E, H, I = wl.num_experts, wl.hidden, wl.intermediate
+    f, c = pl["first"], pl["count"]
+    wg = np.zeros((E, H, I)); wu = np.zeros((E, H, I)); wd = np.zeros((E, I, H))
+    wg[f:f + c], wu[f:f + c], wd[f:f + c] = part_in["w_gate"], part_in["w_up"], part_in["w_down"]
+    zs = np.zeros((H, wl.shared_intermediate))
+    sg = part_in.get("sh_gate", zs)
+    su = part_in.get("sh_up", zs)
+    sd = part_in.get("sh_down", zs.T)
+    part = om.moe_forward(part_in["x"], part_in["router_w"], part_in["router_bias"], wg, wu, wd,
+                          sg, su, sd, top_k=wl.top_k, scale=wl.scale).out
+    total = reduce_partials(torch.from_numpy(part.copy()))
+    full_in = {k: host_f32(v).astype(np.float64) for k, v in make_inputs(wl, "cpu").items()}
+    full = om.moe_forward(full_in["x"], full_in["router_w"], full_in["router_bias"],
+                          full_in["w_gate"], full_in["w_up"], full_in["w_down"],
+                          full_in["sh_gate"], full_in["sh_up"], full_in["sh_down"],
+                          top_k=wl.top_k, scale=wl.scale).out
+    q.put((rank, float(np.max(np.abs(total.numpy() - full))), float(np.max(np.abs(full)))))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_bench_ep_step_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_ep_bench_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=150) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err, scale in res:
+        assert err <= 1e-12 * scale
+
+
+@pytest.mark.gpu
+@pytest.mark.timeout(300)
+def test_gpu_shard_only_loading_matches_full_loading():
+    """moe_load_shard_weights with a shard's own experts gives the same bits
+    as moe_load_weights with the whole tensors."""
+    from sparse_moe_layer_gemm_b200 import binding as B
+    from sparse_moe_layer_gemm_b200.workloads import make_shard_inputs
+    wl = replace(WORKLOADS["tiny"], name="eps", T=300, act_dtype="bf16", weight_dtype="bf16")
+    full = {k: v.cuda() for k, v in make_inputs(wl, "cpu").items()}
+    for first, count, sh in ((0, 7, True), (7, 9, False)):
+        a = B.MoeLayer.from_workload(wl, (first, count, sh))
+        a.load_inputs(full)
+        b = B.MoeLayer.from_workload(wl, (first, count, sh))
+        part = {k: v.cuda() for k, v in make_shard_inputs(wl, first, count, sh, "cpu").items()}
+        b.load_shard_weights(part["router_w"], part["router_bias"], part["w_gate"], part["w_up"],
+                             part["w_down"], part.get("sh_gate"), part.get("sh_up"),
+                             part.get("sh_down"))
+        oa = a.forward(full["x"]).clone()
+        ob = b.forward(full["x"])
+        torch.cuda.synchronize()
+        assert a.device_error() == 0 and b.device_error() == 0
+        assert torch.equal(oa, ob)
+        a.close()
+        b.close()
