@@ -20,6 +20,17 @@ __device__ __forceinline__ void add8(float (&acc)[8], const __nv_bfloat16* p) {
   }
 }
 
+// acc += the 8 bf16 values held in q (already loaded)
+__device__ __forceinline__ void add8(float (&acc)[8], const uint4& q) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    acc[2 * i] += f.x;
+    acc[2 * i + 1] += f.y;
+  }
+}
+
 __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
   uint4 q;
   __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q);

@@ -9,8 +9,9 @@
 // the phases of the layer, separated by grid-wide barriers:
 //
 //   R  router logits on the tensor cores: x . W1|W2|W3 (the three-term bf16
-//      split of W_r, one K part each), pair MMAs of 256 expert rows x 256
-//      tokens, fp32 partial logits                               | barrier
+//      split of W_r; each term's K in two halves: six K parts, so the tiles
+//      fill the pairs in even waves), pair MMAs of 256 expert rows x 256
+//      tokens, fp32 partial logits, summed by the top-k          | barrier
 //   K  top-k, one warp per token over the whole grid (the warp form of the
 //      top-k kernels: boundary candidates recomputed in fp32)     | barrier
 //   S  counting sort: chunk histograms | scan (one CTA) | stable scatter,
@@ -216,6 +217,9 @@ struct FusedParams {
   unsigned int* sync;           // [0] grid barrier; [1 + b] readiness of token block b
   float limit, limit_shared;
   int* status;
+  __nv_bfloat16* x_perm;        // non-null: the routed rows are gathered into x_perm in a
+                                // phase of their own and read by TMA (else by the
+                                // gather warps, straight from x)
   uint64_t wait_ns;             // limit of every bounded wait
   unsigned int ready_extra;     // self-check only: arrivals a down tile waits for beyond
                                 // its token block's gate|up tiles (0 in a forward)
@@ -246,7 +250,7 @@ __device__ __forceinline__ FTile router_tile(const FusedParams& p, int w) {
 }
 
 __device__ __forceinline__ FTile gemm_tile(const GemmParams& gpu, const GemmParams& gpd, int n_gu,
-                                           int w, int E) {
+                                           int w, int E, bool in_producer) {
   FTile t{};
   const bool gu = w < n_gu;
   const Tile d = gu ? decode_tile<kPairBN>(gpu, w) : decode_tile<kPairBN>(gpd, w - n_gu);
@@ -256,7 +260,7 @@ __device__ __forceinline__ FTile gemm_tile(const GemmParams& gpu, const GemmPara
   t.nc = d.nc;
   t.n_valid = d.n_valid;
   t.nch = d.nch;
-  t.gather = gu && d.g != E;
+  t.gather = in_producer && gu && d.g != E;
   t.blk = gpu.tile_start[d.g] / gpu.m_tiles + d.nc;
   return t;
 }
@@ -265,7 +269,7 @@ __device__ __forceinline__ FTile gemm_tile(const GemmParams& gpu, const GemmPara
 // weights of wide / narrow stages for the router, gate|up and down; token rows
 // of x and of h with 128-row x 2 and 32-row x 3 K-block boxes; stores of h, y.
 struct FusedMaps {
-  CUtensorMap rt_w, rt_n, gu_w, gu_n, dn_w, dn_n, x_w, x_n, h_w, h_n, st_h, st_y;
+  CUtensorMap rt_w, rt_n, gu_w, gu_n, dn_w, dn_n, x_w, x_n, h_w, h_n, st_h, st_y, xp_w, xp_n;
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
@@ -295,9 +299,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 2);                 // leader: producer arming + peer forward
+      mbar_init(full0 + 8 * s, 2);                 // leader: producer arming + (peer forward
+                                                   // of gathered rows, or the producer again)
       mbar_init(empty0 + 8 * s, 1);                // one multicast commit
-      mbar_init(gfull0 + 8 * s, kGatherThreads);   // this CTA's gather threads
+      mbar_init(gfull0 + 8 * s, kGatherThreads);   // this CTA's gather threads (gathered
+                                                   // stages only)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull0 + 8 * b, 1);
@@ -308,9 +314,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    const CUtensorMap* maps[12] = {&m.rt_w, &m.rt_n, &m.gu_w, &m.gu_n, &m.dn_w, &m.dn_n,
-                                   &m.x_w,  &m.x_n,  &m.h_w,  &m.h_n,  &m.st_h, &m.st_y};
-    for (int i = 0; i < 12; ++i) prefetch_tmap(maps[i]);
+    const CUtensorMap* maps[14] = {&m.rt_w, &m.rt_n, &m.gu_w, &m.gu_n, &m.dn_w,
+                                   &m.dn_n, &m.x_w,  &m.x_n,  &m.h_w,  &m.h_n,
+                                   &m.st_h, &m.st_y, &m.xp_w, &m.xp_n};
+    for (int i = 0; i < (p.x_perm != nullptr ? 14 : 12); ++i) prefetch_tmap(maps[i]);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), S::TMEM_COLS);
@@ -326,6 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
   uint32_t it = 0;      // pipeline stages (producer, gather, forwarder, issuer)
   uint32_t tc = 0;      // accumulator buffers (issuer, epilogue)
   uint32_t chunks = 0;  // epilogue: staged output chunks (double buffer index)
+  uint32_t gpar = 0;    // per slot: parity of its gather barrier (flips on gathered stages only)
   const uint32_t full_leader = mapa_shared(full0, 0);
   const uint32_t tempty_leader = mapa_shared(tempty0, 0);
   const uint64_t desc0 = sdesc_k_sw<128>(smem_u32(smem));
@@ -335,9 +343,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
   auto run_tiles = [&](int phase, int n_tiles, const GemmParams& gpu, const GemmParams& gpd,
                        int n_gu) {
     auto tile_of = [&](int w) {
-      return phase == 0 ? router_tile(p, w) : gemm_tile(gpu, gpd, n_gu, w, p.E);
+      return phase == 0 ? router_tile(p, w)
+                        : gemm_tile(gpu, gpd, n_gu, w, p.E, p.x_perm == nullptr);
     };
-    const int num_kb_of[3] = {p.H / kBK, p.H / kBK, p.I_pad / kBK};
+    // router parts cover half of one bf16 term's K each (kFusedRouterParts)
+    const int num_kb_of[3] = {p.H / 2 / kBK, p.H / kBK, p.I_pad / kBK};
     if (warp == 0) {
       // ---------------------------------------------------- TMA producer
       if (lane != 0) return;
@@ -354,18 +364,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
         const int n_st = (num_kb + ks - 1) / ks;
         const CUtensorMap* ma;
         const CUtensorMap* mb;
-        int a_row, b_row, a_kb0 = 0;
+        int a_row, b_row, a_kb0 = 0, b_kb0 = 0;
         if (t.kind == kRt) {
+          // part z: K blocks [z, z + 1) * H / 2 of the packed W1 | W2 | W3, against
+          // x's first or second half of K
           ma = narrow ? &m.rt_n : &m.rt_w;
           mb = narrow ? &m.x_n : &m.x_w;
           a_row = t.mt * 2 * kBM + static_cast<int>(rank) * kBM;
-          a_kb0 = t.z * (p.H / kBK);
+          a_kb0 = t.z * (p.H / 2 / kBK);
+          b_kb0 = (t.z & 1) * (p.H / 2 / kBK);
           b_row = t.nc * BN + static_cast<int>(rank) * half;
         } else if (t.kind == kGu) {
           ma = narrow ? &m.gu_n : &m.gu_w;
-          mb = narrow ? &m.x_n : &m.x_w;  // the shared expert's rows are x itself
           a_row = t.g * 2 * p.I_pad + t.mt * 2 * kBM + static_cast<int>(rank) * 64;
-          b_row = t.nc * BN + static_cast<int>(rank) * half;
+          if (t.g == p.E) {  // the shared expert's rows are x itself
+            mb = narrow ? &m.x_n : &m.x_w;
+            b_row = t.nc * BN + static_cast<int>(rank) * half;
+          } else {           // (x_perm: the gathered rows; unused when gathered here)
+            mb = narrow ? &m.xp_n : &m.xp_w;
+            b_row = gpu.row_start[t.g] + t.nc * BN + static_cast<int>(rank) * half;
+          }
         } else {
           ma = narrow ? &m.dn_n : &m.dn_w;
           mb = narrow ? &m.h_n : &m.h_w;
@@ -385,7 +403,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
           const uint32_t s = it % S::STAGES;
           const uint32_t ph = (it / S::STAGES) & 1u;
           if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, p.status, p.wait_ns)) return;
-          if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * (a_bytes + b_bytes));
+          if (rank == 0) {
+            mbar_arrive_expect_tx(full0 + 8 * s, 2 * (a_bytes + b_bytes));
+            // a stage without gathered rows needs no forward from the peer:
+            // its second arrival comes from here
+            if (!t.gather) mbar_arrive(full0 + 8 * s);
+          }
           const uint32_t fb = full_leader + 8 * s;
           const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
           const int kb0 = st * ks;
@@ -393,7 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
             tma_load_4d_pair(sa, ma, fb, 0, a_row, 0, kb0, pol_a);
           else
             tma_load_3d_pair(sa, ma, fb, 0, a_row, a_kb0 + kb0, pol_a);
-          if (!t.gather) tma_load_3d_pair(sa + b_off, mb, fb, 0, b_row, kb0, pol_b);
+          if (!t.gather) tma_load_3d_pair(sa + b_off, mb, fb, 0, b_row, b_kb0 + kb0, pol_b);
           ++it;
         }
       }
@@ -434,14 +457,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
         }
         const uint32_t b_off = narrow ? S::B_OFF_N : S::B_OFF_W;
         const uint32_t sub_b = narrow ? S::SUB_BN : S::SUB_BW;
+        if (!t.gather) {  // nothing to copy; keep the stage count
+          it += n_st;
+          continue;
+        }
         for (int st = 0; st < n_st; ++st) {
           const uint32_t s = it % S::STAGES;
           const uint32_t ph = (it / S::STAGES) & 1u;
           int ok = 1;
-          if (lane == 0) ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, p.status, p.wait_ns) ? 1 : 0;
+          if (lane == 0)
+            ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, abort_flag, p.status, p.wait_ns) ? 1 : 0;
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) return;
-          if (t.gather) {
+          {
             const uint32_t sb = smem_u32(smem + s * S::STAGE_BYTES) + b_off + rg * 128 + swz;
             const int kb0 = st * ks;
             const int nsub = min(ks, num_kb - kb0);
@@ -453,8 +481,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
                 if (src[j] != nullptr) cp_async_16(dh + j * 8 * 128, src[j] + ko);
             }
             cp_async_arrive_noinc(gfull0 + 8 * s);
-          } else {
-            mbar_arrive(gfull0 + 8 * s);
           }
           ++it;
         }
@@ -469,10 +495,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
           const bool narrow = narrow_tile(t.n_valid);
           const int ks = narrow ? S::KS_N : S::KS_W;
           const int n_st = (num_kb_of[t.kind] + ks - 1) / ks;
+          if (!t.gather) {
+            it += n_st;
+            continue;
+          }
           for (int st = 0; st < n_st; ++st) {
             const uint32_t s = it % S::STAGES;
-            const uint32_t ph = (it / S::STAGES) & 1u;
-            if (!mbar_wait(gfull0 + 8 * s, ph, abort_flag, p.status, p.wait_ns)) return;
+            if (!mbar_wait(gfull0 + 8 * s, (gpar >> s) & 1u, abort_flag, p.status, p.wait_ns))
+              return;
+            gpar ^= 1u << s;
             fence_proxy_async_smem();  // the gathered rows, before the leader's MMAs read them
             mbar_arrive_cluster(full_leader + 8 * s);
             ++it;
@@ -500,9 +531,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
         for (int st = 0; st < n_st; ++st) {
           const uint32_t s = it % S::STAGES;
           const uint32_t ph = (it / S::STAGES) & 1u;
-          if (!mbar_wait_cluster(full0 + 8 * s, ph, abort_flag, p.status, p.wait_ns)) return;
-          if (!mbar_wait(gfull0 + 8 * s, ph, abort_flag, p.status, p.wait_ns)) return;
-          if (t.gather) fence_proxy_async_smem();
+          // (cluster-scope acquire only where the peer forwarded gathered rows)
+          if (t.gather ? !mbar_wait_cluster(full0 + 8 * s, ph, abort_flag, p.status, p.wait_ns)
+                       : !mbar_wait(full0 + 8 * s, ph, abort_flag, p.status, p.wait_ns))
+            return;
+          if (t.gather) {
+            if (!mbar_wait(gfull0 + 8 * s, (gpar >> s) & 1u, abort_flag, p.status, p.wait_ns))
+              return;
+            gpar ^= 1u << s;
+            fence_proxy_async_smem();
+          }
           tc_fence_after();
           const uint64_t ad = desc0 + static_cast<uint64_t>((s * S::STAGE_BYTES) >> 4);
           const uint64_t bd = ad + static_cast<uint64_t>(b_off >> 4);
@@ -691,7 +729,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
   // ------------------------------------------------------------ R: router
   {
     const int nb = (p.T + kPairBN - 1) / kPairBN;
-    run_tiles(0, kRouterTcParts * p.rt_mtiles * nb, none, none, 0);
+    run_tiles(0, kFusedRouterParts * p.rt_mtiles * nb, none, none, 0);
   }
   if (!grid_sync(p.sync, nbar++, abort_flag, p.status, p.wait_ns)) goto teardown;
 
@@ -709,7 +747,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
     rf.band = p.band;
     const int gw = blockIdx.x * kFusedWarps + warp;
     for (int t = gw; t < p.T; t += gridDim.x * kFusedWarps)
-      topk::topk_warp_token<kFusedMPL>(t, p.partial, kRouterTcParts, p.T, p.E, p.k, s_bias,
+      topk::topk_warp_token<kFusedMPL>(t, p.partial, kFusedRouterParts, p.T, p.E, p.k, s_bias,
                                        c_lists + warp * 32, p.norm, p.scale, p.topk_idx,
                                        p.topk_w, p.logits_out, rf);
   }
@@ -736,6 +774,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
     }
   }
   if (!grid_sync(p.sync, nbar++, abort_flag, p.status, p.wait_ns)) goto teardown;
+
+  // ------------------------------------------------------------ gather phase
+  if (p.x_perm != nullptr) {
+    // x_perm[r] = x[perm[r] / k], one warp per row at a time over the grid
+    const int rows = p.T * p.k;
+    const int nvec = p.H / 8;
+    for (int r = blockIdx.x * kFusedWarps + warp; r < rows; r += gridDim.x * kFusedWarps) {
+      const int t = p.perm[r] / p.k;
+      const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * p.H);
+      uint4* dst = reinterpret_cast<uint4*>(p.x_perm + static_cast<size_t>(r) * p.H);
+      for (int v = lane; v < nvec; v += 32) dst[v] = src[v];
+    }
+    __threadfence();
+    fence_proxy_async_global();  // before the GEMM phase's TMA reads of x_perm
+    if (!grid_sync(p.sync, nbar++, abort_flag, p.status, p.wait_ns)) goto teardown;
+  }
 
   // ------------------------------------------------------------ G: expert GEMMs
   {
@@ -776,9 +830,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFusedThreads, 1)
       const int v = static_cast<int>(i - static_cast<size_t>(t) * nvec);
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       const int* pt = p.pos + static_cast<size_t>(t) * p.k;
-      for (int j = 0; j < p.k; ++j)
-        combine::add8(acc, p.y + static_cast<size_t>(pt[j]) * p.H + v * 8);
-      combine::add8(acc, p.y + (static_cast<size_t>(p.T) * p.k + t) * p.H + v * 8);
+      const size_t shared_row = static_cast<size_t>(p.T) * p.k + t;
+      if (p.k == 8) {  // the layer's top-8: all nine rows in flight at once
+        uint4 q[9];
+#pragma unroll
+        for (int j = 0; j < 9; ++j)
+          q[j] = *reinterpret_cast<const uint4*>(
+              p.y + (j < 8 ? static_cast<size_t>(pt[j]) : shared_row) * p.H + v * 8);
+#pragma unroll
+        for (int j = 0; j < 9; ++j) combine::add8(acc, q[j]);
+      } else {
+        for (int j = 0; j < p.k; ++j)
+          combine::add8(acc, p.y + static_cast<size_t>(pt[j]) * p.H + v * 8);
+        combine::add8(acc, p.y + shared_row * p.H + v * 8);
+      }
       combine::store8(p.out + static_cast<size_t>(t) * p.H + v * 8, acc);
     }
   }
@@ -854,6 +919,8 @@ cudaError_t launch_fused(const FusedLaunch& f, cudaStream_t st) {
   m.h_n = f.h_n;
   m.st_h = f.st_h;
   m.st_y = f.st_y;
+  m.xp_w = f.xp_w;
+  m.xp_n = f.xp_n;
   FusedParams p{};
   p.x = f.x;
   p.out = f.out;
@@ -888,6 +955,7 @@ cudaError_t launch_fused(const FusedLaunch& f, cudaStream_t st) {
   p.limit = f.limit;
   p.limit_shared = f.limit_shared;
   p.status = f.status;
+  p.x_perm = f.x_perm;
   p.wait_ns = f.wait_ns > 0 ? f.wait_ns : kWaitLimitNs;
   p.ready_extra = f.ready_extra;
   // (not a programmatic-dependent launch: the first phase reads x at once)

@@ -180,6 +180,9 @@ cudaError_t launch_decode_e4m3(const uint8_t* codes, size_t n, __nv_bfloat16* ou
 // experts per lane, kFusedMPL, is fixed).
 constexpr int kFusedMaxExperts = 288;
 constexpr int kFusedMPL = 9;
+// K parts of the fused kernel's tensor-core router: each bf16 term's K in two
+// halves (partial logits [kFusedRouterParts, T, E])
+constexpr int kFusedRouterParts = 6;
 
 struct FusedLaunch {
   // tensor maps: weights of wide / narrow stages (router: encode_bf16_kblocks
@@ -187,6 +190,8 @@ struct FusedLaunch {
   // down: encode_bf16_kblocks, 128 rows), token rows of x and h (128 rows x 2
   // and 32 rows x 3 K blocks), and the TMA stores of h and y
   CUtensorMap rt_w, rt_n, gu_w, gu_n, dn_w, dn_n, x_w, x_n, h_w, h_n, st_h, st_y;
+  CUtensorMap xp_w, xp_n;  // x_perm's K-block maps (gather phase only)
+  __nv_bfloat16* x_perm;   // non-null: gather the routed rows in a phase of their own
   const __nv_bfloat16* x;
   __nv_bfloat16* out;
   int T, H, E, k, I_pad;
@@ -197,7 +202,7 @@ struct FusedLaunch {
   float scale;
   int rt_mtiles;          // ceil(E_pad / 256)
   float* logits_out;      // optional [T, E]
-  float* partial;         // [3, T, E]
+  float* partial;         // [kFusedRouterParts, T, E]
   int *topk_idx;
   float* topk_w;
   uint32_t* masks;
