@@ -5,6 +5,7 @@
 //   -> K5 grouped gate|up + SwiGLU -> K6 grouped down x gate weight -> K7 combine.
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -149,6 +150,27 @@ using moe::encode_bf16_kpair;
 using moe::encode_bf16_store;
 
 namespace {
+
+// NVTX ranges of a forward's stages on the calling host thread (named in the
+// timeline of a profiler; no cost without one).  At most one range is open;
+// the destructor closes it on every return path.
+struct NvtxStages {
+  bool open = false;
+  void enter(const char* name) {
+    if (open) nvtxRangePop();
+    nvtxRangePushA(name);
+    open = true;
+  }
+  void leave() {
+    if (open) nvtxRangePop();
+    open = false;
+  }
+  ~NvtxStages() { leave(); }
+};
+
+const char* const kStageNames[MOE_NUM_STAGES] = {"moe router", "moe top-k", "moe sort",
+                                                 "moe gather", "moe gate|up", "moe down",
+                                                 "moe combine"};
 
 constexpr int kMaxTokens = 1 << 20;
 constexpr size_t kAlign = 1024;
@@ -663,11 +685,19 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   cudaEvent_t* ev = nullptr;
   if (L->timing_capacity > 0 && L->timing_recorded < L->timing_capacity)
     ev = &L->events[static_cast<size_t>(L->timing_recorded++) * (MOE_NUM_STAGES + 1)];
-  auto mark = [&](int i) { return ev == nullptr ? cudaSuccess : cudaEventRecord(ev[i], st); };
+  NvtxStages nvtx;
+  auto mark = [&](int i) {
+    if (i < MOE_NUM_STAGES)
+      nvtx.enter(kStageNames[i]);
+    else
+      nvtx.leave();
+    return ev == nullptr ? cudaSuccess : cudaEventRecord(ev[i], st);
+  };
 
   if (forward_path(L, T) == MOE_PATH_FUSED) {
     // one persistent kernel (fused_moe.cu); the whole forward is stage 0
     MOE_CUDA(mark(0));
+    nvtx.enter("moe fused forward");
     const int r = launch_fused_forward(L, x, T, out, ws, w, st, routing, 0, 0);
     if (r != MOE_OK) return r;
     for (int i = 1; i <= MOE_NUM_STAGES; ++i) MOE_CUDA(mark(i));

@@ -86,6 +86,15 @@ SMALL = {
                                  shared_intermediate=384, act_dtype="bf16",
                                  weight_dtype="bf16", x_dist="rmsnorm_normal",
                                  swiglu_limit=0.9, swiglu_limit_shared=1.2, expert_std=0.08),
+    # tensor-core router (from 512 bf16 tokens) with logits five times the
+    # workloads' spread (router N(0, 0.1): logit std ~6.4 at H = 4096): larger
+    # partial sums, so larger truncation errors of the tensor cores' fp32
+    # accumulation, against the top-k's guard band
+    "large_logits_tc_router": replace(WORKLOADS["tiny"], name="ll", T=1024, hidden=4096,
+                                      num_experts=64, top_k=8, intermediate=128,
+                                      shared_intermediate=128, act_dtype="bf16",
+                                      weight_dtype="bf16", x_dist="rmsnorm_normal",
+                                      router_std=0.1, expert_std=0.02),
     # tensor-core router with the warp-per-token top-k (from 8192 tokens) on a
     # small layer
     "many_tokens_small_layer": replace(WORKLOADS["tiny"], name="mt", T=8448, hidden=256,
