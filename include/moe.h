@@ -402,11 +402,19 @@ int moe_dense_load_weights(moe_dense_t* layer, const void* w_gate, const void* w
  * aligned, caller-allocated).  Host-only. */
 int moe_dense_workspace_size(const moe_dense_t* layer, int T, size_t* bytes);
 
-/* out [T, H] from x [T, H]; x and out must not alias; T = 0 is a no-op. */
+/* out [T, H] from x [T, H]; x and out must not alias; T = 0 is a no-op.
+ * From 1 to 128 tokens with hidden % 256 == 0 the forward is one persistent
+ * launch whose CTAs synchronise through running counters owned by the layer
+ * (never cleared between forwards): the forwards of one layer must then run
+ * on the device in the order they were issued (one stream, or streams
+ * ordered by events).  The result depends only on x's own rows (the same
+ * row gives the same output in any batch of up to 128 tokens). */
 int moe_dense_forward(moe_dense_t* layer, const void* x, int T, void* out,
                       void* workspace, size_t ws_bytes, void* stream);
 
-/* As moe_get_device_error, for the dense layer's status word. */
+/* As moe_get_device_error, for the dense layer's status word.  After a
+ * device error it also clears the layer's forward counters (the aborted
+ * launch left them short), so later forwards start from a clean state. */
 int moe_dense_get_device_error(moe_dense_t* layer, int* device_err);
 
 /* Frees the layer (synchronises the device first).  NULL is ignored. */

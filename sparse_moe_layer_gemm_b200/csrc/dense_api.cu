@@ -6,10 +6,12 @@
 // group of all T rows:
 //   h   = silu(min(x.W_gate, L)) * clip(x.W_up, -L, L)   K5 (gate|up + SwiGLU)
 //   out = h . W_down                                       K6 (down, weight 1)
-// When the tiles of one token block cannot fill the GPU (decode-sized T),
-// both GEMMs split K instead: each part writes raw fp32 accumulators and a
-// reduction kernel sums the parts in fixed order (then applies the SwiGLU, or
-// writes out).  Declared in include/moe.h (moe_dense_*).
+// When the tiles of one token block cannot fill the GPU (decode-sized T):
+// up to 128 tokens with H % 256 == 0, one persistent stream-K launch runs
+// both GEMMs and their reductions (dense_streamk.cu); otherwise both GEMMs
+// split K, each part writes raw fp32 accumulators and a reduction kernel sums
+// the parts in fixed order (then applies the SwiGLU, or writes out).
+// Declared in include/moe.h (moe_dense_*).
 #include <math.h>
 #include <string.h>
 
@@ -27,6 +29,11 @@ struct moe_dense {
   __nv_bfloat16* w_dn;  // [H, I_pad]
   int* status;
   int loaded;
+  // the one-launch stream-K forward (T <= 128): its running counters and
+  // their targets' bases (see dense_streamk.cu)
+  unsigned int* sk_cnt;
+  unsigned int sk_fwd;
+  unsigned int sk_rows;
   CUtensorMap tm_gu;    // box 64 x 256 (one CTA per tile)
   CUtensorMap tm_gu128; // box 64 x 128 (split-K partial tiles)
   CUtensorMap tm_gu_pw; // CTA pairs, wide stages: 64 + 64 rows x 2 K blocks
@@ -130,7 +137,17 @@ unsigned grid_for(size_t n, int num_sms) {
 struct DenseWs {
   size_t xb, h, y, ones, parts, total;
   int s_gu, s_dn;  // split-K parts of the two GEMMs (1: no split)
+  bool sk;         // the one-launch stream-K forward (sk_parts: its slots per pass)
+  int sk_seg[moe::kSkPasses];
+  size_t sk_parts[moe::kSkPasses];
 };
+
+// The one-launch stream-K forward serves decode-sized T when H splits into
+// 256-row down tiles and the grid fits its reduction staging.
+bool use_streamk(const moe_dense* L, int T) {
+  return T <= moe::kSkMaxTokens && L->cfg.hidden % 256 == 0 && L->num_sms <= moe::kSkMaxGrid &&
+         moe::dense_streamk_grid() == L->num_sms;
+}
 
 DenseWs dense_ws(const moe_dense* L, int T) {
   const size_t H = L->cfg.hidden;
@@ -144,6 +161,19 @@ DenseWs dense_ws(const moe_dense* L, int T) {
   const bool xf = L->cfg.act_dtype == MOE_F32;
   w.xb = xf ? take(static_cast<size_t>(T) * H * 2) : 0;    // bf16 copy of fp32 x
   w.h = take(static_cast<size_t>(T) * L->I_pad * 2);
+  if (use_streamk(L, T)) {
+    const size_t G = L->num_sms;
+    moe::SkPass ps[moe::kSkPasses];
+    moe::dense_streamk_passes(L->cfg.hidden, L->I_pad, ps);
+    w.sk = true;
+    w.s_gu = w.s_dn = 1;
+    for (int q = 0; q < moe::kSkPasses; ++q) {
+      w.sk_seg[q] = moe::dense_streamk_max_seg(ps[q].tiles, ps[q].nkb, static_cast<int>(G));
+      w.sk_parts[q] = take(G * w.sk_seg[q] * T * 256 * sizeof(float));
+    }
+    w.total = off;
+    return w;
+  }
   w.y = xf ? take(static_cast<size_t>(T) * H * 2) : 0;     // bf16 result before widening
   w.ones = take(static_cast<size_t>(T) * sizeof(float));  // the down GEMM's row weights
   // split-K only below the CTA-pair range (one token block of tiles)
@@ -199,10 +229,15 @@ int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out) {
   const size_t H = cfg->hidden, Ip = L->I_pad;
   if (moe::gemm_configure_device() != cudaSuccess ||
       moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
+      moe::dense_streamk_configure_device(L->num_sms) != cudaSuccess ||
       cudaMalloc(&L->w_gu, 2 * Ip * H * 2) != cudaSuccess ||
       cudaMalloc(&L->w_dn, H * Ip * 2) != cudaSuccess ||
       cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
       cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&L->sk_cnt, moe::dense_streamk_counters(cfg->hidden, L->I_pad) * 4) !=
+          cudaSuccess ||
+      cudaMemset(L->sk_cnt, 0, moe::dense_streamk_counters(cfg->hidden, L->I_pad) * 4) !=
+          cudaSuccess ||
       !moe::encode_bf16_2d(&L->tm_gu, L->w_gu, 2 * Ip, H, 2 * moe::kBM) ||
       !moe::encode_bf16_2d(&L->tm_gu128, L->w_gu, 2 * Ip, H, moe::kBM) ||
       !moe::encode_bf16_gate_up_pair(&L->tm_gu_pw, L->w_gu, 2 * Ip, H, 2) ||
@@ -272,6 +307,34 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + w.h);
   __nv_bfloat16* y = xf ? reinterpret_cast<__nv_bfloat16*>(ws + w.y)
                         : static_cast<__nv_bfloat16*>(out);
+  if (w.sk) {  // decode-sized T: both GEMMs and their reductions in one launch
+    moe::DenseStreamK d{};
+    d.tm_gu = L->tm_gu128;
+    d.tm_dn = L->tm_dn;
+    const uint32_t n_mma = static_cast<uint32_t>((T + 15) & ~15);
+    if (!moe::encode_bf16_2d(&d.tm_x, xb, T, H, n_mma) ||
+        !moe::encode_bf16_2d(&d.tm_h, h, T, Ip, n_mma))
+      return MOE_ERR_CUDA;
+    d.T = T;
+    d.H = H;
+    d.I_pad = Ip;
+    for (int q = 0; q < moe::kSkPasses; ++q) {
+      d.max_seg[q] = w.sk_seg[q];
+      d.parts[q] = reinterpret_cast<float*>(ws + w.sk_parts[q]);
+    }
+    d.limit = L->cfg.swiglu_limit;
+    d.h = h;
+    d.out = out;
+    d.out_f32 = xf;
+    d.counters = L->sk_cnt;
+    d.fwd = L->sk_fwd + 1u;
+    d.h_rows = L->sk_rows + static_cast<unsigned int>(T);
+    d.status = L->status;
+    MOE_CUDA(moe::launch_dense_streamk(d, st));
+    L->sk_fwd = d.fwd;  // the targets of the launches that follow
+    L->sk_rows = d.h_rows;
+    return MOE_OK;
+  }
   float* ones = reinterpret_cast<float*>(ws + w.ones);
   if (w.s_dn <= 1) {  // the unsplit down GEMM's row weights
     fill_f32_kernel<<<grid_for(static_cast<size_t>(T), L->num_sms), 256, 0, st>>>(ones, 1.f, T);
@@ -423,6 +486,12 @@ int moe_dense_get_device_error(moe_dense_t* L, int* device_err) {
   MOE_CUDA(cudaDeviceSynchronize());
   MOE_CUDA(cudaMemcpy(&v, L->status, sizeof(int), cudaMemcpyDeviceToHost));
   MOE_CUDA(cudaMemset(L->status, 0, sizeof(int)));
+  if (v != 0) {  // an aborted stream-K forward leaves its counters short of their targets
+    MOE_CUDA(cudaMemset(L->sk_cnt, 0,
+                        moe::dense_streamk_counters(L->cfg.hidden, L->I_pad) * sizeof(unsigned int)));
+    L->sk_fwd = 0;
+    L->sk_rows = 0;
+  }
   *device_err = v;
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE_TIMEOUT;
 }
@@ -435,6 +504,7 @@ void moe_dense_destroy(moe_dense_t* L) {
     cudaFree(L->w_gu);
     cudaFree(L->w_dn);
     cudaFree(L->status);
+    cudaFree(L->sk_cnt);
   }
   delete L;
 }

@@ -164,10 +164,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // 16-byte global -> shared copy (cp.async, L2 only) and the arrival on an
 // mbarrier of this CTA once every prior cp.async of the thread has landed
 // (the barrier's count includes it: .noinc).

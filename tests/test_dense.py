@@ -29,6 +29,19 @@ SMALL = {
     # odd H / 128: down tiles of one 128-feature block
     "odd_hidden_fp32": replace(DENSE_WORKLOADS["dense_tiny"], name="do", T=150, hidden=384,
                                intermediate=256),
+    # up to 128 tokens with H % 256 == 0: the one-launch stream-K forward.
+    # Ragged T (not a multiple of 16), padded I, fewer (tile, K block) units
+    # than SMs in both GEMMs (CTAs with empty ranges), clamped SwiGLU:
+    "streamk_ragged_clamped": replace(DENSE_WORKLOADS["dense_tiny"], name="ds", T=77, hidden=512,
+                                      intermediate=700, act_dtype="bf16", weight_dtype="bf16",
+                                      x_dist="rmsnorm_normal", swiglu_limit=0.8),
+    # more units than SMs in both GEMMs (every CTA holds one or two segments),
+    # a full 128-token block, fp32 activations
+    "streamk_full_block_fp32": replace(DENSE_WORKLOADS["dense_tiny"], name="df", T=128,
+                                       hidden=1024, intermediate=2560),
+    # H % 256 != 0 at decode-sized T: the split-K GEMMs and reduction kernels
+    "splitk_odd_hidden": replace(DENSE_WORKLOADS["dense_tiny"], name="dk", T=40, hidden=384,
+                                 intermediate=256, act_dtype="bf16", weight_dtype="bf16"),
 }
 
 
@@ -61,7 +74,9 @@ def test_dense_small_parity(name):
 def test_dense_full_size_parity(name):
     wl = DENSE_WORKLOADS[name]
     rng = np.random.default_rng(5)
-    rows = np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 24)]))
+    # decode: every row (seconds of oracle time); prefill: sampled rows
+    rows = (np.arange(wl.T) if wl.T <= 128 else
+            np.unique(np.concatenate([[0, wl.T - 1], rng.integers(0, wl.T, 24)])))
     rel, mx = _run(wl, rows)
     assert rel <= REL_FRO and mx <= MAX_ABS_OVER_RMS, (rel, mx)
 
@@ -78,4 +93,23 @@ def test_dense_deterministic_and_batch_independent():
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert torch.equal(part, a[100:250])
+    layer.close()
+
+
+@pytest.mark.timeout(120)
+def test_dense_streamk_deterministic_and_batch_independent():
+    """The stream-K forward splits K by (tile, K block) units, which do not
+    depend on T: the same rows give bit-identical outputs in any batch of up
+    to 128 tokens, and twice in a row."""
+    wl = SMALL["streamk_ragged_clamped"]
+    inp = {k: v.cuda() for k, v in make_dense_inputs(wl, "cpu").items()}
+    layer = B.DenseMLP.from_workload(wl)
+    layer.load_inputs(inp)
+    a = layer.forward(inp["x"]).clone()
+    b = layer.forward(inp["x"]).clone()
+    part = layer.forward(inp["x"][30:50].contiguous())
+    torch.cuda.synchronize()
+    assert layer.device_error() == 0
+    assert torch.equal(a, b)
+    assert torch.equal(part, a[30:50])
     layer.close()
