@@ -109,10 +109,11 @@ def _config(wl, world):
             "l2": "inputs > L2: weights streamed from HBM each step"}
 
 
-def _traffic_record(kernel: str, workload: str, groups: int):
+def _traffic_record(kernel: str, workload: str, groups: int, rows: int = 0):
     """ncu DRAM bytes per launch of `kernel`: the committed per-group figure
-    times the launch's groups, or None once the kernel source has changed
-    since the capture."""
+    times the launch's groups, plus (where the record has one) the per-row
+    figure times the launch's token rows; None once the kernel's sources have
+    changed since the capture."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -125,7 +126,9 @@ def _traffic_record(kernel: str, workload: str, groups: int):
             h = hashlib.sha256()
             for src in f[1].split(","):
                 h.update(open(os.path.join(ROOT, src), "rb").read())
-            return int(f[3]) * groups if h.hexdigest() == f[2] else None
+            if h.hexdigest() != f[2]:
+                return None
+            return int(f[3]) * groups + (int(f[4]) * rows if len(f) > 4 else 0)
     except Exception:
         return None
     return None
@@ -374,7 +377,8 @@ def _kernel_roofline(wl, touched, stages_ms, peaks, ms_step, steps, fused=False)
             kname = "K5 gate_up fp8"
         else:
             kname = "K5 gate_up pairs" if wl.T >= 2048 else "K5 gate_up"
-        trec = _traffic_record("gate_up", wl.name, touched + 1)
+        # token rows of the launch: every routed copy plus the shared expert's
+        trec = _traffic_record("gate_up", wl.name, touched + 1, wl.T * (wl.top_k + 1))
     t_bytes = k_bytes / (peaks["hbm"] * 1e9)
     t_flops = k_flops / (tc * 1e12)
     if t_bytes >= t_flops:
@@ -450,8 +454,11 @@ def _dense_secondary(wl, a, dev, world, rank, stream, peaks):
         rl = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": tc,
               "unit": "TFLOP/s"}
     rl["frac"] = rl["achieved"] / rl["peak"]
+    # up to 128 tokens the layer is one kernel (dense_streamk_kernel): its
+    # committed ncu DRAM bytes per launch, while its sources are unchanged
+    traffic = _traffic_record("dense", wl.name, 1) if T <= 128 else None
     rl.update({"scope": "whole dense layer (gate|up + down GEMMs)", "algorithmic_bytes": nbytes,
-               "algorithmic_flops": flops, "traffic": None,
+               "algorithmic_flops": flops, "traffic": traffic,
                "peak_source": f"{peaks['source']}: hbm_gbs, bf16 {tc_kind}"})
     layer.close()
     del inp, x

@@ -96,10 +96,24 @@ def test_traffic_record_follows_the_source_hash(tmp_path, monkeypatch):
     _write_record(root, srcs, h.hexdigest(), 1000)
     monkeypatch.setattr(bench, "ROOT", root)
     assert bench._traffic_record("gate_up", "decode", 33) == 33000
+    assert bench._traffic_record("gate_up", "decode", 33, rows=500) == 33000  # no row term
     assert bench._traffic_record("gate_up", "prefill", 33) is None      # no record
     with open(os.path.join(root, "k.cuh"), "ab") as f:                  # the kernel changes
         f.write(b" ")
     assert bench._traffic_record("gate_up", "decode", 33) is None
+
+
+def test_traffic_record_row_term(tmp_path, monkeypatch):
+    """A fifth column adds bytes per token row of the launch."""
+    root = str(tmp_path)
+    with open(os.path.join(root, "k.cu"), "wb") as f:
+        f.write(b"kernel body")
+    digest = hashlib.sha256(b"kernel body").hexdigest()
+    os.makedirs(os.path.join(root, "profiles"), exist_ok=True)
+    with open(os.path.join(root, "profiles", "dram_traffic.txt"), "w") as f:
+        f.write(f"gate_up:prefill k.cu {digest} 1000 7\n")
+    monkeypatch.setattr(bench, "ROOT", root)
+    assert bench._traffic_record("gate_up", "prefill", 10, rows=100) == 10 * 1000 + 100 * 7
 
 
 def test_committed_traffic_records_match_the_sources():
@@ -112,7 +126,7 @@ def test_committed_traffic_records_match_the_sources():
         f = line.split()
         if not f or f[0].startswith("#"):
             continue
-        assert len(f) == 4, line
+        assert len(f) in (4, 5), line
         for src in f[1].split(","):
             assert os.path.exists(os.path.join(bench.ROOT, src)), src
         keys.append(f[0])
