@@ -349,11 +349,16 @@ __global__ void __launch_bounds__(1024) topk_block_kernel(const float* __restric
 // recomputing the boundary candidates in fp32 after the tensor-core router.
 constexpr int kTopkWarps = 8;
 // Token count from which the warp-per-token form runs (both forms give the
-// same bits).
-constexpr int kTopkWarpMinTokens = 8192;
+// same bits).  Measured at 4096 tokens (288 experts, tensor-core router):
+// 0.063 ms against the block form's 0.088.
+constexpr int kTopkWarpMinTokens = 2048;
 
+// Four blocks (32 warps) per SM: the candidate recomputation is bound by L2
+// latency, so warps in flight matter more than registers (64 a thread, a few
+// spilled; at 80 registers only three blocks fit and the Zipf top-k took
+// 0.284 ms instead of 0.201).
 template <int MPL>
-__global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(
+__global__ void __launch_bounds__(32 * kTopkWarps, 4) topk_warp_kernel(
     const float* __restrict__ partial, int ksplit, int T, int E, int k,
     const float* __restrict__ bias, int norm, float scale, int* __restrict__ topk_idx,
     float* __restrict__ topk_w, float* __restrict__ logits_out, TopkRefine rf) {

@@ -145,7 +145,9 @@ __device__ __forceinline__ float router_dot(const __nv_bfloat16* __restrict__ xt
   return acc;
 }
 
-// Two such dot products (experts e0 and e1) with their loads interleaved.
+// Two such dot products (experts e0 and e1) with their loads interleaved
+// (four iterations' loads in flight: more would cost the registers that let
+// more warps run; the order of each partial sum is the same either way).
 __device__ __forceinline__ void router_dot2(const __nv_bfloat16* __restrict__ xt,
                                             const float* __restrict__ w0,
                                             const float* __restrict__ w1, int H, float& r0,
@@ -156,7 +158,7 @@ __device__ __forceinline__ void router_dot2(const __nv_bfloat16* __restrict__ xt
   const uint2* x4 = reinterpret_cast<const uint2*>(xt);
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   float b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
-#pragma unroll 8
+#pragma unroll 4
   for (int i = lane; i < H / 4; i += 32) {
     const float4 u = __ldg(p0 + i);
     const float4 v = __ldg(p1 + i);
