@@ -95,7 +95,7 @@ SMALL = {
                                       shared_intermediate=128, act_dtype="bf16",
                                       weight_dtype="bf16", x_dist="rmsnorm_normal",
                                       router_std=0.1, expert_std=0.02),
-    # tensor-core router with the warp-per-token top-k (from 8192 tokens) on a
+    # tensor-core router with the warp-per-token top-k (from 2048 tokens) on a
     # small layer
     "many_tokens_small_layer": replace(WORKLOADS["tiny"], name="mt", T=8448, hidden=256,
                                        num_experts=40, top_k=6, intermediate=128,
@@ -168,7 +168,7 @@ TIES = {
                                        num_experts=32, top_k=5, intermediate=128,
                                        shared_intermediate=128, act_dtype="bf16",
                                        weight_dtype="bf16", x_dist="rmsnorm_normal"),
-    # warp-per-token top-k (from 8192 tokens)
+    # warp-per-token top-k (from 2048 tokens)
     "dup_columns_warp_topk": replace(WORKLOADS["tiny"], name="d3", T=8448, hidden=256,
                                      num_experts=40, top_k=5, intermediate=128,
                                      shared_intermediate=128, act_dtype="bf16",

@@ -68,7 +68,8 @@ def test_route_static_matches_forward_twice():
 # sizes with other kernels or another K split):
 #   * T * E * H / 128 > 1,048,576: fewer K splits than moe_forward uses
 #     (here 16 instead of 32), the usual case at the full layer's size;
-#   * T >= 8192: the warp-per-token top-k (T * E <= 1,048,576 needs E <= 124).
+#   * T >= 2048: the warp-per-token top-k (T * E <= 1,048,576 needs E <= 512;
+#     the case below has more tokens than the full layer's prefill).
 REGIMES = {
     "fewer_splits": replace(WORKLOADS["prefill"], name="ns", T=1024, num_experts=64),
     "warp_topk": replace(WORKLOADS["prefill"], name="wt", T=8448, hidden=256,
