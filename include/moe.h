@@ -253,8 +253,8 @@ int moe_check_fused_timeout(moe_layer_t* layer, const void* x, int T, void* out,
                             void* workspace, size_t ws_bytes, int limit_us,
                             int* device_status);
 
-/* Workspace bytes for moe_forward_host: moe_workspace_size plus device
- * staging for x and out. */
+/* Workspace bytes for moe_forward_host and moe_forward_host_async:
+ * moe_workspace_size plus two device staging slots for x and out. */
 int moe_workspace_size_host(const moe_layer_t* layer, int T, size_t* bytes);
 
 /* The forward from and to HOST buffers: copies x_host to the device, runs
@@ -263,6 +263,23 @@ int moe_workspace_size_host(const moe_layer_t* layer, int T, size_t* bytes);
  * copies asynchronous DMA; pageable memory also works. */
 int moe_forward_host(moe_layer_t* layer, const void* x_host, int T, void* out_host,
                      void* workspace, size_t ws_bytes, void* stream);
+
+/* The same for a stream of batches, pipelined: enqueues the copy of x_host
+ * into one of two device staging slots (alternating per call), the forward
+ * on `stream`, and the copy of the result to out_host, and returns without
+ * waiting.  The copies run on two streams owned by the layer, ordered with
+ * `stream` by events, so a call's input copy overlaps the previous call's
+ * forward and its output copy the next call's.  Host buffers must be pinned
+ * (page-locked) and left untouched until the call's copies are done: after
+ * moe_forward_host_join(layer, s) and a synchronisation of s.  Calls of one
+ * layer must come from one host thread; the workspace and the stream as in
+ * moe_forward_host. */
+int moe_forward_host_async(moe_layer_t* layer, const void* x_host, int T, void* out_host,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* Makes `stream` wait until the output copies of every
+ * moe_forward_host_async call issued so far are done (no host wait). */
+int moe_forward_host_join(moe_layer_t* layer, void* stream);
 
 /* Synchronises the device, then reads and clears the layer's device status
  * word: *device_err = 0 when no kernel reported a problem, otherwise a bit

@@ -40,7 +40,8 @@ EXPORTS = (
     "moe_dense_config_check", "moe_dense_create", "moe_dense_load_weights",
     "moe_dense_workspace_size", "moe_dense_forward", "moe_dense_get_device_error",
     "moe_dense_destroy", "moe_create_shard", "moe_set_path", "moe_forward_path",
-    "moe_check_fused_timeout", "moe_load_shard_weights",
+    "moe_check_fused_timeout", "moe_load_shard_weights", "moe_forward_host_async",
+    "moe_forward_host_join",
 )
 MOE_NUM_STAGES = 7
 STAGE_NAMES = ("router", "topk", "sort", "gather", "gate_up", "down", "combine")
@@ -114,6 +115,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_workspace_size_host.argtypes = [vp, i, ctypes.POINTER(sz)]
     lib.moe_forward.argtypes = [vp, vp, i, vp, vp, sz, vp, ctypes.POINTER(moe_routing_t)]
     lib.moe_forward_host.argtypes = [vp, vp, i, vp, vp, sz, vp]
+    lib.moe_forward_host_async.argtypes = [vp, vp, i, vp, vp, sz, vp]
+    lib.moe_forward_host_join.argtypes = [vp, vp]
     lib.moe_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
     lib.moe_status_string.argtypes = [i]
     lib.moe_status_string.restype = ctypes.c_char_p
@@ -271,6 +274,15 @@ def moe_forward(handle, x, T, out, workspace, ws_bytes, stream=None, routing=Non
 def moe_forward_host(handle, x_host, T, out_host, workspace, ws_bytes, stream=None) -> int:
     return load_library().moe_forward_host(ctypes.c_void_p(handle), x_host, T, out_host,
                                            workspace, ws_bytes, _stream(stream))
+
+
+def moe_forward_host_async(handle, x_host, T, out_host, workspace, ws_bytes, stream=None) -> int:
+    return load_library().moe_forward_host_async(ctypes.c_void_p(handle), x_host, T, out_host,
+                                                 workspace, ws_bytes, _stream(stream))
+
+
+def moe_forward_host_join(handle, stream=None) -> int:
+    return load_library().moe_forward_host_join(ctypes.c_void_p(handle), _stream(stream))
 
 
 def moe_get_device_error(handle) -> int:
@@ -488,6 +500,31 @@ class MoeLayer:
         _check(moe_forward_host(self.handle, x_host.data_ptr(), T, out_host.data_ptr(),
                                 ws.data_ptr(), ws.numel(), stream), "moe_forward_host")
         return out_host
+
+    def forward_host_async(self, x_host: torch.Tensor, out_host: torch.Tensor, stream=None):
+        """Pipelined host forward (moe_forward_host_async): returns at once;
+        out_host holds the result after forward_host_join(stream) and a
+        synchronisation of that stream.  Both tensors pinned; neither may be
+        touched before then."""
+        T = x_host.shape[0]
+        for t, name in ((x_host, "x_host"), (out_host, "out_host")):
+            if (t.device.type != "cpu" or not t.is_contiguous() or t.dtype != self.act_dtype
+                    or not t.is_pinned() or tuple(t.shape) != (T, self.cfg.hidden)):
+                raise ValueError(f"{name} must be a pinned contiguous host tensor [T, H] of "
+                                 "the layer's dtype")
+        n = moe_workspace_size_host(self.handle, T)
+        if self._ws is None or self._ws.numel() < n:
+            # a larger workspace: the calls in flight finish with the old one first
+            _check(moe_forward_host_join(self.handle, stream), "moe_forward_host_join")
+            torch.cuda.synchronize(self.device)
+        ws = self.workspace(T, host_io=True)
+        _check(moe_forward_host_async(self.handle, x_host.data_ptr(), T, out_host.data_ptr(),
+                                      ws.data_ptr(), ws.numel(), stream),
+               "moe_forward_host_async")
+
+    def forward_host_join(self, stream=None):
+        """`stream` waits for the output copies of every forward_host_async."""
+        _check(moe_forward_host_join(self.handle, stream), "moe_forward_host_join")
 
     def device_error(self) -> int:
         return moe_get_device_error(self.handle)

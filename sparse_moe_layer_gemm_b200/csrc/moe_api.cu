@@ -53,6 +53,12 @@ struct moe_layer {
   std::vector<cudaEvent_t> events;
   int timing_capacity;
   int timing_recorded;
+  // pipelined host forwards (moe_forward_host_async): input and output copy
+  // streams, per staging slot the events "input copied", "forward done" and
+  // "output copied", and the calls issued so far
+  cudaStream_t st_in, st_out;
+  cudaEvent_t ev_in[2], ev_fwd[2], ev_out[2];
+  unsigned long long host_calls;
 };
 
 namespace moe {
@@ -638,7 +644,7 @@ int moe_workspace_size_host(const moe_layer_t* L, int T, size_t* bytes) {
   if (r != MOE_OK) return r;
   const size_t el = (L->cfg.act_dtype == MOE_BF16) ? 2 : 4;
   const size_t io = align_up(static_cast<size_t>(T) * L->cfg.hidden * el, kAlign);
-  *bytes = b + 2 * io;
+  *bytes = b + 4 * io;  // two staging slots of (x, out)
   return MOE_OK;
 }
 
@@ -910,6 +916,67 @@ int moe_forward_host(moe_layer_t* L, const void* x_host, int T, void* out_host, 
   return MOE_OK;
 }
 
+int moe_forward_host_async(moe_layer_t* L, const void* x_host, int T, void* out_host,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  if (L == nullptr || T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (x_host == nullptr || out_host == nullptr) return MOE_ERR_INVALID_ARG;
+  size_t need = 0;
+  int r = moe_workspace_size_host(L, T, &need);
+  if (r != MOE_OK) return r;
+  if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  if (!L->loaded) return MOE_ERR_NOT_LOADED;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  if (L->st_in == nullptr) {  // first call: the copy streams and the slot events
+    MOE_CUDA(cudaStreamCreateWithFlags(&L->st_in, cudaStreamNonBlocking));
+    MOE_CUDA(cudaStreamCreateWithFlags(&L->st_out, cudaStreamNonBlocking));
+    for (int i = 0; i < 2; ++i) {
+      MOE_CUDA(cudaEventCreateWithFlags(&L->ev_in[i], cudaEventDisableTiming));
+      MOE_CUDA(cudaEventCreateWithFlags(&L->ev_fwd[i], cudaEventDisableTiming));
+      MOE_CUDA(cudaEventCreateWithFlags(&L->ev_out[i], cudaEventDisableTiming));
+    }
+  }
+  const size_t el = (L->cfg.act_dtype == MOE_BF16) ? 2 : 4;
+  const size_t io_bytes = static_cast<size_t>(T) * L->cfg.hidden * el;
+  const size_t io = align_up(io_bytes, kAlign);
+  const size_t base = ws_layout(L, T).total;
+  const int slot = static_cast<int>(L->host_calls & 1ull);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* x_dev = ws + base + slot * 2 * io;
+  void* out_dev = ws + base + slot * 2 * io + io;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // input: once the forward two calls back has read this slot's x
+  MOE_CUDA(cudaStreamWaitEvent(L->st_in, L->ev_fwd[slot], 0));
+  MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, L->st_in));
+  MOE_CUDA(cudaEventRecord(L->ev_in[slot], L->st_in));
+  // forward: after its input, and after the output copy two calls back has
+  // read this slot's out
+  MOE_CUDA(cudaStreamWaitEvent(st, L->ev_in[slot], 0));
+  MOE_CUDA(cudaStreamWaitEvent(st, L->ev_out[slot], 0));
+  r = moe_forward(L, x_dev, T, out_dev, workspace, base, stream, nullptr);
+  if (r != MOE_OK) return r;
+  MOE_CUDA(cudaEventRecord(L->ev_fwd[slot], st));
+  // output
+  MOE_CUDA(cudaStreamWaitEvent(L->st_out, L->ev_fwd[slot], 0));
+  MOE_CUDA(cudaMemcpyAsync(out_host, out_dev, io_bytes, cudaMemcpyDeviceToHost, L->st_out));
+  MOE_CUDA(cudaEventRecord(L->ev_out[slot], L->st_out));
+  ++L->host_calls;
+  return MOE_OK;
+}
+
+int moe_forward_host_join(moe_layer_t* L, void* stream) {
+  if (L == nullptr) return MOE_ERR_INVALID_ARG;
+  if (L->host_calls == 0) return MOE_OK;
+  DeviceGuard dg(L->device);
+  if (!dg.ok) return MOE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the last call's output copy follows every earlier one on the copy stream
+  const int last = static_cast<int>((L->host_calls - 1ull) & 1ull);
+  MOE_CUDA(cudaStreamWaitEvent(st, L->ev_out[last], 0));
+  return MOE_OK;
+}
+
 int moe_get_device_error(moe_layer_t* L, int* device_err) {
   if (L == nullptr || device_err == nullptr) return MOE_ERR_INVALID_ARG;
   DeviceGuard dg(L->device);
@@ -1026,6 +1093,15 @@ void moe_destroy(moe_layer_t* L) {
     DeviceGuard dg(L->device);
     cudaDeviceSynchronize();
     free_events(L);
+    if (L->st_in != nullptr) {
+      for (int i = 0; i < 2; ++i) {
+        cudaEventDestroy(L->ev_in[i]);
+        cudaEventDestroy(L->ev_fwd[i]);
+        cudaEventDestroy(L->ev_out[i]);
+      }
+      cudaStreamDestroy(L->st_in);
+      cudaStreamDestroy(L->st_out);
+    }
     cudaFree(L->w_gu);
     cudaFree(L->w_dn);
     cudaFree(L->sc_gu);

@@ -88,6 +88,9 @@ def test_null_arguments_rejected_without_cuda(lib):
     assert lib.moe_workspace_size_host(None, 64, ctypes.byref(n)) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_forward(None, None, 64, None, None, 0, None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_forward_host(None, None, 64, None, None, 0, None) == B.MOE_ERR_INVALID_ARG
+    assert (lib.moe_forward_host_async(None, None, 64, None, None, 0, None) ==
+            B.MOE_ERR_INVALID_ARG)
+    assert lib.moe_forward_host_join(None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_load_weights(*([None] * 10)) == B.MOE_ERR_INVALID_ARG
     v = ctypes.c_int()
     assert lib.moe_get_device_error(None, ctypes.byref(v)) == B.MOE_ERR_INVALID_ARG
