@@ -272,8 +272,9 @@ int moe_forward_host(moe_layer_t* layer, const void* x_host, int T, void* out_ho
  * forward and its output copy the next call's.  Host buffers must be pinned
  * (page-locked) and left untouched until the call's copies are done: after
  * moe_forward_host_join(layer, s) and a synchronisation of s.  Calls of one
- * layer must come from one host thread; the workspace and the stream as in
- * moe_forward_host. */
+ * layer must come from one host thread, on one stream, with one workspace
+ * (of moe_workspace_size_host bytes for the largest T); a call with another
+ * T than the previous one first waits for every earlier call's copies. */
 int moe_forward_host_async(moe_layer_t* layer, const void* x_host, int T, void* out_host,
                            void* workspace, size_t ws_bytes, void* stream);
 

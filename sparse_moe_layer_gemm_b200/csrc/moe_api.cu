@@ -59,6 +59,7 @@ struct moe_layer {
   cudaStream_t st_in, st_out;
   cudaEvent_t ev_in[2], ev_fwd[2], ev_out[2];
   unsigned long long host_calls;
+  int host_T;  // the last call's T (the staging slots' offsets depend on it)
 };
 
 namespace moe {
@@ -946,6 +947,10 @@ int moe_forward_host_async(moe_layer_t* L, const void* x_host, int T, void* out_
   void* x_dev = ws + base + slot * 2 * io;
   void* out_dev = ws + base + slot * 2 * io + io;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // a new T moves the staging slots: start after every earlier call is done
+  if (L->host_calls > 0 && T != L->host_T)
+    MOE_CUDA(cudaStreamWaitEvent(L->st_in, L->ev_out[(L->host_calls - 1ull) & 1ull], 0));
+  L->host_T = T;
   // input: once the forward two calls back has read this slot's x
   MOE_CUDA(cudaStreamWaitEvent(L->st_in, L->ev_fwd[slot], 0));
   MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, io_bytes, cudaMemcpyHostToDevice, L->st_in));

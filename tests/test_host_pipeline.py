@@ -24,8 +24,11 @@ def test_pipelined_host_forward_matches_device_forward(T):
     g = torch.Generator().manual_seed(3)
     xs = [(inp["x"].float().cpu() * (0.5 + i) + 0.01 * torch.randn(inp["x"].shape, generator=g))
           .to(torch.bfloat16).pin_memory() for i in range(5)]
+    # two more batches of another T (the staging slots move)
+    xs += [x[: T // 2 + 1].clone().pin_memory() for x in xs[:2]]
     outs = [torch.empty_like(x).pin_memory() for x in xs]
     stream = torch.cuda.Stream()
+    layer.workspace(T, host_io=True)  # sized for the largest T up front
     for x, o in zip(xs, outs):
         layer.forward_host_async(x, o, stream=stream)
     layer.forward_host_join(stream=stream)
