@@ -1,14 +1,14 @@
 // The dense SwiGLU MLP at decode-sized T (at most kSkMaxTokens tokens) in ONE
 // persistent launch: stream-K over both GEMMs in 2 kSkGroups passes,
-// synchronised by data flow.  With two groups:
+// synchronised by data flow.  With one group (the setting; more groups were
+// measured slower):
 //
-//   A1 gate|up of the first half of the h tiles   fp32 partials per segment
-//   A2 gate|up of the second half                 (meanwhile: A1 reduced,
-//                                                  h = silu(min(a, L)) *
-//                                                  clip(u, -L, L), bf16)
-//   B1 down over the K blocks of the first half   (meanwhile: A2 reduced)
-//   B2 down over the K blocks of the second half
-//      then out = the B1 and B2 partials summed, bf16 or fp32
+//   A  gate|up                                    fp32 partials per segment
+//      reduced per h tile once its segments are stored:
+//      h = silu(min(a, L)) * clip(u, -L, L), bf16
+//   B  down, each K block's h rows loaded once they exist (the down weights
+//      stream as soon as a CTA's ring is free of gate|up stages)
+//      then out = the down partials summed, bf16 or fp32
 //
 // (sglang-jax issue #1367 "Support Step 3.5 Flash", section "Model
 // configuration", MLP bullet: the first three layers are dense, intermediate
@@ -26,13 +26,14 @@
 // (fixed by the grid size: deterministic, and independent of T and of the
 // batch).
 //
-// Why the passes: the down GEMM needs h, and h needs every gate|up segment.
-// With gate|up in groups, a group's reduction runs on dedicated warps while
-// the SM streams the next group, and the down pass of a group needs only
-// that group's h: the weights stream back to back and only the final
-// reduction is exposed.  (Under full HBM load every global round trip --
-// a counter, a fence, an L2 load -- takes microseconds, so the reductions
-// never run on the warps that drain the accumulators.)
+// Passes: the down GEMM needs h, and h needs every gate|up segment.  With
+// gate|up split into groups of h tiles, a group's reduction could run while
+// the SM streams the next group, and a down pass would need only its group's
+// h; but the extra segment boundaries cost more partials than the overlap
+// gains, so the kernel runs one group (two passes).  Under full HBM load
+// every global round trip -- a counter, a fence, an L2 load -- takes
+// microseconds, so the reductions never run on the warps that drain the
+// accumulators.
 //
 // No grid barrier: counters in device memory owned by the layer carry the
 // dependencies -- per tile of each pass the stored segments (one count per
