@@ -101,12 +101,24 @@ def _sig(v, n=4):
     return int(r) if nd <= 0 else r
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
 def _config(wl, world):
     """The config dict both arms print (identical for the same workload)."""
+    layer_bytes = (wl.num_experts + 1) * wl.weight_bytes_per_expert
+    l2 = ("inputs > L2: weights streamed from HBM each step" if layer_bytes > L2_BYTES else
+          "L2-resident: the whole layer fits in L2 (launch latency, not a roofline case)")
     return {"workload": wl.name, "T": wl.T, "hidden": wl.hidden, "experts": wl.num_experts,
             "top_k": wl.top_k, "intermediate": wl.intermediate, "shared_experts": 1,
-            "parallelism": f"replicas x{world} (weak)",
-            "l2": "inputs > L2: weights streamed from HBM each step"}
+            "parallelism": f"replicas x{world} (weak)", "l2": l2}
+
+
+def _dtype(wl) -> str:
+    """The arithmetic type of the expert GEMMs: fp32 weights take the fp32
+    expert path (tf32 tensor cores over a two-term split, fp32-level
+    results); bf16 and FP8 weights multiply in bf16."""
+    return "f32" if wl.weight_dtype == "f32" else "bf16"
 
 
 def _traffic_record(kernel: str, workload: str, groups: int, rows: int = 0):
@@ -617,7 +629,8 @@ def run_ours(a):
                  "path": "fused" if fused2 else "multi-launch"}
         if wl2.weight_dtype != "bf16":
             entry["weights"] = {"fp8": "fp8_e4m3 codes + fp32 per-feature scales (bf16 MMA)",
-                                "f32": "fp32 (rounded to bf16 at load)"}[wl2.weight_dtype]
+                                "f32": "fp32: tf32 tensor cores over a two-term split of "
+                                       "every operand (fp32 expert path)"}[wl2.weight_dtype]
         if wl2.name == "tiny":
             entry["l2"] = "L2-resident (16 KB experts): launch latency, not a roofline case"
         secondary.append(entry)
@@ -636,7 +649,7 @@ def run_ours(a):
         full = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic",
             "config": _config(wl, world), "roofline": kr, "layer_roofline": lr,
             "stage_ms": stages,
             "routing": {"touched_experts": touched, "max_rows_per_expert": max_rows},
@@ -804,7 +817,7 @@ def run_ep(a):
         full = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "strong", "vs_baseline": None, "dtype": _dtype(wl), "data": "synthetic",
             "config": ep_config(wl, world), "roofline": kr, "layer_roofline": lr,
             "stage_ms": stages, "routing": {}, "cpu_baseline": None, "e2e": e2e,
             "gpu_launches": launches, "clocks": clocks, "secondary": secondary,

@@ -22,17 +22,24 @@
  * Arithmetic: the router, the scores, the selection and the gate weights are
  * fp32 on the CUDA cores (from 512 bf16 tokens the logits are first
  * approximated on the tensor cores and every expert near the selection
- * boundary is recomputed in fp32).  The expert GEMMs are bf16 x bf16 with
- * fp32 accumulation: fp32 x and fp32 expert weights (the act_dtype /
- * weight_dtype MOE_F32 case) are rounded to bf16 (round to nearest even) on
- * the way in, h = SwiGLU(...) and each expert's weighted output row are
- * rounded to bf16, and the k + 1 rows of a token are summed in fp32 and
- * rounded once to the output dtype.  Error budget: each bf16 rounding is a
- * relative error of at most 2^-9; with independent rounding errors over
- * K-term sums the output's relative Frobenius error stays near 2^-9 times a
- * small constant (measured against the fp64 definition: ~5e-3 with fp32
- * inputs of the tiny shape, ~3e-3 at the full layer), inside the 1e-2 bar.
- * There is no fp32 or tf32 expert GEMM.
+ * boundary is recomputed in fp32).  The expert GEMMs follow weight_dtype:
+ *  - bf16 (and FP8) weights: bf16 x bf16 with fp32 accumulation.  fp32 x is
+ *    rounded to bf16 (round to nearest even) on the way in, h = SwiGLU(...)
+ *    and each expert's weighted output row are rounded to bf16, and the
+ *    k + 1 rows of a token are summed in fp32 and rounded once to the output
+ *    dtype.  Error budget: each bf16 rounding is a relative error of at most
+ *    2^-9; with independent rounding errors over K-term sums the output's
+ *    relative Frobenius error stays near 2^-9 times a small constant (~3e-3
+ *    measured at the full layer against the fp64 definition).
+ *  - fp32 weights (weight_dtype MOE_F32): the fp32 expert path.  Every GEMM
+ *    operand (weights, x, h) is split into two tf32 terms v = v_hi + v_lo
+ *    (v_hi = v rounded to tf32, v_lo = v - v_hi), and the tf32 tensor cores
+ *    accumulate w_hi x_hi + w_lo x_hi + w_hi x_lo in fp32: each product to
+ *    within ~2^-21 of fp32's.  h and the output rows stay fp32 and are summed
+ *    in fp32.  Measured against the fp64 definition: ~6e-6 relative
+ *    Frobenius error on the tiny fp32 layer.  Costs: 8 bytes of device memory
+ *    per expert weight and three MMA passes; always on one-SM tiles (no CTA
+ *    pairs, no fused forward).
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers unless the name says _host.
@@ -142,9 +149,10 @@ int moe_create(const moe_config_t* cfg, moe_layer_t** out);
 int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count,
                      int with_shared, moe_layer_t** out);
 
-/* Copies the weights into the layer's packed bf16 layout on `stream`
- * (K-major weight rows; gate and up interleaved in blocks of 128 rows; fp32
- * expert weights are rounded to bf16).  router_w [H, E] and router_bias [E]
+/* Copies the weights into the layer's packed layout on `stream` (K-major
+ * weight rows; gate and up interleaved in blocks of 128 rows): bf16, or for
+ * fp32 expert weights the fp32 expert path's two tf32 terms of each weight
+ * (see the arithmetic note at the top).  router_w [H, E] and router_bias [E]
  * are fp32 and kept fp32; router_bias may be NULL (zero bias).  The expert
  * pointers have the config's weight_dtype (F32 or BF16; a layer created with
  * MOE_FP8_E4M3 weights returns MOE_ERR_INVALID_ARG: it loads through

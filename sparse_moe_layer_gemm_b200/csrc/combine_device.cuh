@@ -20,6 +20,20 @@ __device__ __forceinline__ void add8(float (&acc)[8], const __nv_bfloat16* p) {
   }
 }
 
+// fp32 rows (the fp32 expert path)
+__device__ __forceinline__ void add8(float (&acc)[8], const float* p) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  acc[0] += a.x;
+  acc[1] += a.y;
+  acc[2] += a.z;
+  acc[3] += a.w;
+  acc[4] += b.x;
+  acc[5] += b.y;
+  acc[6] += b.z;
+  acc[7] += b.w;
+}
+
 // acc += the 8 bf16 values held in q (already loaded)
 __device__ __forceinline__ void add8(float (&acc)[8], const uint4& q) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
@@ -47,8 +61,8 @@ __device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
 // Token t's output row, by all threads of the block (threadIdx.x / blockDim.x
 // strides over the row's 8-element vectors); rows_s: k + 1 ints of shared
 // memory.  Ends with a __syncthreads, so rows_s may be reused at once.
-template <typename TO>
-__device__ __forceinline__ void combine_token(int t, const __nv_bfloat16* __restrict__ y,
+template <typename TO, typename TY>
+__device__ __forceinline__ void combine_token(int t, const TY* __restrict__ y,
                                               const int* __restrict__ pos, int T, int k, int H,
                                               int with_shared, TO* __restrict__ out, int* rows_s) {
   if (threadIdx.x < k) rows_s[threadIdx.x] = pos[static_cast<size_t>(t) * k + threadIdx.x];

@@ -9,6 +9,8 @@
 //   split-K partials (dense MLP at small T): part z of a single group's
 //                  product over K slice z, raw fp32 accumulators per packed
 //                  weight row; a reduction kernel finishes the layer.
+//   fp32 expert path (fp32 weights): the same K5 / K6 on the tf32 tensor cores
+//                  over the three-term split of tf32.cuh, h and y kept fp32.
 //   K1 (router, large T):  logits = x . W_r on the bf16 tensor cores: W_r =
 //                  W1 + W2 + W3 split into three bf16 terms concatenated along
 //                  K; the tiles of part z accumulate x . Wz (each bf16 x bf16
@@ -33,7 +35,8 @@
 //                 (BLOCKS 128-feature blocks; gate|up blocks are 128 gate rows
 //                 then 128 up rows) x 64 K and one box of token rows (32 rows
 //                 for tiles of <= 32 tokens, else 128), 128-byte swizzle.
-//   warps 1..NI   tcgen05.mma issuers (kind::f16, bf16 x bf16 -> fp32 TMEM):
+//   warps 1..NI   tcgen05.mma issuers (kind::f16, bf16 x bf16 -> fp32 TMEM;
+//                 the fp32 path kind::tf32 on the same 128-byte rows):
 //                 each owns every NI-th 128-row accumulator of the tile (gate
 //                 and up, or two weight blocks) and keeps its own stage waits
 //                 and commits, so the issue latencies of the accumulator
@@ -46,6 +49,7 @@
 #include "gemm_common.cuh"
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
+#include "tf32.cuh"
 
 namespace moe {
 
@@ -54,10 +58,13 @@ namespace {
 using namespace gemm;
 
 // Tile shape: BLOCKS weight blocks of 128 features per tile (gate|up: each
-// block is 128 gate rows + 128 up rows), BN tokens per tile, BK = 64 reduction
-// elements (one 128-byte swizzled row) per pipeline stage.
-template <int MODE, int BLOCKS, int BN_>
+// block is 128 gate rows + 128 up rows), BN tokens per tile, one 128-byte
+// swizzled row of reduction elements per pipeline stage: BK = 64 bf16, or 32
+// fp32 for the tf32 path (TF).  Either way a stage row takes four MMAs of 32
+// bytes of K (16 bf16 or 8 tf32 elements).
+template <int MODE, int BLOCKS, int BN_, bool TF_ = false>
 struct Shape {
+  static constexpr bool TF = TF_;
   static constexpr bool GU = MODE == kModeGateUp;
   // router with BLOCKS = 2: one weight block, the tile's tokens split into two
   // halves, one accumulator (and issuer) each
@@ -65,8 +72,8 @@ struct Shape {
   // fp32 outputs straight from the accumulators (no tables, no TMA stores)
   static constexpr bool F32OUT = MODE == kModeRouter || MODE == kModePartial;
   static constexpr int BN = BN_;
-  static constexpr int BK = kBK;
-  static constexpr int ROW = BK * 2;                        // bytes per operand row in SMEM
+  static constexpr int BK = TF ? kBK32 : kBK;
+  static constexpr int ROW = 128;                           // bytes per operand row in SMEM
   static constexpr int ACCS = BLOCKS * (GU ? 2 : 1);       // 128-row accumulators per tile
   static constexpr int NI = ACCS >= 2 ? 2 : 1;             // MMA-issuing warps
   static constexpr int THREADS = 32 * (1 + NI + 4);
@@ -101,33 +108,42 @@ struct Shape {
   // descriptor start-address field: 14 bits of (address >> 4), no carries
   static_assert(1024 + STAGES * STAGE_BYTES + BAR_BYTES <= 256 * 1024, "descriptor range");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(!TF || MODE == kModeGateUp || MODE == kModeDown, "tf32: expert GEMMs only");
 };
 
 // tcgen05.mma issue without a memory clobber: the MMA reads shared memory
 // the TMA wrote (ordered by the full-barrier wait and the tcgen05 fence) and
 // writes TMEM; its completion is ordered by the (volatile, clobbering)
 // commit that follows it.
+template <bool TF>
 __device__ __forceinline__ void mma_issue(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+  if (TF)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // tmB / tmBsh: token-row operands with kBBoxRows-row boxes; tmBw / tmBshw
 // the same tensors with BN-row boxes, used when a tile has more than
 // kBBoxRows tokens (one TMA instruction per stage instead of several).
-template <int MODE, int BLOCKS, int BN>
-__global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
+template <int MODE, int BLOCKS, int BN, bool TF>
+__global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN, TF>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBsh,
                         const __grid_constant__ CUtensorMap tmBw,
                         const __grid_constant__ CUtensorMap tmBshw,
                         const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
-  using S = Shape<MODE, BLOCKS, BN>;
+  using S = Shape<MODE, BLOCKS, BN, TF>;
   constexpr bool GU = S::GU;
   constexpr int BK = S::BK;
   extern __shared__ uint8_t smem_raw[];
@@ -219,16 +235,23 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
             ok = false;
             break;
           }
+          // K columns of this stage; the tf32 path's terms hi.hi, lo.hi,
+          // hi.lo read the lo half (kb_term k-blocks in) of A, resp. B
+          int ak = a_k0 + kb * BK, bk = b_k0 + kb * BK;
+          if (TF) {
+            const int term = kb / p.kb_term;
+            const int kk = (kb - term * p.kb_term) * BK;
+            ak = (term == 1 ? p.kb_term * BK : 0) + kk;
+            bk = (term == 2 ? p.kb_term * BK : 0) + kk;
+          }
           const uint32_t fb = full0 + 8 * s;
           mbar_arrive_expect_tx(fb, bytes);
           const uint32_t sa = smem_u32(smem + s * S::STAGE_BYTES);
 #pragma unroll
           for (int i = 0; i < S::A_LOADS; ++i)
-            tma_load_2d(sa + i * S::A_BOX * S::ROW, &tmA, fb, a_k0 + kb * BK, a_row + i * S::A_BOX,
-                        pol_a);
+            tma_load_2d(sa + i * S::A_BOX * S::ROW, &tmA, fb, ak, a_row + i * S::A_BOX, pol_a);
           for (int i = 0; i < nbox; ++i)
-            tma_load_2d(sa + S::A_BYTES + i * kBN * S::ROW, mb, fb, b_k0 + kb * BK,
-                        b_row + i * kBN, pol_b);
+            tma_load_2d(sa + S::A_BYTES + i * kBN * S::ROW, mb, fb, bk, b_row + i * kBN, pol_b);
           ++it;
         }
         if (!ok) break;
@@ -253,7 +276,8 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
         // for a ragged tile's empty second half: it only commits)
         const int n_me = S::TOKSPLIT ? min(S::ACC_N, max(0, t.n_valid - me * S::ACC_N)) : t.n_valid;
         const int n_mma = (n_me + 15) & ~15;
-        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma > 0 ? n_mma : 16);
+        const uint32_t idesc = TF ? idesc_tf32_f32(kBM, n_mma > 0 ? n_mma : 16)
+                                  : idesc_bf16_f32(kBM, n_mma > 0 ? n_mma : 16);
         const uint32_t buf = S::NBUF == 2 ? (tc & 1u) : 0u;
         const uint32_t tph = (S::NBUF == 2 ? (tc >> 1) : tc) & 1u;
         if (!mbar_wait(tempty0 + 8 * buf, tph ^ 1u, abort_flag, p.status)) break;
@@ -274,7 +298,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
           const uint32_t acc0 = kb != 0 ? 1u : 0u;
           if (n_mma > 0) {
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
+            for (int kk = 0; kk < S::ROW / 32; ++kk)
 #pragma unroll
               for (int j = 0; j < S::ACCS / S::NI; ++j) {
                 const int a = j * S::NI + me;
@@ -282,7 +306,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
                 // own half of the token rows
                 const int a_off = S::TOKSPLIT ? 0 : a * kBM * S::ROW;
                 const int b_off = S::TOKSPLIT ? a * S::ACC_N * S::ROW : 0;
-                mma_issue(d + a * S::ACC_N, ad + static_cast<uint64_t>((a_off + kk * 32) >> 4),
+                mma_issue<TF>(d + a * S::ACC_N, ad + static_cast<uint64_t>((a_off + kk * 32) >> 4),
                           bd + static_cast<uint64_t>((b_off + kk * 32) >> 4), idesc,
                           kk == 0 ? acc0 : 1u);
               }
@@ -311,7 +335,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
                                            4 * 2 * kEpiRows * 32 * 2) +
                   (warp - (1 + S::NI)) * BN;
     uint32_t chunks = 0;  // TMA-store chunks this warp has issued
-    if (!S::F32OUT && lane == 0) prefetch_tmap(&tmOut);
+    if (!S::F32OUT && !TF && lane == 0) prefetch_tmap(&tmOut);
     // Writes rows [c0, c0 + 16) of this lane's output feature.  A chunk whose
     // 16 rows all belong to the tile goes through a staging buffer and one
     // TMA store of 16 x 32 values; a ragged one is stored directly, so no row
@@ -395,6 +419,45 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
               if (keep && c0 + i < n_b)
                 lp[static_cast<size_t>(c0 + i) * p.out_ld] = __uint_as_float(ra[i]);
           }
+        } else if (GU && TF) {
+          // h fp32 as its tf32 split: hi in columns [0, ld / 2), lo after
+          float* hp = p.out_f32 + row0 * p.out_ld + feat;
+          const int lo_off = p.out_ld / 2;
+          const float L = (t.g == p.E) ? p.limit_shared : p.limit;
+          const uint32_t tg = taddr + (2 * b) * BN, tu = taddr + (2 * b + 1) * BN;
+          for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t ra[16], rb[16];
+            tmem_ld_x16(tg + c0, ra);
+            tmem_ld_x16(tu + c0, rb);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float a = __uint_as_float(ra[i]);
+              float u = __uint_as_float(rb[i]);
+              if (L > 0.f) {
+                a = fminf(a, L);
+                u = fminf(fmaxf(u, -L), L);
+              }
+              float hi, lo;
+              tf32_split(a / (1.0f + expf(-a)) * u, hi, lo);
+              if (c0 + i < t.n_valid) {
+                hp[static_cast<size_t>(c0 + i) * p.out_ld] = hi;
+                hp[static_cast<size_t>(c0 + i) * p.out_ld + lo_off] = lo;
+              }
+            }
+          }
+        } else if (TF) {
+          // y fp32
+          float* yp = p.out_f32 + row0 * p.out_ld + feat;
+          for (int c0 = 0; c0 < t.n_valid; c0 += 16) {
+            uint32_t ra[16];
+            tmem_ld_x16(taddr + b * BN + c0, ra);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c0 + i < t.n_valid)
+                yp[static_cast<size_t>(c0 + i) * p.out_ld] = __uint_as_float(ra[i]) * wbuf[c0 + i];
+          }
         } else if (GU) {
           __nv_bfloat16* outp = p.out + row0 * p.out_ld + feat;
           const float L = (t.g == p.E) ? p.limit_shared : p.limit;
@@ -435,7 +498,7 @@ __global__ void __launch_bounds__(Shape<MODE, BLOCKS, BN>::THREADS, 1)
       if (lane == 0) mbar_arrive(tempty0 + 8 * buf);
       ++tc;
     }
-    if (!S::F32OUT && lane == 0) bulk_wait_group_all();  // h / y fully written
+    if (!S::F32OUT && !TF && lane == 0) bulk_wait_group_all();  // h / y fully written
   }
 
   tc_fence_before();
@@ -456,10 +519,14 @@ using DnCfg2 = Shape<kModeDown, 2, 128>;
 using DnCfg1 = Shape<kModeDown, 1, 128>;
 using RtCfg = Shape<kModeRouter, 2, 256>;  // 256-token tiles, one accumulator per half
 using PtCfg = Shape<kModePartial, 2, 128>;  // two 128-row blocks, 128-token tiles
+// the fp32 path: the gate|up and down configurations on tf32
+using GuCfgTf = Shape<kModeGateUp, 1, 128, true>;
+using DnCfg2Tf = Shape<kModeDown, 2, 128, true>;
+using DnCfg1Tf = Shape<kModeDown, 1, 128, true>;
 
 template <typename S, int MODE, int BLOCKS>
 cudaError_t set_smem() {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BLOCKS, S::BN>,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<MODE, BLOCKS, S::BN, S::TF>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(S::SMEM));
 }
@@ -472,27 +539,46 @@ cudaError_t gemm_configure_device() {
   if ((e = set_smem<DnCfg2, kModeDown, 2>()) != cudaSuccess) return e;
   if ((e = set_smem<DnCfg1, kModeDown, 1>()) != cudaSuccess) return e;
   if ((e = set_smem<PtCfg, kModePartial, 2>()) != cudaSuccess) return e;
+  if ((e = set_smem<GuCfgTf, kModeGateUp, 1>()) != cudaSuccess) return e;
+  if ((e = set_smem<DnCfg2Tf, kModeDown, 2>()) != cudaSuccess) return e;
+  if ((e = set_smem<DnCfg1Tf, kModeDown, 1>()) != cudaSuccess) return e;
   return set_smem<RtCfg, kModeRouter, 2>();
 }
 
 int gemm_down_blocks(int H) { return (H / kBM) % 2 == 0 ? 2 : 1; }
 
 cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
-  return launch_pdl(grouped_gemm_kernel<kModeGateUp, 1, 128>, dim3(grid), dim3(GuCfg::THREADS),
+  return launch_pdl(grouped_gemm_kernel<kModeGateUp, 1, 128, false>, dim3(grid), dim3(GuCfg::THREADS),
                     GuCfg::SMEM, st, m.a, m.b, m.bsh, m.bw, m.bshw, m.out, p);
 }
 
 cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
                              cudaStream_t st) {
   if (blocks == 2)
-    return launch_pdl(grouped_gemm_kernel<kModeDown, 2, 128>, dim3(grid), dim3(DnCfg2::THREADS),
+    return launch_pdl(grouped_gemm_kernel<kModeDown, 2, 128, false>, dim3(grid), dim3(DnCfg2::THREADS),
                       DnCfg2::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
-  return launch_pdl(grouped_gemm_kernel<kModeDown, 1, 128>, dim3(grid), dim3(DnCfg1::THREADS),
+  return launch_pdl(grouped_gemm_kernel<kModeDown, 1, 128, false>, dim3(grid), dim3(DnCfg1::THREADS),
                     DnCfg1::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 
+cudaError_t launch_gemm_gate_up_tf32(const GemmMaps& m, const GemmParams& p, int grid,
+                                     cudaStream_t st) {
+  return launch_pdl(grouped_gemm_kernel<kModeGateUp, 1, 128, true>, dim3(grid),
+                    dim3(GuCfgTf::THREADS), GuCfgTf::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.b, p);
+}
+
+cudaError_t launch_gemm_down_tf32(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
+                                  cudaStream_t st) {
+  if (blocks == 2)
+    return launch_pdl(grouped_gemm_kernel<kModeDown, 2, 128, true>, dim3(grid),
+                      dim3(DnCfg2Tf::THREADS), DnCfg2Tf::SMEM, st, m.a, m.b, m.b, m.bw, m.bw,
+                      m.b, p);
+  return launch_pdl(grouped_gemm_kernel<kModeDown, 1, 128, true>, dim3(grid),
+                    dim3(DnCfg1Tf::THREADS), DnCfg1Tf::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.b, p);
+}
+
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
-  return launch_pdl(grouped_gemm_kernel<kModeRouter, 2, 256>, dim3(grid), dim3(RtCfg::THREADS),
+  return launch_pdl(grouped_gemm_kernel<kModeRouter, 2, 256, false>, dim3(grid), dim3(RtCfg::THREADS),
                     RtCfg::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 
@@ -501,7 +587,7 @@ cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid,
 namespace moe {
 
 cudaError_t launch_gemm_partial(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st) {
-  return launch_pdl(grouped_gemm_kernel<kModePartial, 2, 128>, dim3(grid), dim3(PtCfg::THREADS),
+  return launch_pdl(grouped_gemm_kernel<kModePartial, 2, 128, false>, dim3(grid), dim3(PtCfg::THREADS),
                     PtCfg::SMEM, st, m.a, m.b, m.b, m.bw, m.bw, m.out, p);
 }
 

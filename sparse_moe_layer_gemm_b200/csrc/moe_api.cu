@@ -24,11 +24,13 @@ struct moe_layer {
   int num_sms;
   int I_pad;
   int fp8;              // expert weights are E4M3 codes (one byte each) + scales
+  int f32;              // fp32 expert weights: the fp32 expert path (tf32 split)
   int first;            // expert shard: the layer holds experts [first, first + E_loc)
   int E_loc;            //   (E_loc = E: all of them)
   int with_shared;      //   and the shared expert if set
-  void* w_gu;           // [(E+1) * 2 * I_pad, H] bf16 or E4M3 codes
-  void* w_dn;           // [(E+1) * H, I_pad] bf16 or E4M3 codes
+  void* w_gu;           // [(E+1) * 2 * I_pad, H] bf16 or E4M3 codes (fp32 path:
+                        //   [.., 2H] fp32, the tf32 split's hi | lo halves)
+  void* w_dn;           // [(E+1) * H, I_pad] bf16 or E4M3 codes (fp32 path: [.., 2 I_pad])
   float* sc_gu;         // FP8: scale of each packed gate|up row [(E+1) * 2 * I_pad]
   float* sc_dn;         // FP8: scale of each packed down row [(E+1) * H]
   float* router_w;      // [H, E]
@@ -88,6 +90,23 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   cuuint32_t box[2] = {static_cast<cuuint32_t>(moe::kBK), box_rows};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// fp32 [rows, cols] row-major, box = 32 columns (128 bytes) x box_rows, 128B
+// swizzle (the fp32 expert path's tf32 operands); out-of-range reads zero.
+bool encode_f32_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(moe::kBK32), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -155,6 +174,7 @@ using moe::encode_bf16_gate_up_pair;
 using moe::encode_bf16_kblocks;
 using moe::encode_bf16_kpair;
 using moe::encode_bf16_store;
+using moe::encode_f32_2d;
 
 namespace {
 
@@ -207,7 +227,8 @@ WsLayout ws_layout(const moe_layer* L, int T) {
   w.ksplit = router_ksplit(T, H, E);
   w.nch = (T + moe::kSortChunk - 1) / moe::kSortChunk;
   w.rows_routed = T * k;
-  w.rows_xperm = T * k + (c.act_dtype == MOE_F32 ? T : 0);
+  // fp32 x, or the fp32 expert path: the shared expert's rows are in x_perm too
+  w.rows_xperm = T * k + (c.act_dtype == MOE_F32 || L->f32 ? T : 0);
   w.rows_all = T * k + T;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -235,9 +256,11 @@ WsLayout ws_layout(const moe_layer* L, int T) {
   w.perm = take(static_cast<size_t>(T) * k * sizeof(int));
   w.pos = take(static_cast<size_t>(T) * k * sizeof(int));
   w.w_perm = take(static_cast<size_t>(w.rows_all) * sizeof(float));
-  w.x_perm = take(static_cast<size_t>(w.rows_xperm) * H * 2);
-  w.h = take(static_cast<size_t>(w.rows_all) * L->I_pad * 2);
-  w.y = take(static_cast<size_t>(w.rows_all) * H * 2);
+  // the fp32 expert path keeps x_perm and h as fp32 [hi | lo] and y as fp32
+  const size_t xh = L->f32 ? 8 : 2, ye = L->f32 ? 4 : 2;
+  w.x_perm = take(static_cast<size_t>(w.rows_xperm) * H * xh);
+  w.h = take(static_cast<size_t>(w.rows_all) * L->I_pad * xh);
+  w.y = take(static_cast<size_t>(w.rows_all) * H * ye);
   // expert shard: the selection in local expert ids (-1: another shard's)
   const bool shard = L->E_loc != E || L->first != 0;
   w.local_idx = shard ? take(static_cast<size_t>(T) * k * sizeof(int)) : 0;
@@ -258,7 +281,7 @@ constexpr bool kFusedGatherPhase = true;
 // The fused persistent forward's conditions (see MOE_PATH_FUSED in moe.h).
 bool fused_eligible(const moe_layer* L, int T) {
   const moe_config_t& c = L->cfg;
-  return c.act_dtype == MOE_BF16 && !L->fp8 && T >= moe::kPairMinTokens &&
+  return c.act_dtype == MOE_BF16 && !L->fp8 && !L->f32 && T >= moe::kPairMinTokens &&
          (c.hidden / moe::kBM) % 2 == 0 && c.num_experts <= moe::kFusedMaxExperts &&
          L->E_loc == c.num_experts && L->first == 0 && L->with_shared != 0;
 }
@@ -432,6 +455,7 @@ int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count
   L->E_loc = expert_count;
   L->with_shared = with_shared;
   L->fp8 = cfg->weight_dtype == MOE_FP8_E4M3 ? 1 : 0;
+  L->f32 = cfg->weight_dtype == MOE_F32 ? 1 : 0;
   L->I_pad = (cfg->intermediate + 127) / 128 * 128;
   L->E_pad = (cfg->num_experts + 127) / 128 * 128;
   if (cudaGetDevice(&L->device) != cudaSuccess ||
@@ -443,7 +467,7 @@ int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count
   // expert weights: the shard's experts + the shared expert (group E_loc);
   // the router covers all experts
   const size_t H = cfg->hidden, E = cfg->num_experts, Ip = L->I_pad, El = L->E_loc;
-  const size_t el = L->fp8 ? 1 : 2;
+  const size_t el = L->fp8 ? 1 : L->f32 ? 8 : 2;  // bytes per weight (fp32: hi + lo)
   const size_t gu_bytes = (El + 1) * 2 * Ip * H * el, dn_bytes = (El + 1) * H * Ip * el;
   if (moe::gemm_configure_device() != cudaSuccess ||
       moe::gemm_fp8_configure_device() != cudaSuccess ||
@@ -466,12 +490,15 @@ int moe_create_shard(const moe_config_t* cfg, int expert_first, int expert_count
   }
   // (FP8 codes are read with plain bulk copies: no tensor maps)
   const bool maps_ok =
-      L->fp8 || (encode_bf16_2d(&L->tm_gu, L->w_gu, (El + 1) * 2 * Ip, H, 2 * moe::kBM) &&
-                 encode_bf16_gate_up_pair(&L->tm_gu_pw, L->w_gu, (El + 1) * 2 * Ip, H, 2) &&
-                 encode_bf16_gate_up_pair(&L->tm_gu_pn, L->w_gu, (El + 1) * 2 * Ip, H, 3) &&
-                 encode_bf16_2d(&L->tm_dn, L->w_dn, (El + 1) * H, Ip, moe::kBM) &&
-                 encode_bf16_kblocks(&L->tm_dn_pw, L->w_dn, (El + 1) * H, Ip, moe::kBM, 2) &&
-                 encode_bf16_kblocks(&L->tm_dn_pn, L->w_dn, (El + 1) * H, Ip, moe::kBM, 3));
+      L->fp8 ||
+      (L->f32 && encode_f32_2d(&L->tm_gu, L->w_gu, (El + 1) * 2 * Ip, 2 * H, 2 * moe::kBM) &&
+       encode_f32_2d(&L->tm_dn, L->w_dn, (El + 1) * H, 2 * Ip, moe::kBM)) ||
+      (!L->f32 && encode_bf16_2d(&L->tm_gu, L->w_gu, (El + 1) * 2 * Ip, H, 2 * moe::kBM) &&
+       encode_bf16_gate_up_pair(&L->tm_gu_pw, L->w_gu, (El + 1) * 2 * Ip, H, 2) &&
+       encode_bf16_gate_up_pair(&L->tm_gu_pn, L->w_gu, (El + 1) * 2 * Ip, H, 3) &&
+       encode_bf16_2d(&L->tm_dn, L->w_dn, (El + 1) * H, Ip, moe::kBM) &&
+       encode_bf16_kblocks(&L->tm_dn_pw, L->w_dn, (El + 1) * H, Ip, moe::kBM, 2) &&
+       encode_bf16_kblocks(&L->tm_dn_pn, L->w_dn, (El + 1) * H, Ip, moe::kBM, 3));
   if (!maps_ok || !encode_bf16_2d(&L->tm_router, L->router_tc, L->E_pad, 3 * H, moe::kBM) ||
       !encode_bf16_kblocks(&L->tm_rt_pw, L->router_tc, L->E_pad, 3 * H, moe::kBM, 2) ||
       !encode_bf16_kblocks(&L->tm_rt_pn, L->router_tc, L->E_pad, 3 * H, moe::kBM, 3)) {
@@ -489,7 +516,8 @@ namespace {
 // Packs the bf16 / fp32 expert weights: the layer's E_loc routed experts start
 // first_in_tensor experts into the caller's tensors (the shard's own first
 // expert for moe_load_weights, 0 for moe_load_shard_weights), then the shared
-// expert if the layer holds it, then the router.
+// expert if the layer holds it, then the router.  fp32 weights become the
+// fp32 expert path's [hi | lo] rows.
 int load_bf16(moe_layer* L, const float* router_w, const float* router_bias, const void* w_gate,
               const void* w_up, const void* w_down, const void* sh_gate, const void* sh_up,
               const void* sh_down, size_t first_in_tensor, cudaStream_t st) {
@@ -497,6 +525,28 @@ int load_bf16(moe_layer* L, const float* router_w, const float* router_bias, con
   const int H = c.hidden, El = L->E_loc, I = c.intermediate, Ip = L->I_pad;
   const bool wb = c.weight_dtype == MOE_BF16;
   const size_t gu_group = static_cast<size_t>(2) * Ip * H, dn_group = static_cast<size_t>(H) * Ip;
+  if (L->f32) {
+    // two fp32 values per weight: groups of 2 * gu_group / 2 * dn_group floats
+    const size_t off = first_in_tensor * H * I * 4;
+    const uint8_t* wg = static_cast<const uint8_t*>(w_gate) + off;
+    const uint8_t* wu = static_cast<const uint8_t*>(w_up) + off;
+    const uint8_t* wd = static_cast<const uint8_t*>(w_down) + off;
+    float* gu = static_cast<float*>(L->w_gu);
+    float* dn = static_cast<float*>(L->w_dn);
+    MOE_CUDA(cudaMemsetAsync(gu, 0, (El + 1) * gu_group * 8, st));
+    MOE_CUDA(cudaMemsetAsync(dn, 0, (El + 1) * dn_group * 8, st));
+    MOE_CUDA(moe::launch_pack_gate_up_split(wg, false, El, H, I, Ip, 0, gu, st));
+    MOE_CUDA(moe::launch_pack_gate_up_split(wu, false, El, H, I, Ip, 1, gu, st));
+    MOE_CUDA(moe::launch_pack_down_split(wd, false, El, H, I, Ip, dn, st));
+    if (L->with_shared) {
+      float* gsh = gu + El * 2 * gu_group;
+      MOE_CUDA(moe::launch_pack_gate_up_split(sh_gate, false, 1, H, I, Ip, 0, gsh, st));
+      MOE_CUDA(moe::launch_pack_gate_up_split(sh_up, false, 1, H, I, Ip, 1, gsh, st));
+      MOE_CUDA(moe::launch_pack_down_split(sh_down, false, 1, H, I, Ip, dn + El * 2 * dn_group,
+                                           st));
+    }
+    return load_router(L, router_w, router_bias, st);
+  }
   __nv_bfloat16* gu = static_cast<__nv_bfloat16*>(L->w_gu);
   __nv_bfloat16* dn = static_cast<__nv_bfloat16*>(L->w_dn);
   const size_t off = first_in_tensor * H * I * (wb ? 2 : 4);
@@ -714,9 +764,11 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   // expert-GEMM tiles: on one SM, 128 tokens x gate|up one 128-feature block
   // (down one or two); on CTA pairs (large T), 256 tokens x gate|up 128
   // features (down 256)
-  // (FP8 weights: always the one-SM tiles, which expand the codes)
-  const bool pair_gu = !L->fp8 && T >= moe::kPairMinTokens;
-  const bool pair_dn = !L->fp8 && T >= moe::kPairMinTokens && (H / moe::kBM) % 2 == 0;
+  // (FP8 weights: always the one-SM tiles, which expand the codes; so does
+  // the fp32 expert path, on tf32)
+  const bool f32 = L->f32 != 0;
+  const bool pair_gu = !L->fp8 && !f32 && T >= moe::kPairMinTokens;
+  const bool pair_dn = !L->fp8 && !f32 && T >= moe::kPairMinTokens && (H / moe::kBM) % 2 == 0;
   const int dn_blocks = moe::gemm_down_blocks(H);
   const int bn_gu = L->fp8 ? moe::kFp8BN : pair_gu ? 2 * moe::kBN : moe::kBN;
   const int bn_dn = L->fp8 ? moe::kFp8BN : pair_dn ? 2 * moe::kBN : moe::kBN;
@@ -728,6 +780,29 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   // kernels read them as K-block maps (32 rows x 3 K blocks, 128 rows x 2).
   moe::GemmMaps gu{}, dn{}, rt{};
   const bool maps_ok = [&] {
+    if (f32) {
+      // fp32 expert path: [hi | lo] rows of x_perm (the shared rows included)
+      // and of h; the router keeps its own path below
+      gu.a = L->tm_gu;
+      dn.a = L->tm_dn;
+      if (!encode_f32_2d(&gu.b, x_perm, w.rows_xperm, 2 * H, moe::kBBoxRows) ||
+          !encode_f32_2d(&gu.bw, x_perm, w.rows_xperm, 2 * H, moe::kBN) ||
+          !encode_f32_2d(&dn.b, hbuf, w.rows_all, 2 * Ip, moe::kBBoxRows) ||
+          !encode_f32_2d(&dn.bw, hbuf, w.rows_all, 2 * Ip, moe::kBN))
+        return false;
+      gu.bsh = gu.b;
+      gu.bshw = gu.bw;
+      dn.bsh = dn.b;
+      dn.bshw = dn.bw;
+      gu.out = gu.b;  // not read
+      dn.out = dn.b;
+      rt.a = L->tm_router;
+      rt.out = dn.b;
+      if (xb && (!encode_bf16_2d(&rt.b, x, T, H, moe::kBBoxRows) ||
+                 !encode_bf16_2d(&rt.bw, x, T, H, moe::kBN)))
+        return false;
+      return true;
+    }
     if (pair_gu) {
       gu.a = L->tm_gu_pw;
       gu.a2 = L->tm_gu_pn;
@@ -840,8 +915,12 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
                             mt_dn, masks, chunk_cnt, chunk_base, counts, row_start, tiles_gu,
                             tiles_dn, perm, pos, w_perm, st));
   MOE_CUDA(mark(3));
-  MOE_CUDA(moe::launch_gather(x, xb, perm, pos, w.rows_routed, k, T, H, !xb, x_perm, L->num_sms,
-                              L->status, st));
+  if (f32)
+    MOE_CUDA(moe::launch_gather_split(x, xb, perm, w.rows_routed, k, T, H,
+                                      reinterpret_cast<float*>(ws + w.x_perm), L->num_sms, st));
+  else
+    MOE_CUDA(moe::launch_gather(x, xb, perm, pos, w.rows_routed, k, T, H, !xb, x_perm,
+                                L->num_sms, L->status, st));
   MOE_CUDA(mark(4));
 
   GemmParams p{};
@@ -864,7 +943,17 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.w_perm = nullptr;
   p.a_scale = L->fp8 ? L->sc_gu : nullptr;
   p.a_codes = L->fp8 ? static_cast<const uint8_t*>(L->w_gu) : nullptr;
-  MOE_CUDA(L->fp8    ? moe::launch_gemm_gate_up_fp8(gu8, p, L->num_sms, st)
+  if (f32) {
+    // three terms of H / 32 k-blocks; h as fp32 [hi | lo] rows of 2 I_pad
+    p.kb_term = H / moe::kBK32;
+    p.num_kb = 3 * p.kb_term;
+    p.shared_b_row0 = T * k;
+    p.out = nullptr;
+    p.out_f32 = reinterpret_cast<float*>(ws + w.h);
+    p.out_ld = 2 * Ip;
+  }
+  MOE_CUDA(f32       ? moe::launch_gemm_gate_up_tf32(gu, p, L->num_sms, st)
+           : L->fp8  ? moe::launch_gemm_gate_up_fp8(gu8, p, L->num_sms, st)
            : pair_gu ? moe::launch_gemm_gate_up_pair(gu, p, st)
                      : moe::launch_gemm_gate_up(gu, p, L->num_sms, st));
   MOE_CUDA(mark(5));
@@ -880,11 +969,24 @@ int moe_forward(moe_layer_t* L, const void* x, int T, void* out, void* workspace
   p.w_perm = w_perm;
   p.a_scale = L->fp8 ? L->sc_dn : nullptr;
   p.a_codes = L->fp8 ? static_cast<const uint8_t*>(L->w_dn) : nullptr;
-  MOE_CUDA(L->fp8    ? moe::launch_gemm_down_fp8(dn8, p, L->num_sms, dn_blocks, st)
+  if (f32) {
+    // three terms of I_pad / 32 k-blocks; y fp32
+    p.kb_term = Ip / moe::kBK32;
+    p.num_kb = 3 * p.kb_term;
+    p.out = nullptr;
+    p.out_f32 = reinterpret_cast<float*>(ws + w.y);
+    p.out_ld = H;
+  }
+  MOE_CUDA(f32       ? moe::launch_gemm_down_tf32(dn, p, L->num_sms, dn_blocks, st)
+           : L->fp8  ? moe::launch_gemm_down_fp8(dn8, p, L->num_sms, dn_blocks, st)
            : pair_dn ? moe::launch_gemm_down_pair(dn, p, st)
                      : moe::launch_gemm_down(dn, p, L->num_sms, dn_blocks, st));
   MOE_CUDA(mark(6));
-  MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, L->with_shared != 0, out, st));
+  if (f32)
+    MOE_CUDA(moe::launch_combine_f32(reinterpret_cast<const float*>(ws + w.y), pos, T, k, H, xb,
+                                     L->with_shared != 0, out, st));
+  else
+    MOE_CUDA(moe::launch_combine(ybuf, pos, T, k, H, xb, L->with_shared != 0, out, st));
   MOE_CUDA(mark(7));
 
   return copy_routing(routing, T, k, El, topk_idx, topk_w, counts, row_start, perm, st);

@@ -14,6 +14,7 @@ namespace moe {
 // the group's tokens its N side).
 constexpr int kBM = 128;        // weight rows per MMA
 constexpr int kBK = 64;         // K elements per pipeline stage (one 128-byte row)
+constexpr int kBK32 = 32;       // the same for fp32 (tf32) operands
 constexpr int kBN = 128;        // tokens per tile (MMA N is rounded up to 16)
 constexpr int kBBoxRows = 32;   // token rows per TMA box of the B operand
 
@@ -75,8 +76,12 @@ struct GemmParams {
                           // k-blocks (A's K offset z * num_kb * kBK, B's 0), each part
                           // stored at out_f32 + z * part_stride (router: W1 | W2 | W3)
   size_t part_stride;
-  float* out_f32;         // router: logits [rows, out_ld]
+  float* out_f32;         // router: logits [rows, out_ld]; fp32 expert path: h as
+                          // [rows, out_ld] with out_ld = 2 * I_pad (tf32 hi | lo), or y
   int valid_feats;        // router: features (experts) actually stored
+  int kb_term;            // fp32 expert path: k-blocks (kBK32) per term; A and B hold
+                          // [hi | lo] halves of kb_term k-blocks each, and num_kb =
+                          // 3 * kb_term walks the terms hi.hi, lo.hi, hi.lo
 };
 
 // Guard band (selection-score units) of the top-k after the tensor-core
@@ -117,6 +122,11 @@ cudaError_t launch_localize(const int* topk_idx, int n, int first, int count, in
 cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, const int* pos,
                           int rows_routed, int k, int T, int H, bool write_shared,
                           __nv_bfloat16* x_perm, int num_sms, int* status, cudaStream_t st);
+// fp32 expert path: x_perm rows as [x_hi | x_lo] fp32 (2H per row, the tf32
+// split), the routed rows (perm) then the shared expert's T rows
+cudaError_t launch_gather_split(const void* x, bool x_bf16, const int* perm, int rows_routed,
+                                int k, int T, int H, float* x_perm, int num_sms,
+                                cudaStream_t st);
 // 128-feature weight blocks per down-projection tile for hidden size H.
 int gemm_down_blocks(int H);
 
@@ -134,6 +144,16 @@ cudaError_t launch_gemm_gate_up(const GemmMaps& m, const GemmParams& p, int grid
 cudaError_t launch_gemm_down(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
                              cudaStream_t st);
 cudaError_t launch_gemm_router(const GemmMaps& m, const GemmParams& p, int grid, cudaStream_t st);
+// fp32 expert path (kind::tf32, the three-term split; see tf32.cuh): m.a the
+// [hi | lo] packed weights (fp32, 32-column x A-rows boxes), m.b / m.bw the
+// [hi | lo] token rows (x_perm, the shared rows included, or h) with 32- and
+// 128-row boxes; num_kb = 3 * kb_term; outputs through p.out_f32 (gate|up: h
+// hi and lo halves, out_ld = 2 * I_pad; down: y fp32, out_ld = H).  m.out is
+// not read.
+cudaError_t launch_gemm_gate_up_tf32(const GemmMaps& m, const GemmParams& p, int grid,
+                                     cudaStream_t st);
+cudaError_t launch_gemm_down_tf32(const GemmMaps& m, const GemmParams& p, int grid, int blocks,
+                                  cudaStream_t st);
 // Split-K partial products of one group (single_rows, k_parts parts of num_kb
 // k-blocks; A and B both offset by the part's K): m.a with 128-row boxes, two
 // 128-row weight blocks per tile; fp32 [T, out_ld] per part.
@@ -159,10 +179,19 @@ cudaError_t launch_pack_router(const float* w, int H, int E, int E_pad, __nv_bfl
                                float* dst_t, cudaStream_t st);
 cudaError_t launch_combine(const __nv_bfloat16* y, const int* pos, int T, int k, int H, bool out_bf16,
                            bool with_shared, void* out, cudaStream_t st);
+// the same over fp32 rows y (the fp32 expert path)
+cudaError_t launch_combine_f32(const float* y, const int* pos, int T, int k, int H, bool out_bf16,
+                               bool with_shared, void* out, cudaStream_t st);
 cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
                                 int half, __nv_bfloat16* dst, cudaStream_t st);
 cudaError_t launch_pack_down(const void* w, bool w_bf16, int groups, int H, int I, int I_pad,
                              __nv_bfloat16* dst, cudaStream_t st);
+// fp32 expert path: the same rows, each as [hi | lo] fp32 halves of the tf32
+// split (row length 2H for gate|up, 2 I_pad for down)
+cudaError_t launch_pack_gate_up_split(const void* w, bool w_bf16, int groups, int H, int I,
+                                      int I_pad, int half, float* dst, cudaStream_t st);
+cudaError_t launch_pack_down_split(const void* w, bool w_bf16, int groups, int H, int I,
+                                   int I_pad, float* dst, cudaStream_t st);
 // FP8 E4M3 weights: the same packing, one byte per code, and the gate|up
 // rows' scales (down's scales need no reordering: row g * H + n)
 cudaError_t launch_pack_codes_gate_up(const uint8_t* w, int groups, int H, int I, int I_pad,

@@ -426,4 +426,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// Instruction descriptor of kind::tf32: tf32 A and B (fp32 containers), fp32
+// D, both K-major, shape M x N (same N rules as kind::f16).
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+  return (1u << 4)                                  // D format f32
+         | (2u << 7)                                // A format tf32
+         | (2u << 10)                               // B format tf32
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
 }  // namespace moe

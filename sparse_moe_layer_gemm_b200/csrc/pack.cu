@@ -6,6 +6,9 @@
 //   down       [G][I][H]  ->  rows g * H + n, columns i (ld I_pad).
 // Rows and columns past I (up to I_pad, a multiple of 128) stay zero, so the
 // padded features compute silu(0) * 0 = 0 and add nothing in the down GEMM.
+// fp32 weights (the fp32 expert path) keep the same rows as fp32 [hi | lo]
+// halves of the tf32 split (tf32.cuh): column k of the row at k (hi) and at
+// K + k (lo), K = H (gate|up) or I_pad (down).
 // FP8 E4M3 weights use the same packed rows, one byte per code, with one fp32
 // scale per packed row (the row's output feature; zero for padded rows), but
 // stored tile-major for the FP8 GEMM: for each tile of TR packed rows (the
@@ -20,6 +23,7 @@
 // K bytes apart.
 #include "fp8.cuh"
 #include "moe_internal.h"
+#include "tf32.cuh"
 
 namespace moe {
 
@@ -51,6 +55,38 @@ __global__ void __launch_bounds__(256) pack_kernel(const TS* __restrict__ src, i
       else
         drow = static_cast<size_t>(g) * H + c;
       dst[drow * dst_ld + r] = __float2bfloat16_rn(tile[threadIdx.x][i]);
+    }
+  }
+}
+
+// pack_kernel's transpose and rows for the fp32 path: dst rows of 2 * dst_ld
+// fp32, the tf32 split's hi half then its lo half.
+template <typename TS, bool GU>
+__global__ void __launch_bounds__(256) pack_split_kernel(const TS* __restrict__ src, int R, int C,
+                                                         float* __restrict__ dst, int dst_ld,
+                                                         int I_pad, int H, int half) {
+  __shared__ float tile[32][33];
+  const int g = blockIdx.z;
+  const TS* s = src + static_cast<size_t>(g) * R * C;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < R && c < C) ? to_f32(s[static_cast<size_t>(r) * C + c]) : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (c < C && r < R) {
+      size_t drow;
+      if (GU)
+        drow = static_cast<size_t>(g) * 2 * I_pad + (c / 128) * 256 + half * 128 + (c % 128);
+      else
+        drow = static_cast<size_t>(g) * H + c;
+      float hi, lo;
+      tf32_split(tile[threadIdx.x][i], hi, lo);
+      float* row = dst + drow * 2 * static_cast<size_t>(dst_ld);
+      row[r] = hi;
+      row[dst_ld + r] = lo;
     }
   }
 }
@@ -203,6 +239,30 @@ cudaError_t launch_pack_gate_up(const void* w, bool w_bf16, int groups, int H, i
   else
     pack_kernel<float, true><<<grid, block, 0, st>>>(static_cast<const float*>(w), H, I, dst, H,
                                                      I_pad, H, half);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_gate_up_split(const void* w, bool w_bf16, int groups, int H, int I,
+                                      int I_pad, int half, float* dst, cudaStream_t st) {
+  dim3 grid((I + 31) / 32, (H + 31) / 32, groups), block(32, 8);
+  if (w_bf16)
+    pack_split_kernel<__nv_bfloat16, true><<<grid, block, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), H, I, dst, H, I_pad, H, half);
+  else
+    pack_split_kernel<float, true><<<grid, block, 0, st>>>(static_cast<const float*>(w), H, I,
+                                                           dst, H, I_pad, H, half);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_down_split(const void* w, bool w_bf16, int groups, int H, int I,
+                                   int I_pad, float* dst, cudaStream_t st) {
+  dim3 grid((H + 31) / 32, (I + 31) / 32, groups), block(32, 8);
+  if (w_bf16)
+    pack_split_kernel<__nv_bfloat16, false><<<grid, block, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(w), I, H, dst, I_pad, I_pad, H, 0);
+  else
+    pack_split_kernel<float, false><<<grid, block, 0, st>>>(static_cast<const float*>(w), I, H,
+                                                            dst, I_pad, I_pad, H, 0);
   return cudaGetLastError();
 }
 

@@ -18,6 +18,7 @@
 // popcount of the mask bits below its token, so the scatter is stable and
 // bit-reproducible.
 #include "moe_internal.h"
+#include "tf32.cuh"
 #include "moe_ptx.cuh"
 #include "sort_device.cuh"
 
@@ -151,6 +152,46 @@ __global__ void __launch_bounds__(256) gather_kernel(const TX* __restrict__ x,
   }
 }
 
+__device__ __forceinline__ float to_float(float v) { return v; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// The fp32 expert path's x_perm: row r = [x_hi | x_lo] of its token (the tf32
+// split, 2H fp32), rows [0, rows_routed) from x[perm[r] / k], then the shared
+// expert's rows [rows_routed, rows_routed + T) from x[r - rows_routed].  One
+// warp per row, four values per lane step.
+template <typename TX>
+__global__ void __launch_bounds__(256) gather_split_kernel(const TX* __restrict__ x,
+                                                           const int* __restrict__ perm,
+                                                           int rows_routed, int k, int T, int H,
+                                                           float* __restrict__ xp) {
+  pdl_wait();  // the previous kernel's results are visible
+  const int lane = threadIdx.x & 31;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int nrows = rows_routed + T;
+  const int nvec = H / 4;
+  for (int r = warp; r < nrows; r += nwarps) {
+    const int t = (r < rows_routed) ? perm[r] / k : r - rows_routed;
+    float4* hi = reinterpret_cast<float4*>(xp + static_cast<size_t>(r) * 2 * H);
+    float4* lo = hi + nvec;
+    if (static_cast<unsigned>(t) >= static_cast<unsigned>(T)) {
+      for (int v = lane; v < nvec; v += 32) hi[v] = lo[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    const TX* src = x + static_cast<size_t>(t) * H;
+    for (int v = lane; v < nvec; v += 32) {
+      float f[4], a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[i] = to_float(src[4 * v + i]);
+        tf32_split(f[i], a[i], b[i]);
+      }
+      hi[v] = make_float4(a[0], a[1], a[2], a[3]);
+      lo[v] = make_float4(b[0], b[1], b[2], b[3]);
+    }
+  }
+}
+
 // Batches from which the bf16 gather runs per token with bulk copies (below,
 // the row-per-warp form spreads a small batch over more SMs).
 constexpr int kGatherRowsMinTokens = 1024;
@@ -244,6 +285,18 @@ cudaError_t launch_sort(const int* topk_idx, const float* topk_w, int T, int k, 
   if (err != cudaSuccess) return err;
   return launch_pdl(sort_scatter_kernel, dim3(nch), dim3(256), smem, st, topk_idx, topk_w, T, k, E,
                     masks, chunk_base, row_start, perm, pos, w_perm);
+}
+
+cudaError_t launch_gather_split(const void* x, bool x_bf16, const int* perm, int rows_routed,
+                                int k, int T, int H, float* x_perm, int num_sms,
+                                cudaStream_t st) {
+  const int want = (rows_routed + T + 7) / 8;
+  const int blocks = max(1, min(want, num_sms * 8));
+  if (x_bf16)
+    return launch_pdl(gather_split_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(x), perm, rows_routed, k, T, H, x_perm);
+  return launch_pdl(gather_split_kernel<float>, dim3(blocks), dim3(256), 0, st,
+                    static_cast<const float*>(x), perm, rows_routed, k, T, H, x_perm);
 }
 
 cudaError_t launch_gather(const void* x, bool x_bf16, const int* perm, const int* pos,

@@ -57,7 +57,7 @@ def _run(wl, rows=None):
     x = host_f32(inp["x"])[rows]
     ref = om.dense_mlp(x, host_f32(inp["w_gate"]), host_f32(inp["w_up"]),
                        host_f32(inp["w_down"]), wl.swiglu_limit)
-    rel, mx = output_errors(host_f32(out)[rows], ref)
+    rel, mx, _ = output_errors(host_f32(out)[rows], ref)
     layer.close()
     return rel, mx
 

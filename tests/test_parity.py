@@ -150,6 +150,39 @@ def test_fp8_decode_every_code():
 def test_small_parity(name):
     rep, _, _ = _run_small(SMALL[name])
     assert rep.ok(), rep
+    if SMALL[name].weight_dtype == "f32":
+        assert rep.ok_fp32(out_bf16=SMALL[name].act_dtype == "bf16"), rep
+
+
+# The fp32 expert path (fp32 weights: tf32 tensor cores over the two-term
+# split, h and y kept fp32) against the tighter bar of tests/parity.py, on
+# one-SM tiles at every size: several weight and token tiles with padded I,
+# down tiles of one and two weight blocks, the clamp, bf16 x (x_lo = 0, the
+# tensor-core router from 512 tokens) and batches past the CTA-pair threshold.
+FP32_PATH = {
+    "f32_multi_tile_ragged": replace(WORKLOADS["tiny"], name="g1", T=777, hidden=512,
+                                     num_experts=32, top_k=4, intermediate=320,
+                                     shared_intermediate=320),
+    "f32_odd_hidden_clamped": replace(WORKLOADS["tiny"], name="g2", T=300, hidden=384,
+                                      num_experts=12, top_k=3, intermediate=192,
+                                      shared_intermediate=192, swiglu_limit=0.9,
+                                      swiglu_limit_shared=1.3, expert_std=0.08),
+    "f32_weights_bf16_x": replace(WORKLOADS["tiny"], name="g3", T=600, hidden=512,
+                                  num_experts=24, top_k=4, intermediate=256,
+                                  shared_intermediate=256, act_dtype="bf16",
+                                  x_dist="rmsnorm_normal"),
+    "f32_many_tokens": replace(WORKLOADS["tiny"], name="g4", T=2304, hidden=512,
+                               num_experts=24, top_k=4, intermediate=256,
+                               shared_intermediate=256),
+    "f32_single_token": replace(WORKLOADS["tiny"], name="g5", T=1),
+}
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("name", list(FP32_PATH))
+def test_fp32_expert_path(name):
+    rep, _, _ = _run_small(FP32_PATH[name])
+    assert rep.ok_fp32(out_bf16=FP32_PATH[name].act_dtype == "bf16"), rep
 
 
 # ------------------------------------------------------------ exact ties
