@@ -175,6 +175,13 @@ FP32_PATH = {
                                num_experts=24, top_k=4, intermediate=256,
                                shared_intermediate=256),
     "f32_single_token": replace(WORKLOADS["tiny"], name="g5", T=1),
+    # the full layer's hidden size: 3 x 128 tf32 k-blocks per gate|up tile,
+    # the longest accumulation the fp32 path meets (1536 MMA k-steps: the
+    # worst-case truncation bound alone would be ~1.8e-4 of the largest
+    # partial sum; the errors seen are an order of magnitude smaller)
+    "f32_long_k": replace(WORKLOADS["tiny"], name="g6", T=96, hidden=4096, num_experts=16,
+                          top_k=4, intermediate=256, shared_intermediate=256,
+                          x_dist="rmsnorm_normal", expert_std=0.02),
 }
 
 
