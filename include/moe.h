@@ -127,9 +127,10 @@ typedef struct {
 int moe_config_check(const moe_config_t* cfg);
 
 /* Creates a layer on the current CUDA device.  Allocates the packed weight
- * copy (3 * (E + 1) * H * round_up(I, 128) bf16, or for FP8 weights as many
- * bytes plus (E + 1) * (2 * round_up(I, 128) + H) fp32 scales, plus the
- * router) and a small device status word.  *out receives the handle (NULL on
+ * copy (3 * (E + 1) * H * round_up(I, 128) bf16; for fp32 weights two fp32
+ * values each; for FP8 weights one byte each plus (E + 1) * (2 *
+ * round_up(I, 128) + H) fp32 scales; plus the router) and a small device
+ * status word.  *out receives the handle (NULL on
  * error). */
 int moe_create(const moe_config_t* cfg, moe_layer_t** out);
 
@@ -396,7 +397,9 @@ int moe_route_static(const void* x, int act_dtype, const float* router_w,
  * (L = 0: no clamp), computed by the MoE layer's expert GEMMs with one group
  * of all T rows.  Same conventions as the MoE entry points: device pointers,
  * caller-owned; x [T, H] and out [T, H] in act_dtype; w_gate, w_up [H, I],
- * w_down [I, H] in weight_dtype (fp32 weights are rounded to bf16 at load);
+ * w_down [I, H] in weight_dtype (fp32 weights take the fp32 expert path of
+ * the MoE layer: tf32 tensor cores over the two-term split, h fp32, one-SM
+ * tiles at every T);
  * stream-ordered, no host synchronisation in the forward; every argument is
  * checked on the host and nothing is enqueued on error. */
 typedef struct moe_dense moe_dense_t;
@@ -415,8 +418,9 @@ typedef struct {
 /* Host-only check of a configuration; no CUDA call. */
 int moe_dense_config_check(const moe_dense_config_t* cfg);
 
-/* Creates the layer on the current device: packed bf16 weights
- * (3 * H * round_up(I, 128) elements) and a device status word. */
+/* Creates the layer on the current device: packed weights (3 * H *
+ * round_up(I, 128) elements: bf16, or two fp32 terms each for fp32 weights)
+ * and a device status word. */
 int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out);
 
 /* Copies the weights into the packed layout on `stream` (the caller's

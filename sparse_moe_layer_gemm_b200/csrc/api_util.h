@@ -16,6 +16,10 @@ namespace moe {
 // swizzle; out-of-range elements read as zero.
 bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows);
+// fp32 [rows, cols] row-major, box = 32 columns (128 bytes) x box_rows, 128B
+// swizzle (the fp32 path's tf32 operands); out-of-range elements read as zero.
+bool encode_f32_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                   uint32_t box_rows);
 // bf16 [rows, cols] as 3-D (64 columns, rows, cols / 64 column blocks), box
 // 64 x box_rows x kblocks column blocks, 128B swizzle: in shared memory the
 // box is k-block-major (kblocks sub-blocks of box_rows 128-byte rows).

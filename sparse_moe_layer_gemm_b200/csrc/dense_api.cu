@@ -11,7 +11,9 @@
 // both GEMMs and their reductions (dense_streamk.cu); otherwise both GEMMs
 // split K, each part writes raw fp32 accumulators and a reduction kernel sums
 // the parts in fixed order (then applies the SwiGLU, or writes out).
-// Declared in include/moe.h (moe_dense_*).
+// fp32 weights take the fp32 expert path at every T: the one-SM tf32 GEMMs
+// over the two-term split of weights, x and h (tf32.cuh), h and the output
+// fp32.  Declared in include/moe.h (moe_dense_*).
 #include <math.h>
 #include <string.h>
 
@@ -27,6 +29,11 @@ struct moe_dense {
   int I_pad;
   __nv_bfloat16* w_gu;  // [2 * I_pad, H]: blocks of 128 gate rows then 128 up rows
   __nv_bfloat16* w_dn;  // [H, I_pad]
+  int f32;              // fp32 weights: the fp32 path (w_gu32 / w_dn32 instead)
+  float* w_gu32;        // [2 * I_pad, 2H]: the same rows as [hi | lo] fp32
+  float* w_dn32;        // [H, 2 * I_pad]
+  CUtensorMap tm_gu32;  // box 32 x 256
+  CUtensorMap tm_dn32;  // box 32 x 128
   int* status;
   int loaded;
   // the one-launch stream-K forward (T <= 128): its running counters and
@@ -136,6 +143,7 @@ unsigned grid_for(size_t n, int num_sms) {
 
 struct DenseWs {
   size_t xb, h, y, ones, parts, total;
+  size_t xs, h32, y32;  // fp32 path: x and h as [hi | lo] rows, y fp32 (bf16 out)
   int s_gu, s_dn;  // split-K parts of the two GEMMs (1: no split)
   bool sk;         // the one-launch stream-K forward (sk_parts: its slots per pass)
   int sk_seg[moe::kSkPasses];
@@ -159,6 +167,15 @@ DenseWs dense_ws(const moe_dense* L, int T) {
     return at;
   };
   const bool xf = L->cfg.act_dtype == MOE_F32;
+  if (L->f32) {  // the fp32 path: one-SM tf32 tiles at every T
+    w.xs = take(static_cast<size_t>(T) * H * 8);
+    w.h32 = take(static_cast<size_t>(T) * L->I_pad * 8);
+    w.y32 = xf ? 0 : take(static_cast<size_t>(T) * H * 4);
+    w.ones = take(static_cast<size_t>(T) * sizeof(float));
+    w.s_gu = w.s_dn = 1;
+    w.total = off;
+    return w;
+  }
   w.xb = xf ? take(static_cast<size_t>(T) * H * 2) : 0;    // bf16 copy of fp32 x
   w.h = take(static_cast<size_t>(T) * L->I_pad * 2);
   if (use_streamk(L, T)) {
@@ -193,6 +210,68 @@ DenseWs dense_ws(const moe_dense* L, int T) {
   return w;
 }
 
+// The fp32 path's forward (L->f32): x split into [hi | lo] rows, gate|up
+// and down on the one-SM tf32 kernels with one group of T rows, h fp32 as
+// [hi | lo], the output fp32 (widened from fp32 y for a bf16 output).
+int dense_forward_f32(moe_dense* L, const void* x, int T, void* out, uint8_t* ws,
+                      const DenseWs& w, cudaStream_t st) {
+  const int H = L->cfg.hidden, Ip = L->I_pad;
+  const bool xf = L->cfg.act_dtype == MOE_F32;
+  float* xs = reinterpret_cast<float*>(ws + w.xs);
+  float* h32 = reinterpret_cast<float*>(ws + w.h32);
+  float* y32 = xf ? static_cast<float*>(out) : reinterpret_cast<float*>(ws + w.y32);
+  float* ones = reinterpret_cast<float*>(ws + w.ones);
+  // the split rows of x: the gather with no routed rows and T identity rows
+  MOE_CUDA(moe::launch_gather_split(x, !xf, nullptr, 0, 1, T, H, xs, L->num_sms, st));
+  fill_f32_kernel<<<grid_for(static_cast<size_t>(T), L->num_sms), 256, 0, st>>>(ones, 1.f, T);
+  MOE_CUDA(cudaGetLastError());
+  moe::GemmMaps gu{}, dn{};
+  gu.a = L->tm_gu32;
+  dn.a = L->tm_dn32;
+  if (!moe::encode_f32_2d(&gu.b, xs, T, 2 * H, moe::kBBoxRows) ||
+      !moe::encode_f32_2d(&gu.bw, xs, T, 2 * H, moe::kBN) ||
+      !moe::encode_f32_2d(&dn.b, h32, T, 2 * Ip, moe::kBBoxRows) ||
+      !moe::encode_f32_2d(&dn.bw, h32, T, 2 * Ip, moe::kBN))
+    return MOE_ERR_CUDA;
+  gu.bsh = gu.b;
+  gu.bshw = gu.bw;
+  dn.bsh = dn.b;
+  dn.bshw = dn.bw;
+  moe::GemmParams p{};
+  p.single_rows = T;
+  p.G = 1;
+  p.E = -1;  // no shared group
+  p.k_parts = 1;
+  p.status = L->status;
+  p.limit = L->cfg.swiglu_limit;
+  p.limit_shared = L->cfg.swiglu_limit;
+  p.kb_term = H / moe::kBK32;
+  p.num_kb = 3 * p.kb_term;
+  p.m_tiles = Ip / moe::kBM;
+  p.a_rows_per_group = 2 * Ip;
+  p.out_f32 = h32;
+  p.out_ld = 2 * Ip;
+  p.out_feats = Ip;
+  MOE_CUDA(moe::launch_gemm_gate_up_tf32(gu, p, L->num_sms, st));
+  const int dn_blocks = moe::gemm_down_blocks(H);
+  p.kb_term = Ip / moe::kBK32;
+  p.num_kb = 3 * p.kb_term;
+  p.m_tiles = H / moe::kBM / dn_blocks;
+  p.a_rows_per_group = H;
+  p.out_f32 = y32;
+  p.out_ld = H;
+  p.out_feats = H;
+  p.w_perm = ones;
+  MOE_CUDA(moe::launch_gemm_down_tf32(dn, p, L->num_sms, dn_blocks, st));
+  if (!xf) {
+    const size_t n = static_cast<size_t>(T) * H;
+    cast_f32_bf16_kernel<<<grid_for(n, L->num_sms), 256, 0, st>>>(
+        y32, static_cast<__nv_bfloat16*>(out), n);
+    MOE_CUDA(cudaGetLastError());
+  }
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -220,6 +299,7 @@ int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out) {
   if (L == nullptr) return MOE_ERR_CUDA;
   L->cfg = *cfg;
   L->I_pad = (cfg->intermediate + 127) / 128 * 128;
+  L->f32 = cfg->weight_dtype == MOE_F32 ? 1 : 0;
   if (cudaGetDevice(&L->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, L->device) !=
           cudaSuccess) {
@@ -227,6 +307,20 @@ int moe_dense_create(const moe_dense_config_t* cfg, moe_dense_t** out) {
     return MOE_ERR_CUDA;
   }
   const size_t H = cfg->hidden, Ip = L->I_pad;
+  if (L->f32) {
+    if (moe::gemm_configure_device() != cudaSuccess ||
+        cudaMalloc(&L->w_gu32, 2 * Ip * H * 8) != cudaSuccess ||
+        cudaMalloc(&L->w_dn32, H * Ip * 8) != cudaSuccess ||
+        cudaMalloc(&L->status, sizeof(int)) != cudaSuccess ||
+        cudaMemset(L->status, 0, sizeof(int)) != cudaSuccess ||
+        !moe::encode_f32_2d(&L->tm_gu32, L->w_gu32, 2 * Ip, 2 * H, 2 * moe::kBM) ||
+        !moe::encode_f32_2d(&L->tm_dn32, L->w_dn32, H, 2 * Ip, moe::kBM)) {
+      moe_dense_destroy(L);
+      return MOE_ERR_CUDA;
+    }
+    *out = L;
+    return MOE_OK;
+  }
   if (moe::gemm_configure_device() != cudaSuccess ||
       moe::gemm_pair_configure_device(L->num_sms) != cudaSuccess ||
       moe::dense_streamk_configure_device(L->num_sms) != cudaSuccess ||
@@ -261,6 +355,15 @@ int moe_dense_load_weights(moe_dense_t* L, const void* w_gate, const void* w_up,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int H = L->cfg.hidden, I = L->cfg.intermediate, Ip = L->I_pad;
   const bool wb = L->cfg.weight_dtype == MOE_BF16;
+  if (L->f32) {
+    MOE_CUDA(cudaMemsetAsync(L->w_gu32, 0, static_cast<size_t>(2) * Ip * H * 8, st));
+    MOE_CUDA(cudaMemsetAsync(L->w_dn32, 0, static_cast<size_t>(H) * Ip * 8, st));
+    MOE_CUDA(moe::launch_pack_gate_up_split(w_gate, false, 1, H, I, Ip, 0, L->w_gu32, st));
+    MOE_CUDA(moe::launch_pack_gate_up_split(w_up, false, 1, H, I, Ip, 1, L->w_gu32, st));
+    MOE_CUDA(moe::launch_pack_down_split(w_down, false, 1, H, I, Ip, L->w_dn32, st));
+    L->loaded = 1;
+    return MOE_OK;
+  }
   MOE_CUDA(cudaMemsetAsync(L->w_gu, 0, static_cast<size_t>(2) * Ip * H * 2, st));
   MOE_CUDA(cudaMemsetAsync(L->w_dn, 0, static_cast<size_t>(H) * Ip * 2, st));
   MOE_CUDA(moe::launch_pack_gate_up(w_gate, wb, 1, H, I, Ip, 0, L->w_gu, st));
@@ -295,6 +398,7 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
   const bool xf = L->cfg.act_dtype == MOE_F32;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t n = static_cast<size_t>(T) * H;
+  if (L->f32) return dense_forward_f32(L, x, T, out, ws, w, st);
   // bf16 operand rows (x itself when bf16)
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (xf) {
@@ -486,7 +590,8 @@ int moe_dense_get_device_error(moe_dense_t* L, int* device_err) {
   MOE_CUDA(cudaDeviceSynchronize());
   MOE_CUDA(cudaMemcpy(&v, L->status, sizeof(int), cudaMemcpyDeviceToHost));
   MOE_CUDA(cudaMemset(L->status, 0, sizeof(int)));
-  if (v != 0) {  // an aborted stream-K forward leaves its counters short of their targets
+  if (v != 0 && L->sk_cnt != nullptr) {  // an aborted stream-K forward leaves its counters
+                                         // short of their targets
     MOE_CUDA(cudaMemset(L->sk_cnt, 0,
                         moe::dense_streamk_counters(L->cfg.hidden, L->I_pad) * sizeof(unsigned int)));
     L->sk_fwd = 0;
@@ -503,6 +608,8 @@ void moe_dense_destroy(moe_dense_t* L) {
     cudaDeviceSynchronize();
     cudaFree(L->w_gu);
     cudaFree(L->w_dn);
+    cudaFree(L->w_gu32);
+    cudaFree(L->w_dn32);
     cudaFree(L->status);
     cudaFree(L->sk_cnt);
   }

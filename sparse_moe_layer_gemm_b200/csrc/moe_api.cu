@@ -96,8 +96,6 @@ bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
   return r == CUDA_SUCCESS;
 }
 
-// fp32 [rows, cols] row-major, box = 32 columns (128 bytes) x box_rows, 128B
-// swizzle (the fp32 expert path's tf32 operands); out-of-range reads zero.
 bool encode_f32_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
                    uint32_t box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
