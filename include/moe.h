@@ -437,8 +437,10 @@ int moe_dense_workspace_size(const moe_dense_t* layer, int T, size_t* bytes);
  * launch whose CTAs synchronise through running counters owned by the layer
  * (never cleared between forwards): the forwards of one layer must then run
  * on the device in the order they were issued (one stream, or streams
- * ordered by events).  The result depends only on x's own rows (the same
- * row gives the same output in any batch of up to 128 tokens). */
+ * ordered by events).  The counters' targets are derived on the device, so
+ * the forward may be captured in a CUDA graph and replayed.  The result
+ * depends only on x's own rows (the same row gives the same output in any
+ * batch of up to 128 tokens). */
 int moe_dense_forward(moe_dense_t* layer, const void* x, int T, void* out,
                       void* workspace, size_t ws_bytes, void* stream);
 

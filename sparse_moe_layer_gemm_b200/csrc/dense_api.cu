@@ -20,6 +20,7 @@
 #include <new>
 
 #include "api_util.h"
+#include "dense_streamk.h"
 #include "moe_internal.h"
 
 struct moe_dense {
@@ -36,11 +37,9 @@ struct moe_dense {
   CUtensorMap tm_dn32;  // box 32 x 128
   int* status;
   int loaded;
-  // the one-launch stream-K forward (T <= 128): its running counters and
-  // their targets' bases (see dense_streamk.cu)
+  // the one-launch stream-K forward (T <= 128): its running counters, with
+  // the words from which each forward derives its targets (dense_streamk.cu)
   unsigned int* sk_cnt;
-  unsigned int sk_fwd;
-  unsigned int sk_rows;
   CUtensorMap tm_gu;    // box 64 x 256 (one CTA per tile)
   CUtensorMap tm_gu128; // box 64 x 128 (split-K partial tiles)
   CUtensorMap tm_gu_pw; // CTA pairs, wide stages: 64 + 64 rows x 2 K blocks
@@ -431,12 +430,8 @@ int moe_dense_forward(moe_dense_t* L, const void* x, int T, void* out, void* wor
     d.out = out;
     d.out_f32 = xf;
     d.counters = L->sk_cnt;
-    d.fwd = L->sk_fwd + 1u;
-    d.h_rows = L->sk_rows + static_cast<unsigned int>(T);
     d.status = L->status;
     MOE_CUDA(moe::launch_dense_streamk(d, st));
-    L->sk_fwd = d.fwd;  // the targets of the launches that follow
-    L->sk_rows = d.h_rows;
     return MOE_OK;
   }
   float* ones = reinterpret_cast<float*>(ws + w.ones);
@@ -594,8 +589,6 @@ int moe_dense_get_device_error(moe_dense_t* L, int* device_err) {
                                          // short of their targets
     MOE_CUDA(cudaMemset(L->sk_cnt, 0,
                         moe::dense_streamk_counters(L->cfg.hidden, L->I_pad) * sizeof(unsigned int)));
-    L->sk_fwd = 0;
-    L->sk_rows = 0;
   }
   *device_err = v;
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE_TIMEOUT;

@@ -41,13 +41,17 @@
 // reset: a forward's targets are the running totals (forward count x
 // segments, and the sum of T over the layer's forwards), so no launch-time
 // clearing breaks the programmatic launch chain, and the forwards of one
-// layer must run on the device in the order they were issued.
+// layer must run on the device in the order they were issued.  The totals
+// live on the device too: each forward reads them after its pdl_wait and
+// the last CTA to finish advances them, so a launch captured in a CUDA graph
+// computes the right targets at every replay.
 //
 // Warps (480 threads): 0 TMA producer; 1, 2 tcgen05.mma issuers (one 128-row
 // accumulator each: gate and up, or two 128-row blocks of H); 3-6 store
 // warps (TMEM -> fp32 slots, one per lane quadrant); 7-14 reducers of h; at
 // the end every warp reduces the output rows.  Every wait is bounded; on expiry the CTA sets its abort flag and the device
 // status bit and winds down.  No TMA multicast.
+#include "dense_streamk.h"
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
 
@@ -81,8 +85,8 @@ struct SkParams {
   float* parts[kSkPasses];        // [grid][max_seg][T][256] fp32
   unsigned int* seg_cnt[kSkPasses];  // per tile of the pass: stored segments x epilogue warps
   unsigned int* h_cnt;            // per h tile: reduced rows
-  unsigned int fwd;               // forwards of the layer on this path, this one included
-  unsigned int h_rows;            // sum of T over those forwards
+  unsigned int* epoch;            // [3]: forwards completed on this path, the sum of their
+                                  // T, CTAs done with the current forward
   float limit;                    // SwiGLU clamp (<= 0: none)
   __nv_bfloat16* h;               // [T, I_pad]
   void* out;                      // [T, H]
@@ -263,6 +267,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   static_assert((2 * kSkMaxStages + 5) * 8 + 8 <= kSkBarBytes, "barrier area");
   __shared__ uint32_t s_lo[kSkPasses][kSkMaxGrid + 1];  // first unit of each CTA, per pass
+  __shared__ unsigned int s_target[2];                   // this forward's counter targets
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -301,10 +306,19 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     tmem_relinquish();
   }
   pdl_wait();  // x and the layer's counters come from the previous kernels of the stream
+  if (threadIdx.x == 0) {
+    // the counters' targets: the running totals of the forwards before this
+    // one (written by the last CTA of the previous forward, whose grid has
+    // completed), plus this one
+    s_target[0] = __ldcg(p.epoch) + 1u;
+    s_target[1] = __ldcg(p.epoch + 1) + static_cast<unsigned int>(p.T);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const unsigned int fwd = s_target[0];     // forwards on this path, this one included
+  const unsigned int h_rows = s_target[1];  // the sum of their T (mod 2^32)
   const uint32_t b_bytes = static_cast<uint32_t>(n_mma) * 128u;
 
   if (warp == 0) {
@@ -339,7 +353,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             // that tile is stored; on an abort the (unused) rows are loaded
             // anyway, so the stage completes and the teardown's wait ends
             if (ps.gemm == 1 && (kb >> 1) != h_ready) {
-              if (ok && wait_count(p.h_cnt + (kb >> 1), p.h_rows, abort_flag, p.status,
+              if (ok && wait_count(p.h_cnt + (kb >> 1), h_rows, abort_flag, p.status,
                                    p.wait_ns, true))
                 h_ready = kb >> 1;
               else
@@ -474,7 +488,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           ts = tile_segs(j, ps.nkb, ps.tiles * ps.nkb, G, s_lo[q], lane);
           int ok = 1;
           if (lane == 0)
-            ok = wait_count(p.seg_cnt[q] + j, kSkEpiWarps * ts.nseg * p.fwd, abort_flag,
+            ok = wait_count(p.seg_cnt[q] + j, kSkEpiWarps * ts.nseg * fwd, abort_flag,
                             p.status, p.wait_ns, false);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           __syncwarp();  // the other lanes' loads after lane 0's acquire
@@ -523,7 +537,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             if (ps.nkb == 0) continue;
             const TileSegs ts = tile_segs(j, ps.nkb, ps.tiles * ps.nkb, G, s_lo[q], lane);
             if (lane == 0)
-              ok = wait_count(p.seg_cnt[q] + j, kSkEpiWarps * ts.nseg * p.fwd, abort_flag,
+              ok = wait_count(p.seg_cnt[q] + j, kSkEpiWarps * ts.nseg * fwd, abort_flag,
                               p.status, p.wait_ns, false);
             ok = __shfl_sync(0xffffffffu, ok, 0);
           }
@@ -554,6 +568,17 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) {
+    // the last CTA to finish moves the running totals on for the next
+    // forward (which reads them after its pdl_wait, once this grid is done)
+    __threadfence();
+    if (atomicAdd(p.epoch + 2, 1u) == static_cast<unsigned int>(G) - 1u) {
+      p.epoch[0] = fwd;
+      p.epoch[1] = h_rows;
+      p.epoch[2] = 0u;
+      __threadfence();
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -613,8 +638,7 @@ cudaError_t launch_dense_streamk(const DenseStreamK& d, cudaStream_t st) {
     cnt += p.pass[q].tiles;
   }
   p.h_cnt = cnt;
-  p.fwd = d.fwd;
-  p.h_rows = d.h_rows;
+  p.epoch = cnt + d.I_pad / kBM;  // after the h tiles' counts (one per 128 features of h)
   p.limit = d.limit;
   p.h = d.h;
   p.out = d.out;
