@@ -1,7 +1,8 @@
 """bench.py host logic on the CPU: the clock sampler against a fake NVML
 (the reasons it reports, the median over samples under load, the fallback
-when NVML cannot start) and the DRAM-traffic records (reported only while
-the captured kernel's sources still hash as recorded)."""
+when NVML cannot start), the DRAM-traffic records (reported only while
+the captured kernel's sources still hash as recorded), and the config and
+dtype a line reports for its workload."""
 import hashlib
 import os
 import time
@@ -197,3 +198,18 @@ def test_both_arms_print_the_same_config():
     wl = WORKLOADS["decode"]
     assert bench._config(wl, 4) == _fake_full()["config"] or bench._config(wl, 8) == \
         _fake_full()["config"]
+
+
+def test_config_and_dtype_follow_the_workload():
+    """The printed config is identical for both arms of a workload; its L2
+    note and the line's dtype follow the workload: the full layer streams its
+    weights from HBM, the tiny fp32 layer fits in L2 and runs the fp32
+    expert path."""
+    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS
+    dec, tiny = WORKLOADS["decode"], WORKLOADS["tiny"]
+    assert bench._config(dec, 1) == bench._config(dec, 1)
+    assert bench._config(dec, 1)["l2"].startswith("inputs > L2")
+    assert bench._config(tiny, 1)["l2"].startswith("L2-resident")
+    assert bench._dtype(dec) == "bf16"
+    assert bench._dtype(WORKLOADS["decode_fp8"]) == "bf16"   # the MMA is bf16 on the codes
+    assert bench._dtype(tiny) == "f32"
