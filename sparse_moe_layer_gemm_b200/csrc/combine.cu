@@ -14,10 +14,12 @@ namespace moe {
 
 namespace {
 
+// Every row of a token is loaded at once (combine_token): the bf16 -> bf16
+// form fits two 512-thread blocks per SM in registers; the others take one.
 template <typename TO, typename TY>
-__global__ void __launch_bounds__(512) combine_kernel(const TY* __restrict__ y,
-                                                      const int* __restrict__ pos, int T, int k,
-                                                      int H, int with_shared, TO* __restrict__ out) {
+__global__ void __launch_bounds__(512, sizeof(TY) == 2 && sizeof(TO) == 2 ? 2 : 1)
+    combine_kernel(const TY* __restrict__ y, const int* __restrict__ pos, int T, int k, int H,
+                   int with_shared, TO* __restrict__ out) {
   pdl_wait();  // the previous kernel's results are visible
   __shared__ int rows[33];
   combine::combine_token<TO, TY>(blockIdx.x, y, pos, T, k, H, with_shared, out, rows);

@@ -45,6 +45,43 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint4& q) {
   }
 }
 
+// 8 consecutive values of a y row, as loaded (bf16: one 16-byte vector;
+// fp32: two)
+struct Row8F32 {
+  float4 a, b;
+};
+template <typename TY>
+struct Row8;
+template <>
+struct Row8<__nv_bfloat16> {
+  using type = uint4;
+};
+template <>
+struct Row8<float> {
+  using type = Row8F32;
+};
+
+__device__ __forceinline__ uint4 load8(const __nv_bfloat16* p) {
+  return *reinterpret_cast<const uint4*>(p);
+}
+__device__ __forceinline__ Row8F32 load8(const float* p) {
+  return Row8F32{*reinterpret_cast<const float4*>(p), *reinterpret_cast<const float4*>(p + 4)};
+}
+__device__ __forceinline__ void add8(float (&acc)[8], const Row8F32& q) {
+  acc[0] += q.a.x;
+  acc[1] += q.a.y;
+  acc[2] += q.a.z;
+  acc[3] += q.a.w;
+  acc[4] += q.b.x;
+  acc[5] += q.b.y;
+  acc[6] += q.b.z;
+  acc[7] += q.b.w;
+}
+
+// Rows a combine thread loads at once (k + 1 <= kPreRows: every row's vector
+// in flight together, then the sum in the fixed order).
+constexpr int kPreRows = 9;
+
 __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
   uint4 q;
   __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&q);
@@ -71,8 +108,21 @@ __device__ __forceinline__ void combine_token(int t, const TY* __restrict__ y,
   const int nvec = H / 8;
   for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j <= k; ++j)  // (-1: another shard's expert, or no shared expert here)
-      if (rows_s[j] >= 0) add8(acc, y + static_cast<size_t>(rows_s[j]) * H + v * 8);
+    // (row -1: another shard's expert, or no shared expert here)
+    if (k + 1 <= kPreRows) {
+      // all rows' loads in flight at once (a latency-bound gather otherwise),
+      // then added in the same order j = 0..k
+      typename Row8<TY>::type q[kPreRows];
+#pragma unroll
+      for (int j = 0; j < kPreRows; ++j)
+        if (j <= k && rows_s[j] >= 0) q[j] = load8(y + static_cast<size_t>(rows_s[j]) * H + v * 8);
+#pragma unroll
+      for (int j = 0; j < kPreRows; ++j)
+        if (j <= k && rows_s[j] >= 0) add8(acc, q[j]);
+    } else {
+      for (int j = 0; j <= k; ++j)
+        if (rows_s[j] >= 0) add8(acc, y + static_cast<size_t>(rows_s[j]) * H + v * 8);
+    }
     store8(out + static_cast<size_t>(t) * H + v * 8, acc);
   }
   __syncthreads();
