@@ -37,7 +37,9 @@
  *    accumulate w_hi x_hi + w_lo x_hi + w_hi x_lo in fp32: each product to
  *    within ~2^-21 of fp32's.  h and the output rows stay fp32 and are summed
  *    in fp32.  Measured against the fp64 definition: ~6e-6 relative
- *    Frobenius error on the tiny fp32 layer.  Costs: 8 bytes of device memory
+ *    Frobenius error on the tiny fp32 layer, dominated by the tensor cores'
+ *    fp32 accumulation, which behaves like truncation at every MMA step and
+ *    so grows with K (~1e-4 expected at H = 4096).  Costs: 8 bytes of device memory
  *    per expert weight and three MMA passes; always on one-SM tiles (no CTA
  *    pairs, no fused forward).
  *

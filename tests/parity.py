@@ -32,7 +32,11 @@ tighter, derived from its arithmetic:
   fp32 roundings;
 so relative Frobenius error <= REL_FRO_F32 = 1e-4 and max |error| <=
 MAX_ABS_OVER_RMS_F32 = 1e-3 * RMS(out) (the bf16 path measures ~5e-3 and
-fails it).  A bf16 output (bf16 x) is the fp32 result rounded once more, by at
+fails it).  The truncation term is linear in the step count, so the bar
+grows with the longest accumulation of the layer (fp32_bar_scale: x8 at
+H = 4096, 1536 steps); tests/test_fp32_bar.py checks the bar against an
+emulation of this arithmetic with an accumulator that truncates every step
+(the tiny fp32 layer: 8e-6 there, 6e-6 measured on the GPU).  A bf16 output (bf16 x) is the fp32 result rounded once more, by at
 most 2^-8 of its magnitude: there the error beyond 2^-8 |out| must meet the
 same max bar (with its own 2^-8 share), and the relative Frobenius error stays
 under 2^-8 + REL_FRO_F32.
@@ -52,6 +56,14 @@ MAX_ABS_OVER_RMS = 5e-2
 REL_FRO_F32 = 1e-4
 MAX_ABS_OVER_RMS_F32 = 1e-3
 BF16_U = 2.0 ** -8      # unit roundoff of bf16 (8 significant bits)
+
+
+def fp32_bar_scale(hidden: int, intermediate: int) -> float:
+    """Factor on the fp32 bar for a layer: its longest accumulation
+    (3 K / 8 MMA steps, K = H for gate|up, I rounded up to 128 for down)
+    over the 192 steps of K = 512 the base bar is derived for."""
+    i_pad = -(-intermediate // 128) * 128
+    return max(1.0, 3 * max(hidden, i_pad) / 8 / 192)
 W_RTOL = 1e-5
 LOGIT_TOL = 1e-5
 LOGIT_TOL_APPROX = 4e-4
@@ -71,13 +83,15 @@ class ParityReport:
     def ok(self) -> bool:
         return self.rel_fro <= REL_FRO and self.max_abs_over_rms <= MAX_ABS_OVER_RMS
 
-    def ok_fp32(self, out_bf16: bool = False) -> bool:
-        """The fp32 expert path's bar (module docstring); out_bf16: the
-        output dtype is bf16, so its own rounding is set apart."""
+    def ok_fp32(self, out_bf16: bool = False, scale: float = 1.0) -> bool:
+        """The fp32 expert path's bar (module docstring) times `scale`
+        (fp32_bar_scale); out_bf16: the output dtype is bf16, so its own
+        rounding is set apart."""
+        rel, mx = REL_FRO_F32 * scale, MAX_ABS_OVER_RMS_F32 * scale
         if out_bf16:
-            return (self.rel_fro <= BF16_U + REL_FRO_F32 and
-                    self.excess_bf16_over_rms <= MAX_ABS_OVER_RMS_F32 * (1 + BF16_U))
-        return self.rel_fro <= REL_FRO_F32 and self.max_abs_over_rms <= MAX_ABS_OVER_RMS_F32
+            return (self.rel_fro <= BF16_U + rel and
+                    self.excess_bf16_over_rms <= mx * (1 + BF16_U))
+        return self.rel_fro <= rel and self.max_abs_over_rms <= mx
 
 
 def order_gaps(beta32: np.ndarray, top_k: int) -> np.ndarray:
