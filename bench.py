@@ -287,6 +287,15 @@ def _sample_inputs_host(wl, x_host, rw, rb, rows, fetch_expert, shared):
     return experts, len(ids)
 
 
+def _arm_config(wl, world: int, parallel: str):
+    """(config, scaling) of a line: both arms print the same for the same
+    workload and GPU count (expert parallelism for N > 1 unless replicas are
+    asked for, strong scaling; else replicas, weak scaling)."""
+    if world > 1 and parallel != "replicas":
+        return ep_config(wl, world), "strong"
+    return _config(wl, world), "weak"
+
+
 def run_reference(a):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -311,12 +320,13 @@ def run_reference(a):
     secs = [_oracle_sample(wl, x, rw, rb, experts, rows) for _ in range(a.steps)]
     total = sum(secs)
     value = sample * a.steps / total
+    config, scaling = _arm_config(wl, int(os.environ.get("WORLD_SIZE", a.gpus)), a.parallel)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
-        "ms_per_step": 1e3 * total / a.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * total / a.steps, "higher_is_better": True, "scaling": scaling,
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": _config(wl, a.gpus),
+        "config": config,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{sample} of {wl.T} tokens per step ({touched} routed experts "
                                    f"+ shared, weights drawn on the host, in RAM before timing)"},

@@ -213,3 +213,15 @@ def test_config_and_dtype_follow_the_workload():
     assert bench._dtype(dec) == "bf16"
     assert bench._dtype(WORKLOADS["decode_fp8"]) == "bf16"   # the MMA is bf16 on the codes
     assert bench._dtype(tiny) == "f32"
+
+
+def test_both_arms_print_the_same_config_at_every_gpu_count():
+    """The reference arm's config and scaling are the ones our arm prints for
+    the same workload and N: the full config at N = 1, expert parallelism
+    (strong scaling) for N > 1 by default, replicas (weak) when asked."""
+    from sparse_moe_layer_gemm_b200.workloads import WORKLOADS
+    wl = WORKLOADS["decode"]
+    assert bench._arm_config(wl, 1, "auto") == (bench._config(wl, 1), "weak")
+    assert bench._arm_config(wl, 4, "auto") == (bench.ep_config(wl, 4), "strong")
+    assert bench._arm_config(wl, 4, "ep") == (bench.ep_config(wl, 4), "strong")
+    assert bench._arm_config(wl, 4, "replicas") == (bench._config(wl, 4), "weak")
