@@ -17,9 +17,8 @@ deterministic) values; a test always hands the same tensors to both sides.
 """
 from __future__ import annotations
 
-import math
-from dataclasses import dataclass, field, replace
-from typing import Dict, Optional
+from dataclasses import dataclass, replace
+from typing import Dict
 
 import torch
 

@@ -6,7 +6,6 @@ ragged last token block of the shared expert (narrow), distinct clamps, the
 gathered token rows of many small experts and exact selection ties."""
 from dataclasses import replace
 
-import numpy as np
 import pytest
 import torch
 

@@ -15,7 +15,7 @@ import torch
 import torch.nn.functional as F
 
 import oracle.moe_oracle as om
-from sparse_moe_layer_gemm_b200.workloads import WORKLOADS, make_inputs, Workload
+from sparse_moe_layer_gemm_b200.workloads import WORKLOADS, make_inputs
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
