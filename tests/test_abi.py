@@ -1,6 +1,6 @@
 """The C ABI without a GPU: the library loads, exports every symbol that
-include/moe.h declares, and rejects bad arguments on the host (no compute call
-is made here)."""
+include/moe.h declares, serves a plain C99 program, and rejects bad arguments
+on the host (no compute call is made here)."""
 import ctypes
 import os
 import re
@@ -150,3 +150,35 @@ def test_dense_host_checks(lib):
     v = ctypes.c_int()
     assert lib.moe_dense_get_device_error(None, ctypes.byref(v)) == B.MOE_ERR_INVALID_ARG
     lib.moe_dense_destroy(None)
+
+
+def test_a_plain_c_program_builds_and_calls_the_library(lib, tmp_path):
+    """The boundary is C: a C99 program that includes only include/moe.h
+    compiles warning-free, links against libmoe.so and calls host-only entry
+    points (no CUDA call is made)."""
+    src = tmp_path / "use_moe.c"
+    src.write_text(
+        '#include <string.h>\n'
+        '#include "moe.h"\n'
+        'int main(void) {\n'
+        '  moe_config_t c;\n'
+        '  memset(&c, 0, sizeof c);\n'
+        '  c.hidden = 4096; c.num_experts = 288; c.top_k = 8;\n'
+        '  c.intermediate = 1280; c.shared_intermediate = 1280;\n'
+        '  c.norm_expert_weight = 1; c.routed_scaling_factor = 3.0f;\n'
+        '  c.use_router_bias = 1; c.act_dtype = MOE_BF16; c.weight_dtype = MOE_BF16;\n'
+        '  if (moe_config_check(&c) != MOE_OK) return 1;\n'
+        '  c.top_k = 289;\n'
+        '  if (moe_config_check(&c) != MOE_ERR_INVALID_ARG) return 2;\n'
+        '  if (moe_config_check(0) != MOE_ERR_INVALID_ARG) return 3;\n'
+        '  if (strcmp(moe_status_string(MOE_OK), "ok") != 0) return 4;\n'
+        '  return 0;\n'
+        '}\n')
+    exe = tmp_path / "use_moe"
+    libdir = os.path.dirname(B.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I" + os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L" + libdir, "-lmoe", "-Wl,-rpath," + libdir],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stderr)
